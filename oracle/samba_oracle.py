@@ -1,0 +1,320 @@
+"""Float64 CPU oracle for Samba's two token mixers (test infrastructure only).
+
+This module is the slow, plain reference that the CUDA library is checked
+against.  It is test infrastructure: only the test suite, the smoke check in
+``__graft_entry__`` and the ``cpu_baseline`` / reference leg of ``bench.py``
+may import it.  It shares no code, constants or helpers with the CUDA path,
+and the CUDA path never imports it.
+
+Sources (pages on Samba, "Samba: Simple Hybrid State Space Models for
+Efficient Unlimited Context Language Modeling", Ren et al.):
+
+* "SAMBA混合注意力状态空间模型" (metaphor-xennon.pages.dev), section
+  "数学框架 / Mamba层": the selective recurrence h_t = Ā_t h_{t-1} + B̄_t x_t,
+  y_t = C_t h_t, with B_t, C_t and Δ_t = τ_Δ(Linear_Δ(x_t)) depending on the
+  input (the selective-parameter equation that follows it).
+* same page, section "滑动窗口注意力": softmax(Q Kᵀ / √d_k + M) V with a
+  window mask M.
+* same page, section "推理效率": the prefill ``forward`` followed by
+  ``mamba_step`` / ``swa_step`` decoding.
+* hackernoon page, §2.1.2 "Sliding Window Attention (SWA) Layer": a window
+  that slides over the sequence (w = 2048 in the paper).
+
+Readings taken where the pages are silent or garbled (each one is listed in
+the design notes as well):
+
+* Discretisation: Ā = exp(Δ·A) with a diagonal real A (one value per
+  channel and state), B̄·x = Δ·B·x.  The pages write Ā_t and B̄_t without a
+  formula; this is the zero-order-hold decay with an Euler input term of the
+  Mamba layer the paper builds on.
+* τ_Δ = softplus, applied to the raw per-channel input ``delta`` when
+  ``delta_softplus`` is set; no bias is added.
+* In front of the scan: a depthwise causal conv1d of width K (K = 4) with a
+  bias, followed by SiLU when ``conv_silu`` is set.  The scan input u is the
+  conv output.
+* Output: y = (C_t · h_t + D ⊙ u_t) ⊙ silu(z_t); the D skip and the z gate are
+  optional.
+* One group for B and C: B_t, C_t have N entries shared by all channels.
+* Window mask: key j is visible to query i exactly when 0 <= i - j < W
+  (causal, W keys including the query itself).  The page writes the mask
+  inverted and symmetric (|i - j| > W ↦ 0, else -inf); that cannot be meant
+  literally, since it would attend only to far-away keys.
+* Grouped-query attention: query head h reads key/value head
+  h // (H_q / H_kv).
+* Softmax scale 1/√d_k, as on the page.
+
+Every function works in float64.  Parity unpinned: none (each function has a
+pin in ``tests/test_oracle.py``).
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "softplus",
+    "silu",
+    "causal_conv1d",
+    "selective_scan",
+    "swa",
+    "swa_rows",
+    "scan_step",
+    "swa_step",
+    "ring_fill",
+]
+
+
+def _f64(a):
+    return None if a is None else np.asarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------- activations
+def softplus(w):
+    """τ_Δ = softplus(w) = log(1 + e^w), written to stay exact for large |w|.
+
+    Page "SAMBA混合注意力状态空间模型", §数学框架 / Mamba层, the selective-
+    parameter equation Δ_t = τ_Δ(Linear_Δ(x_t)).
+    """
+    w = _f64(w)
+    out = np.empty_like(w)
+    pos = w > 0
+    out[pos] = w[pos] + np.log1p(np.exp(-w[pos]))
+    out[~pos] = np.log1p(np.exp(w[~pos]))
+    return out
+
+
+def silu(x):
+    """SiLU / swish: x · σ(x) = x / (1 + e^{-x}).
+
+    The page's training configuration names "swish" (SiLU) as the activation.
+    """
+    x = _f64(x)
+    return x / (1.0 + np.exp(-x))
+
+
+# ----------------------------------------------------------------------- conv
+def causal_conv1d(x, weight, bias=None, state=None, apply_silu=True):
+    """Depthwise causal conv1d over time, channel-last.
+
+    u[b, t, c] = bias[c] + sum_{k=0}^{K-1} weight[c, k] * xpad[b, t + k, c]
+
+    where xpad is x with K-1 earlier inputs in front of it: ``state`` (shape
+    [B, D, K-1], oldest first) when given, else zeros.  weight[c, K-1] thus
+    multiplies x_t itself.  Returns (u, new_state) with new_state the last
+    K-1 inputs of xpad, i.e. the state a following call continues from.
+
+    x: [B, L, D]; weight: [D, K]; bias: [D] or None.
+    """
+    x = _f64(x)
+    weight = _f64(weight)
+    Bsz, L, D = x.shape
+    K = weight.shape[1]
+    if state is None:
+        state = np.zeros((Bsz, D, K - 1))
+    state = _f64(state)
+    xpad = np.concatenate([np.transpose(state, (0, 2, 1)), x], axis=1)  # [B, L+K-1, D]
+    u = np.zeros((Bsz, L, D))
+    for k in range(K):
+        u += weight[None, None, :, k] * xpad[:, k:k + L, :]
+    if bias is not None:
+        u += _f64(bias)[None, None, :]
+    if apply_silu:
+        u = silu(u)
+    new_state = np.transpose(xpad[:, L:L + K - 1, :], (0, 2, 1)).copy()
+    return u, new_state
+
+
+# ----------------------------------------------------------------------- scan
+def selective_scan(x, delta, A, Bm, Cm, Dskip=None, z=None, h0=None,
+                   conv_w=None, conv_b=None, conv_state=None,
+                   delta_softplus=True, conv_silu=True):
+    """Selective SSM prefill, sequential in time.
+
+    Page "SAMBA混合注意力状态空间模型", §数学框架 / Mamba层:
+        h_t = Ā_t h_{t-1} + B̄_t x_t,   y_t = C_t h_t
+    with, per channel c and state n (readings in the module docstring):
+        Δ[t, c]      = softplus(delta[t, c])          (if delta_softplus)
+        Ā[t, c, n]   = exp(Δ[t, c] * A[c, n])
+        B̄x[t, c, n]  = Δ[t, c] * B[t, n] * u[t, c]
+        y[t, c]      = (sum_n C[t, n] h[t, c, n] + D[c] u[t, c]) * silu(z[t, c])
+    where u = SiLU(conv1d(x)) if conv_w is given, else u = x.
+
+    Shapes: x, delta, z: [B, L, D]; A: [D, N]; Bm, Cm: [B, L, N]; Dskip: [D];
+    h0: [B, D, N]; conv_w: [D, K]; conv_b: [D]; conv_state: [B, D, K-1].
+    Returns dict(y [B, L, D], h [B, D, N], conv_state [B, D, K-1] or None).
+    """
+    x = _f64(x)
+    delta = _f64(delta)
+    A = _f64(A)
+    Bm = _f64(Bm)
+    Cm = _f64(Cm)
+    Bsz, L, D = x.shape
+    N = A.shape[1]
+
+    if conv_w is not None:
+        u, conv_state_out = causal_conv1d(x, conv_w, conv_b, conv_state, apply_silu=conv_silu)
+    else:
+        u, conv_state_out = x, None
+    dt = softplus(delta) if delta_softplus else delta
+
+    h = np.zeros((Bsz, D, N)) if h0 is None else _f64(h0).copy()
+    y = np.empty((Bsz, L, D))
+    for t in range(L):
+        dA = np.exp(dt[:, t, :, None] * A[None, :, :])                       # [B, D, N]
+        dBx = (dt[:, t, :] * u[:, t, :])[:, :, None] * Bm[:, t, None, :]      # [B, D, N]
+        h = dA * h + dBx
+        y[:, t, :] = np.einsum("bdn,bn->bd", h, Cm[:, t, :])
+    if Dskip is not None:
+        y = y + _f64(Dskip)[None, None, :] * u
+    if z is not None:
+        y = y * silu(z)
+    return {"y": y, "h": h, "conv_state": conv_state_out}
+
+
+def scan_step(h, conv_state, x_t, delta_t, A, B_t, C_t, Dskip=None, z_t=None,
+              conv_w=None, conv_b=None, delta_softplus=True, conv_silu=True):
+    """One decoding step of the selective scan (``mamba_step`` on the page's
+    §推理效率 pseudo-code): the recurrence of ``selective_scan`` with L = 1,
+    carrying the SSM state h [B, D, N] and the conv state [B, D, K-1].
+
+    x_t, delta_t, z_t: [B, D]; B_t, C_t: [B, N].  Returns (y_t, h, conv_state).
+    """
+    out = selective_scan(_f64(x_t)[:, None, :], _f64(delta_t)[:, None, :], A,
+                         _f64(B_t)[:, None, :], _f64(C_t)[:, None, :], Dskip,
+                         None if z_t is None else _f64(z_t)[:, None, :], h,
+                         conv_w, conv_b, conv_state, delta_softplus, conv_silu)
+    return out["y"][:, 0, :], out["h"], out["conv_state"]
+
+
+# ------------------------------------------------------------------------ SWA
+def _visible(i, j, window):
+    """Band mask of the sliding window: key j is visible to query i."""
+    return (i - j >= 0) & (i - j < window)
+
+
+def swa_rows(q, k, v, window, rows, scale=None):
+    """Sliding-window attention for the query rows ``rows`` only.
+
+    Page "SAMBA混合注意力状态空间模型", §滑动窗口注意力:
+        o_i = sum_j softmax_j(q_i · k_j / √d_k + M_ij) v_j
+    with M_ij = 0 for visible keys (0 <= i - j < W) and -inf otherwise, and
+    query head h reading kv head h // (H_q / H_kv).
+
+    q: [B, L, Hq, d]; k, v: [B, L, Hkv, d].  Returns (o [B, R, Hq, d],
+    lse [B, Hq, R]) for the R requested rows (natural-log logsumexp of the
+    scaled scores).
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    Bsz, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    group = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rows = np.asarray(rows, dtype=np.int64)
+    R = rows.shape[0]
+    o = np.zeros((Bsz, R, Hq, d))
+    lse = np.zeros((Bsz, Hq, R))
+    every_key = np.arange(L)
+    for r, i in enumerate(rows):
+        js = every_key[_visible(int(i), every_key, window)]
+        for h in range(Hq):
+            kv = h // group
+            s = np.einsum("bd,bjd->bj", q[:, i, h, :], k[:, js, kv, :]) * scale   # [B, J]
+            m = s.max(axis=1, keepdims=True)
+            p = np.exp(s - m)
+            den = p.sum(axis=1, keepdims=True)
+            o[:, r, h, :] = np.einsum("bj,bjd->bd", p / den, v[:, js, kv, :])
+            lse[:, h, r] = (m + np.log(den))[:, 0]
+    return o, lse
+
+
+def swa(q, k, v, window, scale=None, block=64):
+    """Sliding-window attention over all rows, processed per query block with
+    the banded slice of keys each block needs (same definition as swa_rows).
+
+    Returns (o [B, L, Hq, d], lse [B, Hq, L]).
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    Bsz, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    group = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = np.zeros((Bsz, L, Hq, d))
+    lse = np.zeros((Bsz, Hq, L))
+    for i0 in range(0, L, block):
+        i1 = min(L, i0 + block)
+        j0 = max(0, i0 - window + 1)
+        ii = np.arange(i0, i1)[:, None]
+        jj = np.arange(j0, i1)[None, :]
+        mask = _visible(ii, jj, window)                                     # [I, J]
+        for h in range(Hq):
+            kv = h // group
+            s = np.einsum("bid,bjd->bij", q[:, i0:i1, h, :], k[:, j0:i1, kv, :]) * scale
+            s = np.where(mask[None], s, -np.inf)
+            m = s.max(axis=2, keepdims=True)
+            p = np.exp(s - m)
+            den = p.sum(axis=2, keepdims=True)
+            o[:, i0:i1, h, :] = np.einsum("bij,bjd->bid", p / den, v[:, j0:i1, kv, :])
+            lse[:, h, i0:i1] = (m + np.log(den))[:, :, 0]
+    return o, lse
+
+
+def ring_fill(k, v, window):
+    """Decode state after a prefill of L tokens (the page's ``forward(prompt)``
+    filling the cache): the last min(L, W) keys and values, key of absolute
+    position p stored in slot p mod W, and the next position pos = L.
+
+    k, v: [B, L, Hkv, d].  Returns (k_ring, v_ring [B, W, Hkv, d], pos [B]).
+    """
+    k = _f64(k)
+    v = _f64(v)
+    Bsz, L, Hkv, d = k.shape
+    k_ring = np.zeros((Bsz, window, Hkv, d))
+    v_ring = np.zeros((Bsz, window, Hkv, d))
+    for p in range(max(0, L - window), L):
+        k_ring[:, p % window] = k[:, p]
+        v_ring[:, p % window] = v[:, p]
+    return k_ring, v_ring, np.full((Bsz,), L, dtype=np.int64)
+
+
+def swa_step(q_t, k_t, v_t, k_ring, v_ring, pos, window, scale=None):
+    """One decoding step of sliding-window attention (``swa_step`` on the
+    page's §推理效率 pseudo-code).
+
+    The new key/value (absolute position p = pos[b]) goes into slot p mod W;
+    the query then attends the keys of positions max(0, p - W + 1) .. p, which
+    are exactly the filled slots.  Softmax does not depend on the order of
+    the keys, so the slot order is irrelevant.
+
+    q_t: [B, Hq, d]; k_t, v_t: [B, Hkv, d]; rings [B, W, Hkv, d]; pos [B].
+    Returns (o_t [B, Hq, d], k_ring, v_ring, pos + 1) (rings updated copies).
+    """
+    q_t = _f64(q_t)
+    k_ring = _f64(k_ring).copy()
+    v_ring = _f64(v_ring).copy()
+    pos = np.asarray(pos, dtype=np.int64).copy()
+    Bsz, Hq, d = q_t.shape
+    Hkv = k_ring.shape[2]
+    group = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = np.zeros((Bsz, Hq, d))
+    for b in range(Bsz):
+        p = int(pos[b])
+        k_ring[b, p % window] = _f64(k_t)[b]
+        v_ring[b, p % window] = _f64(v_t)[b]
+        slots = np.array([a % window for a in range(max(0, p - window + 1), p + 1)])
+        for h in range(Hq):
+            kv = h // group
+            s = k_ring[b, slots, kv, :] @ q_t[b, h] * scale
+            e = np.exp(s - s.max())
+            o[b, h] = (e / e.sum()) @ v_ring[b, slots, kv, :]
+        pos[b] = p + 1
+    return o, k_ring, v_ring, pos

@@ -1,0 +1,361 @@
+"""Pins for the float64 oracle: each check ties it to something other than
+itself -- hand-worked values, closed forms, library routines on special
+cases, invariants and brute force on tiny inputs.  CPU only.
+
+A second group plants plausible mistakes in the oracle (monkeypatched, on
+the CPU) and shows that some pin catches each one.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle.samba_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+def _tiny_scan_inputs(seed=0, Bsz=1, L=64, D=16, N=4, K=4):
+    r = _rng(seed)
+    step = np.exp(r.uniform(math.log(1e-3), math.log(1e-1), size=(Bsz, L, D)))
+    return dict(
+        x=r.standard_normal((Bsz, L, D)),
+        z=r.standard_normal((Bsz, L, D)),
+        delta=np.log(np.expm1(step)),
+        A=-np.tile(np.arange(1, N + 1, dtype=np.float64), (D, 1)),
+        Bm=r.standard_normal((Bsz, L, N)),
+        Cm=r.standard_normal((Bsz, L, N)),
+        Dskip=r.standard_normal(D),
+        conv_w=r.uniform(-0.5, 0.5, size=(D, K)),
+        conv_b=r.uniform(-0.5, 0.5, size=D),
+    )
+
+
+# ----------------------------------------------------------- hand-worked values
+def test_scan_handworked_golden():
+    g = _load("scan_handworked.json")
+    i = g["inputs"]
+    out = orc.selective_scan(i["x"], i["delta"], i["A"], i["B"], i["C"], Dskip=i["D"],
+                             delta_softplus=False)
+    np.testing.assert_allclose(out["y"], g["expected"]["y"], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(out["h"], g["expected"]["h"], rtol=0, atol=1e-13)
+
+
+def test_conv_handworked_golden():
+    g = _load("conv_handworked.json")
+    i = g["inputs"]
+    u, st = orc.causal_conv1d(i["x"], i["w"], i["bias"], None, apply_silu=False)
+    np.testing.assert_allclose(u, g["expected"]["u_zero_state"], atol=1e-13)
+    np.testing.assert_allclose(st, g["expected"]["state_out"], atol=1e-13)
+    x3 = np.asarray(i["x"])[:, :3]
+    u2, _ = orc.causal_conv1d(x3, i["w"], i["bias"], i["state"], apply_silu=False)
+    np.testing.assert_allclose(u2, g["expected"]["u_with_state_first3"], atol=1e-13)
+
+
+def test_swa_handworked_golden():
+    g = _load("swa_handworked.json")
+    i = g["inputs"]
+    for fn in (orc.swa, lambda q, k, v, w: orc.swa_rows(q, k, v, w, np.arange(3))):
+        o, lse = fn(i["q"], i["k"], i["v"], i["window"])
+        np.testing.assert_allclose(o, g["expected"]["o"], atol=1e-13)
+        np.testing.assert_allclose(lse, g["expected"]["lse"], atol=1e-13)
+
+
+# ------------------------------------------------------------------ activations
+def test_softplus_closed_forms():
+    w = np.linspace(-40, 40, 2001)
+    sp = orc.softplus(w)
+    assert abs(orc.softplus(np.array([0.0]))[0] - math.log(2.0)) < 1e-15
+    np.testing.assert_allclose(sp - orc.softplus(-w), w, atol=1e-12)        # sp(w) - sp(-w) = w
+    # derivative is the logistic function (central differences)
+    eps = 1e-5
+    deriv = (orc.softplus(w + eps) - orc.softplus(w - eps)) / (2 * eps)
+    np.testing.assert_allclose(deriv, scipy.special.expit(w), atol=1e-8)
+    # inverse used by the input recipe: softplus(log(expm1(s))) = s
+    s = np.exp(np.linspace(math.log(1e-3), math.log(1e-1), 101))
+    np.testing.assert_allclose(orc.softplus(np.log(np.expm1(s))), s, rtol=1e-13)
+
+
+def test_silu_closed_forms():
+    x = np.linspace(-30, 30, 1201)
+    y = orc.silu(x)
+    assert orc.silu(np.array([0.0]))[0] == 0.0
+    np.testing.assert_allclose(y - orc.silu(-x), x, atol=1e-12)              # odd part is x/2
+    np.testing.assert_allclose(y, x * scipy.special.expit(x), rtol=1e-14, atol=1e-300)
+
+
+# ------------------------------------------------------------------------- conv
+def test_conv_matches_torch_conv1d():
+    i = _tiny_scan_inputs(1, Bsz=2, L=37, D=8)
+    x = torch.from_numpy(i["x"])                                              # [B, L, D]
+    w = torch.from_numpy(i["conv_w"])                                         # [D, K]
+    b = torch.from_numpy(i["conv_b"])
+    ref = torch.nn.functional.conv1d(x.transpose(1, 2), w[:, None, :], b, padding=3,
+                                     groups=x.shape[2])[..., :x.shape[1]].transpose(1, 2)
+    u, _ = orc.causal_conv1d(i["x"], i["conv_w"], i["conv_b"], apply_silu=False)
+    np.testing.assert_allclose(u, ref.numpy(), atol=1e-13)
+    u_silu, _ = orc.causal_conv1d(i["x"], i["conv_w"], i["conv_b"], apply_silu=True)
+    np.testing.assert_allclose(u_silu, torch.nn.functional.silu(ref).numpy(), atol=1e-13)
+
+
+def test_conv_state_carry_equals_one_pass():
+    i = _tiny_scan_inputs(2, Bsz=2, L=40, D=8)
+    full, st_full = orc.causal_conv1d(i["x"], i["conv_w"], i["conv_b"])
+    for cut in (1, 2, 3, 17, 39):
+        a, st = orc.causal_conv1d(i["x"][:, :cut], i["conv_w"], i["conv_b"])
+        b, st2 = orc.causal_conv1d(i["x"][:, cut:], i["conv_w"], i["conv_b"], st)
+        np.testing.assert_allclose(np.concatenate([a, b], 1), full, atol=1e-13)
+        np.testing.assert_allclose(st2, st_full, atol=0)
+
+
+# ------------------------------------------------------------------------- scan
+def _brute_force_scan(i, h0=None):
+    """Unrolled sum, written from the definition with explicit loops:
+    y_t = (C_t . sum_{s<=t} (prod_{r=s+1}^{t} exp(Δ_r A)) Δ_s B_s u_s
+           + C_t . (prod_{r<=t} exp(Δ_r A)) h0 + D u_t) * silu(z_t)."""
+    x, z = i["x"], i["z"]
+    Bsz, L, D = x.shape
+    K = i["conv_w"].shape[1]
+    N = i["A"].shape[1]
+    u = np.zeros_like(x)
+    for b in range(Bsz):
+        for t in range(L):
+            for c in range(D):
+                acc = i["conv_b"][c]
+                for k in range(K):
+                    tt = t - (K - 1) + k
+                    if tt >= 0:
+                        acc += i["conv_w"][c, k] * x[b, tt, c]
+                u[b, t, c] = acc / (1.0 + math.exp(-acc))
+    dt = np.vectorize(lambda w: math.log1p(math.exp(w)))(i["delta"])
+    y = np.zeros_like(x)
+    for b in range(Bsz):
+        for c in range(D):
+            for t in range(L):
+                tot = 0.0
+                for n in range(N):
+                    hn = 0.0
+                    if h0 is not None:
+                        hn = math.exp(i["A"][c, n] * dt[b, :t + 1, c].sum()) * h0[b, c, n]
+                    for s in range(t + 1):
+                        decay = math.exp(i["A"][c, n] * dt[b, s + 1:t + 1, c].sum())
+                        hn += decay * dt[b, s, c] * i["Bm"][b, s, n] * u[b, s, c]
+                    tot += i["Cm"][b, t, n] * hn
+                g = z[b, t, c] / (1.0 + math.exp(-z[b, t, c]))
+                y[b, t, c] = (tot + i["Dskip"][c] * u[b, t, c]) * g
+    return y
+
+
+def test_scan_matches_unrolled_sum():
+    i = _tiny_scan_inputs(0, L=24, D=6, N=4)
+    out = orc.selective_scan(**i)
+    np.testing.assert_allclose(out["y"], _brute_force_scan(i), rtol=1e-12, atol=1e-12)
+    h0 = _rng(5).standard_normal((1, 6, 4))
+    out = orc.selective_scan(**i, h0=h0)
+    np.testing.assert_allclose(out["y"], _brute_force_scan(i, h0), rtol=1e-12, atol=1e-12)
+
+
+def test_scan_A_zero_is_prefix_sum():
+    i = _tiny_scan_inputs(3, Bsz=2, L=50, D=5, N=3)
+    dt = np.exp(_rng(4).uniform(-5, 0, size=i["x"].shape))
+    out = orc.selective_scan(i["x"], dt, np.zeros((5, 3)), i["Bm"], i["Cm"], delta_softplus=False)
+    inc = (dt * i["x"])[..., None] * i["Bm"][:, :, None, :]                  # [B, L, D, N]
+    h = np.cumsum(inc, axis=1)
+    np.testing.assert_allclose(out["h"], h[:, -1], rtol=1e-12)
+    np.testing.assert_allclose(out["y"], np.einsum("bldn,bln->bld", h, i["Cm"]), rtol=1e-12, atol=1e-12)
+
+
+def test_scan_delta_zero_keeps_state():
+    i = _tiny_scan_inputs(5, Bsz=2, L=20, D=4, N=4)
+    h0 = _rng(6).standard_normal((2, 4, 4))
+    out = orc.selective_scan(i["x"], np.zeros_like(i["x"]), i["A"], i["Bm"], i["Cm"], i["Dskip"],
+                             h0=h0, delta_softplus=False)
+    np.testing.assert_array_equal(out["h"], h0)
+    exp_y = np.einsum("bdn,bln->bld", h0, i["Cm"]) + i["Dskip"] * i["x"]
+    np.testing.assert_allclose(out["y"], exp_y, rtol=1e-13, atol=1e-13)
+
+
+def test_scan_linear_in_input_and_state():
+    i = _tiny_scan_inputs(7, Bsz=1, L=30, D=4, N=4)
+    r = _rng(8)
+    u1, u2 = r.standard_normal(i["x"].shape), r.standard_normal(i["x"].shape)
+    h1, h2 = r.standard_normal((1, 4, 4)), r.standard_normal((1, 4, 4))
+    a, b = 0.7, -1.9
+
+    def run(u, h):
+        o = orc.selective_scan(u, i["delta"], i["A"], i["Bm"], i["Cm"], i["Dskip"], h0=h)
+        return o["y"], o["h"]
+
+    y, h = run(a * u1 + b * u2, a * h1 + b * h2)
+    ya, ha = run(u1, h1)
+    yb, hb = run(u2, h2)
+    np.testing.assert_allclose(y, a * ya + b * yb, atol=1e-11)
+    np.testing.assert_allclose(h, a * ha + b * hb, atol=1e-11)
+
+
+def test_scan_split_with_carry_equals_one_pass():
+    i = _tiny_scan_inputs(9, Bsz=2, L=64, D=8, N=4)
+    full = orc.selective_scan(**i)
+    for cut in (1, 3, 31, 63):
+        first = {k: (v[:, :cut] if k in ("x", "z", "delta", "Bm", "Cm") else v) for k, v in i.items()}
+        rest = {k: (v[:, cut:] if k in ("x", "z", "delta", "Bm", "Cm") else v) for k, v in i.items()}
+        a = orc.selective_scan(**first)
+        b = orc.selective_scan(**rest, h0=a["h"], conv_state=a["conv_state"])
+        np.testing.assert_allclose(np.concatenate([a["y"], b["y"]], 1), full["y"], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(b["h"], full["h"], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(b["conv_state"], full["conv_state"], atol=0)
+
+
+def test_scan_step_sequence_equals_prefill():
+    i = _tiny_scan_inputs(10, Bsz=2, L=40, D=8, N=4)
+    full = orc.selective_scan(**i)
+    L1 = 25
+    pre = orc.selective_scan(**{k: (v[:, :L1] if k in ("x", "z", "delta", "Bm", "Cm") else v)
+                                for k, v in i.items()})
+    h, cs = pre["h"], pre["conv_state"]
+    for t in range(L1, 40):
+        y_t, h, cs = orc.scan_step(h, cs, i["x"][:, t], i["delta"][:, t], i["A"], i["Bm"][:, t],
+                                   i["Cm"][:, t], i["Dskip"], i["z"][:, t], i["conv_w"], i["conv_b"])
+        np.testing.assert_allclose(y_t, full["y"][:, t], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(h, full["h"], rtol=1e-12, atol=1e-12)
+
+
+# -------------------------------------------------------------------------- SWA
+def _attn_inputs(seed, Bsz, L, Hq, Hkv, d):
+    r = _rng(seed)
+    return (r.standard_normal((Bsz, L, Hq, d)), r.standard_normal((Bsz, L, Hkv, d)),
+            r.standard_normal((Bsz, L, Hkv, d)))
+
+
+def _sdpa_causal(q, k, v):
+    group = q.shape[2] // k.shape[2]
+    qt = torch.from_numpy(q).permute(0, 2, 1, 3)
+    kt = torch.from_numpy(np.repeat(k, group, axis=2)).permute(0, 2, 1, 3)
+    vt = torch.from_numpy(np.repeat(v, group, axis=2)).permute(0, 2, 1, 3)
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True)
+    return o.permute(0, 2, 1, 3).numpy()
+
+
+@pytest.mark.parametrize("W", [40, 41, 1000])
+def test_swa_wide_window_is_full_causal_sdpa(W):
+    q, k, v = _attn_inputs(11, 2, 40, 8, 2, 16)
+    ref = _sdpa_causal(q, k, v)
+    o, _ = orc.swa(q, k, v, W, block=16)
+    np.testing.assert_allclose(o, ref, atol=1e-12)
+    o2, _ = orc.swa_rows(q, k, v, W, np.arange(40))
+    np.testing.assert_allclose(o2, ref, atol=1e-12)
+
+
+def test_swa_window_one_returns_v():
+    q, k, v = _attn_inputs(12, 2, 33, 4, 2, 16)
+    o, lse = orc.swa(q, k, v, 1, block=8)
+    np.testing.assert_allclose(o, np.repeat(v, 2, axis=2), atol=1e-14)
+    s = np.einsum("blhd,blhd->bhl", q, np.repeat(k, 2, axis=2)) / 4.0
+    np.testing.assert_allclose(lse, s, atol=1e-12)
+
+
+@pytest.mark.parametrize("W", [1, 5, 16, 70])
+def test_swa_equal_scores_give_window_mean(W):
+    _, k, v = _attn_inputs(13, 1, 50, 4, 4, 8)
+    q = np.zeros((1, 50, 4, 8))
+    o, lse = orc.swa(q, k, v, W, block=16)
+    for i in range(50):
+        j0 = max(0, i - W + 1)
+        np.testing.assert_allclose(o[0, i], v[0, j0:i + 1].mean(axis=0), atol=1e-13)
+        np.testing.assert_allclose(lse[0, :, i], math.log(i + 1 - j0), atol=1e-13)
+
+
+def test_swa_gqa_equals_mha_with_repeated_kv():
+    q, k, v = _attn_inputs(14, 2, 45, 8, 2, 16)
+    o, lse = orc.swa(q, k, v, 9, block=16)
+    o2, lse2 = orc.swa(q, np.repeat(k, 4, axis=2), np.repeat(v, 4, axis=2), 9, block=16)
+    np.testing.assert_allclose(o, o2, atol=1e-14)
+    np.testing.assert_allclose(lse, lse2, atol=1e-14)
+
+
+@pytest.mark.parametrize("W", [1, 3, 16, 64])
+def test_swa_matches_full_masked_softmax(W):
+    q, k, v = _attn_inputs(15, 1, 64, 2, 2, 16)
+    L, d = 64, 16
+    o, lse = orc.swa(q, k, v, W, block=16)
+    for h in range(2):
+        s = q[0, :, h, :] @ k[0, :, h, :].T / math.sqrt(d)
+        i, j = np.meshgrid(np.arange(L), np.arange(L), indexing="ij")
+        s = np.where((j <= i) & (j > i - W), s, -np.inf)
+        p = scipy.special.softmax(s, axis=1)
+        np.testing.assert_allclose(o[0, :, h, :], p @ v[0, :, h, :], atol=1e-12)
+        np.testing.assert_allclose(lse[0, h], scipy.special.logsumexp(s, axis=1), atol=1e-12)
+
+
+def test_swa_rows_equals_blocked():
+    q, k, v = _attn_inputs(16, 2, 70, 8, 2, 16)
+    o, lse = orc.swa(q, k, v, 20, block=32)
+    rows = np.array([0, 1, 19, 20, 21, 45, 69])
+    o2, lse2 = orc.swa_rows(q, k, v, 20, rows)
+    np.testing.assert_allclose(o2, o[:, rows], atol=1e-13)
+    np.testing.assert_allclose(lse2, lse[:, :, rows], atol=1e-13)
+
+
+@pytest.mark.parametrize("L1,W", [(10, 16), (40, 16), (16, 16), (1, 4)])
+def test_swa_decode_steps_equal_prefill(L1, W):
+    L = L1 + 20
+    q, k, v = _attn_inputs(17, 2, L, 8, 2, 16)
+    full, _ = orc.swa(q, k, v, W, block=16)
+    kr, vr, pos = orc.ring_fill(k[:, :L1], v[:, :L1], W)
+    assert np.all(pos == L1)
+    for t in range(L1, L):
+        o_t, kr, vr, pos = orc.swa_step(q[:, t], k[:, t], v[:, t], kr, vr, pos, W)
+        np.testing.assert_allclose(o_t, full[:, t], atol=1e-12)
+    assert np.all(pos == L)
+
+
+# ----------------------------------------------- planted mistakes are caught
+def test_planted_symmetric_mask_is_caught(monkeypatch):
+    """The page's literal symmetric band |i - j| <= W is non-causal."""
+    monkeypatch.setattr(orc, "_visible", lambda i, j, W: np.abs(i - j) < W)
+    q, k, v = _attn_inputs(18, 1, 30, 2, 2, 8)
+    o, _ = orc.swa_rows(q, k, v, 1000, np.arange(30))
+    assert not np.allclose(o, _sdpa_causal(q, k, v), atol=1e-6)
+
+
+def test_planted_window_off_by_one_is_caught(monkeypatch):
+    monkeypatch.setattr(orc, "_visible", lambda i, j, W: (i - j >= 0) & (i - j <= W))
+    q, k, v = _attn_inputs(19, 1, 30, 2, 2, 8)
+    o, _ = orc.swa_rows(q, k, v, 1, np.arange(30))
+    assert not np.allclose(o, v, atol=1e-6)
+
+
+def test_planted_scan_mistakes_are_caught(monkeypatch):
+    i = _tiny_scan_inputs(20, L=12, D=3, N=2)
+    ref = _brute_force_scan(i)
+    good = orc.selective_scan(**i)["y"]
+    assert np.allclose(good, ref, atol=1e-12)
+    # (a) softplus dropped
+    monkeypatch.setattr(orc, "softplus", lambda w: np.asarray(w, dtype=np.float64))
+    assert not np.allclose(orc.selective_scan(**i)["y"], ref, atol=1e-6)
+    monkeypatch.undo()
+    # (b) SiLU after the conv dropped
+    bad = orc.selective_scan(**i, conv_silu=False)["y"]
+    assert not np.allclose(bad, ref, atol=1e-6)
+    # (c) D skip dropped
+    j = dict(i)
+    j["Dskip"] = None
+    assert not np.allclose(orc.selective_scan(**j)["y"], ref, atol=1e-6)
+    # (d) conv taps reversed (weight[c, 0] on x_t)
+    j = dict(i)
+    j["conv_w"] = i["conv_w"][:, ::-1].copy()
+    assert not np.allclose(orc.selective_scan(**j)["y"], ref, atol=1e-6)
