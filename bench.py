@@ -1,0 +1,400 @@
+#!/usr/bin/env python
+"""Throughput of the Samba mixer prefill on B200.
+
+One step = one samba_mixer_prefill call: the fused selective scan (conv,
+softplus, scan, D skip, gate; bf16 y, fp32 final state and conv state) and
+the banded sliding-window attention (bf16, 32 q / 4 kv heads, d = 64,
+W = 2048) over one batch of the 128K-token workload (B = 1, L = 131072,
+d_inner = 4096, N = 16).  Inputs are synthetic (seeded) and resident in HBM;
+each input is larger than L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl samba|reference]
+
+With N > 1 (torchrun) every rank runs its own batch (weak scaling, no
+collective on the data path); the time is the max over ranks.  --impl
+reference times the float64 CPU oracle on bounded samples of the same
+workload.  Prints one JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Samba mixer prefill tokens/s @128K; scan HBM GB/s; SWA tensor-pipe %"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="samba", choices=["samba", "reference"])
+    ap.add_argument("--workload", default="prefill_128k")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--kernel-steps", type=int, default=50)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mp = json.load(f)
+        return {"hbm_gbs": mp["hbm_gbs"], "bf16_tflops": mp["bf16_tflops"],
+                "bf16_tflops_sustained": mp.get("bf16_tflops_sustained", mp["bf16_tflops"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def workload_config(wl):
+    return {"workload": wl.name, "batch": wl.batch, "seq_len": wl.seqlen, "d_inner": wl.dim, "d_state": wl.dstate,
+            "d_conv": wl.dconv, "heads_q": wl.heads_q, "heads_kv": wl.heads_kv, "head_dim": wl.head_dim,
+            "window": wl.window, "l2": "no flush: every input tensor is larger than the 126 MB L2"}
+
+
+# ----------------------------------------------------------------- algorithmic work
+def scan_bytes(wl):
+    """HBM bytes the scan must move once: x, z (bf16), delta (fp32) in, y
+    (bf16) out per (token, channel); B and C per token; the final state and
+    conv state out and the small per-channel parameters."""
+    tc = wl.batch * wl.seqlen * wl.dim
+    per_token = 2 * wl.dstate * 4
+    small = wl.batch * wl.dim * (wl.dstate + 3) * 4 + wl.dim * (wl.dstate + wl.dconv + 2) * 4
+    return tc * (2 + 2 + 4 + 2) + wl.batch * wl.seqlen * per_token + small
+
+
+def swa_flops(wl):
+    """Band FLOPs 4·L·W·d per (batch, query head)."""
+    return 4.0 * wl.seqlen * wl.window * wl.head_dim * wl.batch * wl.heads_q
+
+
+def swa_exact_band_flops(wl):
+    L, W = wl.seqlen, wl.window
+    pairs = sum(min(i + 1, W) for i in range(0, min(L, W))) + max(0, L - W) * W
+    return 4.0 * pairs * wl.head_dim * wl.batch * wl.heads_q
+
+
+# ----------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------- oracle leg
+def oracle_throughput(wl, n_chan=256, n_tok=2048, n_rows=64, seed=0):
+    """Times the float64 oracle, as it stands, on a bounded sample of the
+    workload and extrapolates to tokens/s of the whole mixer pair: the scan
+    on n_chan channels x n_tok tokens (cost scaled by D / n_chan), SWA on
+    n_rows query rows of every head (rows past the window's ramp)."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    import oracle.samba_oracle as orc
+
+    rng = np.random.default_rng(seed)
+    N, K = wl.dstate, wl.dconv
+    x = rng.standard_normal((1, n_tok, n_chan))
+    z = rng.standard_normal((1, n_tok, n_chan))
+    delta = np.log(np.expm1(np.exp(rng.uniform(math.log(1e-3), math.log(1e-1), (1, n_tok, n_chan)))))
+    A = -np.tile(np.arange(1, N + 1, dtype=np.float64), (n_chan, 1))
+    Bm = rng.standard_normal((1, n_tok, N))
+    Cm = rng.standard_normal((1, n_tok, N))
+    Ds = rng.standard_normal(n_chan)
+    cw = rng.uniform(-0.5, 0.5, (n_chan, K))
+    cb = rng.uniform(-0.5, 0.5, n_chan)
+    span = wl.window + n_rows
+    q = rng.standard_normal((1, span, wl.heads_q, wl.head_dim))
+    k = rng.standard_normal((1, span, wl.heads_kv, wl.head_dim))
+    v = rng.standard_normal((1, span, wl.heads_kv, wl.head_dim))
+    rows = np.arange(span - n_rows, span)
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        orc.selective_scan(x, delta, A, Bm, Cm, Ds, z, conv_w=cw, conv_b=cb)
+        t_scan = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        orc.swa_rows(q, k, v, wl.window, rows)
+        t_swa = time.perf_counter() - t0
+    per_token = t_scan / n_tok * (wl.dim / n_chan) + t_swa / n_rows
+    sample = (f"scan: {n_chan} of {wl.dim} channels x {n_tok} tokens ({t_scan:.1f} s, scaled by channels); "
+              f"swa: {n_rows} query rows x {wl.heads_q} heads at full window ({t_swa:.1f} s); "
+              f"float64 NumPy, extrapolated to whole-workload tokens/s")
+    return 1.0 / per_token, 1, sample
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from hybrid_ssm_sliding_b200.workloads import WORKLOADS
+
+    wl = WORKLOADS[args.workload]
+    # Each step is a bounded sample (a few hundred ms), so K steps stay short.
+    for _ in range(max(0, args.warmup)):
+        oracle_throughput(wl, n_chan=64, n_tok=64, n_rows=1)
+    vals, samples = [], ""
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        v, cores, samples = oracle_throughput(wl, n_chan=256, n_tok=128, n_rows=2, seed=s)
+        vals.append(v)
+    wall = time.perf_counter() - t0
+    value = statistics.median(vals)
+    tokens_per_step = wl.batch * wl.seqlen
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": tokens_per_step / value * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": samples + f"; median of {args.steps} samples ({wall:.1f} s)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# -------------------------------------------------------------------- GPU leg
+def main():
+    args = parse()
+    if args.impl == "reference":
+        sys.exit(run_reference(args))
+
+    import torch
+    import torch.distributed as dist
+
+    from hybrid_ssm_sliding_b200 import _lib as L
+    from hybrid_ssm_sliding_b200 import build as B
+    from hybrid_ssm_sliding_b200 import ops
+    from hybrid_ssm_sliding_b200.workloads import WORKLOADS, make_prefill_inputs
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+    if local == 0:
+        B.build()
+    if world > 1:
+        dist.barrier()
+    lib = L.load()
+
+    wl = WORKLOADS[args.workload]
+    from dataclasses import replace
+    wl_rank = replace(wl, seed=wl.seed + 1000 * rank)   # each rank its own batch
+    inp = make_prefill_inputs(wl_rank, device=dev)
+    Bsz, Ln, D, N, K = wl.batch, wl.seqlen, wl.dim, wl.dstate, wl.dconv
+    y = torch.empty((Bsz, Ln, D), dtype=torch.bfloat16, device=dev)
+    h_final = torch.empty((Bsz, D, N), dtype=torch.float32, device=dev)
+    cs_out = torch.empty((Bsz, D, K - 1), dtype=torch.float32, device=dev)
+    o = torch.empty_like(inp["q"])
+    scan_kw = dict(x=inp["x"], delta=inp["delta"], A=inp["A"], B=inp["B"], C=inp["C"], D=inp["D"], z=inp["z"],
+                   conv_w=inp["conv_w"], conv_b=inp["conv_b"], y=y, h_final=h_final, conv_state_out=cs_out)
+    swa_kw = dict(q=inp["q"], k=inp["k"], v=inp["v"], window=wl.window, o=o)
+    sa, _ = ops._scan_struct(**scan_kw)
+    wa, _ = ops._swa_struct(**swa_kw)
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+
+    def step():
+        rc = lib.samba_mixer_prefill(ctypes.byref(sa), ctypes.byref(wa), sh, None)
+        if rc != 0:
+            L.check(rc)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K mixer-prefill steps
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = e0.elapsed_time(e1)
+    clk = clocks.stop()
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    tokens_all = world * Bsz * Ln
+    value = tokens_all / (ms_step / 1e3)
+    status = ops.get_status()
+
+    # ---- per-kernel times (each kernel alone, back to back, same stream)
+    def time_kernel(fn, n):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    ms_scan = time_kernel(lambda: L.check(lib.samba_selective_scan_fwd(ctypes.byref(sa), sh)), args.kernel_steps)
+    ms_swa = time_kernel(lambda: L.check(lib.samba_swa_fwd(ctypes.byref(wa), sh)), args.kernel_steps)
+    peaks = load_peaks()
+    sb = scan_bytes(wl)
+    sf = swa_flops(wl)
+    scan_gbs = sb / (ms_scan / 1e3) / 1e9
+    swa_tfs = sf / (ms_swa / 1e3) / 1e12
+    scan_roof = {"bound": "hbm", "achieved": scan_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                 "frac": scan_gbs / peaks["hbm_gbs"], "traffic": None, "ms": ms_scan,
+                 "algorithmic_bytes": sb, "peak_source": peaks["source"]}
+    swa_roof = {"bound": "tensor", "achieved": swa_tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": swa_tfs / peaks["bf16_tflops"], "traffic": None, "ms": ms_swa, "band_flops": sf,
+                "exact_band_flops": swa_exact_band_flops(wl), "peak_source": peaks["source"] + " burst"}
+    traffic_file = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(traffic_file):
+        try:
+            tr = json.load(open(traffic_file))
+            for name, roof in (("scan", scan_roof), ("swa", swa_roof)):
+                ent = tr.get(name, {}).get(wl.name)
+                if ent and ent.get("source_hash") == B.source_hash():
+                    roof["traffic"] = ent["bytes_per_launch"]
+        except Exception:
+            pass
+    dominant = swa_roof if ms_swa >= ms_scan else scan_roof
+    roofline = {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+    roofline["kernel"] = "swa_fwd_kernel" if dominant is swa_roof else "scan_fwd_kernel"
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = {k: v.to("cpu").pin_memory() for k, v in inp.items()}
+        dev_in = {k: torch.empty_like(v) for k, v in inp.items()}
+        y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = y_h.numel() * y_h.element_size() + o_h.numel() * o_h.element_size()
+        skw = dict(scan_kw)
+        wkw = dict(swa_kw)
+        for kk in ("x", "delta", "A", "B", "C", "D", "z", "conv_w", "conv_b"):
+            skw[kk] = dev_in[kk]
+        for kk in ("q", "k", "v"):
+            wkw[kk] = dev_in[kk]
+
+        def e2e_step():
+            for kk in host:
+                dev_in[kk].copy_(host[kk], non_blocking=True)
+            ops.mixer_prefill(skw, wkw)
+            y_h.copy_(y, non_blocking=True)
+            o_h.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = a.elapsed_time(b) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": tokens_all / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = oracle_throughput(wl)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(wl),
+            "roofline": roofline, "kernels": {"scan": scan_roof, "swa": swa_roof},
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "gpu_launches": 2 * args.steps,
+            "status": status,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,385 @@
+// Standalone conv1d and the single-token decode kernels (mamba_step and
+// swa_step of the decode loop in the "推理效率" section of the page
+// "SAMBA混合注意力状态空间模型"), plus the prefill -> decode ring hand-off.
+#include <algorithm>
+#include <cmath>
+
+#include "common.cuh"
+#include "host.hpp"
+
+namespace samba {
+
+int take_status_misc(cudaStream_t s) { return take_status_word(s); }
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float silu_dev(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
+__device__ __forceinline__ float softplus_dev(float w) {
+  return w > 20.0f ? w : (w > 0.0f ? w + log1pf(__expf(-w)) : log1pf(__expf(w)));
+}
+
+template <typename T>
+__device__ __forceinline__ float ld_any(const void* p, int64_t i) {
+  return to_f32<T>(reinterpret_cast<const T*>(p)[i]);
+}
+
+// ---------------------------------------------------------------- conv1d
+// u[b,t,c] = bias[c] + sum_k w[c,k] x[b,t-K+1+k,c] (earlier inputs from the
+// conv state), then SiLU.  One thread per output element.
+template <typename XT, typename UT>
+__global__ void conv1d_kernel(const XT* __restrict__ x, const float* __restrict__ w, const float* __restrict__ bias,
+                              const float* __restrict__ cs_in, UT* __restrict__ u, int64_t B, int64_t L, int64_t D,
+                              int K, int silu) {
+  const int64_t n = B * L * D;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t c = e % D;
+    const int64_t t = (e / D) % L;
+    const int64_t b = e / (D * L);
+    float acc = bias ? bias[c] : 0.f;
+    for (int k = 0; k < K; ++k) {
+      const int64_t tt = t - (K - 1) + k;
+      float xv;
+      if (tt >= 0) xv = to_f32<XT>(x[(b * L + tt) * D + c]);
+      else xv = cs_in ? cs_in[(b * D + c) * (K - 1) + (K - 1) + tt] : 0.f;
+      acc = fmaf(w[c * K + k], xv, acc);
+    }
+    if (silu) acc = silu_dev(acc);
+    u[e] = from_f32<UT>(acc);
+  }
+}
+
+template <typename XT>
+__global__ void conv_state_kernel(const XT* __restrict__ x, const float* __restrict__ cs_in,
+                                  float* __restrict__ cs_out, int64_t B, int64_t L, int64_t D, int K) {
+  const int64_t n = B * D * (K - 1);
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const int j = (int)(e % (K - 1));
+    const int64_t c = (e / (K - 1)) % D;
+    const int64_t b = e / ((K - 1) * D);
+    const int64_t src = L + j - (K - 1);
+    float v;
+    if (src >= 0) v = to_f32<XT>(x[(b * L + src) * D + c]);
+    else v = cs_in ? cs_in[(b * D + c) * (K - 1) + (K - 1) + src] : 0.f;
+    cs_out[e] = v;
+  }
+}
+
+template <typename XT, typename UT>
+static void conv1d_go(const void* x, const float* w, const float* bias, const float* cs_in, void* u, float* cs_out,
+                      int64_t B, int64_t L, int64_t D, int K, int silu, cudaStream_t s) {
+  const int64_t n = B * L * D;
+  const int threads = 256;
+  const int blocks = (int)std::min<int64_t>((n + threads - 1) / threads, (int64_t)sm_count() * 16);
+  conv1d_kernel<XT, UT><<<blocks, threads, 0, s>>>(reinterpret_cast<const XT*>(x), w, bias, cs_in,
+                                                    reinterpret_cast<UT*>(u), B, L, D, K, silu);
+  if (cs_out) {
+    const int64_t m = B * D * (K - 1);
+    conv_state_kernel<XT><<<(int)std::min<int64_t>((m + 255) / 256, 4096), 256, 0, s>>>(
+        reinterpret_cast<const XT*>(x), cs_in, cs_out, B, L, D, K);
+  }
+}
+
+int launch_conv1d(const void* x, int x_dtype, const float* w, const float* bias, const float* cs_in, void* u,
+                  int u_dtype, float* cs_out, int64_t B, int64_t L, int64_t D, int K, int silu, cudaStream_t s) {
+  const bool xb = x_dtype == SAMBA_BF16, ub = u_dtype == SAMBA_BF16;
+  if (xb && ub) conv1d_go<__nv_bfloat16, __nv_bfloat16>(x, w, bias, cs_in, u, cs_out, B, L, D, K, silu, s);
+  else if (xb) conv1d_go<__nv_bfloat16, float>(x, w, bias, cs_in, u, cs_out, B, L, D, K, silu, s);
+  else if (ub) conv1d_go<float, __nv_bfloat16>(x, w, bias, cs_in, u, cs_out, B, L, D, K, silu, s);
+  else conv1d_go<float, float>(x, w, bias, cs_in, u, cs_out, B, L, D, K, silu, s);
+  return check_launch("samba_conv1d_fwd");
+}
+
+// -------------------------------------------------------------- scan step
+// One thread per (batch, channel) holding its N states.  Same arithmetic as
+// the prefill kernel with L = 1.
+template <int N, typename XT, typename YT>
+__global__ void scan_step_kernel(float* __restrict__ h, float* __restrict__ cs, const XT* __restrict__ x_t,
+                                 const XT* __restrict__ z_t, const float* __restrict__ delta_t,
+                                 const float* __restrict__ B_t, const float* __restrict__ C_t,
+                                 const float* __restrict__ A, const float* __restrict__ Dskip,
+                                 const float* __restrict__ conv_w, const float* __restrict__ conv_b,
+                                 YT* __restrict__ y_t, int64_t Bsz, int64_t D, int K, uint32_t flags) {
+  const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (e >= Bsz * D) return;
+  const int64_t b = e / D, c = e % D;
+  const float xv = to_f32<XT>(x_t[e]);
+  float u;
+  if (flags & SAMBA_SCAN_FUSE_CONV) {
+    float* st = cs + e * (K - 1);
+    float acc = conv_b ? conv_b[c] : 0.f;
+    for (int k = 0; k < K - 1; ++k) acc = fmaf(conv_w[c * K + k], st[k], acc);
+    acc = fmaf(conv_w[c * K + K - 1], xv, acc);
+    for (int k = 0; k + 1 < K - 1; ++k) st[k] = st[k + 1];
+    st[K - 2] = xv;
+    u = (flags & SAMBA_SCAN_CONV_SILU) ? silu_dev(acc) : acc;
+  } else {
+    u = xv;
+  }
+  const float wr = delta_t[e];
+  const float dlt = (flags & SAMBA_SCAN_DELTA_SOFTPLUS) ? softplus_dev(wr) : wr;
+  const float du = dlt * u;
+  float* hp = h + e * N;
+  const float* Ap = A + c * N;
+  const float* Bp = B_t + b * N;
+  const float* Cp = C_t + b * N;
+  float acc = 0.f;
+#pragma unroll
+  for (int n = 0; n < N; n += 4) {
+    float4 hv = *reinterpret_cast<float4*>(hp + n);
+    const float4 av = *reinterpret_cast<const float4*>(Ap + n);
+    const float4 bv = *reinterpret_cast<const float4*>(Bp + n);
+    const float4 cv = *reinterpret_cast<const float4*>(Cp + n);
+    constexpr float kLog2e = 1.4426950408889634f;
+    hv.x = fmaf(ex2_approx(dlt * (av.x * kLog2e)), hv.x, du * bv.x);
+    hv.y = fmaf(ex2_approx(dlt * (av.y * kLog2e)), hv.y, du * bv.y);
+    hv.z = fmaf(ex2_approx(dlt * (av.z * kLog2e)), hv.z, du * bv.z);
+    hv.w = fmaf(ex2_approx(dlt * (av.w * kLog2e)), hv.w, du * bv.w);
+    acc = fmaf(cv.x, hv.x, acc);
+    acc = fmaf(cv.y, hv.y, acc);
+    acc = fmaf(cv.z, hv.z, acc);
+    acc = fmaf(cv.w, hv.w, acc);
+    *reinterpret_cast<float4*>(hp + n) = hv;
+  }
+  float yv = acc + (Dskip ? Dskip[c] * u : 0.f);
+  if (z_t) yv *= silu_dev(to_f32<XT>(z_t[e]));
+  y_t[e] = from_f32<YT>(yv);
+}
+
+template <int N, typename XT, typename YT>
+static void scan_step_go(float* h, float* cs, const void* x_t, const void* z_t, const float* delta_t, const float* B_t,
+                         const float* C_t, const float* A, const float* Dskip, const float* conv_w,
+                         const float* conv_b, void* y_t, int64_t B, int64_t D, int K, uint32_t flags,
+                         cudaStream_t s) {
+  const int64_t n = B * D;
+  scan_step_kernel<N, XT, YT><<<(unsigned)((n + 127) / 128), 128, 0, s>>>(
+      h, cs, reinterpret_cast<const XT*>(x_t), reinterpret_cast<const XT*>(z_t), delta_t, B_t, C_t, A, Dskip, conv_w,
+      conv_b, reinterpret_cast<YT*>(y_t), B, D, K, flags);
+}
+
+template <int N>
+static void scan_step_n(float* h, float* cs, const void* x_t, int xdt, const void* z_t, const float* delta_t,
+                        const float* B_t, const float* C_t, const float* A, const float* Dskip, const float* conv_w,
+                        const float* conv_b, void* y_t, int ydt, int64_t B, int64_t D, int K, uint32_t flags,
+                        cudaStream_t s) {
+  const bool xb = xdt == SAMBA_BF16, yb = ydt == SAMBA_BF16;
+  if (xb && yb) scan_step_go<N, __nv_bfloat16, __nv_bfloat16>(h, cs, x_t, z_t, delta_t, B_t, C_t, A, Dskip, conv_w, conv_b, y_t, B, D, K, flags, s);
+  else if (xb) scan_step_go<N, __nv_bfloat16, float>(h, cs, x_t, z_t, delta_t, B_t, C_t, A, Dskip, conv_w, conv_b, y_t, B, D, K, flags, s);
+  else if (yb) scan_step_go<N, float, __nv_bfloat16>(h, cs, x_t, z_t, delta_t, B_t, C_t, A, Dskip, conv_w, conv_b, y_t, B, D, K, flags, s);
+  else scan_step_go<N, float, float>(h, cs, x_t, z_t, delta_t, B_t, C_t, A, Dskip, conv_w, conv_b, y_t, B, D, K, flags, s);
+}
+
+int launch_scan_step(float* h, float* conv_state, const void* x_t, int x_dtype, const void* z_t, int z_dtype,
+                     const float* delta_t, const float* B_t, const float* C_t, const float* A, const float* Dskip,
+                     const float* conv_w, const float* conv_b, void* y_t, int y_dtype, int64_t B, int64_t D, int N,
+                     int K, uint32_t flags, cudaStream_t s) {
+  if (z_t && z_dtype != x_dtype) return fail(SAMBA_ERR_UNSUPPORTED, "samba_scan_step: z dtype must equal x dtype");
+  const void* vec[] = {h, A, B_t, C_t};
+  for (const void* p : vec)
+    if (!aligned16(p)) return fail(SAMBA_ERR_INVALID_ARG, "samba_scan_step: h, A, B_t, C_t must be 16-byte aligned");
+  switch (N) {
+    case 4: scan_step_n<4>(h, conv_state, x_t, x_dtype, z_t, delta_t, B_t, C_t, A, Dskip, conv_w, conv_b, y_t, y_dtype, B, D, K, flags, s); break;
+    case 8: scan_step_n<8>(h, conv_state, x_t, x_dtype, z_t, delta_t, B_t, C_t, A, Dskip, conv_w, conv_b, y_t, y_dtype, B, D, K, flags, s); break;
+    default: scan_step_n<16>(h, conv_state, x_t, x_dtype, z_t, delta_t, B_t, C_t, A, Dskip, conv_w, conv_b, y_t, y_dtype, B, D, K, flags, s); break;
+  }
+  return check_launch("samba_scan_step");
+}
+
+// -------------------------------------------------------------- ring fill
+// Copies 16-byte chunks of the last min(L, W) positions into their slots.
+__global__ void ring_fill_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, uint4* __restrict__ kr,
+                                 uint4* __restrict__ vr, int64_t* __restrict__ pos, int64_t B, int64_t L, int64_t W,
+                                 int row_chunks) {
+  const int64_t keep = L < W ? L : W;
+  const int64_t n = B * keep * row_chunks;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t ch = e % row_chunks;
+    const int64_t r = (e / row_chunks) % keep;
+    const int64_t b = e / (row_chunks * keep);
+    const int64_t p = L - keep + r;
+    const int64_t slot = p % W;
+    kr[(b * W + slot) * row_chunks + ch] = k[(b * L + p) * row_chunks + ch];
+    vr[(b * W + slot) * row_chunks + ch] = v[(b * L + p) * row_chunks + ch];
+  }
+  if (blockIdx.x == 0)
+    for (int64_t b = threadIdx.x; b < B; b += blockDim.x) pos[b] = L;
+}
+
+int launch_ring_fill(const void* k, const void* v, int64_t L, void* k_ring, void* v_ring, int64_t* pos, int64_t B,
+                     int Hkv, int d, int64_t W, cudaStream_t s) {
+  const int row_chunks = Hkv * d * 2 / 16;
+  const int64_t n = B * std::min(L, W) * row_chunks;
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, (int64_t)sm_count() * 8));
+  ring_fill_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v),
+                                          reinterpret_cast<uint4*>(k_ring), reinterpret_cast<uint4*>(v_ring), pos, B,
+                                          L, W, row_chunks);
+  return check_launch("samba_swa_ring_fill");
+}
+
+// --------------------------------------------------------------- SWA step
+// Split over the window: CTA (split, kv head g, batch b) handles CH consecutive
+// positions of the window for the `group` query heads of g, writing a partial
+// (max, sum, unnormalised output) per head; a second kernel combines the
+// splits.  The newest position is read from k_t/v_t, which split 0 also
+// stores into its ring slot (that slot held a position outside the window, so
+// no other CTA reads it in this step).
+constexpr int kStepChunk = 256;
+
+template <int HD>
+__global__ void __launch_bounds__(256) swa_step_split_kernel(
+    const __nv_bfloat16* __restrict__ q_t, const __nv_bfloat16* __restrict__ k_t,
+    const __nv_bfloat16* __restrict__ v_t, __nv_bfloat16* __restrict__ k_ring, __nv_bfloat16* __restrict__ v_ring,
+    const int64_t* __restrict__ pos, float* __restrict__ ws, int Hq, int Hkv, int64_t W, float scale_log2,
+    int nsplit) {
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int group = Hq / Hkv;
+  const int64_t p = pos[b];
+  const int64_t lo = p - W + 1 > 0 ? p - W + 1 : 0;
+  const int64_t a0 = lo + (int64_t)split * kStepChunk;
+  __shared__ float qs[16][HD];
+  __shared__ float sc[16][kStepChunk];
+  __shared__ float red_m[16], red_l[16];
+
+  const int tid = threadIdx.x;
+  for (int i = tid; i < group * HD; i += blockDim.x) {
+    const int hh = i / HD, dd = i % HD;
+    qs[hh][dd] = __bfloat162float(q_t[((int64_t)b * Hq + g * group + hh) * HD + dd]);
+  }
+  if (split == 0) {  // store the new key/value into its slot
+    const int64_t slot = p % W;
+    for (int i = tid; i < HD; i += blockDim.x) {
+      k_ring[(((int64_t)b * W + slot) * Hkv + g) * HD + i] = k_t[((int64_t)b * Hkv + g) * HD + i];
+      v_ring[(((int64_t)b * W + slot) * Hkv + g) * HD + i] = v_t[((int64_t)b * Hkv + g) * HD + i];
+    }
+  }
+  __syncthreads();
+
+  // scores: thread = position
+  {
+    const int64_t a = a0 + tid;
+    const bool valid = a <= p;
+    const __nv_bfloat16* krow = (a == p) ? k_t + ((int64_t)b * Hkv + g) * HD
+                                         : k_ring + (((int64_t)b * W + (valid ? a % W : 0)) * Hkv + g) * HD;
+    float kv[HD];
+    if (valid) {
+#pragma unroll
+      for (int dd = 0; dd < HD; dd += 8) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(krow + dd);
+        const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(pr[q]);
+          kv[dd + 2 * q] = f.x;
+          kv[dd + 2 * q + 1] = f.y;
+        }
+      }
+    }
+    for (int hh = 0; hh < group; ++hh) {
+      float s = 0.f;
+#pragma unroll
+      for (int dd = 0; dd < HD; ++dd) s = fmaf(qs[hh][dd], kv[dd], s);
+      sc[hh][tid] = valid ? s * scale_log2 : -INFINITY;
+    }
+  }
+  __syncthreads();
+  // per head max and exp-sum (one warp per head, heads strided over 8 warps)
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int hh = warp; hh < group; hh += 8) {
+    float m = -INFINITY;
+    for (int i = lane; i < kStepChunk; i += 32) m = fmaxf(m, sc[hh][i]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float mu = (m == -INFINITY) ? 0.f : m;
+    float l = 0.f;
+    for (int i = lane; i < kStepChunk; i += 32) {
+      const float e = ex2_approx(sc[hh][i] - mu);
+      sc[hh][i] = e;
+      l += e;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      red_m[hh] = m;
+      red_l[hh] = l;
+    }
+  }
+  __syncthreads();
+  // partial outputs: thread = (head, dim pair)
+  constexpr int PAIRS = HD / 2;
+  for (int job = tid; job < group * PAIRS; job += blockDim.x) {
+    const int hh = job / PAIRS, dp = job % PAIRS;
+    float o0 = 0.f, o1 = 0.f;
+    const int64_t n_here = p - a0 + 1 < kStepChunk ? p - a0 + 1 : kStepChunk;
+    for (int i = 0; i < n_here; ++i) {
+      const int64_t a = a0 + i;
+      const __nv_bfloat16* vrow = (a == p) ? v_t + ((int64_t)b * Hkv + g) * HD
+                                           : v_ring + (((int64_t)b * W + a % W) * Hkv + g) * HD;
+      const float2 vv = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(vrow)[dp]);
+      const float pw = sc[hh][i];
+      o0 = fmaf(pw, vv.x, o0);
+      o1 = fmaf(pw, vv.y, o1);
+    }
+    float* dst = ws + ((((int64_t)b * Hq + g * group + hh) * nsplit + split) * (HD + 2));
+    dst[2 + 2 * dp] = o0;
+    dst[2 + 2 * dp + 1] = o1;
+    if (dp == 0) {
+      dst[0] = red_m[hh];
+      dst[1] = red_l[hh];
+    }
+  }
+}
+
+template <int HD>
+__global__ void swa_step_combine_kernel(const float* __restrict__ ws, __nv_bfloat16* __restrict__ o_t,
+                                        int64_t* __restrict__ pos, int Hq, int nsplit) {
+  const int hq = blockIdx.x, b = blockIdx.y;
+  const int dd = threadIdx.x;
+  const float* base = ws + ((int64_t)b * Hq + hq) * nsplit * (HD + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, base[s * (HD + 2)]);
+  float l = 0.f, acc = 0.f;
+  for (int s = 0; s < nsplit; ++s) {
+    const float m = base[s * (HD + 2)];
+    const float f = (m == -INFINITY) ? 0.f : ex2_approx(m - M);
+    l = fmaf(base[s * (HD + 2) + 1], f, l);
+    acc = fmaf(base[s * (HD + 2) + 2 + dd], f, acc);
+  }
+  o_t[((int64_t)b * Hq + hq) * HD + dd] = __float2bfloat16_rn(acc / l);
+  if (hq == 0 && dd == 0) pos[b] += 1;
+}
+
+size_t swa_step_workspace(int64_t B, int Hq, int d, int64_t W) {
+  const int64_t nsplit = (W + kStepChunk - 1) / kStepChunk;
+  return static_cast<size_t>(B * Hq * nsplit * (d + 2)) * sizeof(float);
+}
+
+template <int HD>
+static void swa_step_go(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring, int64_t* pos,
+                        void* o_t, int64_t B, int Hq, int Hkv, int64_t W, float scale, void* ws, cudaStream_t s) {
+  const int nsplit = (int)((W + kStepChunk - 1) / kStepChunk);
+  dim3 g1(nsplit, Hkv, (unsigned)B);
+  swa_step_split_kernel<HD><<<g1, 256, 0, s>>>(
+      reinterpret_cast<const __nv_bfloat16*>(q_t), reinterpret_cast<const __nv_bfloat16*>(k_t),
+      reinterpret_cast<const __nv_bfloat16*>(v_t), reinterpret_cast<__nv_bfloat16*>(k_ring),
+      reinterpret_cast<__nv_bfloat16*>(v_ring), pos, reinterpret_cast<float*>(ws), Hq, Hkv, W,
+      scale * 1.4426950408889634f, nsplit);
+  dim3 g2(Hq, (unsigned)B);
+  swa_step_combine_kernel<HD><<<g2, HD, 0, s>>>(reinterpret_cast<const float*>(ws),
+                                                 reinterpret_cast<__nv_bfloat16*>(o_t), pos, Hq, nsplit);
+}
+
+int launch_swa_step(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring, int64_t* pos,
+                    void* o_t, int64_t B, int Hq, int Hkv, int d, int64_t W, float scale, void* ws, cudaStream_t s) {
+  if (B > 65535) return fail(SAMBA_ERR_UNSUPPORTED, "samba_swa_step: batch too large");
+  switch (d) {
+    case 16: swa_step_go<16>(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, B, Hq, Hkv, W, scale, ws, s); break;
+    case 32: swa_step_go<32>(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, B, Hq, Hkv, W, scale, ws, s); break;
+    case 64: swa_step_go<64>(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, B, Hq, Hkv, W, scale, ws, s); break;
+    default: swa_step_go<128>(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, B, Hq, Hkv, W, scale, ws, s); break;
+  }
+  return check_launch("samba_swa_step");
+}
+
+}  // namespace samba

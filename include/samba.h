@@ -1,0 +1,226 @@
+/*
+ * samba.h -- C ABI of the B200 (sm_100a) kernels for Samba's two token mixers.
+ *
+ * Samba ("Samba: Simple Hybrid State Space Models for Efficient Unlimited
+ * Context Language Modeling", Ren et al.) interleaves a Mamba layer (a
+ * selective state-space scan) with a sliding-window attention (SWA) layer.
+ * This library runs the prefill forward of both mixers and their single-token
+ * decode steps:
+ *
+ *   - causal depthwise conv1d (width K, K = 4) in front of the scan;
+ *   - selective scan h_t = exp(Δ_t A) h_{t-1} + Δ_t B_t u_t,
+ *     y_t = (C_t . h_t + D u_t) * silu(z_t), with Δ_t = softplus(delta_t)
+ *     (page "SAMBA混合注意力状态空间模型", section 数学框架 / Mamba层: the
+ *     recurrence h_t = Ā_t h_{t-1} + B̄_t x_t, y_t = C_t h_t and its
+ *     input-dependent B_t, C_t, Δ_t);
+ *   - causal sliding-window attention with grouped KV heads, where query i
+ *     sees key j exactly when 0 <= i - j < W (same page, section
+ *     滑动窗口注意力; its mask is printed inverted, this is the causal band);
+ *   - the decode steps mamba_step / swa_step of the page's section 推理效率.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer is a DEVICE pointer owned by the caller.  The library never
+ *    allocates or frees device memory and never synchronises, except in
+ *    samba_get_status().
+ *  - Every call is asynchronous on the given stream (a cudaStream_t; NULL is
+ *    the legacy default stream) and returns an int status.  Arguments are
+ *    checked on the host before any launch; a rejected call launches nothing.
+ *  - Tensors are dense and row-major in the layouts written beside each
+ *    argument (channel-last activations).  Base pointers must be 16-byte
+ *    aligned.
+ *  - bf16 is IEEE bfloat16 (round-to-nearest-even on store).  All arithmetic
+ *    of the scan is fp32; attention multiplies in bf16 on the tensor cores
+ *    with fp32 accumulation and an fp32 softmax.
+ *  - Errors: SAMBA_ERR_INVALID_ARG (null pointer where one is required, bad
+ *    shape, misaligned pointer), SAMBA_ERR_UNSUPPORTED (dtype, state size,
+ *    head_dim or head grouping outside what the kernels implement),
+ *    SAMBA_ERR_WORKSPACE (workspace too small), SAMBA_ERR_CUDA (a CUDA call
+ *    or launch failed).  samba_last_error() gives a one-line description of
+ *    the last failure on the calling host thread.
+ *  - Kernels never spin without a limit.  A device-side wait that runs out
+ *    (which only a library bug can cause) stops the kernel cleanly and
+ *    records SAMBA_ERR_TIMEOUT in a per-device status word that
+ *    samba_get_status() returns.
+ */
+#ifndef SAMBA_H_
+#define SAMBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so the header needs no CUDA. */
+typedef struct CUstream_st* samba_stream_t;
+
+/* element types */
+enum { SAMBA_F32 = 0, SAMBA_BF16 = 1 };
+
+/* status codes */
+enum {
+  SAMBA_OK = 0,
+  SAMBA_ERR_INVALID_ARG = -1,
+  SAMBA_ERR_UNSUPPORTED = -2,
+  SAMBA_ERR_WORKSPACE = -3,
+  SAMBA_ERR_CUDA = -4,
+  SAMBA_ERR_TIMEOUT = -5
+};
+
+/* flags of samba_scan_args.flags */
+enum {
+  SAMBA_SCAN_FUSE_CONV = 1,      /* x is the conv input; u = conv1d(x) (+ SiLU) */
+  SAMBA_SCAN_DELTA_SOFTPLUS = 2, /* Δ = softplus(delta); otherwise Δ = delta    */
+  SAMBA_SCAN_CONV_SILU = 4       /* apply SiLU to the conv output               */
+};
+
+/* Library version, major*10000 + minor*100 + patch. */
+int samba_version(void);
+
+/* One-line text of the last error reported on this host thread ("" if none). */
+const char* samba_last_error(void);
+
+/* Synchronises `stream`, then returns and clears this device's status word:
+ * SAMBA_OK, or SAMBA_ERR_TIMEOUT if a kernel gave up a device-side wait since
+ * the last call.  Returns SAMBA_ERR_CUDA if the synchronisation itself fails. */
+int samba_get_status(samba_stream_t stream);
+
+/* ------------------------------------------------------------------ conv1d
+ * Causal depthwise conv1d over time (the conv that Samba's Mamba layer puts in
+ * front of its selective scan):
+ *   u[b,t,c] = bias[c] + sum_{k<K} w[c,k] * xpad[b,t+k,c],  then SiLU if silu,
+ * where xpad is x preceded by the K-1 inputs of conv_state_in (oldest first;
+ * zeros when conv_state_in is NULL), so w[c,K-1] multiplies x_t.
+ *
+ *   x              [B, L, D]   x_dtype (SAMBA_F32 or SAMBA_BF16)
+ *   w              [D, K]      fp32
+ *   bias           [D]         fp32, or NULL (no bias)
+ *   conv_state_in  [B, D, K-1] fp32, or NULL (zeros)
+ *   u              [B, L, D]   u_dtype
+ *   conv_state_out [B, D, K-1] fp32, or NULL: the last K-1 entries of xpad.
+ *                  May not alias conv_state_in.
+ * K must be 2..4; B, L >= 1; D >= 1.  L may be smaller than K-1.
+ */
+int samba_conv1d_fwd(const void* x, int x_dtype, const float* w, const float* bias,
+                     const float* conv_state_in, void* u, int u_dtype, float* conv_state_out,
+                     int64_t batch, int64_t seqlen, int64_t dim, int dconv, int silu,
+                     samba_stream_t stream);
+
+/* ------------------------------------------------------------------- scan
+ * Selective-scan prefill, fused with the conv, softplus, D skip and gate:
+ *   u      = SiLU(conv1d(x))  with SAMBA_SCAN_FUSE_CONV (|CONV_SILU), else x
+ *   Δ      = softplus(delta)  with SAMBA_SCAN_DELTA_SOFTPLUS, else delta
+ *   h_t[n] = exp(Δ_t A[c,n]) h_{t-1}[n] + Δ_t B_t[n] u_t        (fp32 state)
+ *   y_t    = (sum_n C_t[n] h_t[n] + Dskip[c] u_t) * silu(z_t)
+ * for every batch b and channel c, t = 0..L-1, starting from h0 (zeros if
+ * NULL).  B and C are shared by all channels (one group).
+ */
+typedef struct samba_scan_args {
+  const void* x;               /* [B, L, D]   x_dtype                         */
+  const void* z;               /* [B, L, D]   z_dtype, or NULL (no gate)      */
+  const float* delta;          /* [B, L, D]   fp32                            */
+  const float* A;              /* [D, N]      fp32                            */
+  const float* Bm;             /* [B, L, N]   fp32                            */
+  const float* Cm;             /* [B, L, N]   fp32                            */
+  const float* Dskip;          /* [D]         fp32, or NULL (no skip)         */
+  const float* conv_w;         /* [D, K]      fp32 (needed with FUSE_CONV)    */
+  const float* conv_b;         /* [D]         fp32, or NULL                   */
+  const float* conv_state_in;  /* [B, D, K-1] fp32, or NULL (zeros)           */
+  float* conv_state_out;       /* [B, D, K-1] fp32, or NULL                   */
+  const float* h0;             /* [B, D, N]   fp32, or NULL (zeros)           */
+  float* h_final;              /* [B, D, N]   fp32, or NULL; may alias h0     */
+  void* y;                     /* [B, L, D]   y_dtype                         */
+  int64_t batch, seqlen, dim;  /* B >= 1, L >= 1, D >= 1 with D % 8 == 0      */
+  int32_t dstate, dconv;       /* N in {4, 8, 16}; K in 2..4                  */
+  int32_t x_dtype, z_dtype, y_dtype;
+  uint32_t flags;
+} samba_scan_args;
+
+int samba_selective_scan_fwd(const samba_scan_args* args, samba_stream_t stream);
+
+/* -------------------------------------------------------------------- SWA
+ * Causal sliding-window attention prefill with grouped KV heads:
+ *   o[b,i,h] = sum_{j : 0 <= i-j < W} softmax_j(scale * q[b,i,h] . k[b,j,g])
+ *              * v[b,j,g],   g = h / (Hq / Hkv)
+ * computed with tcgen05 bf16 MMAs (fp32 accumulate in tensor memory) and an
+ * fp32 online softmax; o is rounded to bf16 once.  lse (optional) receives the
+ * natural-log logsumexp of the scaled scores of every row.
+ * W >= L gives plain causal attention.
+ */
+typedef struct samba_swa_args {
+  const void* q;      /* [B, L, Hq, d]   bf16 */
+  const void* k;      /* [B, L, Hkv, d]  bf16 */
+  const void* v;      /* [B, L, Hkv, d]  bf16 */
+  void* o;            /* [B, L, Hq, d]   bf16 */
+  float* lse;         /* [B, Hq, L]      fp32, or NULL */
+  int64_t batch, seqlen, window;   /* B >= 1, L >= 1, W >= 1 */
+  int32_t heads_q, heads_kv, head_dim;  /* Hq % Hkv == 0, Hq/Hkv divides 128; d in {16, 32, 64} */
+  float scale;        /* softmax scale; <= 0 selects 1/sqrt(d) */
+} samba_swa_args;
+
+int samba_swa_fwd(const samba_swa_args* args, samba_stream_t stream);
+
+/* ------------------------------------------------------------ mixer prefill
+ * One Mamba mixer (scan) and one SWA mixer on their own inputs (the two token
+ * mixers of a Samba block: the forward pseudo-code of the page's section
+ * 推理效率 runs mamba(x), then swa(x) after the MLP).  The two are independent: with aux == NULL both run
+ * in order on `stream`; otherwise the attention runs on `aux`, forked from
+ * and joined back into `stream` with events, so that the call as a whole is
+ * still ordered on `stream`.
+ */
+int samba_mixer_prefill(const samba_scan_args* scan, const samba_swa_args* swa,
+                        samba_stream_t stream, samba_stream_t aux);
+
+/* ------------------------------------------------------------- decode: scan
+ * One token of the selective scan (mamba_step): updates h and the conv state
+ * in place and writes y_t.  Same arithmetic as the prefill with L = 1.
+ *   h          [B, D, N]   fp32, read and written
+ *   conv_state [B, D, K-1] fp32, read and written (oldest first)
+ *   x_t, z_t   [B, D]      x_dtype / z_dtype (z_t may be NULL)
+ *   delta_t    [B, D]      fp32 (softplus applied with DELTA_SOFTPLUS)
+ *   B_t, C_t   [B, N]      fp32;  A [D, N], Dskip [D] (or NULL), conv_w
+ *                          [D, K], conv_b [D] (or NULL) as in the prefill
+ *   y_t        [B, D]      y_dtype
+ * flags: as samba_scan_args.flags (FUSE_CONV requires conv_state and conv_w).
+ */
+int samba_scan_step(float* h, float* conv_state, const void* x_t, int x_dtype, const void* z_t,
+                    int z_dtype, const float* delta_t, const float* B_t, const float* C_t,
+                    const float* A, const float* Dskip, const float* conv_w, const float* conv_b,
+                    void* y_t, int y_dtype, int64_t batch, int64_t dim, int dstate, int dconv,
+                    uint32_t flags, samba_stream_t stream);
+
+/* -------------------------------------------------------------- decode: SWA
+ * Ring-buffer KV window.  Slot p mod W of k_ring/v_ring holds the key/value
+ * of absolute position p; pos[b] is the next position of sequence b.
+ *
+ * samba_swa_ring_fill: after a prefill of L tokens, copy the last min(L, W)
+ * keys/values of k, v ([B, L, Hkv, d] bf16) into their slots and set
+ * pos[b] = L.  Slots of positions < L - W are left untouched.
+ */
+int samba_swa_ring_fill(const void* k, const void* v, int64_t seqlen, void* k_ring, void* v_ring,
+                        int64_t* pos, int64_t batch, int heads_kv, int head_dim, int64_t window,
+                        samba_stream_t stream);
+
+/* Bytes of device workspace samba_swa_step needs for these sizes. */
+size_t samba_swa_step_workspace_size(int64_t batch, int heads_q, int head_dim, int64_t window);
+
+/* samba_swa_step (swa_step): writes k_t, v_t ([B, Hkv, d]) into slot
+ * pos[b] mod W, then each query q_t ([B, Hq, d]) attends the keys of
+ * positions max(0, pos-W+1) .. pos and writes o_t ([B, Hq, d] bf16); finally
+ * pos[b] += 1.  All of it happens on the device (pos is a device int64 [B]),
+ * so consecutive steps can be captured in one CUDA graph.  `workspace` is
+ * caller-owned device memory of at least samba_swa_step_workspace_size()
+ * bytes (split partial results); it needs no initialisation.
+ */
+int samba_swa_step(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring,
+                   int64_t* pos, void* o_t, int64_t batch, int heads_q, int heads_kv, int head_dim,
+                   int64_t window, float scale, void* workspace, size_t workspace_bytes,
+                   samba_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAMBA_H_ */

@@ -129,7 +129,7 @@ def causal_conv1d(x, weight, bias=None, state=None, apply_silu=True):
 # ----------------------------------------------------------------------- scan
 def selective_scan(x, delta, A, Bm, Cm, Dskip=None, z=None, h0=None,
                    conv_w=None, conv_b=None, conv_state=None,
-                   delta_softplus=True, conv_silu=True):
+                   delta_softplus=True, conv_silu=True, magnitudes=False):
     """Selective SSM prefill, sequential in time.
 
     Page "SAMBA混合注意力状态空间模型", §数学框架 / Mamba层:
@@ -144,6 +144,14 @@ def selective_scan(x, delta, A, Bm, Cm, Dskip=None, z=None, h0=None,
     Shapes: x, delta, z: [B, L, D]; A: [D, N]; Bm, Cm: [B, L, N]; Dskip: [D];
     h0: [B, D, N]; conv_w: [D, K]; conv_b: [D]; conv_state: [B, D, K-1].
     Returns dict(y [B, L, D], h [B, D, N], conv_state [B, D, K-1] or None).
+
+    With ``magnitudes`` the dict also holds y_mag and h_mag: the same
+    recurrence run on the absolute values of its terms,
+        hm_t = Ā_t hm_{t-1} + |B̄x_t|,   y_mag = (sum_n |C| hm + |D u|) |silu(z)|
+    (Ā > 0), i.e. the size of the sums that produce y and h.  Rounding error
+    of a finite-precision evaluation scales with these, not with |y|, which
+    can be far smaller through cancellation; the tests measure relative
+    error against them.
     """
     x = _f64(x)
     delta = _f64(delta)
@@ -161,16 +169,30 @@ def selective_scan(x, delta, A, Bm, Cm, Dskip=None, z=None, h0=None,
 
     h = np.zeros((Bsz, D, N)) if h0 is None else _f64(h0).copy()
     y = np.empty((Bsz, L, D))
+    if magnitudes:
+        hm = np.abs(h)
+        ym = np.empty((Bsz, L, D))
     for t in range(L):
         dA = np.exp(dt[:, t, :, None] * A[None, :, :])                       # [B, D, N]
         dBx = (dt[:, t, :] * u[:, t, :])[:, :, None] * Bm[:, t, None, :]      # [B, D, N]
         h = dA * h + dBx
         y[:, t, :] = np.einsum("bdn,bn->bd", h, Cm[:, t, :])
+        if magnitudes:
+            hm = dA * hm + np.abs(dBx)
+            ym[:, t, :] = np.einsum("bdn,bn->bd", hm, np.abs(Cm[:, t, :]))
     if Dskip is not None:
         y = y + _f64(Dskip)[None, None, :] * u
+        if magnitudes:
+            ym = ym + np.abs(_f64(Dskip)[None, None, :] * u)
     if z is not None:
         y = y * silu(z)
-    return {"y": y, "h": h, "conv_state": conv_state_out}
+        if magnitudes:
+            ym = ym * np.abs(silu(z))
+    out = {"y": y, "h": h, "conv_state": conv_state_out}
+    if magnitudes:
+        out["y_mag"] = ym
+        out["h_mag"] = hm
+    return out
 
 
 def scan_step(h, conv_state, x_t, delta_t, A, B_t, C_t, Dskip=None, z_t=None,

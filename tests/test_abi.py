@@ -1,0 +1,125 @@
+"""CPU checks of the C ABI: the library builds and loads, exports every
+function the header declares, and rejects bad arguments on the host (no
+kernel is launched and no GPU is needed)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from hybrid_ssm_sliding_b200 import _lib as L
+from hybrid_ssm_sliding_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.load()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "samba.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\**(samba_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("samba_conv1d_fwd", "samba_selective_scan_fwd", "samba_swa_fwd", "samba_mixer_prefill",
+              "samba_scan_step", "samba_swa_step", "samba_swa_ring_fill", "samba_get_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version(lib):
+    assert lib.samba_version() >= 100
+
+
+def _scan_args(**over):
+    a = L.ScanArgs()
+    fake = 0x10000  # 16-byte aligned dummy address; never dereferenced on rejected calls
+    for f in ("x", "delta", "A", "Bm", "Cm", "y", "conv_w"):
+        setattr(a, f, fake)
+    a.batch, a.seqlen, a.dim, a.dstate, a.dconv = 1, 64, 16, 16, 4
+    a.x_dtype = a.y_dtype = a.z_dtype = L.SAMBA_BF16
+    a.flags = L.SCAN_FUSE_CONV | L.SCAN_DELTA_SOFTPLUS | L.SCAN_CONV_SILU
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(x=None), L.SAMBA_ERR_INVALID_ARG),
+    (dict(y=None), L.SAMBA_ERR_INVALID_ARG),
+    (dict(batch=0), L.SAMBA_ERR_INVALID_ARG),
+    (dict(seqlen=0), L.SAMBA_ERR_INVALID_ARG),
+    (dict(dim=12), L.SAMBA_ERR_INVALID_ARG),
+    (dict(dstate=32), L.SAMBA_ERR_UNSUPPORTED),
+    (dict(dconv=5), L.SAMBA_ERR_UNSUPPORTED),
+    (dict(x_dtype=7), L.SAMBA_ERR_UNSUPPORTED),
+    (dict(conv_w=None), L.SAMBA_ERR_INVALID_ARG),
+    (dict(flags=64), L.SAMBA_ERR_INVALID_ARG),
+    (dict(x=0x10008), L.SAMBA_ERR_INVALID_ARG),
+])
+def test_scan_rejects_bad_arguments_on_host(lib, over, code):
+    a = _scan_args(**over)
+    assert lib.samba_selective_scan_fwd(ctypes.byref(a), None) == code
+    assert lib.samba_last_error().decode()
+
+
+def test_scan_rejects_null_struct(lib):
+    assert lib.samba_selective_scan_fwd(None, None) == L.SAMBA_ERR_INVALID_ARG
+
+
+def _swa_args(**over):
+    a = L.SwaArgs()
+    for f in ("q", "k", "v", "o"):
+        setattr(a, f, 0x20000)
+    a.batch, a.seqlen, a.window, a.heads_q, a.heads_kv, a.head_dim = 1, 128, 64, 32, 4, 64
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), L.SAMBA_ERR_INVALID_ARG),
+    (dict(window=0), L.SAMBA_ERR_INVALID_ARG),
+    (dict(heads_kv=5), L.SAMBA_ERR_INVALID_ARG),
+    (dict(heads_q=96, heads_kv=3), L.SAMBA_ERR_UNSUPPORTED),
+    (dict(head_dim=80), L.SAMBA_ERR_UNSUPPORTED),
+    (dict(o=0x20004), L.SAMBA_ERR_INVALID_ARG),
+])
+def test_swa_rejects_bad_arguments_on_host(lib, over, code):
+    a = _swa_args(**over)
+    assert lib.samba_swa_fwd(ctypes.byref(a), None) == code
+    assert lib.samba_mixer_prefill(ctypes.byref(_scan_args()), ctypes.byref(a), None, None) == code
+
+
+def test_conv_rejects_bad_arguments_on_host(lib):
+    f = 0x30000
+    assert lib.samba_conv1d_fwd(None, 1, f, None, None, f, 1, None, 1, 8, 8, 4, 1, None) == L.SAMBA_ERR_INVALID_ARG
+    assert lib.samba_conv1d_fwd(f, 1, f, None, None, f, 1, None, 1, 8, 8, 7, 1, None) == L.SAMBA_ERR_UNSUPPORTED
+    assert lib.samba_conv1d_fwd(f, 1, f, None, f, f, 1, f, 1, 8, 8, 4, 1, None) == L.SAMBA_ERR_INVALID_ARG
+
+
+def test_decode_rejects_bad_arguments_on_host(lib):
+    f = 0x40000
+    assert lib.samba_scan_step(None, None, f, 1, None, 1, f, f, f, f, None, None, None, f, 1, 1, 8, 16, 4, 0,
+                               None) == L.SAMBA_ERR_INVALID_ARG
+    assert lib.samba_scan_step(f, None, f, 1, None, 1, f, f, f, f, None, None, None, f, 1, 1, 8, 16, 4,
+                               L.SCAN_FUSE_CONV, None) == L.SAMBA_ERR_INVALID_ARG
+    assert lib.samba_swa_ring_fill(f, f, 8, f, f, None, 1, 4, 64, 16, None) == L.SAMBA_ERR_INVALID_ARG
+    assert lib.samba_swa_ring_fill(f, f, 8, f, f, f, 1, 4, 80, 16, None) == L.SAMBA_ERR_UNSUPPORTED
+    need = lib.samba_swa_step_workspace_size(16, 32, 64, 2048)
+    assert need == 16 * 32 * 8 * 66 * 4
+    assert lib.samba_swa_step(f, f, f, f, f, f, f, 16, 32, 4, 64, 2048, 0.0, f, need - 1, None) == \
+        L.SAMBA_ERR_WORKSPACE
+    assert lib.samba_swa_step(f, f, f, f, f, f, f, 16, 32, 4, 64, 2048, 0.0, None, 0, None) == \
+        L.SAMBA_ERR_WORKSPACE

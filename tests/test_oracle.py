@@ -359,3 +359,31 @@ def test_planted_scan_mistakes_are_caught(monkeypatch):
     j = dict(i)
     j["conv_w"] = i["conv_w"][:, ::-1].copy()
     assert not np.allclose(orc.selective_scan(**j)["y"], ref, atol=1e-6)
+
+
+# --------------------------------------------------- error-scale magnitudes
+def test_scan_magnitudes_bound_the_outputs():
+    i = _tiny_scan_inputs(21, Bsz=2, L=40, D=8, N=4)
+    h0 = _rng(22).standard_normal((2, 8, 4))
+    out = orc.selective_scan(**i, h0=h0, magnitudes=True)
+    assert np.all(out["y_mag"] >= np.abs(out["y"]) * (1 - 1e-12))
+    assert np.all(out["h_mag"] >= np.abs(out["h"]) * (1 - 1e-12))
+    # the magnitudes do not change the outputs themselves
+    plain = orc.selective_scan(**i, h0=h0)
+    np.testing.assert_array_equal(plain["y"], out["y"])
+
+
+def test_scan_magnitudes_equal_outputs_when_no_term_is_negative():
+    """With every term of the sums non-negative (u, B, C, D > 0, no gate,
+    no conv) nothing cancels and the magnitudes equal the outputs."""
+    r = _rng(23)
+    Bsz, L, D, N = 1, 30, 5, 4
+    x = r.uniform(0.1, 2.0, (Bsz, L, D))
+    dt = r.uniform(0.01, 0.3, (Bsz, L, D))
+    A = -r.uniform(0.5, 3.0, (D, N))
+    Bm = r.uniform(0.1, 1.0, (Bsz, L, N))
+    Cm = r.uniform(0.1, 1.0, (Bsz, L, N))
+    Ds = r.uniform(0.1, 1.0, D)
+    out = orc.selective_scan(x, dt, A, Bm, Cm, Ds, delta_softplus=False, magnitudes=True)
+    np.testing.assert_allclose(out["y_mag"], out["y"], rtol=1e-13)
+    np.testing.assert_allclose(out["h_mag"], out["h"], rtol=1e-13)
