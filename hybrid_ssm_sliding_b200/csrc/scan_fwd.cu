@@ -12,20 +12,39 @@
 //   h_t   = exp(Δ_t A) ⊙ h_{t-1} + Δ_t u_t B_t        (N states, fp32)
 //   y_t   = (C_t · h_t + D u_t) · silu(z_t)
 //
-// Work split.  The recurrence is sequential in t but independent across
-// (batch, channel, state).  A channel's N states are spread over GL = N/NS
-// lanes (NS states per lane), so a warp covers 32/GL channels and the whole
-// grid keeps B·D·N/NS threads busy without splitting time.  Inputs stream
-// through shared memory in tiles of T tokens × CB channels, loaded by TMA
-// from a producer warp into a STAGES-deep ring (mbarrier full/empty pairs).
+// The recurrence is sequential in t but independent across (batch, channel,
+// state), and on B200 it is bound by arithmetic (one exp per state and token
+// on a 16/clk/SM MUFU pipe), not by HBM.  So the kernel spends as few
+// instructions as it can per (token, channel, state) and keeps every SM busy:
 //
-// Per GL-token sub-tile, lane j of a channel group first computes the
-// per-(token, channel) prologue (conv, SiLU, softplus, gate) for token j of
-// the sub-tile -- once per (t, c), not once per lane -- and shares (Δ, Δu)
-// through shared memory.  Every lane then advances its NS states over the GL
-// tokens, and the partial sums C·h of the GL lanes are reduced through shared
-// memory so that lane j ends up with y of the token whose prologue it holds.
+//   * A CTA owns CU consecutive channels of one batch row (CU chosen on the
+//     host so that the CTAs spread evenly over the SMs) and walks the whole
+//     sequence in tiles of T tokens.
+//   * Warp roles.  One producer warp streams x, z, delta, B, C tiles into a
+//     STAGES-deep shared-memory ring with TMA.  NPRO "prologue" warps compute,
+//     once per (token, channel), the conv, SiLU, softplus and gate, leaving
+//     (Δ, Δu) for the scan and (D·u, silu(z)) for the output; the same warps
+//     later finish y = (Σ partials + D·u)·silu(z) and store it.  The scan
+//     warps hold the state: a channel's N states are spread over GL lanes
+//     (NS states per lane) and each lane writes its partial C·h per token.
+//   * Prologue, scan and epilogue of consecutive tiles overlap through
+//     double-buffered exchange arrays guarded by mbarriers.
+//   * The scan core uses packed f32x2 arithmetic; a compile-time share of the
+//     exps is evaluated on the FMA pipe with a polynomial (exp2 split into
+//     2^j · 2^f, degree-5 fit of 2^f on [-1/2, 1/2] with p(0) = 1 and
+//     p'(0) = ln 2), so the MUFU and FMA pipes share the load.
+//   * Every wait is bounded; a wait that runs out stops the CTA cleanly.
 #include "common.cuh"
+
+// Every SAMBA_SCAN_POLY-th token evaluates its exps on the FMA pipe
+// (0: never).  A build-time constant, fixed by measurement.
+#ifndef SAMBA_SCAN_POLY
+#define SAMBA_SCAN_POLY 4
+#endif
+// States per scan lane at N = 16 (2 or 4); also fixed by measurement.
+#ifndef SAMBA_SCAN_NS16
+#define SAMBA_SCAN_NS16 2
+#endif
 
 namespace samba {
 
@@ -42,107 +61,202 @@ struct ScanParams {
   void* y;
   int64_t L, D;
   int K;
+  int CU;  // channels per CTA
   int has_z, fuse_conv, conv_silu, softplus;
 };
 
-template <int N, int NS, int WARPS, int T, int STAGES, typename XT, typename ZT, typename YT>
-struct ScanCfg {
-  static constexpr int GL = N / NS;       // lanes per channel
-  static constexpr int CPW = 32 / GL;     // channels per warp
-  static constexpr int CB = WARPS * CPW;  // channels per CTA
-  static constexpr int HALO = 3;          // conv taps before the tile (K <= 4)
-  static constexpr int XROWS = T + HALO;
-  static_assert(T % GL == 0, "tile must hold whole sub-tiles");
-  static constexpr int XB = XROWS * CB * (int)sizeof(XT);
-  static constexpr int ZB = T * CB * (int)sizeof(ZT);
+template <int N> struct ScanShape;
+template <> struct ScanShape<16> { static constexpr int NS = SAMBA_SCAN_NS16, GL = 16 / SAMBA_SCAN_NS16; };
+template <> struct ScanShape<8> { static constexpr int NS = 1, GL = 8; };
+template <> struct ScanShape<4> { static constexpr int NS = 1, GL = 4; };
+
+constexpr int kScanCB = 32;     // channels in one TMA box (>= CU + alignment offset)
+constexpr int kScanT = 32;      // tokens per tile
+constexpr int kScanStages = 4;  // TMA ring depth
+constexpr int kScanPro = 4;     // prologue / epilogue warps
+
+template <int N, typename XT>
+struct ScanLayout {
+  static constexpr int GL = ScanShape<N>::GL;
+  static constexpr int CB = kScanCB, T = kScanT, STAGES = kScanStages, HALO = 3;
+  static constexpr int al(int v) { return (v + 127) / 128 * 128; }
+  static constexpr int XB = (T + HALO) * CB * (int)sizeof(XT);
+  static constexpr int ZB = T * CB * (int)sizeof(XT);
   static constexpr int WB = T * CB * 4;
   static constexpr int BB = T * N * 4;
-  static constexpr int al(int v) { return (v + 127) / 128 * 128; }
-  static constexpr int X_OFF = 0;
-  static constexpr int Z_OFF = al(XB);
-  static constexpr int W_OFF = Z_OFF + al(ZB);
-  static constexpr int B_OFF = W_OFF + al(WB);
-  static constexpr int C_OFF = B_OFF + al(BB);
-  static constexpr int STAGE_BYTES = C_OFF + al(BB);
-  // per-warp scratch: exchange of (Δ, Δu) and the y reduction
-  static constexpr int XCH_FLOATS = CPW * GL * 2;
-  static constexpr int RS = GL * (GL + 1);  // row stride of a channel group, bank-conflict free
-  static constexpr int RED_FLOATS = CPW * RS;
-  static constexpr int WARP_SCRATCH = (XCH_FLOATS + RED_FLOATS) * 4;
-  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  static constexpr int SCRATCH_OFF = BAR_OFF + 128;
-  static constexpr int SMEM = SCRATCH_OFF + WARPS * al(WARP_SCRATCH);
-  static constexpr int THREADS = (WARPS + 1) * 32;
+  static constexpr int X_OFF = 0, Z_OFF = al(XB), W_OFF = Z_OFF + al(ZB), B_OFF = W_OFF + al(WB),
+                       C_OFF = B_OFF + al(BB), STAGE_BYTES = C_OFF + al(BB);
+  static constexpr int XCH_OFF = STAGES * STAGE_BYTES;        // float4 [2][T][CB]
+  static constexpr int EPI_OFF = XCH_OFF + 2 * T * CB * 16;   // float2 [2][T][CB]
+  static constexpr int PART_OFF = EPI_OFF + 2 * T * CB * 8;   // float  [2][T][CB][GL]
+  static constexpr int BAR_OFF = PART_OFF + 2 * T * CB * GL * 4;
+  static constexpr int SMEM = BAR_OFF + 256;
 };
 
-__device__ __forceinline__ float fast_ex2(float x) {
+// ------------------------------------------------------------ math helpers
+__device__ __forceinline__ float mufu_ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-
-__device__ __forceinline__ float silu_f(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
-
-__device__ __forceinline__ float softplus_f(float w) {
-  // log(1 + e^w); the identity softplus(w) = w + log1p(e^-w) keeps large w exact.
-  return w > 20.0f ? w : (w > 0.0f ? w + log1pf(__expf(-w)) : log1pf(__expf(w)));
+__device__ __forceinline__ float mufu_rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
-template <int N, int NS, int WARPS, int T, int STAGES, typename XT, typename ZT, typename YT>
-__global__ void __launch_bounds__((WARPS + 1) * 32, 1)
+typedef unsigned long long f2;  // two packed fp32 (f32x2 operand)
+__device__ __forceinline__ f2 pk2(float lo, float hi) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 up2(f2 v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+  f2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+  f2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 sub2(f2 a, f2 b) {
+  f2 d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// 2^x on the FMA pipe for a pair of arguments: x = j + f with j = rint(x)
+// (magic-number rounding), 2^f by a degree-5 polynomial fitted on
+// [-1/2, 1/2] for relative error (fit made for this library; c0 = 1 and
+// c1 = ln 2 are pinned so that 2^f - 1 stays accurate for tiny f), and the
+// exponent j added to the bits of 2^f.  x is clamped to [-125, 127]; below
+// that the true value is under 2^-125 and is returned as 2^-125.
+__device__ __forceinline__ f2 ex2_poly2(f2 x) {
+  float2 xv = up2(x);
+  xv.x = fminf(fmaxf(xv.x, -125.f), 127.f);
+  xv.y = fminf(fmaxf(xv.y, -125.f), 127.f);
+  const f2 xc = pk2(xv.x, xv.y);
+  const f2 magic = pk2(12582912.f, 12582912.f);  // 1.5 * 2^23
+  const f2 t = add2(xc, magic);
+  const f2 j = sub2(t, magic);
+  const f2 f = sub2(xc, j);
+  f2 p = pk2(0x1.59c4aap-10f, 0x1.59c4aap-10f);
+  p = fma2(p, f, pk2(0x1.3c6c98p-7f, 0x1.3c6c98p-7f));
+  p = fma2(p, f, pk2(0x1.c6b7f4p-5f, 0x1.c6b7f4p-5f));
+  p = fma2(p, f, pk2(0x1.ebfb30p-3f, 0x1.ebfb30p-3f));
+  p = fma2(p, f, pk2(0x1.62e430p-1f, 0x1.62e430p-1f));
+  p = fma2(p, f, pk2(1.f, 1.f));
+  const float2 tv = up2(t), pv = up2(p);
+  const float r0 = __int_as_float(__float_as_int(pv.x) + (__float_as_int(tv.x) << 23));
+  const float r1 = __int_as_float(__float_as_int(pv.y) + (__float_as_int(tv.y) << 23));
+  return pk2(r0, r1);
+}
+
+__device__ __forceinline__ float silu_fast(float v) {
+  return v * mufu_rcp(1.0f + mufu_ex2(v * -1.4426950408889634f));
+}
+
+// softplus(w) = log(1 + e^w).  For w <= 0 with e = e^w: log1p(e) = 2 atanh(s),
+// s = e / (2 + e) in (0, 1/3], summed as 2s(1 + s²/3 + ... + s¹²/13) (the
+// next term is below 1.5e-8 relative).  For w > 0 the identity
+// softplus(w) = w + softplus(-w) is used, and for w > 20 softplus(w) = w in
+// fp32.
+__device__ __forceinline__ float softplus_fast(float w) {
+  const float e = mufu_ex2(-fabsf(w) * 1.4426950408889634f);
+  const float s = e * mufu_rcp(2.0f + e);
+  const float s2 = s * s;
+  float p = 1.f / 13.f;
+  p = fmaf(p, s2, 1.f / 11.f);
+  p = fmaf(p, s2, 1.f / 9.f);
+  p = fmaf(p, s2, 1.f / 7.f);
+  p = fmaf(p, s2, 1.f / 5.f);
+  p = fmaf(p, s2, 1.f / 3.f);
+  p = fmaf(p, s2, 1.f);
+  const float l = 2.f * s * p;
+  return w > 20.f ? w : (w > 0.f ? w + l : l);
+}
+
+// ------------------------------------------------------------------ kernel
+template <int N, typename XT, typename YT, int POLY>
+__global__ void __launch_bounds__(416, 1)
     scan_fwd_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_z,
                     const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_b,
                     const __grid_constant__ CUtensorMap map_c, const ScanParams p) {
-  using Cfg = ScanCfg<N, NS, WARPS, T, STAGES, XT, ZT, YT>;
-  constexpr int GL = Cfg::GL, CPW = Cfg::CPW, CB = Cfg::CB;
+  using Ly = ScanLayout<N, XT>;
+  constexpr int NS = ScanShape<N>::NS, GL = ScanShape<N>::GL, CPW = 32 / GL;
+  constexpr int T = Ly::T, CB = Ly::CB, STAGES = Ly::STAGES, HALO = Ly::HALO;
+  constexpr int PRO_THREADS = kScanPro * 32;
   extern __shared__ __align__(1024) unsigned char smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::BAR_OFF);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Ly::BAR_OFF);
   uint64_t* empty = full + STAGES;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + STAGES);
+  uint64_t* pro_full = empty + STAGES;  // [2]
+  uint64_t* scan_done = pro_full + 2;   // [2]
+  uint64_t* epi_done = scan_done + 2;   // [2]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(epi_done + 2);
+  float4* XCH = reinterpret_cast<float4*>(smem + Ly::XCH_OFF);
+  float2* EPI = reinterpret_cast<float2*>(smem + Ly::EPI_OFF);
+  float* PART = reinterpret_cast<float*>(smem + Ly::PART_OFF);
 
+  const int CU = p.CU;
+  const int NSW = (CU + CPW - 1) / CPW;  // scan warps
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
-  const int c_cta = blockIdx.x * CB;
+  const int c_start = blockIdx.x * CU;
+  const int c_box = c_start & ~7;
+  const int off = c_start - c_box;
   const int64_t L = p.L;
   const int ntiles = static_cast<int>((L + T - 1) / T);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], WARPS);
+      mbar_init(&empty[s], NSW + kScanPro);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&pro_full[s], kScanPro);
+      mbar_init(&scan_done[s], NSW);
+      mbar_init(&epi_done[s], kScanPro);
     }
     *abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
 
-  if (warp == WARPS) {
-    // ------------------------------------------------------------ producer
+  if (warp == NSW + kScanPro) {
+    // ================================================================ TMA
     if (lane == 0) {
       tma_prefetch_desc(&map_x);
       tma_prefetch_desc(&map_w);
       tma_prefetch_desc(&map_b);
       tma_prefetch_desc(&map_c);
       if (p.has_z) tma_prefetch_desc(&map_z);
-      const uint32_t bytes = Cfg::XB + (p.has_z ? Cfg::ZB : 0) + Cfg::WB + 2 * Cfg::BB;
+      const uint32_t bytes = Ly::XB + (p.has_z ? Ly::ZB : 0) + Ly::WB + 2 * Ly::BB;
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % STAGES;
-        if (i >= STAGES) {
-          if (!mbar_wait(&empty[s], ((i / STAGES) - 1) & 1, abort_flag)) break;
-        }
-        unsigned char* st = smem + s * Cfg::STAGE_BYTES;
+        if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) - 1) & 1, abort_flag)) break;
+        unsigned char* st = smem + s * Ly::STAGE_BYTES;
         const int t0 = i * T;
         mbar_arrive_expect_tx(&full[s], bytes);
-        tma_load_3d(st + Cfg::X_OFF, &map_x, &full[s], c_cta, t0 - Cfg::HALO, b);
-        if (p.has_z) tma_load_3d(st + Cfg::Z_OFF, &map_z, &full[s], c_cta, t0, b);
-        tma_load_3d(st + Cfg::W_OFF, &map_w, &full[s], c_cta, t0, b);
-        tma_load_3d(st + Cfg::B_OFF, &map_b, &full[s], 0, t0, b);
-        tma_load_3d(st + Cfg::C_OFF, &map_c, &full[s], 0, t0, b);
+        tma_load_3d(st + Ly::X_OFF, &map_x, &full[s], c_box, t0 - HALO, b);
+        if (p.has_z) tma_load_3d(st + Ly::Z_OFF, &map_z, &full[s], c_box, t0, b);
+        tma_load_3d(st + Ly::W_OFF, &map_w, &full[s], c_box, t0, b);
+        tma_load_3d(st + Ly::B_OFF, &map_b, &full[s], 0, t0, b);
+        tma_load_3d(st + Ly::C_OFF, &map_c, &full[s], 0, t0, b);
         issued = i + 1;
       }
-      // Drain: make sure no copy is still in flight when the CTA exits (only
-      // matters after an abort; in normal runs every stage was consumed).
       for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i) {
         volatile int never = 0;
         mbar_wait(&full[i % STAGES], (i / STAGES) & 1, &never);
@@ -151,128 +265,221 @@ __global__ void __launch_bounds__((WARPS + 1) * 32, 1)
     return;
   }
 
-  // -------------------------------------------------------------- consumers
-  const int cg = lane / GL;        // channel within the warp
-  const int j = lane % GL;         // state group / sub-tile token index
-  const int cl = warp * CPW + cg;  // channel within the CTA tile
-  const int c = c_cta + cl;
-  const bool cvalid = c < p.D;
-  const int n0 = j * NS;
-  const int K = p.K;
-
-  float* xch = reinterpret_cast<float*>(smem + Cfg::SCRATCH_OFF + warp * Cfg::al(Cfg::WARP_SCRATCH));
-  float* red = xch + Cfg::XCH_FLOATS;
-
-  constexpr float kLog2e = 1.4426950408889634f;
-  float a2[NS], h[NS];
-#pragma unroll
-  for (int s = 0; s < NS; ++s) {
-    a2[s] = cvalid ? p.A[(int64_t)c * N + n0 + s] * kLog2e : 0.f;
-    h[s] = (cvalid && p.h0) ? p.h0[((int64_t)b * p.D + c) * N + n0 + s] : 0.f;
-  }
-  float cw[4] = {0.f, 0.f, 0.f, 0.f};
-  float cbias = 0.f, dskip = 0.f;
-  if (cvalid) {
-    if (p.fuse_conv) {
-      for (int k = 0; k < K; ++k) cw[4 - K + k] = p.conv_w[(int64_t)c * K + k];
-      if (p.conv_b) cbias = p.conv_b[c];
-    }
-    if (p.Dskip) dskip = p.Dskip[c];
-  }
-  const float* cstate = (cvalid && p.conv_state_in) ? p.conv_state_in + ((int64_t)b * p.D + c) * (K - 1) : nullptr;
-
-  for (int i = 0; i < ntiles; ++i) {
-    const int s = i % STAGES;
-    const bool ok = mbar_wait(&full[s], (i / STAGES) & 1, abort_flag);
-    if (!__all_sync(0xffffffffu, ok)) break;
-    const unsigned char* st = smem + s * Cfg::STAGE_BYTES;
-    const XT* xs = reinterpret_cast<const XT*>(st + Cfg::X_OFF);
-    const ZT* zs = reinterpret_cast<const ZT*>(st + Cfg::Z_OFF);
-    const float* ws = reinterpret_cast<const float*>(st + Cfg::W_OFF);
-    const float* bs = reinterpret_cast<const float*>(st + Cfg::B_OFF);
-    const float* cs = reinterpret_cast<const float*>(st + Cfg::C_OFF);
-    const int64_t t0 = (int64_t)i * T;
-
-#pragma unroll 1
-    for (int sub = 0; sub < T / GL; ++sub) {
-      // ---- prologue for token (sub*GL + j) of this channel
-      const int tl = sub * GL + j;
-      const int64_t t = t0 + tl;
-      const bool tvalid = t < L;
-      float u, dlt, g = 1.f;
+  if (warp >= NSW) {
+    // ================================================== prologue / epilogue
+    // Thread (tg, cl): channel cl of the CTA (lane), tokens [tg·TPT, (tg+1)·TPT)
+    // of every tile, so its per-channel constants stay in registers and the
+    // conv taps slide along consecutive tokens.
+    constexpr int TPT = T / kScanPro;  // tokens per thread per tile
+    const int cl = lane;
+    const int tg = warp - NSW;
+    const int cb = off + cl;
+    const int64_t c = c_start + cl;
+    const bool cact = cl < CU;           // lane owns a channel of this CTA
+    const bool cval = cact && c < p.D;   // ... that exists
+    const int K = p.K;
+    float cw[4] = {0.f, 0.f, 0.f, 0.f};
+    float cbias = 0.f, dsk = 0.f;
+    float hist[3] = {0.f, 0.f, 0.f};  // x of the 3 tokens before the first tile (conv state)
+    if (cval) {
       if (p.fuse_conv) {
-        float acc = cbias;
+        // tap k (0..3) multiplies x_{t-3+k}: weight k - (4 - K), if any
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          // tap k multiplies x_{t-3+k}; smem row tl + k holds token t - 3 + k
-          float xv = to_f32<XT>(xs[(tl + k) * CB + cl]);
-          if (cstate && t - 3 + k < 0 && k >= 4 - K) xv = cstate[(K - 1) + (t - 3 + k)];
-          acc = fmaf(cw[k], xv, acc);
+          const int kk = k - (4 - K);
+          cw[k] = kk >= 0 ? p.conv_w[c * K + kk] : 0.f;
         }
-        u = p.conv_silu ? silu_f(acc) : acc;
-      } else {
-        u = to_f32<XT>(xs[(tl + Cfg::HALO) * CB + cl]);
-      }
-      const float wraw = ws[tl * CB + cl];
-      dlt = p.softplus ? softplus_f(wraw) : wraw;
-      if (p.has_z) g = silu_f(to_f32<ZT>(zs[tl * CB + cl]));
-      if (!tvalid) dlt = 0.f;  // padding tokens leave the state untouched
-      const float du = dlt * u;
-      reinterpret_cast<float2*>(xch)[cg * GL + j] = make_float2(dlt, du);
-      __syncwarp();
-
-      // ---- recurrence over the GL tokens of the sub-tile
-      float part[GL];
+        if (p.conv_b) cbias = p.conv_b[c];
+        if (p.conv_state_in) {
 #pragma unroll
-      for (int k = 0; k < GL; ++k) {
-        const float2 e = reinterpret_cast<const float2*>(xch)[cg * GL + k];
-        const float* brow = bs + (sub * GL + k) * N + n0;
-        const float* crow = cs + (sub * GL + k) * N + n0;
+          for (int k = 0; k < 3; ++k) {  // hist[k] = x_{k-3}: state entry k - (4 - K)
+            const int kk = k - (4 - K);
+            hist[k] = kk >= 0 ? p.conv_state_in[((int64_t)b * p.D + c) * (K - 1) + kk] : 0.f;
+          }
+        }
+      }
+      if (p.Dskip) dsk = p.Dskip[c];
+    }
+
+    auto epilogue = [&](int i) -> bool {
+      const int slot = i & 1;
+      const bool ok = mbar_wait(&scan_done[slot], (i >> 1) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) return false;
+      const int64_t t0 = (int64_t)i * T;
+#pragma unroll
+      for (int q = 0; q < TPT; ++q) {
+        const int t = tg * TPT + q;
+        const float* part = PART + ((slot * T + t) * CB + cl) * GL;
         float acc = 0.f;
 #pragma unroll
-        for (int q = 0; q < NS; ++q) {
-          const float dA = fast_ex2(e.x * a2[q]);
-          h[q] = fmaf(dA, h[q], e.y * brow[q]);
-          acc = fmaf(crow[q], h[q], acc);
+        for (int r = 0; r < GL; r += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(part + r);
+          acc += (v.x + v.y) + (v.z + v.w);
         }
-        part[k] = acc;
+        const float2 e = EPI[(slot * T + t) * CB + cl];
+        const int64_t tok = t0 + t;
+        if (cval && tok < L)
+          reinterpret_cast<YT*>(p.y)[((int64_t)b * L + tok) * p.D + c] = from_f32<YT>((acc + e.x) * e.y);
       }
-      // ---- reduce C·h over the GL lanes of the channel: lane j gets token j
-#pragma unroll
-      for (int k = 0; k < GL; ++k) red[cg * Cfg::RS + k * GL + j] = part[k];
       __syncwarp();
-      float ysum = 0.f;
-#pragma unroll
-      for (int m = 0; m < GL; ++m) ysum += red[cg * Cfg::RS + j * GL + m];
-      __syncwarp();
+      if (lane == 0) mbar_arrive(&epi_done[slot]);
+      return true;
+    };
 
-      if (tvalid && cvalid) {
-        const float yv = (ysum + dskip * u) * g;
-        reinterpret_cast<YT*>(p.y)[((int64_t)b * L + t) * p.D + c] = from_f32<YT>(yv);
+    bool ok_all = true;
+    for (int i = 0; i < ntiles && ok_all; ++i) {
+      const int s = i % STAGES, slot = i & 1;
+      const bool ok = mbar_wait(&full[s], (i / STAGES) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) { ok_all = false; break; }
+      const unsigned char* st = smem + s * Ly::STAGE_BYTES;
+      const XT* xs = reinterpret_cast<const XT*>(st + Ly::X_OFF);
+      const XT* zs = reinterpret_cast<const XT*>(st + Ly::Z_OFF);
+      const float* ws = reinterpret_cast<const float*>(st + Ly::W_OFF);
+      const int64_t t0 = (int64_t)i * T;
+      const int tb = tg * TPT;  // first token of this thread in the tile
+      // conv window: smem row r holds token t0 - 3 + r
+      float xw[TPT + 3];
+#pragma unroll
+      for (int r = 0; r < TPT + 3; ++r) xw[r] = to_f32<XT>(xs[(tb + r) * CB + cb]);
+      if (i == 0 && tb == 0) {  // tokens before the sequence come from the conv state
+        xw[0] = hist[0];
+        xw[1] = hist[1];
+        xw[2] = hist[2];
       }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
-  }
-
-  if (*abort_flag) return;
-  if (cvalid) {
-    if (p.h_final) {
 #pragma unroll
-      for (int s = 0; s < NS; ++s) p.h_final[((int64_t)b * p.D + c) * N + n0 + s] = h[s];
-    }
-    if (p.conv_state_out) {
-      for (int jj = j; jj < K - 1; jj += GL) {
-        // new state entry jj = xpad[L + jj] (xpad = old state followed by x)
-        const int64_t src = L + jj - (K - 1);  // index into x (negative: old state)
-        float v;
-        if (src >= 0) {
-          v = to_f32<XT>(reinterpret_cast<const XT*>(p.x)[((int64_t)b * L + src) * p.D + c]);
+      for (int q = 0; q < TPT; ++q) {
+        const int t = tb + q;
+        const int64_t tok = t0 + t;
+        float u;
+        if (p.fuse_conv) {
+          float acc = cbias;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) acc = fmaf(cw[k], xw[q + k], acc);
+          u = p.conv_silu ? silu_fast(acc) : acc;
         } else {
-          v = cstate ? cstate[(K - 1) + src] : 0.f;
+          u = xw[q + HALO];
         }
+        const float wr = ws[t * CB + cb];
+        float dlt = p.softplus ? softplus_fast(wr) : wr;
+        if (tok >= L || !cact) dlt = 0.f;  // padding tokens leave the state untouched
+        const float du = dlt * u;
+        const float g = p.has_z ? silu_fast(to_f32<XT>(zs[t * CB + cb])) : 1.f;
+        if (cact) {
+          XCH[(slot * T + t) * CB + cl] = make_float4(dlt, dlt, du, du);
+          EPI[(slot * T + t) * CB + cl] = make_float2(dsk * u, g);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&pro_full[slot]);
+        mbar_arrive(&empty[s]);
+      }
+      if (i > 0 && !epilogue(i - 1)) { ok_all = false; break; }
+    }
+    if (ok_all && ntiles > 0) ok_all = epilogue(ntiles - 1);
+    if (!ok_all || *abort_flag) return;
+    // final conv state: the last K-1 entries of (old state, x)
+    if (p.conv_state_out && cval && tg == 0) {
+      for (int jj = 0; jj < K - 1; ++jj) {
+        const int64_t src = L + jj - (K - 1);
+        float v;
+        if (src >= 0) v = to_f32<XT>(reinterpret_cast<const XT*>(p.x)[((int64_t)b * L + src) * p.D + c]);
+        else v = p.conv_state_in ? p.conv_state_in[((int64_t)b * p.D + c) * (K - 1) + (K - 1) + src] : 0.f;
         p.conv_state_out[((int64_t)b * p.D + c) * (K - 1) + jj] = v;
       }
+    }
+    return;
+  }
+
+  // ==================================================================== scan
+  // Lane (cg, j): channel cl of the CTA, states [j·NS, (j+1)·NS) held as NP
+  // packed pairs.  Lanes past the CTA's channels (last warp, CU % CPW != 0)
+  // run along on zeros and write partials nobody reads.
+  constexpr int NP = (NS + 1) / 2;
+  const int cg = lane / GL, j = lane % GL;
+  const int cl = warp * CPW + cg;
+  const int64_t c = c_start + cl;
+  const bool cval = cl < CU && c < p.D;
+  const int n0 = j * NS;
+  constexpr float kLog2e = 1.4426950408889634f;
+  f2 a2p[NP], hp[NP];
+#pragma unroll
+  for (int q = 0; q < NP; ++q) {
+    float a[2] = {0.f, 0.f}, hh[2] = {0.f, 0.f};
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int n = n0 + 2 * q + r;
+      if (2 * q + r < NS && cval) {
+        a[r] = p.A[c * N + n] * kLog2e;
+        if (p.h0) hh[r] = p.h0[((int64_t)b * p.D + c) * N + n];
+      }
+    }
+    a2p[q] = pk2(a[0], a[1]);
+    hp[q] = pk2(hh[0], hh[1]);
+  }
+
+  for (int i = 0; i < ntiles; ++i) {
+    const int s = i % STAGES, slot = i & 1;
+    bool ok = mbar_wait(&pro_full[slot], (i >> 1) & 1, abort_flag);
+    ok = ok && mbar_wait(&full[s], (i / STAGES) & 1, abort_flag);
+    if (i >= 2) ok = ok && mbar_wait(&epi_done[slot], ((i - 2) >> 1) & 1, abort_flag);
+    if (!__all_sync(0xffffffffu, ok)) break;
+    const unsigned char* st = smem + s * Ly::STAGE_BYTES;
+    const float* bs = reinterpret_cast<const float*>(st + Ly::B_OFF);
+    const float* cs = reinterpret_cast<const float*>(st + Ly::C_OFF);
+    const float4* xch = XCH + slot * T * CB + cl;
+    float* part = PART + (slot * T * CB + cl) * GL + j;
+#pragma unroll 8
+    for (int t = 0; t < T; ++t) {
+      const float4 e = xch[t * CB];
+      f2 bb[NP], cc[NP];
+      if (NS == 4) {
+        const float4 bv = *reinterpret_cast<const float4*>(bs + t * N + n0);
+        const float4 cv = *reinterpret_cast<const float4*>(cs + t * N + n0);
+        bb[0] = pk2(bv.x, bv.y);
+        bb[NP - 1] = pk2(bv.z, bv.w);
+        cc[0] = pk2(cv.x, cv.y);
+        cc[NP - 1] = pk2(cv.z, cv.w);
+      } else if (NS == 2) {
+        const float2 bv = *reinterpret_cast<const float2*>(bs + t * N + n0);
+        const float2 cv = *reinterpret_cast<const float2*>(cs + t * N + n0);
+        bb[0] = pk2(bv.x, bv.y);
+        cc[0] = pk2(cv.x, cv.y);
+      } else {
+        bb[0] = pk2(bs[t * N + n0], 0.f);
+        cc[0] = pk2(cs[t * N + n0], 0.f);
+      }
+      const f2 dlt2 = pk2(e.x, e.y), du2 = pk2(e.z, e.w);
+      f2 acc;
+#pragma unroll
+      for (int q = 0; q < NP; ++q) {
+        const f2 xx = mul2(dlt2, a2p[q]);
+        f2 dA;
+        if (POLY > 0 && (t % POLY) == POLY - 1) {
+          dA = ex2_poly2(xx);
+        } else {
+          const float2 xv = up2(xx);
+          dA = pk2(mufu_ex2(xv.x), NS >= 2 ? mufu_ex2(xv.y) : 0.f);
+        }
+        hp[q] = fma2(dA, hp[q], mul2(du2, bb[q]));
+        acc = q == 0 ? mul2(cc[q], hp[q]) : fma2(cc[q], hp[q], acc);
+      }
+      const float2 pr = up2(acc);
+      part[t * CB * GL] = pr.x + pr.y;
+    }
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&scan_done[slot]);
+      mbar_arrive(&empty[s]);
+    }
+  }
+  if (*abort_flag) return;
+  if (cval && p.h_final) {
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+      const float2 hv = up2(hp[q]);
+      p.h_final[((int64_t)b * p.D + c) * N + n0 + 2 * q] = hv.x;
+      if (2 * q + 1 < NS) p.h_final[((int64_t)b * p.D + c) * N + n0 + 2 * q + 1] = hv.y;
     }
   }
 }
@@ -286,17 +493,39 @@ namespace samba {
 
 int take_status_scan(cudaStream_t s) { return take_status_word(s); }
 
+// Channels per CTA: the largest multiple of 4 (<= 32, and <= 28 unless a
+// multiple of 8 so that the 16-byte-aligned TMA box of 32 channels covers it)
+// that minimises (waves of CTAs) x (channels per CTA) on this GPU.
+static int choose_cu(int64_t B, int64_t D) {
+  const int sms = sm_count();
+  int best = 32;
+  int64_t best_cost = INT64_MAX;
+  for (int cu = 32; cu >= 8; cu -= 4) {
+    if (cu % 8 != 0 && cu > 28) continue;
+    const int64_t ctas = B * ((D + cu - 1) / cu);
+    const int64_t waves = (ctas + sms - 1) / sms;
+    const int64_t cost = waves * cu;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = cu;
+    }
+  }
+  return best;
+}
+
 template <int N, typename XT, typename YT>
 static int launch_scan_t(const samba_scan_args& a, cudaStream_t stream) {
-  constexpr int NS = 2, WARPS = (N == 16 ? 8 : (N == 8 ? 4 : 2)), T = 64, STAGES = 4;
-  using Cfg = ScanCfg<N, NS, WARPS, T, STAGES, XT, XT, YT>;
-  auto kern = scan_fwd_kernel<N, NS, WARPS, T, STAGES, XT, XT, YT>;
-  static bool attr_done = false;  // per instantiation; harmless if set twice
+  using Ly = ScanLayout<N, XT>;
+  constexpr int POLY = SAMBA_SCAN_POLY;
+  auto kern = scan_fwd_kernel<N, XT, YT, POLY>;
+  static bool attr_done = false;
   if (!attr_done) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::SMEM) != cudaSuccess)
       return fail(SAMBA_ERR_CUDA, "scan: cannot set shared memory size");
     attr_done = true;
   }
+  constexpr int CPW = 32 / ScanShape<N>::GL;
+  const int CU = choose_cu(a.batch, a.dim);
   const uint64_t Bsz = a.batch, L = a.seqlen, D = a.dim;
   const uint32_t xs = sizeof(XT);
   const CUtensorMapDataType xdt = sizeof(XT) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -304,8 +533,8 @@ static int launch_scan_t(const samba_scan_args& a, cudaStream_t stream) {
   {
     const uint64_t dims[3] = {D, L, Bsz};
     const uint64_t st[2] = {D * xs, L * D * xs};
-    const uint32_t boxx[3] = {(uint32_t)Cfg::CB, (uint32_t)Cfg::XROWS, 1};
-    const uint32_t boxz[3] = {(uint32_t)Cfg::CB, (uint32_t)T, 1};
+    const uint32_t boxx[3] = {(uint32_t)Ly::CB, (uint32_t)(Ly::T + Ly::HALO), 1};
+    const uint32_t boxz[3] = {(uint32_t)Ly::CB, (uint32_t)Ly::T, 1};
     int rc = encode_tiled(&mx, xdt, 3, a.x, dims, st, boxx, CU_TENSOR_MAP_SWIZZLE_NONE, "scan x");
     if (rc) return rc;
     rc = encode_tiled(&mz, xdt, 3, a.z ? a.z : a.x, dims, st, boxz, CU_TENSOR_MAP_SWIZZLE_NONE, "scan z");
@@ -316,7 +545,7 @@ static int launch_scan_t(const samba_scan_args& a, cudaStream_t stream) {
     if (rc) return rc;
     const uint64_t dimb[3] = {(uint64_t)N, L, Bsz};
     const uint64_t stb[2] = {(uint64_t)N * 4, L * N * 4};
-    const uint32_t boxb[3] = {(uint32_t)N, (uint32_t)T, 1};
+    const uint32_t boxb[3] = {(uint32_t)N, (uint32_t)Ly::T, 1};
     rc = encode_tiled(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.Bm, dimb, stb, boxb, CU_TENSOR_MAP_SWIZZLE_NONE, "scan B");
     if (rc) return rc;
     rc = encode_tiled(&mc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.Cm, dimb, stb, boxb, CU_TENSOR_MAP_SWIZZLE_NONE, "scan C");
@@ -336,12 +565,14 @@ static int launch_scan_t(const samba_scan_args& a, cudaStream_t stream) {
   p.L = a.seqlen;
   p.D = a.dim;
   p.K = a.dconv;
+  p.CU = CU;
   p.has_z = a.z != nullptr;
   p.fuse_conv = (a.flags & SAMBA_SCAN_FUSE_CONV) != 0;
   p.conv_silu = (a.flags & SAMBA_SCAN_CONV_SILU) != 0;
   p.softplus = (a.flags & SAMBA_SCAN_DELTA_SOFTPLUS) != 0;
-  dim3 grid((unsigned)((D + Cfg::CB - 1) / Cfg::CB), (unsigned)Bsz);
-  kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(mx, mz, mw, mb, mc, p);
+  const int threads = ((CU + CPW - 1) / CPW + kScanPro + 1) * 32;
+  dim3 grid((unsigned)((D + CU - 1) / CU), (unsigned)Bsz);
+  kern<<<grid, threads, Ly::SMEM, stream>>>(mx, mz, mw, mb, mc, p);
   return check_launch("samba_selective_scan_fwd");
 }
 
@@ -355,7 +586,8 @@ static int launch_scan_n(const samba_scan_args& a, cudaStream_t s) {
 }
 
 int launch_scan(const samba_scan_args& a, cudaStream_t s) {
-  if (a.z && a.z_dtype != a.x_dtype) return fail(SAMBA_ERR_UNSUPPORTED, "samba_selective_scan_fwd: z dtype must equal x dtype");
+  if (a.z && a.z_dtype != a.x_dtype)
+    return fail(SAMBA_ERR_UNSUPPORTED, "samba_selective_scan_fwd: z dtype must equal x dtype");
   switch (a.dstate) {
     case 4: return launch_scan_n<4>(a, s);
     case 8: return launch_scan_n<8>(a, s);

@@ -63,6 +63,9 @@ WORKLOADS = {
     "batched_32k": Workload("batched_32k", 8, 32768, 4096, 16, 4, 32, 4, 64, 2048, 3),
     "decode_64k": Workload("decode_64k", 16, 4096, 4096, 16, 4, 32, 4, 64, 2048, 4,
                            decode_steps=65536),
+    # one 32K-token prompt at the same widths: every input still exceeds L2,
+    # but the whole problem holds ~1.5 GB, small enough for profiler captures
+    "prefill_32k": Workload("prefill_32k", 1, 32768, 4096, 16, 4, 32, 4, 64, 2048, 5),
 }
 
 
