@@ -39,11 +39,11 @@
 // Every SAMBA_SCAN_POLY-th token evaluates its exps on the FMA pipe
 // (0: never).  A build-time constant, fixed by measurement.
 #ifndef SAMBA_SCAN_POLY
-#define SAMBA_SCAN_POLY 4
+#define SAMBA_SCAN_POLY 0
 #endif
 // States per scan lane at N = 16 (2 or 4); also fixed by measurement.
 #ifndef SAMBA_SCAN_NS16
-#define SAMBA_SCAN_NS16 2
+#define SAMBA_SCAN_NS16 4
 #endif
 
 namespace samba {
@@ -73,7 +73,7 @@ template <> struct ScanShape<4> { static constexpr int NS = 1, GL = 4; };
 constexpr int kScanCB = 32;     // channels in one TMA box (>= CU + alignment offset)
 constexpr int kScanT = 32;      // tokens per tile
 constexpr int kScanStages = 4;  // TMA ring depth
-constexpr int kScanPro = 4;     // prologue / epilogue warps
+constexpr int kScanPro = 8;     // prologue / epilogue warps
 
 template <int N, typename XT>
 struct ScanLayout {
@@ -86,8 +86,8 @@ struct ScanLayout {
   static constexpr int BB = T * N * 4;
   static constexpr int X_OFF = 0, Z_OFF = al(XB), W_OFF = Z_OFF + al(ZB), B_OFF = W_OFF + al(WB),
                        C_OFF = B_OFF + al(BB), STAGE_BYTES = C_OFF + al(BB);
-  static constexpr int XCH_OFF = STAGES * STAGE_BYTES;        // float4 [2][T][CB]
-  static constexpr int EPI_OFF = XCH_OFF + 2 * T * CB * 16;   // float2 [2][T][CB]
+  static constexpr int XCH_OFF = STAGES * STAGE_BYTES;        // float2 [2][T][CB] (Δ, Δu)
+  static constexpr int EPI_OFF = XCH_OFF + 2 * T * CB * 8;    // float2 [2][T][CB] (D·u, silu(z))
   static constexpr int PART_OFF = EPI_OFF + 2 * T * CB * 8;   // float  [2][T][CB][GL]
   static constexpr int BAR_OFF = PART_OFF + 2 * T * CB * GL * 4;
   static constexpr int SMEM = BAR_OFF + 256;
@@ -190,7 +190,7 @@ __device__ __forceinline__ float softplus_fast(float w) {
 
 // ------------------------------------------------------------------ kernel
 template <int N, typename XT, typename YT, int POLY>
-__global__ void __launch_bounds__(416, 1)
+__global__ void __launch_bounds__(544, 1)
     scan_fwd_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_z,
                     const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_b,
                     const __grid_constant__ CUtensorMap map_c, const ScanParams p) {
@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(416, 1)
   uint64_t* scan_done = pro_full + 2;   // [2]
   uint64_t* epi_done = scan_done + 2;   // [2]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(epi_done + 2);
-  float4* XCH = reinterpret_cast<float4*>(smem + Ly::XCH_OFF);
+  float2* XCH = reinterpret_cast<float2*>(smem + Ly::XCH_OFF);
   float2* EPI = reinterpret_cast<float2*>(smem + Ly::EPI_OFF);
   float* PART = reinterpret_cast<float*>(smem + Ly::PART_OFF);
 
@@ -346,6 +346,12 @@ __global__ void __launch_bounds__(416, 1)
         xw[1] = hist[1];
         xw[2] = hist[2];
       }
+      float wv[TPT], zv[TPT];
+#pragma unroll
+      for (int q = 0; q < TPT; ++q) {
+        wv[q] = ws[(tb + q) * CB + cb];
+        zv[q] = p.has_z ? to_f32<XT>(zs[(tb + q) * CB + cb]) : 0.f;
+      }
 #pragma unroll
       for (int q = 0; q < TPT; ++q) {
         const int t = tb + q;
@@ -359,13 +365,13 @@ __global__ void __launch_bounds__(416, 1)
         } else {
           u = xw[q + HALO];
         }
-        const float wr = ws[t * CB + cb];
+        const float wr = wv[q];
         float dlt = p.softplus ? softplus_fast(wr) : wr;
         if (tok >= L || !cact) dlt = 0.f;  // padding tokens leave the state untouched
         const float du = dlt * u;
-        const float g = p.has_z ? silu_fast(to_f32<XT>(zs[t * CB + cb])) : 1.f;
+        const float g = p.has_z ? silu_fast(zv[q]) : 1.f;
         if (cact) {
-          XCH[(slot * T + t) * CB + cl] = make_float4(dlt, dlt, du, du);
+          XCH[(slot * T + t) * CB + cl] = make_float2(dlt, du);
           EPI[(slot * T + t) * CB + cl] = make_float2(dsk * u, g);
         }
       }
@@ -427,45 +433,57 @@ __global__ void __launch_bounds__(416, 1)
     const unsigned char* st = smem + s * Ly::STAGE_BYTES;
     const float* bs = reinterpret_cast<const float*>(st + Ly::B_OFF);
     const float* cs = reinterpret_cast<const float*>(st + Ly::C_OFF);
-    const float4* xch = XCH + slot * T * CB + cl;
+    const float2* xch = XCH + slot * T * CB + cl;
     float* part = PART + (slot * T * CB + cl) * GL + j;
-#pragma unroll 8
-    for (int t = 0; t < T; ++t) {
-      const float4 e = xch[t * CB];
-      f2 bb[NP], cc[NP];
-      if (NS == 4) {
-        const float4 bv = *reinterpret_cast<const float4*>(bs + t * N + n0);
-        const float4 cv = *reinterpret_cast<const float4*>(cs + t * N + n0);
-        bb[0] = pk2(bv.x, bv.y);
-        bb[NP - 1] = pk2(bv.z, bv.w);
-        cc[0] = pk2(cv.x, cv.y);
-        cc[NP - 1] = pk2(cv.z, cv.w);
-      } else if (NS == 2) {
-        const float2 bv = *reinterpret_cast<const float2*>(bs + t * N + n0);
-        const float2 cv = *reinterpret_cast<const float2*>(cs + t * N + n0);
-        bb[0] = pk2(bv.x, bv.y);
-        cc[0] = pk2(cv.x, cv.y);
-      } else {
-        bb[0] = pk2(bs[t * N + n0], 0.f);
-        cc[0] = pk2(cs[t * N + n0], 0.f);
-      }
-      const f2 dlt2 = pk2(e.x, e.y), du2 = pk2(e.z, e.w);
-      f2 acc;
+    constexpr int G8 = 8;  // tokens whose operands are loaded before any is used
+#pragma unroll 1
+    for (int t8 = 0; t8 < T; t8 += G8) {
+      float2 ev[G8];
+      f2 bb[G8][NP], cc[G8][NP];
 #pragma unroll
-      for (int q = 0; q < NP; ++q) {
-        const f2 xx = mul2(dlt2, a2p[q]);
-        f2 dA;
-        if (POLY > 0 && (t % POLY) == POLY - 1) {
-          dA = ex2_poly2(xx);
+      for (int k = 0; k < G8; ++k) {
+        const int t = t8 + k;
+        ev[k] = xch[t * CB];
+        if (NS == 4) {
+          const float4 bv = *reinterpret_cast<const float4*>(bs + t * N + n0);
+          const float4 cv = *reinterpret_cast<const float4*>(cs + t * N + n0);
+          bb[k][0] = pk2(bv.x, bv.y);
+          bb[k][NP - 1] = pk2(bv.z, bv.w);
+          cc[k][0] = pk2(cv.x, cv.y);
+          cc[k][NP - 1] = pk2(cv.z, cv.w);
+        } else if (NS == 2) {
+          const float2 bv = *reinterpret_cast<const float2*>(bs + t * N + n0);
+          const float2 cv = *reinterpret_cast<const float2*>(cs + t * N + n0);
+          bb[k][0] = pk2(bv.x, bv.y);
+          cc[k][0] = pk2(cv.x, cv.y);
         } else {
-          const float2 xv = up2(xx);
-          dA = pk2(mufu_ex2(xv.x), NS >= 2 ? mufu_ex2(xv.y) : 0.f);
+          bb[k][0] = pk2(bs[t * N + n0], 0.f);
+          cc[k][0] = pk2(cs[t * N + n0], 0.f);
         }
-        hp[q] = fma2(dA, hp[q], mul2(du2, bb[q]));
-        acc = q == 0 ? mul2(cc[q], hp[q]) : fma2(cc[q], hp[q], acc);
       }
-      const float2 pr = up2(acc);
-      part[t * CB * GL] = pr.x + pr.y;
+      float pv[G8];
+#pragma unroll
+      for (int k = 0; k < G8; ++k) {
+        const f2 dlt2 = pk2(ev[k].x, ev[k].x), du2 = pk2(ev[k].y, ev[k].y);
+        f2 acc;
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+          const f2 xx = mul2(dlt2, a2p[q]);
+          f2 dA;
+          if (POLY > 0 && (k % POLY) == POLY - 1) {
+            dA = ex2_poly2(xx);
+          } else {
+            const float2 xv = up2(xx);
+            dA = pk2(mufu_ex2(xv.x), NS >= 2 ? mufu_ex2(xv.y) : 0.f);
+          }
+          hp[q] = fma2(dA, hp[q], mul2(du2, bb[k][q]));
+          acc = q == 0 ? mul2(cc[k][q], hp[q]) : fma2(cc[k][q], hp[q], acc);
+        }
+        const float2 pr = up2(acc);
+        pv[k] = pr.x + pr.y;
+      }
+#pragma unroll
+      for (int k = 0; k < G8; ++k) part[(t8 + k) * CB * GL] = pv[k];
     }
     __syncwarp();
     if (lane == 0) {
