@@ -72,13 +72,26 @@ template <> struct ScanShape<4> { static constexpr int NS = 1, GL = 4; };
 
 constexpr int kScanCB = 32;     // channels in one TMA box (>= CU + alignment offset)
 constexpr int kScanT = 32;      // tokens per tile
-constexpr int kScanStages = 4;  // TMA ring depth
-constexpr int kScanPro = 8;     // prologue / epilogue warps
+constexpr int kScanPro = 8;     // prologue warps
+constexpr int kScanEpi = 4;     // epilogue warps
+// Upper bound on the block size (sets the register budget per thread).
+#ifndef SAMBA_SCAN_MAXTHREADS
+#define SAMBA_SCAN_MAXTHREADS 672
+#endif
+// Tokens per load / exp / update group of the scan warps.
+#ifndef SAMBA_SCAN_GROUP
+#define SAMBA_SCAN_GROUP 8
+#endif
+#ifndef SAMBA_SCAN_SLOTS
+#define SAMBA_SCAN_SLOTS 3
+#endif
+constexpr int kScanSlots = SAMBA_SCAN_SLOTS;  // depth of the prologue -> scan -> epilogue hand-off
+constexpr int kScanSmemBudget = 227 * 1024;
 
 template <int N, typename XT>
 struct ScanLayout {
   static constexpr int GL = ScanShape<N>::GL;
-  static constexpr int CB = kScanCB, T = kScanT, STAGES = kScanStages, HALO = 3;
+  static constexpr int CB = kScanCB, T = kScanT, HALO = 3, SLOTS = kScanSlots;
   static constexpr int al(int v) { return (v + 127) / 128 * 128; }
   static constexpr int XB = (T + HALO) * CB * (int)sizeof(XT);
   static constexpr int ZB = T * CB * (int)sizeof(XT);
@@ -86,12 +99,24 @@ struct ScanLayout {
   static constexpr int BB = T * N * 4;
   static constexpr int X_OFF = 0, Z_OFF = al(XB), W_OFF = Z_OFF + al(ZB), B_OFF = W_OFF + al(WB),
                        C_OFF = B_OFF + al(BB), STAGE_BYTES = C_OFF + al(BB);
-  static constexpr int XCH_OFF = STAGES * STAGE_BYTES;        // float2 [2][T][CB] (Δ, Δu)
-  static constexpr int EPI_OFF = XCH_OFF + 2 * T * CB * 8;    // float2 [2][T][CB] (D·u, silu(z))
-  static constexpr int PART_OFF = EPI_OFF + 2 * T * CB * 8;   // float  [2][T][CB][GL]
-  static constexpr int BAR_OFF = PART_OFF + 2 * T * CB * GL * 4;
-  static constexpr int SMEM = BAR_OFF + 256;
+  static constexpr int XCH_BYTES = SLOTS * T * CB * 8;       // float2 [SLOTS][T][CB] (Δ, Δu)
+  static constexpr int EPI_BYTES = SLOTS * T * CB * 8;       // float2 [SLOTS][T][CB] (D·u, silu(z))
+  static constexpr int PART_BYTES = SLOTS * T * CB * GL * 4; // float  [SLOTS][T][CB][GL]
+  static constexpr int FIXED = XCH_BYTES + EPI_BYTES + PART_BYTES + 512;
+  // TMA ring: as many stages (up to 6) as fit next to the hand-off buffers
+  static constexpr int STAGES_FIT = (kScanSmemBudget - FIXED) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+  static_assert(STAGES >= 2, "scan tile does not fit in shared memory");
+  static constexpr int XCH_OFF = STAGES * STAGE_BYTES;
+  static constexpr int EPI_OFF = XCH_OFF + XCH_BYTES;
+  static constexpr int PART_OFF = EPI_OFF + EPI_BYTES;
+  static constexpr int BAR_OFF = PART_OFF + PART_BYTES;
+  static constexpr int SMEM = BAR_OFF + 512;
 };
+
+__host__ __device__ constexpr int scan_warps(int cu, int cpw) {
+  return (((cu + cpw - 1) / cpw) + 3) / 4 * 4;
+}
 
 // ------------------------------------------------------------ math helpers
 __device__ __forceinline__ float mufu_ex2(float x) {
@@ -189,28 +214,41 @@ __device__ __forceinline__ float softplus_fast(float w) {
 }
 
 // ------------------------------------------------------------------ kernel
+// Warp roles (index ranges): [0, NSW) scan, then kScanPro prologue, then
+// kScanEpi epilogue, then one TMA producer.  Per tile i (slot k = i % SLOTS):
+//   producer : full[s] <- TMA of x, z, delta, B, C          (waits empty[s])
+//   prologue : XCH[k], EPI[k] <- conv/softplus/gate; arrives pro_full[k]
+//              (waits full[s]; scan_done[k] and epi_done[k] of tile i-SLOTS)
+//   scan     : PART[k] <- partial C·h of its states; arrives scan_done[k]
+//              (waits pro_full[k], full[s]; epi_done[k] of tile i-SLOTS)
+//   epilogue : y <- (Σ PART[k] + D·u)·silu(z); arrives epi_done[k]
+//              (waits scan_done[k])
+// empty[s] collects the prologue and scan warps (the readers of stage s).
 template <int N, typename XT, typename YT, int POLY>
-__global__ void __launch_bounds__(544, 1)
+__global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
     scan_fwd_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_z,
                     const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_b,
                     const __grid_constant__ CUtensorMap map_c, const ScanParams p) {
   using Ly = ScanLayout<N, XT>;
   constexpr int NS = ScanShape<N>::NS, GL = ScanShape<N>::GL, CPW = 32 / GL;
-  constexpr int T = Ly::T, CB = Ly::CB, STAGES = Ly::STAGES, HALO = Ly::HALO;
-  constexpr int PRO_THREADS = kScanPro * 32;
+  constexpr int T = Ly::T, CB = Ly::CB, STAGES = Ly::STAGES, HALO = Ly::HALO, SLOTS = Ly::SLOTS;
   extern __shared__ __align__(1024) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Ly::BAR_OFF);
   uint64_t* empty = full + STAGES;
-  uint64_t* pro_full = empty + STAGES;  // [2]
-  uint64_t* scan_done = pro_full + 2;   // [2]
-  uint64_t* epi_done = scan_done + 2;   // [2]
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(epi_done + 2);
+  uint64_t* pro_full = empty + STAGES;      // [SLOTS]
+  uint64_t* scan_done = pro_full + SLOTS;   // [SLOTS]
+  uint64_t* epi_done = scan_done + SLOTS;   // [SLOTS]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(epi_done + SLOTS);
   float2* XCH = reinterpret_cast<float2*>(smem + Ly::XCH_OFF);
   float2* EPI = reinterpret_cast<float2*>(smem + Ly::EPI_OFF);
   float* PART = reinterpret_cast<float*>(smem + Ly::PART_OFF);
 
   const int CU = p.CU;
-  const int NSW = (CU + CPW - 1) / CPW;  // scan warps
+  // Scan warps: a multiple of 4 (one per SM sub-partition, whose MUFU pipes
+  // are separate), channels spread evenly over them.
+  const int NSW = scan_warps(CU, CPW);
+  const int CPWE = (CU + NSW - 1) / NSW;  // channels per scan warp
+  const int PRO0 = NSW, EPI0 = NSW + kScanPro, PROD = NSW + kScanPro + kScanEpi;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
   const int c_start = blockIdx.x * CU;
@@ -224,17 +262,17 @@ __global__ void __launch_bounds__(544, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], NSW + kScanPro);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&pro_full[s], kScanPro);
-      mbar_init(&scan_done[s], NSW);
-      mbar_init(&epi_done[s], kScanPro);
+    for (int k = 0; k < SLOTS; ++k) {
+      mbar_init(&pro_full[k], kScanPro);
+      mbar_init(&scan_done[k], NSW);
+      mbar_init(&epi_done[k], kScanEpi);
     }
     *abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
 
-  if (warp == NSW + kScanPro) {
+  if (warp == PROD) {
     // ================================================================ TMA
     if (lane == 0) {
       tma_prefetch_desc(&map_x);
@@ -265,14 +303,55 @@ __global__ void __launch_bounds__(544, 1)
     return;
   }
 
-  if (warp >= NSW) {
-    // ================================================== prologue / epilogue
+  if (warp >= EPI0) {
+    // ============================================================ epilogue
+    // Thread (eg, cl): channel cl (lane), tokens [eg·TPE, (eg+1)·TPE) of every tile.
+    constexpr int TPE = T / kScanEpi;
+    const int cl = lane, eg = warp - EPI0;
+    const int64_t c = c_start + cl;
+    const bool cval = cl < CU && c < p.D;
+    for (int i = 0; i < ntiles; ++i) {
+      const int k = i % SLOTS, r = i / SLOTS;
+      const bool ok = mbar_wait(&scan_done[k], r & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const int64_t t0 = (int64_t)i * T;
+      float4 pv[TPE];
+      float2 ev[TPE];
+#pragma unroll
+      for (int q = 0; q < TPE; ++q) {
+        const int t = eg * TPE + q;
+        const float* part = PART + ((k * T + t) * CB + cl) * GL;
+        pv[q] = *reinterpret_cast<const float4*>(part);
+        if (GL == 8) {
+          const float4 v2 = *reinterpret_cast<const float4*>(part + 4);
+          pv[q].x += v2.x;
+          pv[q].y += v2.y;
+          pv[q].z += v2.z;
+          pv[q].w += v2.w;
+        }
+        ev[q] = EPI[(k * T + t) * CB + cl];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&epi_done[k]);
+#pragma unroll
+      for (int q = 0; q < TPE; ++q) {
+        const int64_t tok = t0 + eg * TPE + q;
+        const float acc = (pv[q].x + pv[q].y) + (pv[q].z + pv[q].w);
+        if (cval && tok < L)
+          reinterpret_cast<YT*>(p.y)[((int64_t)b * L + tok) * p.D + c] = from_f32<YT>((acc + ev[q].x) * ev[q].y);
+      }
+    }
+    return;
+  }
+
+  if (warp >= PRO0) {
+    // ============================================================ prologue
     // Thread (tg, cl): channel cl of the CTA (lane), tokens [tg·TPT, (tg+1)·TPT)
     // of every tile, so its per-channel constants stay in registers and the
     // conv taps slide along consecutive tokens.
     constexpr int TPT = T / kScanPro;  // tokens per thread per tile
     const int cl = lane;
-    const int tg = warp - NSW;
+    const int tg = warp - PRO0;
     const int cb = off + cl;
     const int64_t c = c_start + cl;
     const bool cact = cl < CU;           // lane owns a channel of this CTA
@@ -301,36 +380,14 @@ __global__ void __launch_bounds__(544, 1)
       if (p.Dskip) dsk = p.Dskip[c];
     }
 
-    auto epilogue = [&](int i) -> bool {
-      const int slot = i & 1;
-      const bool ok = mbar_wait(&scan_done[slot], (i >> 1) & 1, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) return false;
-      const int64_t t0 = (int64_t)i * T;
-#pragma unroll
-      for (int q = 0; q < TPT; ++q) {
-        const int t = tg * TPT + q;
-        const float* part = PART + ((slot * T + t) * CB + cl) * GL;
-        float acc = 0.f;
-#pragma unroll
-        for (int r = 0; r < GL; r += 4) {
-          const float4 v = *reinterpret_cast<const float4*>(part + r);
-          acc += (v.x + v.y) + (v.z + v.w);
-        }
-        const float2 e = EPI[(slot * T + t) * CB + cl];
-        const int64_t tok = t0 + t;
-        if (cval && tok < L)
-          reinterpret_cast<YT*>(p.y)[((int64_t)b * L + tok) * p.D + c] = from_f32<YT>((acc + e.x) * e.y);
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = i % STAGES, k = i % SLOTS, r = i / SLOTS;
+      bool ok = mbar_wait(&full[s], (i / STAGES) & 1, abort_flag);
+      if (r >= 1) {
+        ok = ok && mbar_wait(&scan_done[k], (r - 1) & 1, abort_flag);
+        ok = ok && mbar_wait(&epi_done[k], (r - 1) & 1, abort_flag);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&epi_done[slot]);
-      return true;
-    };
-
-    bool ok_all = true;
-    for (int i = 0; i < ntiles && ok_all; ++i) {
-      const int s = i % STAGES, slot = i & 1;
-      const bool ok = mbar_wait(&full[s], (i / STAGES) & 1, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) { ok_all = false; break; }
+      if (!__all_sync(0xffffffffu, ok)) break;
       const unsigned char* st = smem + s * Ly::STAGE_BYTES;
       const XT* xs = reinterpret_cast<const XT*>(st + Ly::X_OFF);
       const XT* zs = reinterpret_cast<const XT*>(st + Ly::Z_OFF);
@@ -338,19 +395,20 @@ __global__ void __launch_bounds__(544, 1)
       const int64_t t0 = (int64_t)i * T;
       const int tb = tg * TPT;  // first token of this thread in the tile
       // conv window: smem row r holds token t0 - 3 + r
-      float xw[TPT + 3];
+      float xw[TPT + 3], wv[TPT], zv[TPT];
 #pragma unroll
-      for (int r = 0; r < TPT + 3; ++r) xw[r] = to_f32<XT>(xs[(tb + r) * CB + cb]);
-      if (i == 0 && tb == 0) {  // tokens before the sequence come from the conv state
-        xw[0] = hist[0];
-        xw[1] = hist[1];
-        xw[2] = hist[2];
-      }
-      float wv[TPT], zv[TPT];
+      for (int q = 0; q < TPT + 3; ++q) xw[q] = to_f32<XT>(xs[(tb + q) * CB + cb]);
 #pragma unroll
       for (int q = 0; q < TPT; ++q) {
         wv[q] = ws[(tb + q) * CB + cb];
         zv[q] = p.has_z ? to_f32<XT>(zs[(tb + q) * CB + cb]) : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);  // x, z, delta of stage s consumed
+      if (i == 0 && tb == 0) {  // tokens before the sequence come from the conv state
+        xw[0] = hist[0];
+        xw[1] = hist[1];
+        xw[2] = hist[2];
       }
 #pragma unroll
       for (int q = 0; q < TPT; ++q) {
@@ -360,7 +418,7 @@ __global__ void __launch_bounds__(544, 1)
         if (p.fuse_conv) {
           float acc = cbias;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) acc = fmaf(cw[k], xw[q + k], acc);
+          for (int kk = 0; kk < 4; ++kk) acc = fmaf(cw[kk], xw[q + kk], acc);
           u = p.conv_silu ? silu_fast(acc) : acc;
         } else {
           u = xw[q + HALO];
@@ -371,19 +429,14 @@ __global__ void __launch_bounds__(544, 1)
         const float du = dlt * u;
         const float g = p.has_z ? silu_fast(zv[q]) : 1.f;
         if (cact) {
-          XCH[(slot * T + t) * CB + cl] = make_float2(dlt, du);
-          EPI[(slot * T + t) * CB + cl] = make_float2(dsk * u, g);
+          XCH[(k * T + t) * CB + cl] = make_float2(dlt, du);
+          EPI[(k * T + t) * CB + cl] = make_float2(dsk * u, g);
         }
       }
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&pro_full[slot]);
-        mbar_arrive(&empty[s]);
-      }
-      if (i > 0 && !epilogue(i - 1)) { ok_all = false; break; }
+      if (lane == 0) mbar_arrive(&pro_full[k]);
     }
-    if (ok_all && ntiles > 0) ok_all = epilogue(ntiles - 1);
-    if (!ok_all || *abort_flag) return;
+    if (*abort_flag) return;
     // final conv state: the last K-1 entries of (old state, x)
     if (p.conv_state_out && cval && tg == 0) {
       for (int jj = 0; jj < K - 1; ++jj) {
@@ -403,9 +456,10 @@ __global__ void __launch_bounds__(544, 1)
   // run along on zeros and write partials nobody reads.
   constexpr int NP = (NS + 1) / 2;
   const int cg = lane / GL, j = lane % GL;
-  const int cl = warp * CPW + cg;
+  const int cl = warp * CPWE + cg;
   const int64_t c = c_start + cl;
-  const bool cval = cl < CU && c < p.D;
+  const bool cown = cg < CPWE && cl < CU;  // lane owns one of this warp's channels
+  const bool cval = cown && c < p.D;
   const int n0 = j * NS;
   constexpr float kLog2e = 1.4426950408889634f;
   f2 a2p[NP], hp[NP];
@@ -425,69 +479,79 @@ __global__ void __launch_bounds__(544, 1)
   }
 
   for (int i = 0; i < ntiles; ++i) {
-    const int s = i % STAGES, slot = i & 1;
-    bool ok = mbar_wait(&pro_full[slot], (i >> 1) & 1, abort_flag);
+    const int s = i % STAGES, k = i % SLOTS, r = i / SLOTS;
+    bool ok = mbar_wait(&pro_full[k], r & 1, abort_flag);
     ok = ok && mbar_wait(&full[s], (i / STAGES) & 1, abort_flag);
-    if (i >= 2) ok = ok && mbar_wait(&epi_done[slot], ((i - 2) >> 1) & 1, abort_flag);
+    if (r >= 1) ok = ok && mbar_wait(&epi_done[k], (r - 1) & 1, abort_flag);
     if (!__all_sync(0xffffffffu, ok)) break;
     const unsigned char* st = smem + s * Ly::STAGE_BYTES;
     const float* bs = reinterpret_cast<const float*>(st + Ly::B_OFF);
     const float* cs = reinterpret_cast<const float*>(st + Ly::C_OFF);
-    const float2* xch = XCH + slot * T * CB + cl;
-    float* part = PART + (slot * T * CB + cl) * GL + j;
-    constexpr int G8 = 8;  // tokens whose operands are loaded before any is used
-#pragma unroll 1
-    for (int t8 = 0; t8 < T; t8 += G8) {
-      float2 ev[G8];
-      f2 bb[G8][NP], cc[G8][NP];
+    const float2* xch = XCH + k * T * CB + cl;
+    float* part = PART + (k * T * CB + cl) * GL + j;
+    // Groups of G tokens in three phases: load every operand, issue every exp
+    // (they do not depend on the state, so the MUFU pipe is fed back to
+    // back), then run the dependent state updates and store the partials.
+    constexpr int G = SAMBA_SCAN_GROUP;
+#pragma unroll 2
+    for (int tg0 = 0; tg0 < T; tg0 += G) {
+      float2 ev[G];
+      f2 bb[G][NP], cc[G][NP], dA[G][NP];
 #pragma unroll
-      for (int k = 0; k < G8; ++k) {
-        const int t = t8 + k;
-        ev[k] = xch[t * CB];
+      for (int q = 0; q < G; ++q) {
+        const int t = tg0 + q;
+        ev[q] = xch[t * CB];
         if (NS == 4) {
           const float4 bv = *reinterpret_cast<const float4*>(bs + t * N + n0);
           const float4 cv = *reinterpret_cast<const float4*>(cs + t * N + n0);
-          bb[k][0] = pk2(bv.x, bv.y);
-          bb[k][NP - 1] = pk2(bv.z, bv.w);
-          cc[k][0] = pk2(cv.x, cv.y);
-          cc[k][NP - 1] = pk2(cv.z, cv.w);
+          bb[q][0] = pk2(bv.x, bv.y);
+          bb[q][NP - 1] = pk2(bv.z, bv.w);
+          cc[q][0] = pk2(cv.x, cv.y);
+          cc[q][NP - 1] = pk2(cv.z, cv.w);
         } else if (NS == 2) {
           const float2 bv = *reinterpret_cast<const float2*>(bs + t * N + n0);
           const float2 cv = *reinterpret_cast<const float2*>(cs + t * N + n0);
-          bb[k][0] = pk2(bv.x, bv.y);
-          cc[k][0] = pk2(cv.x, cv.y);
+          bb[q][0] = pk2(bv.x, bv.y);
+          cc[q][0] = pk2(cv.x, cv.y);
         } else {
-          bb[k][0] = pk2(bs[t * N + n0], 0.f);
-          cc[k][0] = pk2(cs[t * N + n0], 0.f);
+          bb[q][0] = pk2(bs[t * N + n0], 0.f);
+          cc[q][0] = pk2(cs[t * N + n0], 0.f);
         }
       }
-      float pv[G8];
 #pragma unroll
-      for (int k = 0; k < G8; ++k) {
-        const f2 dlt2 = pk2(ev[k].x, ev[k].x), du2 = pk2(ev[k].y, ev[k].y);
-        f2 acc;
+      for (int q = 0; q < G; ++q) {
+        const f2 dlt2 = pk2(ev[q].x, ev[q].x);
 #pragma unroll
-        for (int q = 0; q < NP; ++q) {
-          const f2 xx = mul2(dlt2, a2p[q]);
-          f2 dA;
-          if (POLY > 0 && (k % POLY) == POLY - 1) {
-            dA = ex2_poly2(xx);
+        for (int m = 0; m < NP; ++m) {
+          const f2 xx = mul2(dlt2, a2p[m]);
+          if (POLY > 0 && (q % (POLY > 0 ? POLY : 1)) == POLY - 1) {
+            dA[q][m] = ex2_poly2(xx);
           } else {
             const float2 xv = up2(xx);
-            dA = pk2(mufu_ex2(xv.x), NS >= 2 ? mufu_ex2(xv.y) : 0.f);
+            dA[q][m] = pk2(mufu_ex2(xv.x), NS >= 2 ? mufu_ex2(xv.y) : 0.f);
           }
-          hp[q] = fma2(dA, hp[q], mul2(du2, bb[k][q]));
-          acc = q == 0 ? mul2(cc[k][q], hp[q]) : fma2(cc[k][q], hp[q], acc);
+        }
+      }
+      float pv[G];
+#pragma unroll
+      for (int q = 0; q < G; ++q) {
+        const f2 du2 = pk2(ev[q].y, ev[q].y);
+        f2 acc;
+#pragma unroll
+        for (int m = 0; m < NP; ++m) {
+          hp[m] = fma2(dA[q][m], hp[m], mul2(du2, bb[q][m]));
+          acc = m == 0 ? mul2(cc[q][m], hp[m]) : fma2(cc[q][m], hp[m], acc);
         }
         const float2 pr = up2(acc);
-        pv[k] = pr.x + pr.y;
+        pv[q] = pr.x + pr.y;
       }
 #pragma unroll
-      for (int k = 0; k < G8; ++k) part[(t8 + k) * CB * GL] = pv[k];
+      for (int q = 0; q < G; ++q)
+        if (cown) part[(tg0 + q) * CB * GL] = pv[q];  // idle lanes alias other warps' channels
     }
     __syncwarp();
     if (lane == 0) {
-      mbar_arrive(&scan_done[slot]);
+      mbar_arrive(&scan_done[k]);
       mbar_arrive(&empty[s]);
     }
   }
@@ -588,7 +652,7 @@ static int launch_scan_t(const samba_scan_args& a, cudaStream_t stream) {
   p.fuse_conv = (a.flags & SAMBA_SCAN_FUSE_CONV) != 0;
   p.conv_silu = (a.flags & SAMBA_SCAN_CONV_SILU) != 0;
   p.softplus = (a.flags & SAMBA_SCAN_DELTA_SOFTPLUS) != 0;
-  const int threads = ((CU + CPW - 1) / CPW + kScanPro + 1) * 32;
+  const int threads = (scan_warps(CU, CPW) + kScanPro + kScanEpi + 1) * 32;
   dim3 grid((unsigned)((D + CU - 1) / CU), (unsigned)Bsz);
   kern<<<grid, threads, Ly::SMEM, stream>>>(mx, mz, mw, mb, mc, p);
   return check_launch("samba_selective_scan_fwd");
