@@ -18,10 +18,10 @@
 //     the band of both Q tiles; tiles outside the band are never loaded.
 //     Only tiles crossing the diagonal, the window's lower edge or key 0 are
 //     masked element by element.
-//   * Warp 0 issues TMA (Q once per unit, K and V per tile into a STG-deep
-//     ring).  Warp 1 owns tensor memory and one thread of it issues every
+//   * Warp 8 issues TMA (Q once per unit, K and V per tile into a STG-deep
+//     ring).  Warp 9 owns tensor memory and one thread of it issues every
 //     tcgen05.mma: S = Q·Kᵀ (bf16, fp32 accumulate into TMEM) and
-//     O += P·V with P read straight from TMEM.  Warps 4-7 and 8-11 are the
+//     O += P·V with P read straight from TMEM.  Warps 0-3 and 4-7 are the
 //     softmax warpgroups of Q tiles A and B: each thread owns one row, reads
 //     its S row from TMEM, keeps the running max and sum in fp32, writes P
 //     back to TMEM as bf16, and rescales O in TMEM only when the running max
@@ -55,10 +55,14 @@ struct SwaCfg {
   static constexpr int SMEM = BAR_OFF + 256 + 1024;        // + alignment slack
   static constexpr uint32_t SWZ = HD == 64 ? 2u : (HD == 32 ? 4u : 6u);  // descriptor swizzle code
   static constexpr uint32_t ATOM = 8 * ROW_BYTES;          // 8-row swizzle atom
-  static constexpr int THREADS = 384;
+  static constexpr int THREADS = 320;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_P = 256, COL_O = 384;
 };
+
+// Warp roles: 0-3 softmax of Q tile A, 4-7 softmax of Q tile B (warp % 4 is
+// the TMEM lane quarter a warp may access), 8 TMA producer, 9 MMA issuer.
+constexpr int kWarpTma = 8, kWarpMma = 9;
 
 // Barrier indices inside the barrier block.
 enum : int {
@@ -69,6 +73,35 @@ __device__ __forceinline__ float ex2f(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Every SWA_POLY-th pair of probabilities is evaluated on the FMA pipe
+// (0: never); the rest use the MUFU ex2.  Build-time, fixed by measurement.
+#ifndef SWA_POLY
+#define SWA_POLY 4
+#endif
+
+// 2^x for a pair of arguments on the FMA pipe, accurate to ~1e-4 relative
+// (ample for probabilities that are rounded to bf16): x = j + f with
+// j = rint(x) by magic-number rounding, 2^f by a degree-3 polynomial fitted
+// on [-1/2, 1/2] for relative error with p(0) = 1 (fit made for this
+// library), and j added to the exponent bits.  x is clamped below at -125,
+// so masked scores (-inf) give 2^-125 instead of 0, which no sum can notice.
+__device__ __forceinline__ f2 ex2_poly3x2(f2 x) {
+  float2 xv = up2(x);
+  xv.x = fmaxf(xv.x, -125.f);
+  xv.y = fmaxf(xv.y, -125.f);
+  const f2 xc = pk2(xv.x, xv.y);
+  const f2 magic = pk2(12582912.f, 12582912.f);  // 1.5 * 2^23
+  const f2 t = add2(xc, magic);
+  const f2 f = sub2(xc, sub2(t, magic));
+  f2 p = pk2(0x1.c2a212p-5f, 0x1.c2a212p-5f);
+  p = fma2(p, f, pk2(0x1.f00c4ep-3f, 0x1.f00c4ep-3f));
+  p = fma2(p, f, pk2(0x1.62f5fap-1f, 0x1.62f5fap-1f));
+  p = fma2(p, f, pk2(1.f, 1.f));
+  const float2 tv = up2(t), pv = up2(p);
+  return pk2(__int_as_float(__float_as_int(pv.x) + (__float_as_int(tv.x) << 23)),
+             __int_as_float(__float_as_int(pv.y) + (__float_as_int(tv.y) << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -94,7 +127,7 @@ __device__ __forceinline__ int unit_tiles(int64_t top, int64_t W, int tok2) {
 }
 
 template <int HD, int GROUP, int STG>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(320, 1)
     swa_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v, const SwaParams p) {
   using Cfg = SwaCfg<HD, GROUP, STG>;
@@ -131,7 +164,7 @@ __global__ void __launch_bounds__(384, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
@@ -140,7 +173,7 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == kWarpTma) {
     // ================================================================ TMA
     if (lane == 0) {
       tma_prefetch_desc(&map_q);
@@ -177,7 +210,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpMma) {
     // ================================================================ MMA
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
@@ -261,9 +294,9 @@ __global__ void __launch_bounds__(384, 1)
       volatile int never = 0;
       mbar_wait(&bars[BMMA_DONE], 0, &never);
     }
-  } else if (warp >= 4) {
+  } else {
     // ============================================================ softmax
-    const int x = (warp >= 8) ? 1 : 0;        // Q tile A or B
+    const int x = (warp >= 4) ? 1 : 0;        // Q tile A or B
     const int wq = warp & 3;                  // TMEM lane quarter
     const int r = wq * 32 + lane;             // row of the tile
     const int tok = r / GROUP, hh = r % GROUP;
@@ -295,28 +328,32 @@ __global__ void __launch_bounds__(384, 1)
         const bool okw = mbar_wait(bar_s, tcount & 1, abort_flag);
         if (!__all_sync(0xffffffffu, okw)) { ok = false; break; }
         tc_fence_after();
-        float s[128];
-        {
-          uint32_t rr[32];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            tmem_ld32(tS + 32 * q, rr);
-            tc_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) s[32 * q + c] = __uint_as_float(rr[c]);
-          }
-        }
+        // The whole 128-column row in four loads, one wait.
+        uint32_t sr[128];
+        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        tc_wait_ld();
+        float* s = reinterpret_cast<float*>(sr);
         if (need_mask) {
+          // visible: 0 <= irow - (k0 + c) < W and k0 + c >= 0, i.e. c in [lo, hi]
+          const int64_t lo64 = k0 < 0 ? -k0 : 0;
+          const int64_t lw = irow - p.W + 1 - k0;
+          const int lo = (int)(lo64 > lw ? lo64 : lw);
+          const int hi = (int)(irow - k0);
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const int64_t jk = k0 + c;
-            const int64_t dd = irow - jk;
-            if (!(dd >= 0 && dd < p.W && jk >= 0)) s[c] = -INFINITY;
-          }
+          for (int c = 0; c < 128; ++c)
+            if (c < lo || c > hi) s[c] = -INFINITY;
         }
-        float mx = -INFINITY;
+        // Row max over 8 independent partial maxima (short dependency chains).
+        float m8[8];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        for (int q = 0; q < 8; ++q) m8[q] = s[q];
+#pragma unroll
+        for (int c = 8; c < 128; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         const float m_tile = mx * sl;  // scale > 0
         float factor = 1.f;
         bool rescale = false;
@@ -326,15 +363,27 @@ __global__ void __launch_bounds__(384, 1)
           rescale = true;
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        // p = 2^(s·scale·log2e - m) in packed pairs; every SWA_POLY-th pair on
+        // the FMA pipe, the rest on MUFU; four partial sums.
         uint32_t pk[64];
-        float rs = 0.f;
+        const f2 sl2 = pk2(sl, sl), nm2 = pk2(-m_use, -m_use);
+        f2 acc4[4] = {pk2(0.f, 0.f), pk2(0.f, 0.f), pk2(0.f, 0.f), pk2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float p0 = ex2f(fmaf(s[2 * c], sl, -m_use));
-          const float p1 = ex2f(fmaf(s[2 * c + 1], sl, -m_use));
-          rs += p0 + p1;
-          pk[c] = pack_bf16(p0, p1);
+          const f2 xx = fma2(pk2(s[2 * c], s[2 * c + 1]), sl2, nm2);
+          f2 pv;
+          if (SWA_POLY > 0 && (c % (SWA_POLY > 0 ? SWA_POLY : 1)) == SWA_POLY - 1) {
+            pv = ex2_poly3x2(xx);
+          } else {
+            const float2 xv = up2(xx);
+            pv = pk2(ex2f(xv.x), ex2f(xv.y));
+          }
+          acc4[c & 3] = add2(acc4[c & 3], pv);
+          const float2 pp = up2(pv);
+          pk[c] = pack_bf16(pp.x, pp.y);
         }
+        const float2 r01 = up2(add2(add2(acc4[0], acc4[1]), add2(acc4[2], acc4[3])));
+        const float rs = r01.x + r01.y;
         l_run = l_run * factor + rs;
         // P_X and O_X are still read by the previous PV: wait for it.
         if (jt > 0) {
@@ -402,7 +451,7 @@ __global__ void __launch_bounds__(384, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::TMEM_COLS);
   }
