@@ -65,6 +65,7 @@ def load() -> ctypes.CDLL:
     lib.samba_version.restype = ctypes.c_int
     lib.samba_last_error.restype = ctypes.c_char_p
     lib.samba_get_status.argtypes = [_vp]
+    lib.samba_selftest_wait_timeout.argtypes = [_vp]
     lib.samba_conv1d_fwd.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _vp, ctypes.c_int, _vp,
                                      _i64, _i64, _i64, ctypes.c_int, ctypes.c_int, _vp]
     lib.samba_selective_scan_fwd.argtypes = [ctypes.POINTER(ScanArgs), _vp]
@@ -80,7 +81,8 @@ def load() -> ctypes.CDLL:
     lib.samba_swa_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, ctypes.c_int, ctypes.c_int,
                                    ctypes.c_int, _i64, ctypes.c_float, _vp, ctypes.c_size_t, _vp]
     for name in ("samba_conv1d_fwd", "samba_selective_scan_fwd", "samba_swa_fwd", "samba_mixer_prefill",
-                 "samba_scan_step", "samba_swa_ring_fill", "samba_swa_step", "samba_get_status"):
+                 "samba_scan_step", "samba_swa_ring_fill", "samba_swa_step", "samba_get_status",
+                 "samba_selftest_wait_timeout"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib

@@ -35,6 +35,7 @@ int sm_count();
 int take_status_scan(cudaStream_t s);
 int take_status_swa(cudaStream_t s);
 int take_status_misc(cudaStream_t s);
+int launch_selftest_wait(cudaStream_t s);
 
 // Launchers (validated arguments only).
 int launch_conv1d(const void* x, int x_dtype, const float* w, const float* bias, const float* cs_in, void* u,

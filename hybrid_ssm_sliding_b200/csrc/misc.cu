@@ -383,3 +383,25 @@ int launch_swa_step(const void* q_t, const void* k_t, const void* v_t, void* k_r
 }
 
 }  // namespace samba
+
+// ------------------------------------------------------- bounded-wait self-test
+namespace samba {
+
+// One thread waits on a barrier that expects one arrival which never comes.
+__global__ void selftest_wait_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+    (void)mbar_wait(&bar, 0, &abort_flag);  // gives up after the limit, records the timeout
+  }
+}
+
+int launch_selftest_wait(cudaStream_t s) {
+  selftest_wait_kernel<<<1, 32, 0, s>>>();
+  return check_launch("samba_selftest_wait_timeout");
+}
+
+}  // namespace samba

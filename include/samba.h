@@ -87,6 +87,15 @@ const char* samba_last_error(void);
  * the last call.  Returns SAMBA_ERR_CUDA if the synchronisation itself fails. */
 int samba_get_status(samba_stream_t stream);
 
+/* Self-test of the failure path: launches one small kernel that waits on an
+ * mbarrier nothing ever completes.  The bounded wait gives up after its limit
+ * (200 ms), the kernel records SAMBA_ERR_TIMEOUT in the status word and
+ * returns, and the CUDA context stays usable; samba_get_status(stream) then
+ * returns SAMBA_ERR_TIMEOUT (and clears it).  Returns SAMBA_OK if the launch
+ * was issued.  Not part of the mixers; it exists so the timeout handling can
+ * be tested on a GPU without faulting or hanging it. */
+int samba_selftest_wait_timeout(samba_stream_t stream);
+
 /* ------------------------------------------------------------------ conv1d
  * Causal depthwise conv1d over time (the conv that Samba's Mamba layer puts in
  * front of its selective scan):
