@@ -80,9 +80,11 @@ def load() -> ctypes.CDLL:
     lib.samba_swa_step_workspace_size.restype = ctypes.c_size_t
     lib.samba_swa_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, ctypes.c_int, ctypes.c_int,
                                    ctypes.c_int, _i64, ctypes.c_float, _vp, ctypes.c_size_t, _vp]
+    lib.samba_swa_step_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, _i64, ctypes.c_float, _vp]
     for name in ("samba_conv1d_fwd", "samba_selective_scan_fwd", "samba_swa_fwd", "samba_mixer_prefill",
                  "samba_scan_step", "samba_swa_ring_fill", "samba_swa_step", "samba_get_status",
-                 "samba_selftest_wait_timeout"):
+                 "samba_selftest_wait_timeout", "samba_swa_step_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib

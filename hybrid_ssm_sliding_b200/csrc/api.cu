@@ -264,4 +264,22 @@ int samba_swa_step(const void* q_t, const void* k_t, const void* v_t, void* k_ri
                          scale, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int samba_swa_step_noalloc(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring,
+                           int64_t* pos, void* o_t, int64_t batch, int heads_q, int heads_kv, int head_dim,
+                           int64_t window, float scale, samba_stream_t stream) {
+  const char* who = "samba_swa_step_noalloc";
+  if (!q_t || !k_t || !v_t || !k_ring || !v_ring || !pos || !o_t)
+    return fail(SAMBA_ERR_INVALID_ARG, "%s: null pointer", who);
+  int rc = check_ring(batch, heads_kv, head_dim, window, who);
+  if (rc != SAMBA_OK) return rc;
+  if (heads_q < 1 || heads_q % heads_kv != 0) return fail(SAMBA_ERR_INVALID_ARG, "%s: heads_q %% heads_kv", who);
+  if (heads_q / heads_kv > 16) return fail(SAMBA_ERR_UNSUPPORTED, "%s: heads_q / heads_kv must be <= 16", who);
+  const void* ptrs[] = {q_t, k_t, v_t, k_ring, v_ring, o_t};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return fail(SAMBA_ERR_INVALID_ARG, "%s: misaligned pointer", who);
+  if (!(scale > 0.f)) scale = 1.0f / std::sqrt(static_cast<float>(head_dim));
+  return launch_swa_step_noalloc(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, batch, heads_q, heads_kv, head_dim, window,
+                                 scale, reinterpret_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

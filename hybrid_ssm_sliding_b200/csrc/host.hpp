@@ -50,6 +50,9 @@ int launch_scan_step(float* h, float* conv_state, const void* x_t, int x_dtype, 
 int launch_ring_fill(const void* k, const void* v, int64_t L, void* k_ring, void* v_ring, int64_t* pos, int64_t B,
                      int Hkv, int d, int64_t W, cudaStream_t stream);
 size_t swa_step_workspace(int64_t B, int Hq, int d, int64_t W);
+int launch_swa_step_noalloc(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring,
+                            int64_t* pos, void* o_t, int64_t B, int Hq, int Hkv, int d, int64_t W, float scale,
+                            cudaStream_t stream);
 int launch_swa_step(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring, int64_t* pos,
                     void* o_t, int64_t B, int Hq, int Hkv, int d, int64_t W, float scale, void* ws,
                     cudaStream_t stream);

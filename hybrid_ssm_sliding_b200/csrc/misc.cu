@@ -405,3 +405,53 @@ int launch_selftest_wait(cudaStream_t s) {
 }
 
 }  // namespace samba
+
+// ------------------------------------------- SWA step without allocations
+// Scratch for samba_swa_step_noalloc: the split partials of swa_step live in
+// this file-scope device array instead of caller-provided workspace.  Every
+// GPU that loads the library holds it (4 MiB) until the process exits.
+#include <mutex>
+
+namespace samba {
+
+constexpr size_t kSwaStepScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) unsigned char g_swa_step_scratch[kSwaStepScratchBytes];
+
+// In host code g_swa_step_scratch names a host-side stand-in, not device
+// memory: the device address must be looked up once per device, with that
+// device current, and passed to the kernels.
+static std::mutex g_scratch_mu;
+static void* g_scratch_addr[128];
+
+static int scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128)
+    return fail(SAMBA_ERR_CUDA, "samba_swa_step_noalloc: no usable current device");
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_swa_step_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(SAMBA_ERR_CUDA, "samba_swa_step_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return SAMBA_OK;
+}
+
+int launch_swa_step_noalloc(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring,
+                            int64_t* pos, void* o_t, int64_t B, int Hq, int Hkv, int d, int64_t W, float scale,
+                            cudaStream_t s) {
+  const size_t need = swa_step_workspace(B, Hq, d, W);
+  if (need > kSwaStepScratchBytes)
+    return fail(SAMBA_ERR_WORKSPACE,
+                "samba_swa_step_noalloc: these sizes need %zu bytes of scratch but the built-in array holds %zu; "
+                "call samba_swa_step with a workspace instead",
+                need, kSwaStepScratchBytes);
+  void* ws = nullptr;
+  const int rc = scratch_address(&ws);
+  if (rc != SAMBA_OK) return rc;
+  return launch_swa_step(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, B, Hq, Hkv, d, W, scale, ws, s);
+}
+
+}  // namespace samba

@@ -228,6 +228,39 @@ int samba_swa_step(const void* q_t, const void* k_t, const void* v_t, void* k_ri
                    int64_t window, float scale, void* workspace, size_t workspace_bytes,
                    samba_stream_t stream);
 
+/* samba_swa_step_noalloc: the same decode step as samba_swa_step, for
+ * callers that cannot allocate device memory.  Examples are a host framework
+ * that owns every device allocation and hands plug-ins only tensors, or code
+ * running where a cudaMalloc would be refused or would synchronise the device.
+ * Such a caller has no way to pass samba_swa_step a workspace.
+ *
+ * The split partials live in a 4 MiB array inside the library (a file-scope
+ * __device__ array), which every GPU that loads the library holds until the
+ * process exits.  Calls whose partials do not fit, that is
+ * samba_swa_step_workspace_size(batch, heads_q, head_dim, window) > 4 MiB,
+ * are rejected with SAMBA_ERR_WORKSPACE before anything is launched; the
+ * 16 x 32-head, d = 64, W = 2048 decode needs 1.08 MB.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current, and keeps it; make that
+ * first call before any stream capture.  The function calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *
+ * Every call shares the one array and finds the previous call's partials in
+ * it.  That is harmless, because each step writes every partial it reads and
+ * nothing has to start at zero.  But two calls that may run at the same time
+ * on the GPU (different streams, or different threads without ordering)
+ * race on the array and give wrong results; order them, or use
+ * samba_swa_step with separate workspaces.
+ *
+ * Arguments, layouts and errors are those of samba_swa_step without the
+ * workspace.  The paper has no counterpart to this entry point; it exists
+ * only for callers that cannot allocate.
+ */
+int samba_swa_step_noalloc(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring,
+                           int64_t* pos, void* o_t, int64_t batch, int heads_q, int heads_kv, int head_dim,
+                           int64_t window, float scale, samba_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
