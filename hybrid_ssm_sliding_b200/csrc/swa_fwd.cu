@@ -18,15 +18,22 @@
 //     the band of both Q tiles; tiles outside the band are never loaded.
 //     Only tiles crossing the diagonal, the window's lower edge or key 0 are
 //     masked element by element.
-//   * Warp 8 issues TMA (Q once per unit, K and V per tile into a STG-deep
-//     ring).  Warp 9 owns tensor memory and one thread of it issues every
-//     tcgen05.mma: S = Q·Kᵀ (bf16, fp32 accumulate into TMEM) and
-//     O += P·V with P read straight from TMEM.  Warps 0-3 and 4-7 are the
-//     softmax warpgroups of Q tiles A and B: each thread owns one row, reads
-//     its S row from TMEM, keeps the running max and sum in fp32, writes P
-//     back to TMEM as bf16, and rescales O in TMEM only when the running max
-//     grows by more than 2^8 (the result does not depend on the reference
-//     max; the threshold only bounds P <= 256).
+//   * Warp 8 issues TMA: Q once per unit into one of two buffers (so the
+//     next unit's Q lands while this one is finishing), K and V per key tile
+//     into a STG-deep ring.  Warp 9 owns tensor memory and issues every
+//     tcgen05.mma, the whole warp in lock-step with one elected lane issuing:
+//     S = Q·Kᵀ (bf16, fp32 accumulate into TMEM) and O += P·V with P read
+//     straight from TMEM.  Over the flat sequence of key tiles (crossing
+//     unit boundaries) it issues S of tile t+1 into the columns of S(t) as
+//     soon as the softmax has read them, so Q·Kᵀ runs under the exps.
+//   * Warps 0-3 and 4-7 are the softmax warpgroups of Q tiles A and B:
+//     each thread owns one row, reads its S row from TMEM, keeps the running
+//     max and sum in fp32, writes P back to TMEM as bf16 (16 packed pairs at
+//     a time), and rescales O in TMEM only when the running max grows by
+//     more than 2^8 (the result does not depend on the reference max; the
+//     threshold only bounds P <= 256).  The exp2 of the probabilities
+//     (special-function unit, with every SWA_POLY-th pair on the FMA pipe)
+//     bounds this kernel.
 //   * TMEM columns: S_A 0-127, S_B 128-255, P_A 256-319, P_B 320-383,
 //     O_A 384-447, O_B 448-511 (fp32, one row per lane).
 #include "common.cuh"
@@ -48,8 +55,8 @@ struct SwaCfg {
   static constexpr int TOK = 128 / GROUP;
   static constexpr int ROW_BYTES = HD * 2;                 // one K-major row (= swizzle span)
   static constexpr int TILE_BYTES = 128 * ROW_BYTES;       // 128 rows
-  static constexpr int Q_OFF = 0;                          // Q_A, Q_B
-  static constexpr int K_OFF = 2 * TILE_BYTES;
+  static constexpr int Q_OFF = 0;                          // two buffers of (Q_A, Q_B)
+  static constexpr int K_OFF = 4 * TILE_BYTES;
   static constexpr int V_OFF = K_OFF + STG * TILE_BYTES;
   static constexpr int BAR_OFF = V_OFF + STG * TILE_BYTES;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;        // + alignment slack
@@ -61,12 +68,18 @@ struct SwaCfg {
 };
 
 // Warp roles: 0-3 softmax of Q tile A, 4-7 softmax of Q tile B (warp % 4 is
-// the TMEM lane quarter a warp may access), 8 TMA producer, 9 MMA issuer.
-constexpr int kWarpTma = 8, kWarpMma = 9;
+// the TMEM lane quarter a warp may access; thread i of warp w owns row
+// 32 (w % 4) + i of its tile), 8 TMA producer, 9 MMA issuer.
+constexpr int kSoftmaxWarps = 8, kWarpTma = 8, kWarpMma = 9;
 
-// Barrier indices inside the barrier block.
+// Barrier indices inside the barrier block.  Per Q tile X in {A, B}:
+// BS_X  S_X of the next key tile is in TMEM          (tcgen05.commit)
+// BSF_X the softmax of X has read S_X into registers (one arrival per warp)
+// BP_X  P_X is in TMEM                               (one arrival per warp)
+// BO_X  O_X += P_X V has completed                   (tcgen05.commit)
 enum : int {
-  BQ_FULL = 0, BQ_EMPTY, BS_A, BS_B, BP_A, BP_B, BO_A, BO_B, BOE_A, BOE_B, BMMA_DONE, B_STAGE0
+  BQ_FULL0 = 0, BQ_FULL1, BQ_EMPTY0, BQ_EMPTY1, BS_A, BS_B, BSF_A, BSF_B, BP_A, BP_B, BO_A, BO_B,
+  BMMA_DONE, B_STAGE0
 };
 
 __device__ __forceinline__ float ex2f(float x) {
@@ -104,6 +117,13 @@ __device__ __forceinline__ f2 ex2_poly3x2(f2 x) {
              __int_as_float(__float_as_int(pv.y) + (__float_as_int(tv.y) << 23)));
 }
 
+// max(a, b, c) in one instruction (three-input form of sm_100).
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -126,39 +146,74 @@ __device__ __forceinline__ int unit_tiles(int64_t top, int64_t W, int tok2) {
   return static_cast<int>(n_band < n_pos ? n_band : n_pos);
 }
 
+
+// Position in the flat sequence of key tiles a CTA walks through: work unit
+// u (the nu-th unit of this CTA), key tile jt of the unit's nt tiles.
+struct TileCursor {
+  int u;
+  uint32_t nu;
+  int jt, nt;
+};
+
+__device__ __forceinline__ int tiles_of_unit(int u, const SwaParams& p, int tok2) {
+  int b, g;
+  int64_t i0;
+  unit_coords(u, p, tok2, b, g, i0);
+  return unit_tiles(i0 + tok2, p.W, tok2);
+}
+
+__device__ __forceinline__ bool cursor_begin(TileCursor& c, const SwaParams& p, int tok2) {
+  c.u = blockIdx.x;
+  c.nu = 0;
+  c.jt = 0;
+  if (c.u >= p.total_units) return false;
+  c.nt = tiles_of_unit(c.u, p, tok2);
+  return true;
+}
+
+__device__ __forceinline__ bool cursor_next(TileCursor& c, const SwaParams& p, int tok2) {
+  if (++c.jt < c.nt) return true;
+  c.u += gridDim.x;
+  ++c.nu;
+  c.jt = 0;
+  if (c.u >= p.total_units) return false;
+  c.nt = tiles_of_unit(c.u, p, tok2);
+  return true;
+}
+
+
 template <int HD, int GROUP, int STG>
 __global__ void __launch_bounds__(320, 1)
     swa_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v, const SwaParams p) {
   using Cfg = SwaCfg<HD, GROUP, STG>;
+  static_assert((B_STAGE0 + 2 * STG) * 8 + 8 <= 256, "barrier block overflows its 256 bytes");
+  static_assert(HD == 16 || HD == 32 || HD == 64, "head dim");
   constexpr int TOK = Cfg::TOK;
   constexpr int TOK2 = 2 * TOK;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::BAR_OFF);
-  uint64_t* kfull = bars + B_STAGE0;
-  uint64_t* vfull = kfull + STG;
-  uint64_t* kvempty = vfull + STG;
+  uint64_t* kvfull = bars + B_STAGE0;  // K and V tile of a stage landed
+  uint64_t* kvempty = kvfull + STG;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(kvempty + STG);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars[BQ_FULL], 1);
-    mbar_init(&bars[BQ_EMPTY], 1);
+    for (int i = BQ_FULL0; i <= BQ_EMPTY1; ++i) mbar_init(&bars[i], 1);
     mbar_init(&bars[BS_A], 1);
     mbar_init(&bars[BS_B], 1);
-    mbar_init(&bars[BP_A], 128);
-    mbar_init(&bars[BP_B], 128);
+    mbar_init(&bars[BSF_A], kSoftmaxWarps / 2);
+    mbar_init(&bars[BSF_B], kSoftmaxWarps / 2);
+    mbar_init(&bars[BP_A], kSoftmaxWarps / 2);
+    mbar_init(&bars[BP_B], kSoftmaxWarps / 2);
     mbar_init(&bars[BO_A], 1);
     mbar_init(&bars[BO_B], 1);
-    mbar_init(&bars[BOE_A], 128);
-    mbar_init(&bars[BOE_B], 128);
     mbar_init(&bars[BMMA_DONE], 1);
     for (int s = 0; s < STG; ++s) {
-      mbar_init(&kfull[s], 1);
-      mbar_init(&vfull[s], 1);
+      mbar_init(&kvfull[s], 1);
       mbar_init(&kvempty[s], 1);
     }
     *abort_flag = 0;
@@ -187,116 +242,127 @@ __global__ void __launch_bounds__(320, 1)
         unit_coords(u, p, TOK2, b, g, i0);
         const int64_t top = i0 + TOK2;
         const int nt = unit_tiles(top, p.W, TOK2);
-        if (nu > 0 && !mbar_wait(&bars[BQ_EMPTY], (nu - 1) & 1, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(&bars[BQ_FULL], 2 * Cfg::TILE_BYTES);
-        tma_load_4d(smem + Cfg::Q_OFF, &map_q, &bars[BQ_FULL], 0, g * GROUP, (int)i0, b);
-        tma_load_4d(smem + Cfg::Q_OFF + Cfg::TILE_BYTES, &map_q, &bars[BQ_FULL], 0, g * GROUP, (int)(i0 + TOK), b);
+        // Q of unit nu goes to buffer nu % 2 once unit nu - 2 has issued its last Q·Kᵀ.
+        const uint32_t qb = nu & 1;
+        if (nu >= 2 && !mbar_wait(&bars[BQ_EMPTY0 + qb], ((nu >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+        unsigned char* qdst = smem + Cfg::Q_OFF + 2 * qb * Cfg::TILE_BYTES;
+        mbar_arrive_expect_tx(&bars[BQ_FULL0 + qb], 2 * Cfg::TILE_BYTES);
+        tma_load_4d(qdst, &map_q, &bars[BQ_FULL0 + qb], 0, g * GROUP, (int)i0, b);
+        tma_load_4d(qdst + Cfg::TILE_BYTES, &map_q, &bars[BQ_FULL0 + qb], 0, g * GROUP, (int)(i0 + TOK), b);
         for (int m = 0; m < nt; ++m, ++it) {
           const int s = it % STG;
           if (it >= STG && !mbar_wait(&kvempty[s], ((it / STG) - 1) & 1, abort_flag)) { ok = false; break; }
           const int k0 = (int)(top - 128 * (m + 1));
-          mbar_arrive_expect_tx(&kfull[s], Cfg::TILE_BYTES);
-          tma_load_4d(smem + Cfg::K_OFF + s * Cfg::TILE_BYTES, &map_k, &kfull[s], 0, g, k0, b);
-          mbar_arrive_expect_tx(&vfull[s], Cfg::TILE_BYTES);
-          tma_load_4d(smem + Cfg::V_OFF + s * Cfg::TILE_BYTES, &map_v, &vfull[s], 0, g, k0, b);
+          mbar_arrive_expect_tx(&kvfull[s], 2 * Cfg::TILE_BYTES);
+          tma_load_4d(smem + Cfg::K_OFF + s * Cfg::TILE_BYTES, &map_k, &kvfull[s], 0, g, k0, b);
+          tma_load_4d(smem + Cfg::V_OFF + s * Cfg::TILE_BYTES, &map_v, &kvfull[s], 0, g, k0, b);
         }
       }
       // Drain copies that may still be in flight (after an abort only).
       if (!ok) {
         volatile int never = 0;
-        for (uint32_t i = (it > STG ? it - STG : 0); i < it; ++i) {
-          mbar_wait(&kfull[i % STG], (i / STG) & 1, &never);
-          mbar_wait(&vfull[i % STG], (i / STG) & 1, &never);
-        }
+        for (uint32_t i = (it > STG ? it - STG : 0); i < it; ++i) mbar_wait(&kvfull[i % STG], (i / STG) & 1, &never);
+        for (uint32_t n = (nu > 2 ? nu - 2 : 0); n < nu; ++n) mbar_wait(&bars[BQ_FULL0 + (n & 1)], (n >> 1) & 1, &never);
       }
     }
   } else if (warp == kWarpMma) {
     // ================================================================ MMA
-    if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t IDESC_O = idesc_bf16_f32(128, HD, 0, 1);
-      const uint32_t q_base = smem_u32(smem + Cfg::Q_OFF);
-      const uint32_t k_base = smem_u32(smem + Cfg::K_OFF);
-      const uint32_t v_base = smem_u32(smem + Cfg::V_OFF);
-      const uint32_t tS[2] = {tmem + Cfg::COL_S, tmem + Cfg::COL_S + 128};
-      const uint32_t tP[2] = {tmem + Cfg::COL_P, tmem + Cfg::COL_P + 64};
-      const uint32_t tO[2] = {tmem + Cfg::COL_O, tmem + Cfg::COL_O + 64};
-      uint32_t it = 0, tcount = 0, nu = 0;
-      bool ok = true;
-
-      auto issue_s = [&](int x, uint32_t stage) {
-        const uint32_t qa = q_base + x * Cfg::TILE_BYTES;
-        const uint32_t ka = k_base + stage * Cfg::TILE_BYTES;
+    // The whole warp runs this loop in lock-step; each tcgen05 instruction
+    // is issued by one elected lane.  Over the flat sequence of key tiles t
+    // (crossing unit boundaries) the issue order is S_A(t+1) and S_B(t+1) as
+    // soon as the softmax has read S(t), then O_A += P_A(t) V(t) and
+    // O_B += P_B(t) V(t) as P arrives; the stage of tile t is then free.
+    constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
+    constexpr uint32_t IDESC_O = idesc_bf16_f32(128, HD, 0, 1);
+    const uint32_t q_base = smem_u32(smem + Cfg::Q_OFF);
+    const uint32_t k_base = smem_u32(smem + Cfg::K_OFF);
+    const uint32_t v_base = smem_u32(smem + Cfg::V_OFF);
+    bool ok = true;
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
+    // Descriptors are built once: the upper halves are constant, and the
+    // start-address field of the lower half (address / 16, below 2^14 for
+    // any shared-memory address) advances by 2 per 16 K-elements of Q and K
+    // and by ROW_BYTES per 16 keys of V without carrying out of its field.
+    const uint64_t d_q0 = smem_desc(q_base, 16, Cfg::ATOM, Cfg::SWZ);
+    const uint64_t d_k0 = smem_desc(k_base, 16, Cfg::ATOM, Cfg::SWZ);
+    const uint64_t d_v0 = smem_desc(v_base, 4096, Cfg::ATOM, Cfg::SWZ);
+    const uint32_t hi_qk = static_cast<uint32_t>(d_q0 >> 32), hi_v = static_cast<uint32_t>(d_v0 >> 32);
+    const uint32_t lo_q0 = static_cast<uint32_t>(d_q0), lo_k0 = static_cast<uint32_t>(d_k0);
+    const uint32_t lo_v0 = static_cast<uint32_t>(d_v0);
+    constexpr uint32_t kTileDesc = Cfg::TILE_BYTES >> 4;
+    auto desc64 = [](uint32_t lo, uint32_t hi) { return (static_cast<uint64_t>(hi) << 32) | lo; };
+    auto issue_s = [&](int x, uint32_t qb, uint32_t stage) {
+      const uint32_t lq = lo_q0 + (2 * qb + x) * kTileDesc;
+      const uint32_t lk = lo_k0 + stage * kTileDesc;
 #pragma unroll
-        for (int k = 0; k < HD / 16; ++k) {
-          const uint64_t da = smem_desc(qa + 32 * k, 16, Cfg::ATOM, Cfg::SWZ);
-          const uint64_t db = smem_desc(ka + 32 * k, 16, Cfg::ATOM, Cfg::SWZ);
-          umma_ss(tS[x], da, db, IDESC_S, k > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int x, uint32_t stage, bool first) {
-        const uint32_t va = v_base + stage * Cfg::TILE_BYTES;
+      for (int k = 0; k < HD / 16; ++k)
+        umma_ss_w(tmem + Cfg::COL_S + 128 * x, desc64(lq + 2 * k, hi_qk), desc64(lk + 2 * k, hi_qk), IDESC_S,
+                  k > 0 ? 1u : 0u);
+    };
+    auto issue_pv = [&](int x, uint32_t stage, bool first) {
+      const uint32_t lv = lo_v0 + stage * kTileDesc;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          // 16 keys per step = two 8-row atoms of V
-          const uint64_t db = smem_desc(va + k * 2 * Cfg::ATOM, 4096, Cfg::ATOM, Cfg::SWZ);
-          umma_ts(tO[x], tP[x] + 8 * k, db, IDESC_O, (first && k == 0) ? 0u : 1u);
-        }
-      };
+      for (int k = 0; k < 8; ++k)  // 16 keys per step = two 8-row atoms of V
+        umma_ts_w(tmem + Cfg::COL_O + 64 * x, tmem + Cfg::COL_P + 64 * x + 8 * k,
+                  desc64(lv + k * (Cfg::ROW_BYTES), hi_v), IDESC_O, (first && k == 0) ? 0u : 1u);
+    };
 
-      for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x, ++nu) {
-        int b, g;
-        int64_t i0;
-        unit_coords(u, p, TOK2, b, g, i0);
-        const int nt = unit_tiles(i0 + TOK2, p.W, TOK2);
-        if (!mbar_wait(&bars[BQ_FULL], nu & 1, abort_flag)) { ok = false; break; }
-        uint32_t s0 = it % STG;
-        if (!mbar_wait(&kfull[s0], (it / STG) & 1, abort_flag)) { ok = false; break; }
+    TileCursor cs;  // tile t
+    bool more = cursor_begin(cs, p, TOK2);
+    bool first_cur = true;
+    if (more) {
+      ok = wait(&bars[BQ_FULL0], 0) && wait(&kvfull[0], 0);
+      if (ok) {
         tc_fence_after();
-        issue_s(0, s0);
-        tc_commit(&bars[BS_A]);
-        issue_s(1, s0);
-        tc_commit(&bars[BS_B]);
-        for (int jt = 0; jt < nt; ++jt, ++it, ++tcount) {
-          const uint32_t s = it % STG;
-          const uint32_t sn = (it + 1) % STG;
-          // ---- tile A: O_A += P_A V, then S_A of the next tile
-          if (!mbar_wait(&vfull[s], (it / STG) & 1, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&bars[BP_A], tcount & 1, abort_flag)) { ok = false; break; }
-          if (jt == 0 && nu > 0 && !mbar_wait(&bars[BOE_A], (nu - 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(0, s, jt == 0);
-          tc_commit(&bars[BO_A]);
-          if (jt + 1 < nt) {
-            if (!mbar_wait(&kfull[sn], ((it + 1) / STG) & 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            issue_s(0, sn);
-            tc_commit(&bars[BS_A]);
-          }
-          // ---- tile B
-          if (!mbar_wait(&bars[BP_B], tcount & 1, abort_flag)) { ok = false; break; }
-          if (jt == 0 && nu > 0 && !mbar_wait(&bars[BOE_B], (nu - 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(1, s, jt == 0);
-          tc_commit(&bars[BO_B]);
-          tc_commit(&kvempty[s]);
-          if (jt + 1 < nt) {
-            issue_s(1, sn);
-            tc_commit(&bars[BS_B]);
-          }
-        }
-        if (!ok) break;
-        tc_commit(&bars[BQ_EMPTY]);  // every MMA reading this unit's Q has been issued
+        issue_s(0, 0, 0);
+        tc_commit_w(&bars[BS_A]);
+        issue_s(1, 0, 0);
+        tc_commit_w(&bars[BS_B]);
+        if (cs.nt == 1) tc_commit_w(&bars[BQ_EMPTY0]);
       }
-      // Wait until every MMA issued by this thread has finished before the
-      // tensor memory can be released.
-      tc_commit(&bars[BMMA_DONE]);
-      volatile int never = 0;
-      mbar_wait(&bars[BMMA_DONE], 0, &never);
     }
-  } else {
+    for (uint32_t t = 0; more && ok; ++t) {
+      TileCursor cn = cs;  // tile t + 1
+      const bool has_next = cursor_next(cn, p, TOK2);
+      const bool first_next = has_next && cn.jt == 0;
+      const uint32_t s = t % STG, sn = (t + 1) % STG;
+      const uint32_t qbn = cn.nu & 1;
+      if (has_next) {
+        if (first_next && !wait(&bars[BQ_FULL0 + qbn], (cn.nu >> 1) & 1)) { ok = false; break; }
+        if (!wait(&kvfull[sn], ((t + 1) / STG) & 1)) { ok = false; break; }
+        if (!wait(&bars[BSF_A], t & 1)) { ok = false; break; }
+        tc_fence_after();
+        issue_s(0, qbn, sn);
+        tc_commit_w(&bars[BS_A]);
+        if (!wait(&bars[BSF_B], t & 1)) { ok = false; break; }
+        tc_fence_after();
+        issue_s(1, qbn, sn);
+        tc_commit_w(&bars[BS_B]);
+        if (cn.jt == cn.nt - 1) tc_commit_w(&bars[BQ_EMPTY0 + qbn]);
+      }
+      if (!wait(&bars[BP_A], t & 1)) { ok = false; break; }
+      tc_fence_after();
+      issue_pv(0, s, first_cur);
+      tc_commit_w(&bars[BO_A]);
+      if (!wait(&bars[BP_B], t & 1)) { ok = false; break; }
+      tc_fence_after();
+      issue_pv(1, s, first_cur);
+      tc_commit_w(&bars[BO_B]);
+      tc_commit_w(&kvempty[s]);
+      first_cur = first_next;
+      cs = cn;
+      more = has_next;
+    }
+    // Wait until every MMA issued by this warp has finished before the
+    // tensor memory can be released.
+    tc_commit_w(&bars[BMMA_DONE]);
+    volatile int never = 0;
+    mbar_wait(&bars[BMMA_DONE], 0, &never);
+  } else if (warp < kSoftmaxWarps) {
     // ============================================================ softmax
-    const int x = (warp >= 4) ? 1 : 0;        // Q tile A or B
+    const int x = warp >> 2;                  // Q tile A or B
     const int wq = warp & 3;                  // TMEM lane quarter
     const int r = wq * 32 + lane;             // row of the tile
     const int tok = r / GROUP, hh = r % GROUP;
@@ -305,12 +371,22 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t tP = tmem + lane_off + Cfg::COL_P + 64 * x;
     const uint32_t tO = tmem + lane_off + Cfg::COL_O + 64 * x;
     uint64_t* bar_s = &bars[BS_A + x];
+    uint64_t* bar_sf = &bars[BSF_A + x];
     uint64_t* bar_p = &bars[BP_A + x];
     uint64_t* bar_o = &bars[BO_A + x];
-    uint64_t* bar_oe = &bars[BOE_A + x];
     const float sl = p.scale_log2;
-    uint32_t tcount = 0;
+    uint32_t t = 0;  // flat key-tile index
     bool ok = true;
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
+    // One arrival per warp: the tcgen05 loads and stores before it are
+    // warp-collective and complete in every lane, so after the warp has
+    // converged one lane signals for all of them.
+    auto warp_arrive = [&](uint64_t* bar) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
 
     for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
       int b, g;
@@ -322,11 +398,10 @@ __global__ void __launch_bounds__(320, 1)
       const int64_t first_tok = i0 + TOK * x, last_tok = first_tok + TOK - 1;
       float m_run = -INFINITY, l_run = 0.f;
 
-      for (int jt = 0; jt < nt; ++jt, ++tcount) {
+      for (int jt = 0; jt < nt; ++jt, ++t) {
         const int64_t k0 = top - 128 * (jt + 1);
         const bool need_mask = (k0 + 127 > first_tok) || (k0 < last_tok - p.W + 1) || (k0 < 0);
-        const bool okw = mbar_wait(bar_s, tcount & 1, abort_flag);
-        if (!__all_sync(0xffffffffu, okw)) { ok = false; break; }
+        if (!wait(bar_s, t & 1)) { ok = false; break; }
         tc_fence_after();
         // The whole 128-column row in four loads, one wait.
         uint32_t sr[128];
@@ -335,7 +410,9 @@ __global__ void __launch_bounds__(320, 1)
         tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
         tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
         tc_wait_ld();
-        float* s = reinterpret_cast<float*>(sr);
+        tc_fence_before();
+        warp_arrive(bar_sf);  // S_X may now be overwritten by the next tile's Q·Kᵀ
+        float* sc = reinterpret_cast<float*>(sr);
         if (need_mask) {
           // visible: 0 <= irow - (k0 + c) < W and k0 + c >= 0, i.e. c in [lo, hi]
           const int64_t lo64 = k0 < 0 ? -k0 : 0;
@@ -344,16 +421,19 @@ __global__ void __launch_bounds__(320, 1)
           const int hi = (int)(irow - k0);
 #pragma unroll
           for (int c = 0; c < 128; ++c)
-            if (c < lo || c > hi) s[c] = -INFINITY;
+            if (c < lo || c > hi) sc[c] = -INFINITY;
         }
-        // Row max over 8 independent partial maxima (short dependency chains).
+        // Row max: eight chains of three-input maxima, chain q over the
+        // columns c = q (mod 8).
         float m8[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) m8[q] = s[q];
+        for (int q = 0; q < 8; ++q) {
+          float m = fmax3f(sc[q], sc[q + 8], sc[q + 16]);
 #pragma unroll
-        for (int c = 8; c < 128; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
-        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          for (int c = 24; c < 120; c += 16) m = fmax3f(m, sc[c + q], sc[c + 8 + q]);
+          m8[q] = fmaxf(m, sc[120 + q]);
+        }
+        const float mx = fmaxf(fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]), m8[6]), m8[7]);
         const float m_tile = mx * sl;  // scale > 0
         float factor = 1.f;
         bool rescale = false;
@@ -363,60 +443,58 @@ __global__ void __launch_bounds__(320, 1)
           rescale = true;
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        // P_X and O_X are still read by the previous O += P·V of this unit:
+        // wait for it before P is overwritten.  At the first tile of a unit
+        // the epilogue of the previous unit has already waited for it.
+        if (jt > 0) {
+          if (!wait(bar_o, (t - 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+        }
         // p = 2^(s·scale·log2e - m) in packed pairs; every SWA_POLY-th pair on
-        // the FMA pipe, the rest on MUFU; four partial sums.
-        uint32_t pk[64];
+        // the FMA pipe, the rest on MUFU; four partial sums; each 16 packed
+        // pairs go to TMEM as soon as they are ready.
         const f2 sl2 = pk2(sl, sl), nm2 = pk2(-m_use, -m_use);
         f2 acc4[4] = {pk2(0.f, 0.f), pk2(0.f, 0.f), pk2(0.f, 0.f), pk2(0.f, 0.f)};
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const f2 xx = fma2(pk2(s[2 * c], s[2 * c + 1]), sl2, nm2);
-          f2 pv;
-          if (SWA_POLY > 0 && (c % (SWA_POLY > 0 ? SWA_POLY : 1)) == SWA_POLY - 1) {
-            pv = ex2_poly3x2(xx);
-          } else {
-            const float2 xv = up2(xx);
-            pv = pk2(ex2f(xv.x), ex2f(xv.y));
+        for (int k = 0; k < 4; ++k) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int c = 16 * k + j;
+            const f2 xx = fma2(pk2(sc[2 * c], sc[2 * c + 1]), sl2, nm2);
+            f2 pv;
+            if (SWA_POLY > 0 && (c % (SWA_POLY > 0 ? SWA_POLY : 1)) == SWA_POLY - 1) {
+              pv = ex2_poly3x2(xx);
+            } else {
+              const float2 xv = up2(xx);
+              pv = pk2(ex2f(xv.x), ex2f(xv.y));
+            }
+            acc4[c & 3] = add2(acc4[c & 3], pv);
+            const float2 pp = up2(pv);
+            pk[j] = pack_bf16(pp.x, pp.y);
           }
-          acc4[c & 3] = add2(acc4[c & 3], pv);
-          const float2 pp = up2(pv);
-          pk[c] = pack_bf16(pp.x, pp.y);
+          tmem_st16(tP + 16 * k, pk);
         }
         const float2 r01 = up2(add2(add2(acc4[0], acc4[1]), add2(acc4[2], acc4[3])));
-        const float rs = r01.x + r01.y;
-        l_run = l_run * factor + rs;
-        // P_X and O_X are still read by the previous PV: wait for it.
-        if (jt > 0) {
-          const bool oko = mbar_wait(bar_o, (tcount - 1) & 1, abort_flag);
-          if (!__all_sync(0xffffffffu, oko)) { ok = false; break; }
-          tc_fence_after();
-          if (rescale) {
-            uint32_t o[16];
+        l_run = l_run * factor + (r01.x + r01.y);
+        if (jt > 0 && rescale) {
+          uint32_t o[16];
 #pragma unroll
-            for (int q = 0; q < HD / 16; ++q) {
-              tmem_ld16(tO + 16 * q, o);
-              tc_wait_ld();
+          for (int q = 0; q < HD / 16; ++q) {
+            tmem_ld16(tO + 16 * q, o);
+            tc_wait_ld();
 #pragma unroll
-              for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * factor);
-              tmem_st16(tO + 16 * q, o);
-            }
+            for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * factor);
+            tmem_st16(tO + 16 * q, o);
           }
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t w[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) w[c] = pk[16 * q + c];
-          tmem_st16(tP + 16 * q, w);
         }
         tc_wait_st();
         tc_fence_before();
-        mbar_arrive(bar_p);
+        warp_arrive(bar_p);  // also tells the MMA warp that O_X has been read, if this starts a unit
       }
       if (!ok) break;
       // ---- epilogue: O / l  -> bf16 rows
-      const bool oko = mbar_wait(bar_o, (tcount - 1) & 1, abort_flag);
-      if (!__all_sync(0xffffffffu, oko)) { ok = false; break; }
+      if (!wait(bar_o, (t - 1) & 1)) { ok = false; break; }
       tc_fence_after();
       uint32_t o[HD];
 #pragma unroll
@@ -427,8 +505,6 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int c = 0; c < 16; ++c) o[16 * q + c] = t16[c];
       }
-      tc_fence_before();
-      mbar_arrive(bar_oe);  // O_X may be overwritten by the next unit
       if (irow < p.L) {
         const float inv = 1.f / l_run;
         const int h = g * GROUP + hh;
@@ -468,9 +544,14 @@ namespace samba {
 
 int take_status_swa(cudaStream_t s) { return take_status_word(s); }
 
+// K/V ring depth (stages of one K and one V tile each); build-time.
+#ifndef SWA_STAGES
+#define SWA_STAGES 4
+#endif
+
 template <int HD, int GROUP>
 static int launch_swa_t(const samba_swa_args& a, cudaStream_t stream) {
-  constexpr int STG = 3;
+  constexpr int STG = SWA_STAGES;
   using Cfg = SwaCfg<HD, GROUP, STG>;
   auto kern = swa_fwd_kernel<HD, GROUP, STG>;
   static bool attr_done = false;
