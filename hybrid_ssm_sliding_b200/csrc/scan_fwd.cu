@@ -21,18 +21,20 @@
 //     host so that the CTAs spread evenly over the SMs) and walks the whole
 //     sequence in tiles of T tokens.
 //   * Warp roles.  One producer warp streams x, z, delta, B, C tiles into a
-//     STAGES-deep shared-memory ring with TMA.  NPRO "prologue" warps compute,
-//     once per (token, channel), the conv, SiLU, softplus and gate, leaving
-//     (Δ, Δu) for the scan and (D·u, silu(z)) for the output; the same warps
-//     later finish y = (Σ partials + D·u)·silu(z) and store it.  The scan
-//     warps hold the state: a channel's N states are spread over GL lanes
-//     (NS states per lane) and each lane writes its partial C·h per token.
+//     STAGES-deep shared-memory ring with TMA.  Prologue warps compute, once
+//     per (token, channel), the conv, SiLU and softplus, leaving (Δ, Δu) for
+//     the scan and (D·u, z) for the output.  The scan warps hold the state: a
+//     channel's N states are spread over GL lanes (NS states per lane) and
+//     each lane writes its partial C·h per token.  Epilogue warps finish
+//     y = (Σ partials + D·u)·silu(z) and store it.
 //   * Prologue, scan and epilogue of consecutive tiles overlap through
-//     double-buffered exchange arrays guarded by mbarriers.
-//   * The scan core uses packed f32x2 arithmetic; a compile-time share of the
-//     exps is evaluated on the FMA pipe with a polynomial (exp2 split into
-//     2^j · 2^f, degree-5 fit of 2^f on [-1/2, 1/2] with p(0) = 1 and
-//     p'(0) = ln 2), so the MUFU and FMA pipes share the load.
+//     SLOTS-deep exchange arrays guarded by mbarriers.
+//   * The scan warps software-pipeline groups of G tokens: the decays
+//     exp(Δ A) of group g+1, which do not depend on the state, are issued
+//     next to the dependent updates of group g.  The core uses packed f32x2
+//     arithmetic; a compile-time share of the exps can be evaluated on the
+//     FMA pipe with a polynomial (exp2 split into 2^j · 2^f, degree-5 fit of
+//     2^f on [-1/2, 1/2] with p(0) = 1 and p'(0) = ln 2).
 //   * Every wait is bounded; a wait that runs out stops the CTA cleanly.
 #include "common.cuh"
 
@@ -78,13 +80,14 @@ constexpr int kScanEpi = 4;     // epilogue warps
 #ifndef SAMBA_SCAN_MAXTHREADS
 #define SAMBA_SCAN_MAXTHREADS 672
 #endif
-// Tokens per load / exp / update group of the scan warps.
+// Tokens per group of the scan warps' software pipeline.
 #ifndef SAMBA_SCAN_GROUP
-#define SAMBA_SCAN_GROUP 8
+#define SAMBA_SCAN_GROUP 4
 #endif
 #ifndef SAMBA_SCAN_SLOTS
 #define SAMBA_SCAN_SLOTS 3
 #endif
+
 constexpr int kScanSlots = SAMBA_SCAN_SLOTS;  // depth of the prologue -> scan -> epilogue hand-off
 constexpr int kScanSmemBudget = 227 * 1024;
 
@@ -100,7 +103,7 @@ struct ScanLayout {
   static constexpr int X_OFF = 0, Z_OFF = al(XB), W_OFF = Z_OFF + al(ZB), B_OFF = W_OFF + al(WB),
                        C_OFF = B_OFF + al(BB), STAGE_BYTES = C_OFF + al(BB);
   static constexpr int XCH_BYTES = SLOTS * T * CB * 8;       // float2 [SLOTS][T][CB] (Δ, Δu)
-  static constexpr int EPI_BYTES = SLOTS * T * CB * 8;       // float2 [SLOTS][T][CB] (D·u, silu(z))
+  static constexpr int EPI_BYTES = SLOTS * T * CB * 8;       // float2 [SLOTS][T][CB] (D·u, z)
   static constexpr int PART_BYTES = SLOTS * T * CB * GL * 4; // float  [SLOTS][T][CB][GL]
   static constexpr int FIXED = XCH_BYTES + EPI_BYTES + PART_BYTES + 512;
   // TMA ring: as many stages (up to 6) as fit next to the hand-off buffers
@@ -185,7 +188,7 @@ __device__ __forceinline__ float softplus_fast(float w) {
 // Warp roles (index ranges): [0, NSW) scan, then kScanPro prologue, then
 // kScanEpi epilogue, then one TMA producer.  Per tile i (slot k = i % SLOTS):
 //   producer : full[s] <- TMA of x, z, delta, B, C          (waits empty[s])
-//   prologue : XCH[k], EPI[k] <- conv/softplus/gate; arrives pro_full[k]
+//   prologue : XCH[k], EPI[k] <- conv/softplus, D·u, z; arrives pro_full[k]
 //              (waits full[s]; scan_done[k] and epi_done[k] of tile i-SLOTS)
 //   scan     : PART[k] <- partial C·h of its states; arrives scan_done[k]
 //              (waits pro_full[k], full[s]; epi_done[k] of tile i-SLOTS)
@@ -305,8 +308,9 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
       for (int q = 0; q < TPE; ++q) {
         const int64_t tok = t0 + eg * TPE + q;
         const float acc = (pv[q].x + pv[q].y) + (pv[q].z + pv[q].w);
+        const float g = p.has_z ? silu_fast(ev[q].y) : 1.f;
         if (cval && tok < L)
-          reinterpret_cast<YT*>(p.y)[((int64_t)b * L + tok) * p.D + c] = from_f32<YT>((acc + ev[q].x) * ev[q].y);
+          reinterpret_cast<YT*>(p.y)[((int64_t)b * L + tok) * p.D + c] = from_f32<YT>((acc + ev[q].x) * g);
       }
     }
     return;
@@ -395,7 +399,9 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
         float dlt = p.softplus ? softplus_fast(wr) : wr;
         if (tok >= L || !cact) dlt = 0.f;  // padding tokens leave the state untouched
         const float du = dlt * u;
-        const float g = p.has_z ? silu_fast(zv[q]) : 1.f;
+        // z itself goes to the epilogue warps, which wait on the scan most
+        // of the time and evaluate the gate silu(z) there
+        const float g = p.has_z ? zv[q] : 1.f;
         if (cact) {
           XCH[(k * T + t) * CB + cl] = make_float2(dlt, du);
           EPI[(k * T + t) * CB + cl] = make_float2(dsk * u, g);
@@ -457,65 +463,92 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
     const float* cs = reinterpret_cast<const float*>(st + Ly::C_OFF);
     const float2* xch = XCH + k * T * CB + cl;
     float* part = PART + (k * T * CB + cl) * GL + j;
-    // Groups of G tokens in three phases: load every operand, issue every exp
-    // (they do not depend on the state, so the MUFU pipe is fed back to
-    // back), then run the dependent state updates and store the partials.
     constexpr int G = SAMBA_SCAN_GROUP;
-#pragma unroll 2
-    for (int tg0 = 0; tg0 < T; tg0 += G) {
-      float2 ev[G];
-      f2 bb[G][NP], cc[G][NP], dA[G][NP];
+    // B and C of token t for this lane's states, as packed pairs.
+    auto load_bc = [&](int t, f2 (&bq)[NP], f2 (&cq)[NP]) {
+      if (NS == 4) {
+        const float4 bv = *reinterpret_cast<const float4*>(bs + t * N + n0);
+        const float4 cv = *reinterpret_cast<const float4*>(cs + t * N + n0);
+        bq[0] = pk2(bv.x, bv.y);
+        bq[NP - 1] = pk2(bv.z, bv.w);
+        cq[0] = pk2(cv.x, cv.y);
+        cq[NP - 1] = pk2(cv.z, cv.w);
+      } else if (NS == 2) {
+        const float2 bv = *reinterpret_cast<const float2*>(bs + t * N + n0);
+        const float2 cv = *reinterpret_cast<const float2*>(cs + t * N + n0);
+        bq[0] = pk2(bv.x, bv.y);
+        cq[0] = pk2(cv.x, cv.y);
+      } else {
+        bq[0] = pk2(bs[t * N + n0], 0.f);
+        cq[0] = pk2(cs[t * N + n0], 0.f);
+      }
+    };
+    // exp(Δ A) for this lane's states (A pre-scaled by log2 e).
+    auto decay = [&](float dlt, int q, f2 (&dq)[NP]) {
+      const f2 dlt2 = pk2(dlt, dlt);
 #pragma unroll
-      for (int q = 0; q < G; ++q) {
-        const int t = tg0 + q;
-        ev[q] = xch[t * CB];
-        if (NS == 4) {
-          const float4 bv = *reinterpret_cast<const float4*>(bs + t * N + n0);
-          const float4 cv = *reinterpret_cast<const float4*>(cs + t * N + n0);
-          bb[q][0] = pk2(bv.x, bv.y);
-          bb[q][NP - 1] = pk2(bv.z, bv.w);
-          cc[q][0] = pk2(cv.x, cv.y);
-          cc[q][NP - 1] = pk2(cv.z, cv.w);
-        } else if (NS == 2) {
-          const float2 bv = *reinterpret_cast<const float2*>(bs + t * N + n0);
-          const float2 cv = *reinterpret_cast<const float2*>(cs + t * N + n0);
-          bb[q][0] = pk2(bv.x, bv.y);
-          cc[q][0] = pk2(cv.x, cv.y);
+      for (int m = 0; m < NP; ++m) {
+        const f2 xx = mul2(dlt2, a2p[m]);
+        if (POLY > 0 && (q % (POLY > 0 ? POLY : 1)) == POLY - 1) {
+          dq[m] = ex2_poly2(xx);
         } else {
-          bb[q][0] = pk2(bs[t * N + n0], 0.f);
-          cc[q][0] = pk2(cs[t * N + n0], 0.f);
+          const float2 xv = up2(xx);
+          dq[m] = pk2(mufu_ex2(xv.x), NS >= 2 ? mufu_ex2(xv.y) : 0.f);
         }
       }
+    };
+    // h <- exp(Δ A) h + Δu B for one token; returns this lane's part of C·h.
+    auto update = [&](const f2 (&dq)[NP], float du, const f2 (&bq)[NP], const f2 (&cq)[NP]) {
+      const f2 du2 = pk2(du, du);
+      f2 acc;
 #pragma unroll
-      for (int q = 0; q < G; ++q) {
-        const f2 dlt2 = pk2(ev[q].x, ev[q].x);
-#pragma unroll
-        for (int m = 0; m < NP; ++m) {
-          const f2 xx = mul2(dlt2, a2p[m]);
-          if (POLY > 0 && (q % (POLY > 0 ? POLY : 1)) == POLY - 1) {
-            dA[q][m] = ex2_poly2(xx);
-          } else {
-            const float2 xv = up2(xx);
-            dA[q][m] = pk2(mufu_ex2(xv.x), NS >= 2 ? mufu_ex2(xv.y) : 0.f);
-          }
-        }
+      for (int m = 0; m < NP; ++m) {
+        hp[m] = fma2(dq[m], hp[m], mul2(du2, bq[m]));
+        acc = m == 0 ? mul2(cq[m], hp[m]) : fma2(cq[m], hp[m], acc);
       }
-      float pv[G];
+      const float2 pr = up2(acc);
+      return pr.x + pr.y;
+    };
+    {
+      // Software pipeline over groups of G tokens: the decays of group g+1
+      // (MUFU, independent of the state) are issued next to the dependent
+      // updates of group g, so the special-function pipe is fed steadily.
+      constexpr int NG = T / G;
+      float2 evn[G];
+      f2 dAn[G][NP];
 #pragma unroll
-      for (int q = 0; q < G; ++q) {
-        const f2 du2 = pk2(ev[q].y, ev[q].y);
-        f2 acc;
+      for (int q = 0; q < G; ++q) evn[q] = xch[q * CB];
 #pragma unroll
-        for (int m = 0; m < NP; ++m) {
-          hp[m] = fma2(dA[q][m], hp[m], mul2(du2, bb[q][m]));
-          acc = m == 0 ? mul2(cc[q][m], hp[m]) : fma2(cc[q][m], hp[m], acc);
+      for (int q = 0; q < G; ++q) decay(evn[q].x, q, dAn[q]);
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        const int tg0 = g * G;
+        float duc[G];
+        f2 dAc[G][NP];
+#pragma unroll
+        for (int q = 0; q < G; ++q) {
+          duc[q] = evn[q].y;
+#pragma unroll
+          for (int m = 0; m < NP; ++m) dAc[q][m] = dAn[q][m];
         }
-        const float2 pr = up2(acc);
-        pv[q] = pr.x + pr.y;
-      }
+        if (g + 1 < NG) {
 #pragma unroll
-      for (int q = 0; q < G; ++q)
-        if (cown) part[(tg0 + q) * CB * GL] = pv[q];  // idle lanes alias other warps' channels
+          for (int q = 0; q < G; ++q) evn[q] = xch[(tg0 + G + q) * CB];
+        }
+        f2 bb[G][NP], cc[G][NP];
+#pragma unroll
+        for (int q = 0; q < G; ++q) load_bc(tg0 + q, bb[q], cc[q]);
+        if (g + 1 < NG) {
+#pragma unroll
+          for (int q = 0; q < G; ++q) decay(evn[q].x, q, dAn[q]);
+        }
+        float pv[G];
+#pragma unroll
+        for (int q = 0; q < G; ++q) pv[q] = update(dAc[q], duc[q], bb[q], cc[q]);
+#pragma unroll
+        for (int q = 0; q < G; ++q)
+          if (cown) part[(tg0 + q) * CB * GL] = pv[q];  // idle lanes alias other warps' channels
+      }
     }
     __syncwarp();
     if (lane == 0) {
