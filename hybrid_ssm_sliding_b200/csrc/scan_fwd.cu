@@ -73,7 +73,10 @@ template <> struct ScanShape<8> { static constexpr int NS = 1, GL = 8; };
 template <> struct ScanShape<4> { static constexpr int NS = 1, GL = 4; };
 
 constexpr int kScanCB = 32;     // channels in one TMA box (>= CU + alignment offset)
-constexpr int kScanT = 32;      // tokens per tile
+#ifndef SAMBA_SCAN_T
+#define SAMBA_SCAN_T 32
+#endif
+constexpr int kScanT = SAMBA_SCAN_T;  // tokens per tile
 constexpr int kScanPro = 8;     // prologue warps
 constexpr int kScanEpi = 4;     // epilogue warps
 // Upper bound on the block size (sets the register budget per thread).
@@ -94,7 +97,8 @@ constexpr int kScanSmemBudget = 227 * 1024;
 template <int N, typename XT>
 struct ScanLayout {
   static constexpr int GL = ScanShape<N>::GL;
-  static constexpr int CB = kScanCB, T = kScanT, HALO = 3, SLOTS = kScanSlots;
+  // tiles of kScanT tokens at N = 16; 32 at smaller N (more partials per channel)
+  static constexpr int CB = kScanCB, T = N == 16 ? kScanT : 32, HALO = 3, SLOTS = kScanSlots;
   static constexpr int al(int v) { return (v + 127) / 128 * 128; }
   static constexpr int XB = (T + HALO) * CB * (int)sizeof(XT);
   static constexpr int ZB = T * CB * (int)sizeof(XT);
@@ -191,7 +195,8 @@ __device__ __forceinline__ float softplus_fast(float w) {
 //   prologue : XCH[k], EPI[k] <- conv/softplus, D·u, z; arrives pro_full[k]
 //              (waits full[s]; scan_done[k] and epi_done[k] of tile i-SLOTS)
 //   scan     : PART[k] <- partial C·h of its states; arrives scan_done[k]
-//              (waits pro_full[k], full[s]; epi_done[k] of tile i-SLOTS)
+//              (waits pro_full[k], full[s]; pro_full[k] follows the
+//              prologue's own wait for epi_done[k] of tile i-SLOTS)
 //   epilogue : y <- (Σ PART[k] + D·u)·silu(z); arrives epi_done[k]
 //              (waits scan_done[k])
 // empty[s] collects the prologue and scan warps (the readers of stage s).
@@ -454,9 +459,11 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
 
   for (int i = 0; i < ntiles; ++i) {
     const int s = i % STAGES, k = i % SLOTS, r = i / SLOTS;
+    // PART[k] may be rewritten once the epilogue has read tile i - SLOTS:
+    // the prologue waits for that (epi_done[k]) before it arrives on
+    // pro_full[k], so the wait on pro_full[k] covers it.
     bool ok = mbar_wait(&pro_full[k], r & 1, abort_flag);
     ok = ok && mbar_wait(&full[s], (i / STAGES) & 1, abort_flag);
-    if (r >= 1) ok = ok && mbar_wait(&epi_done[k], (r - 1) & 1, abort_flag);
     if (!__all_sync(0xffffffffu, ok)) break;
     const unsigned char* st = smem + s * Ly::STAGE_BYTES;
     const float* bs = reinterpret_cast<const float*>(st + Ly::B_OFF);
