@@ -23,9 +23,10 @@
 //   * Warp roles.  One producer warp streams x, z, delta, B, C tiles into a
 //     STAGES-deep shared-memory ring with TMA.  Prologue warps compute, once
 //     per (token, channel), the conv, SiLU and softplus, leaving (Δ, Δu) for
-//     the scan and (D·u, z) for the output.  The scan warps hold the state: a
-//     channel's N states are spread over GL lanes (NS states per lane) and
-//     each lane writes its partial C·h per token.  Epilogue warps finish
+//     the scan and (D·u, z) for the output.  The scan warps hold the state:
+//     lane = channel, and each of the GL scan warps holds NS of a channel's N
+//     states, so all lanes of a warp read the same B and C entries; each lane
+//     writes its partial C·h per token.  Epilogue warps finish
 //     y = (Σ partials + D·u)·silu(z) and store it.
 //   * Prologue, scan and epilogue of consecutive tiles overlap through
 //     SLOTS-deep exchange arrays guarded by mbarriers.
@@ -108,7 +109,7 @@ struct ScanLayout {
                        C_OFF = B_OFF + al(BB), STAGE_BYTES = C_OFF + al(BB);
   static constexpr int XCH_BYTES = SLOTS * T * CB * 8;       // float2 [SLOTS][T][CB] (Δ, Δu)
   static constexpr int EPI_BYTES = SLOTS * T * CB * 8;       // float2 [SLOTS][T][CB] (D·u, z)
-  static constexpr int PART_BYTES = SLOTS * T * CB * GL * 4; // float  [SLOTS][T][CB][GL]
+  static constexpr int PART_BYTES = SLOTS * T * CB * GL * 4; // float  [SLOTS][T][GL][CB]
   static constexpr int FIXED = XCH_BYTES + EPI_BYTES + PART_BYTES + 512;
   // TMA ring: as many stages (up to 6) as fit next to the hand-off buffers
   static constexpr int STAGES_FIT = (kScanSmemBudget - FIXED) / STAGE_BYTES;
@@ -121,9 +122,8 @@ struct ScanLayout {
   static constexpr int SMEM = BAR_OFF + 512;
 };
 
-__host__ __device__ constexpr int scan_warps(int cu, int cpw) {
-  return (((cu + cpw - 1) / cpw) + 3) / 4 * 4;
-}
+// Scan warps: one per group of NS states (GL of them); lane = channel (CU <= 32).
+__host__ __device__ constexpr int scan_warps(int gl) { return gl; }
 
 // ------------------------------------------------------------ math helpers
 __device__ __forceinline__ float mufu_ex2(float x) {
@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
                     const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_b,
                     const __grid_constant__ CUtensorMap map_c, const ScanParams p) {
   using Ly = ScanLayout<N, XT>;
-  constexpr int NS = ScanShape<N>::NS, GL = ScanShape<N>::GL, CPW = 32 / GL;
+  constexpr int NS = ScanShape<N>::NS, GL = ScanShape<N>::GL;
   constexpr int T = Ly::T, CB = Ly::CB, STAGES = Ly::STAGES, HALO = Ly::HALO, SLOTS = Ly::SLOTS;
   extern __shared__ __align__(1024) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Ly::BAR_OFF);
@@ -220,10 +220,7 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
   float* PART = reinterpret_cast<float*>(smem + Ly::PART_OFF);
 
   const int CU = p.CU;
-  // Scan warps: a multiple of 4 (one per SM sub-partition, whose MUFU pipes
-  // are separate), channels spread evenly over them.
-  const int NSW = scan_warps(CU, CPW);
-  const int CPWE = (CU + NSW - 1) / NSW;  // channels per scan warp
+  constexpr int NSW = scan_warps(GL);
   const int PRO0 = NSW, EPI0 = NSW + kScanPro, PROD = NSW + kScanPro + kScanEpi;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
@@ -296,14 +293,13 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
 #pragma unroll
       for (int q = 0; q < TPE; ++q) {
         const int t = eg * TPE + q;
-        const float* part = PART + ((k * T + t) * CB + cl) * GL;
-        pv[q] = *reinterpret_cast<const float4*>(part);
+        const float* part = PART + (k * T + t) * GL * CB + cl;
+        pv[q] = make_float4(part[0], part[CB], part[2 * CB], part[3 * CB]);
         if (GL == 8) {
-          const float4 v2 = *reinterpret_cast<const float4*>(part + 4);
-          pv[q].x += v2.x;
-          pv[q].y += v2.y;
-          pv[q].z += v2.z;
-          pv[q].w += v2.w;
+          pv[q].x += part[4 * CB];
+          pv[q].y += part[5 * CB];
+          pv[q].z += part[6 * CB];
+          pv[q].w += part[7 * CB];
         }
         ev[q] = EPI[(k * T + t) * CB + cl];
       }
@@ -430,14 +426,14 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
   }
 
   // ==================================================================== scan
-  // Lane (cg, j): channel cl of the CTA, states [j·NS, (j+1)·NS) held as NP
-  // packed pairs.  Lanes past the CTA's channels (last warp, CU % CPW != 0)
-  // run along on zeros and write partials nobody reads.
+  // Warp j, lane cl: channel cl of the CTA, states [j·NS, (j+1)·NS) held as
+  // NP packed pairs.  Every lane of a warp reads the same B and C entries of
+  // a token (a shared-memory broadcast).  Lanes past the CTA's channels run
+  // along on zeros and write no partials.
   constexpr int NP = (NS + 1) / 2;
-  const int cg = lane / GL, j = lane % GL;
-  const int cl = warp * CPWE + cg;
+  const int j = warp, cl = lane;
   const int64_t c = c_start + cl;
-  const bool cown = cg < CPWE && cl < CU;  // lane owns one of this warp's channels
+  const bool cown = cl < CU;  // lane owns a channel
   const bool cval = cown && c < p.D;
   const int n0 = j * NS;
   constexpr float kLog2e = 1.4426950408889634f;
@@ -469,7 +465,7 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
     const float* bs = reinterpret_cast<const float*>(st + Ly::B_OFF);
     const float* cs = reinterpret_cast<const float*>(st + Ly::C_OFF);
     const float2* xch = XCH + k * T * CB + cl;
-    float* part = PART + (k * T * CB + cl) * GL + j;
+    float* part = PART + (k * T * GL + j) * CB + cl;
     constexpr int G = SAMBA_SCAN_GROUP;
     // B and C of token t for this lane's states, as packed pairs.
     auto load_bc = [&](int t, f2 (&bq)[NP], f2 (&cq)[NP]) {
@@ -554,7 +550,7 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
         for (int q = 0; q < G; ++q) pv[q] = update(dAc[q], duc[q], bb[q], cc[q]);
 #pragma unroll
         for (int q = 0; q < G; ++q)
-          if (cown) part[(tg0 + q) * CB * GL] = pv[q];  // idle lanes alias other warps' channels
+          if (cown) part[(tg0 + q) * CB * GL] = pv[q];  // idle lanes would alias other channels
       }
     }
     __syncwarp();
@@ -614,7 +610,6 @@ static int launch_scan_t(const samba_scan_args& a, cudaStream_t stream) {
       return fail(SAMBA_ERR_CUDA, "scan: cannot set shared memory size");
     attr_done = true;
   }
-  constexpr int CPW = 32 / ScanShape<N>::GL;
   const int CU = choose_cu(a.batch, a.dim);
   const uint64_t Bsz = a.batch, L = a.seqlen, D = a.dim;
   const uint32_t xs = sizeof(XT);
@@ -660,7 +655,7 @@ static int launch_scan_t(const samba_scan_args& a, cudaStream_t stream) {
   p.fuse_conv = (a.flags & SAMBA_SCAN_FUSE_CONV) != 0;
   p.conv_silu = (a.flags & SAMBA_SCAN_CONV_SILU) != 0;
   p.softplus = (a.flags & SAMBA_SCAN_DELTA_SOFTPLUS) != 0;
-  const int threads = (scan_warps(CU, CPW) + kScanPro + kScanEpi + 1) * 32;
+  const int threads = (scan_warps(ScanShape<N>::GL) + kScanPro + kScanEpi + 1) * 32;
   dim3 grid((unsigned)((D + CU - 1) / CU), (unsigned)Bsz);
   kern<<<grid, threads, Ly::SMEM, stream>>>(mx, mz, mw, mb, mc, p);
   return check_launch("samba_selective_scan_fwd");
