@@ -14,6 +14,15 @@ With N > 1 (torchrun) every rank runs its own batch (weak scaling, no
 collective on the data path); the time is the max over ranks.  --impl
 reference times the float64 CPU oracle on bounded samples of the same
 workload.  Prints one JSON line on rank 0.
+
+    python bench.py --workload decode_64k [--steps K] [--warmup W]
+
+times decoding instead: after a 4096-token prefill of 16 sequences, one step
+is samba_scan_step + samba_swa_step of one layer for all 16 sequences (one
+token each; the SWA step reads the full 2048-slot K/V ring).  Four layer
+states (scan state, conv state, K/V rings: 154 MB, more than L2) rotate from
+step to step, as in a multi-layer model, so every step reads its state from
+HBM; 32 steps per CUDA graph, inputs of 32 distinct steps resident in HBM.
 """
 
 from __future__ import annotations
@@ -35,6 +44,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "Samba mixer prefill tokens/s @128K; scan HBM GB/s; SWA tensor-pipe %"
 UNIT = "tokens/s"
+DECODE_METRIC = "Samba mixer decode tokens/s (16 sequences, one token each per step; SWA ring W = 2048)"
+DECODE_GRAPH_STEPS = 32
+DECODE_LAYERS = 4
 
 
 def parse():
@@ -48,6 +60,9 @@ def parse():
     ap.add_argument("--kernel-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--graphs", type=int, default=0,
+                    help="decode workloads: timed replays of the 32-step graph (default: the workload's decode "
+                         "steps / 32)")
     return ap.parse_args()
 
 
@@ -76,6 +91,22 @@ def scan_bytes(wl):
     per_token = 2 * wl.dstate * 4
     small = wl.batch * wl.dim * (wl.dstate + 3) * 4 + wl.dim * (wl.dstate + wl.dconv + 2) * 4
     return tc * (2 + 2 + 4 + 2) + wl.batch * wl.seqlen * per_token + small
+
+
+def decode_bytes(wl):
+    """Algorithmic HBM bytes of one decode step for the whole batch: the scan
+    step reads and writes h [B, D, N] f32 and the conv state [B, D, K-1] f32,
+    reads x_t, z_t (bf16), delta_t (f32), A, conv weights and writes y_t
+    (bf16); the SWA step reads the valid K and V ring slots (all W of them
+    after a prefill longer than W), q_t, writes k_t, v_t into the ring and
+    o_t."""
+    Bsz, D, N, K = wl.batch, wl.dim, wl.dstate, wl.dconv
+    scan = (2 * Bsz * D * N * 4 + 2 * Bsz * D * (K - 1) * 4 + Bsz * D * (2 + 2 + 4) + Bsz * D * 2
+            + D * N * 4 + D * (K + 2) * 4 + 2 * Bsz * N * 4)
+    slots = min(wl.window, wl.seqlen + 1)
+    kv = Bsz * wl.heads_kv * wl.head_dim * 2
+    swa = 2 * slots * kv + 2 * kv + 2 * Bsz * wl.heads_q * wl.head_dim * 2
+    return scan, swa
 
 
 def swa_flops(wl):
@@ -191,6 +222,24 @@ def run_reference(args):
     from hybrid_ssm_sliding_b200.workloads import WORKLOADS
 
     wl = WORKLOADS[args.workload]
+    if wl.decode_steps > 0:
+        vals = []
+        t0 = time.perf_counter()
+        for s in range(max(1, args.steps)):
+            v, cores, sample = oracle_decode_throughput(wl, seed=s)
+            vals.append(v)
+        wall = time.perf_counter() - t0
+        value = statistics.median(vals)
+        print(json.dumps({
+            "impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.batch / value * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(wl),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample + f"; median of {args.steps} samples ({wall:.1f} s)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}))
+        return 0
     # Each step is a bounded sample (a few hundred ms), so K steps stay short.
     for _ in range(max(0, args.warmup)):
         oracle_throughput(wl, n_chan=64, n_tok=64, n_rows=1)
@@ -214,6 +263,214 @@ def run_reference(args):
     }
     print(json.dumps(line))
     return 0
+
+
+# ------------------------------------------------------------ decode GPU leg
+def run_decode(args, wl, lib, dev, rank, world):
+    """Times decode steps (scan step + SWA step over the whole batch) in
+    CUDA graphs of DECODE_GRAPH_STEPS steps; returns the JSON line."""
+    import torch
+    import torch.distributed as dist
+    from dataclasses import replace
+
+    from hybrid_ssm_sliding_b200 import _lib as L
+    from hybrid_ssm_sliding_b200 import build as B
+    from hybrid_ssm_sliding_b200 import ops
+    from hybrid_ssm_sliding_b200.workloads import make_decode_step_inputs, make_prefill_inputs
+
+    wl_rank = replace(wl, seed=wl.seed + 1000 * rank)
+    Bsz, D, N, K = wl.batch, wl.dim, wl.dstate, wl.dconv
+    # state after a prefill of wl.seqlen tokens, through the library itself
+    pre = make_prefill_inputs(wl_rank, device=dev)
+    h = torch.empty((Bsz, D, N), dtype=torch.float32, device=dev)
+    cs = torch.empty((Bsz, D, K - 1), dtype=torch.float32, device=dev)
+    ops.selective_scan_fwd(pre["x"], pre["delta"], pre["A"], pre["B"], pre["C"], D=pre["D"], z=pre["z"],
+                           conv_w=pre["conv_w"], conv_b=pre["conv_b"], h_final=h, conv_state_out=cs,
+                           y_dtype=torch.bfloat16)
+    k_ring, v_ring, pos = ops.swa_ring_fill(pre["k"], pre["v"], wl.window)
+    A, Dsk, cw, cb = pre["A"], pre["D"], pre["conv_w"], pre["conv_b"]
+    del pre
+    NLY = DECODE_LAYERS
+    layers = [dict(h=h.clone(), cs=cs.clone(), k_ring=k_ring.clone(), v_ring=v_ring.clone(), pos=pos.clone())
+              for _ in range(NLY)]
+    del h, cs, k_ring, v_ring, pos
+    G = DECODE_GRAPH_STEPS
+    steps_in = [make_decode_step_inputs(wl_rank, s, device=dev) for s in range(G)]
+    y_t = torch.empty((Bsz, D), dtype=torch.bfloat16, device=dev)
+    o_t = torch.empty((Bsz, wl.heads_q, wl.head_dim), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty((max(ops.swa_step_workspace_size(Bsz, wl.heads_q, wl.head_dim, wl.window), 16),),
+                     dtype=torch.uint8, device=dev)
+
+    def scan_one(si, ly):
+        ops.scan_step(ly["h"], ly["cs"], si["x"], si["delta"], A, si["B"], si["C"], D=Dsk, z_t=si["z"], conv_w=cw,
+                      conv_b=cb, y_t=y_t)
+
+    def swa_one(si, ly):
+        ops.swa_step(si["q"], si["k"], si["v"], ly["k_ring"], ly["v_ring"], ly["pos"], wl.window, o_t=o_t,
+                     workspace=ws)
+
+    def capture(body):
+        for s_ in range(2):  # warm-up outside capture (first-call setup, attributes)
+            body(steps_in[s_], layers[s_ % NLY])
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for s_, si in enumerate(steps_in):
+                body(si, layers[s_ % NLY])
+        return g
+
+    g_step = capture(lambda si, ly: (scan_one(si, ly), swa_one(si, ly)))
+    g_scan = capture(scan_one)
+    g_swa = capture(swa_one)
+    stream = torch.cuda.current_stream()
+    reps = args.graphs if args.graphs > 0 else max(1, wl.decode_steps // G)
+    for _ in range(max(1, args.warmup)):
+        g_step.replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g_step.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = e0.elapsed_time(e1)
+    clk = clocks.stop()
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    n_steps = reps * G
+    ms_step = ms_total / n_steps
+    value = world * Bsz / (ms_step / 1e3)
+
+    def time_graph(g, n=max(4, reps // 2)):
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / (n * G)
+
+    ms_scan = time_graph(g_scan)
+    ms_swa = time_graph(g_swa)
+    status = ops.get_status()
+    peaks = load_peaks()
+    sb, wb = decode_bytes(wl)
+    kern = {}
+    for name, ms, nb in (("scan_step", ms_scan, sb), ("swa_step", ms_swa, wb)):
+        gbs = nb / (ms / 1e3) / 1e9
+        kern[name] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                      "frac": gbs / peaks["hbm_gbs"], "traffic": None, "ms": ms, "algorithmic_bytes": nb,
+                      "peak_source": peaks["source"]}
+    dom = "swa_step" if ms_swa >= ms_scan else "scan_step"
+    roofline = {k: kern[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+    roofline["kernel"] = dom
+
+    # end to end: per step, copy that step's inputs from pinned host memory
+    # and read y_t and o_t back, through the public API, outside graphs
+    e2e = None
+    if not args.no_e2e:
+        host = [{k: v.to("cpu").pin_memory() for k, v in si.items()} for si in steps_in]
+        dev_in = {k: torch.empty_like(v) for k, v in steps_in[0].items()}
+        y_h = torch.empty(y_t.shape, dtype=y_t.dtype).pin_memory()
+        o_h = torch.empty(o_t.shape, dtype=o_t.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host[0].values())
+        d2h = y_h.numel() * y_h.element_size() + o_h.numel() * o_h.element_size()
+
+        def e2e_step(hs, ly):
+            for kk in hs:
+                dev_in[kk].copy_(hs[kk], non_blocking=True)
+            scan_one(dev_in, ly)
+            swa_one(dev_in, ly)
+            y_h.copy_(y_t, non_blocking=True)
+            o_h.copy_(o_t, non_blocking=True)
+
+        e2e_step(host[0], layers[0])
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        n_e2e = 4 * G
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(n_e2e):
+            e2e_step(host[i % G], layers[i % NLY])
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = a.elapsed_time(b) / n_e2e
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": world * Bsz / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = oracle_decode_throughput(wl)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+    cfg = workload_config(wl)
+    sb_state = Bsz * D * N * 4 + Bsz * D * (K - 1) * 4
+    ring_bytes = Bsz * wl.window * wl.heads_kv * wl.head_dim * 2
+    cfg.update({"prefill_tokens": wl.seqlen, "graph_steps": G, "layers": NLY,
+                "l2": f"inputs larger than L2: {NLY} layer states (scan state, conv state, K/V rings; "
+                      f"{NLY * (sb_state + 2 * ring_bytes) / 1e6:.0f} MB) rotate from step to step"})
+    return {
+        "metric": DECODE_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": n_steps,
+        "warmup": max(1, args.warmup) * G, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg, "roofline": roofline,
+        "kernels": kern, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+        "gpu_launches": n_steps * 3, "status": status,
+    }
+
+
+def oracle_decode_throughput(wl, n_seq=2, n_chan=512, seed=0):
+    """Times the float64 oracle's decode step, as it stands, on n_seq
+    sequences (n_chan channels of the scan, every head of SWA at a full ring)
+    and extrapolates to tokens/s of the whole batch."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    import oracle.samba_oracle as orc
+
+    rng = np.random.default_rng(seed)
+    N, K, W = wl.dstate, wl.dconv, wl.window
+    h = rng.standard_normal((n_seq, n_chan, N)) * 0.1
+    cs = rng.standard_normal((n_seq, n_chan, K - 1))
+    A = -np.tile(np.arange(1, N + 1, dtype=np.float64), (n_chan, 1))
+    kr = rng.standard_normal((n_seq, W, wl.heads_kv, wl.head_dim))
+    vr = rng.standard_normal((n_seq, W, wl.heads_kv, wl.head_dim))
+    pos = np.full((n_seq,), W + 7, dtype=np.int64)
+    reps = 8
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            orc.scan_step(h, cs, rng.standard_normal((n_seq, n_chan)), rng.uniform(-6.9, -2.3, (n_seq, n_chan)), A,
+                          rng.standard_normal((n_seq, N)), rng.standard_normal((n_seq, N)),
+                          rng.standard_normal(n_chan), rng.standard_normal((n_seq, n_chan)),
+                          conv_w=rng.uniform(-0.5, 0.5, (n_chan, K)), conv_b=rng.uniform(-0.5, 0.5, n_chan))
+        t_scan = (time.perf_counter() - t0) / reps
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            orc.swa_step(rng.standard_normal((n_seq, wl.heads_q, wl.head_dim)),
+                         rng.standard_normal((n_seq, wl.heads_kv, wl.head_dim)),
+                         rng.standard_normal((n_seq, wl.heads_kv, wl.head_dim)), kr, vr, pos, W)
+        t_swa = (time.perf_counter() - t0) / reps
+    per_token = t_scan * (wl.dim / n_chan) / n_seq + t_swa / n_seq
+    sample = (f"{n_seq} sequences; scan step on {n_chan} of {wl.dim} channels ({t_scan * 1e3:.1f} ms, scaled by "
+              f"channels), SWA step over a full {W}-slot ring ({t_swa * 1e3:.1f} ms); float64 NumPy, {reps} reps")
+    return 1.0 / per_token, 1, sample
 
 
 # -------------------------------------------------------------------- GPU leg
@@ -244,6 +501,14 @@ def main():
     lib = L.load()
 
     wl = WORKLOADS[args.workload]
+    if wl.decode_steps > 0:
+        line = run_decode(args, wl, lib, dev, rank, world)
+        if rank == 0:
+            print(json.dumps(line))
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
     from dataclasses import replace
     wl_rank = replace(wl, seed=wl.seed + 1000 * rank)   # each rank its own batch
     inp = make_prefill_inputs(wl_rank, device=dev)

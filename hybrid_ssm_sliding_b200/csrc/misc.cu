@@ -224,58 +224,86 @@ int launch_ring_fill(const void* k, const void* v, int64_t L, void* k_ring, void
 // (max, sum, unnormalised output) per head; a second kernel combines the
 // splits.  The newest position is read from k_t/v_t, which split 0 also
 // stores into its ring slot (that slot held a position outside the window, so
-// no other CTA reads it in this step).
-constexpr int kStepChunk = 256;
+// no other CTA reads it in this step).  Thread i of a CTA owns position i of
+// its chunk: it loads that position's K row into registers and its V row into
+// shared memory in one burst (all rows of the chunk in flight at once), so
+// the P·V loop runs from shared memory.
+template <int HD> struct StepCfg {
+  static constexpr int CH = HD <= 64 ? 128 : 64;  // positions per CTA (= threads)
+};
 
 template <int HD>
-__global__ void __launch_bounds__(256) swa_step_split_kernel(
+__global__ void __launch_bounds__(StepCfg<HD>::CH) swa_step_split_kernel(
     const __nv_bfloat16* __restrict__ q_t, const __nv_bfloat16* __restrict__ k_t,
     const __nv_bfloat16* __restrict__ v_t, __nv_bfloat16* __restrict__ k_ring, __nv_bfloat16* __restrict__ v_ring,
     const int64_t* __restrict__ pos, float* __restrict__ ws, int Hq, int Hkv, int64_t W, float scale_log2,
     int nsplit) {
+  constexpr int CH = StepCfg<HD>::CH;
+  constexpr int NW = CH / 32;       // warps
+  constexpr int PAIRS = HD / 2;
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int group = Hq / Hkv;
+  const int group = Hq / Hkv;  // <= 16
   const int64_t p = pos[b];
   const int64_t lo = p - W + 1 > 0 ? p - W + 1 : 0;
-  const int64_t a0 = lo + (int64_t)split * kStepChunk;
+  const int64_t a0 = lo + (int64_t)split * CH;
+  // positions a0 .. a0 + n_here - 1 of this chunk are valid; their ring slots
+  // are consecutive modulo W, starting at slot0 (one 64-bit remainder per CTA)
+  const int n_here = (int)(p - a0 + 1 < CH ? (p - a0 + 1 > 0 ? p - a0 + 1 : 0) : CH);
+  const int slot0 = (int)(a0 % W);
+  const int Wi = (int)W;
   __shared__ float qs[16][HD];
-  __shared__ float sc[16][kStepChunk];
+  __shared__ float sc[16][CH];
+  __shared__ __align__(16) __nv_bfloat162 vs[CH][PAIRS];
   __shared__ float red_m[16], red_l[16];
 
   const int tid = threadIdx.x;
-  for (int i = tid; i < group * HD; i += blockDim.x) {
+  // this thread's position: K row to registers, V row to shared memory
+  uint4 kraw[HD / 8];
+  {
+    const bool valid = tid < n_here;
+    int slot = slot0 + tid;
+    slot = slot >= Wi ? slot - Wi : slot;
+    const bool is_new = a0 + tid == p;
+    const int64_t roff = (((int64_t)b * W + (valid ? slot : 0)) * Hkv + g) * HD;
+    const int64_t noff = ((int64_t)b * Hkv + g) * HD;
+    const uint4* krow = reinterpret_cast<const uint4*>(is_new ? k_t + noff : k_ring + roff);
+    const uint4* vrow = reinterpret_cast<const uint4*>(is_new ? v_t + noff : v_ring + roff);
+    uint4 vraw[HD / 8];
+#pragma unroll
+    for (int c = 0; c < HD / 8; ++c) {
+      kraw[c] = valid ? krow[c] : make_uint4(0u, 0u, 0u, 0u);
+      vraw[c] = valid ? vrow[c] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int c = 0; c < HD / 8; ++c) reinterpret_cast<uint4*>(&vs[tid][0])[c] = vraw[c];
+  }
+  for (int i = tid; i < group * HD; i += CH) {
     const int hh = i / HD, dd = i % HD;
     qs[hh][dd] = __bfloat162float(q_t[((int64_t)b * Hq + g * group + hh) * HD + dd]);
   }
   if (split == 0) {  // store the new key/value into its slot
     const int64_t slot = p % W;
-    for (int i = tid; i < HD; i += blockDim.x) {
+    for (int i = tid; i < HD; i += CH) {
       k_ring[(((int64_t)b * W + slot) * Hkv + g) * HD + i] = k_t[((int64_t)b * Hkv + g) * HD + i];
       v_ring[(((int64_t)b * W + slot) * Hkv + g) * HD + i] = v_t[((int64_t)b * Hkv + g) * HD + i];
     }
   }
   __syncthreads();
 
-  // scores: thread = position
+  // scores of this thread's position for every head of the group
   {
-    const int64_t a = a0 + tid;
-    const bool valid = a <= p;
-    const __nv_bfloat16* krow = (a == p) ? k_t + ((int64_t)b * Hkv + g) * HD
-                                         : k_ring + (((int64_t)b * W + (valid ? a % W : 0)) * Hkv + g) * HD;
     float kv[HD];
-    if (valid) {
 #pragma unroll
-      for (int dd = 0; dd < HD; dd += 8) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(krow + dd);
-        const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    for (int c = 0; c < HD / 8; ++c) {
+      const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&kraw[c]);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(pr[q]);
-          kv[dd + 2 * q] = f.x;
-          kv[dd + 2 * q + 1] = f.y;
-        }
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(pr[q]);
+        kv[8 * c + 2 * q] = f.x;
+        kv[8 * c + 2 * q + 1] = f.y;
       }
     }
+    const bool valid = tid < n_here;
     for (int hh = 0; hh < group; ++hh) {
       float s = 0.f;
 #pragma unroll
@@ -284,16 +312,16 @@ __global__ void __launch_bounds__(256) swa_step_split_kernel(
     }
   }
   __syncthreads();
-  // per head max and exp-sum (one warp per head, heads strided over 8 warps)
+  // per head max and exp-sum (one warp per head, heads strided over the warps)
   const int warp = tid >> 5, lane = tid & 31;
-  for (int hh = warp; hh < group; hh += 8) {
+  for (int hh = warp; hh < group; hh += NW) {
     float m = -INFINITY;
-    for (int i = lane; i < kStepChunk; i += 32) m = fmaxf(m, sc[hh][i]);
+    for (int i = lane; i < CH; i += 32) m = fmaxf(m, sc[hh][i]);
 #pragma unroll
     for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     const float mu = (m == -INFINITY) ? 0.f : m;
     float l = 0.f;
-    for (int i = lane; i < kStepChunk; i += 32) {
+    for (int i = lane; i < CH; i += 32) {
       const float e = ex2_approx(sc[hh][i] - mu);
       sc[hh][i] = e;
       l += e;
@@ -306,24 +334,25 @@ __global__ void __launch_bounds__(256) swa_step_split_kernel(
     }
   }
   __syncthreads();
-  // partial outputs: thread = (head, dim pair)
-  constexpr int PAIRS = HD / 2;
-  for (int job = tid; job < group * PAIRS; job += blockDim.x) {
+  // partial outputs: job = (head, dim pair); V from shared memory (invalid
+  // positions hold zeros and zero probabilities)
+  for (int job = tid; job < group * PAIRS; job += CH) {
     const int hh = job / PAIRS, dp = job % PAIRS;
-    float o0 = 0.f, o1 = 0.f;
-    const int64_t n_here = p - a0 + 1 < kStepChunk ? p - a0 + 1 : kStepChunk;
-    for (int i = 0; i < n_here; ++i) {
-      const int64_t a = a0 + i;
-      const __nv_bfloat16* vrow = (a == p) ? v_t + ((int64_t)b * Hkv + g) * HD
-                                           : v_ring + (((int64_t)b * W + a % W) * Hkv + g) * HD;
-      const float2 vv = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(vrow)[dp]);
-      const float pw = sc[hh][i];
-      o0 = fmaf(pw, vv.x, o0);
-      o1 = fmaf(pw, vv.y, o1);
+    float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+    const int n4 = (n_here + 3) & ~3;
+#pragma unroll 4
+    for (int i = 0; i < n4; i += 2) {
+      const float2 va = __bfloat1622float2(vs[i][dp]);
+      const float2 vb = __bfloat1622float2(vs[i + 1][dp]);
+      const float pa = sc[hh][i], pb = sc[hh][i + 1];
+      o0 = fmaf(pa, va.x, o0);
+      o1 = fmaf(pa, va.y, o1);
+      o2 = fmaf(pb, vb.x, o2);
+      o3 = fmaf(pb, vb.y, o3);
     }
     float* dst = ws + ((((int64_t)b * Hq + g * group + hh) * nsplit + split) * (HD + 2));
-    dst[2 + 2 * dp] = o0;
-    dst[2 + 2 * dp + 1] = o1;
+    dst[2 + 2 * dp] = o0 + o2;
+    dst[2 + 2 * dp + 1] = o1 + o3;
     if (dp == 0) {
       dst[0] = red_m[hh];
       dst[1] = red_l[hh];
@@ -351,16 +380,18 @@ __global__ void swa_step_combine_kernel(const float* __restrict__ ws, __nv_bfloa
 }
 
 size_t swa_step_workspace(int64_t B, int Hq, int d, int64_t W) {
-  const int64_t nsplit = (W + kStepChunk - 1) / kStepChunk;
+  const int ch = d <= 64 ? StepCfg<64>::CH : StepCfg<128>::CH;
+  const int64_t nsplit = (W + ch - 1) / ch;
   return static_cast<size_t>(B * Hq * nsplit * (d + 2)) * sizeof(float);
 }
 
 template <int HD>
 static void swa_step_go(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring, int64_t* pos,
                         void* o_t, int64_t B, int Hq, int Hkv, int64_t W, float scale, void* ws, cudaStream_t s) {
-  const int nsplit = (int)((W + kStepChunk - 1) / kStepChunk);
+  constexpr int CH = StepCfg<HD>::CH;
+  const int nsplit = (int)((W + CH - 1) / CH);
   dim3 g1(nsplit, Hkv, (unsigned)B);
-  swa_step_split_kernel<HD><<<g1, 256, 0, s>>>(
+  swa_step_split_kernel<HD><<<g1, CH, 0, s>>>(
       reinterpret_cast<const __nv_bfloat16*>(q_t), reinterpret_cast<const __nv_bfloat16*>(k_t),
       reinterpret_cast<const __nv_bfloat16*>(v_t), reinterpret_cast<__nv_bfloat16*>(k_ring),
       reinterpret_cast<__nv_bfloat16*>(v_ring), pos, reinterpret_cast<float*>(ws), Hq, Hkv, W,

@@ -63,7 +63,7 @@ def test_noalloc_step_matches_workspace_step_on_two_calls():
 
 def test_noalloc_step_refuses_sizes_beyond_its_scratch():
     lib = L.load()
-    Bsz, Hq, Hkv, d, W = 64, 64, 4, 128, 4096  # partials need 64*64*16*130*4 B = 34 MB > 4 MiB
+    Bsz, Hq, Hkv, d, W = 64, 64, 4, 128, 4096  # the split partials need far more than 4 MiB
     assert lib.samba_swa_step_workspace_size(Bsz, Hq, d, W) > (4 << 20)
     buf = torch.empty((16,), dtype=torch.uint8, device="cuda")
     pos = torch.zeros((Bsz,), dtype=torch.int64, device="cuda")
