@@ -305,9 +305,10 @@ __global__ void __launch_bounds__(StepCfg<HD>::CH) swa_step_split_kernel(
     }
     const bool valid = tid < n_here;
     for (int hh = 0; hh < group; ++hh) {
-      float s = 0.f;
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};  // four short chains instead of one of length HD
 #pragma unroll
-      for (int dd = 0; dd < HD; ++dd) s = fmaf(qs[hh][dd], kv[dd], s);
+      for (int dd = 0; dd < HD; ++dd) s4[dd & 3] = fmaf(qs[hh][dd], kv[dd], s4[dd & 3]);
+      const float s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       sc[hh][tid] = valid ? s * scale_log2 : -INFINITY;
     }
   }
@@ -366,9 +367,12 @@ __global__ void swa_step_combine_kernel(const float* __restrict__ ws, __nv_bfloa
   const int hq = blockIdx.x, b = blockIdx.y;
   const int dd = threadIdx.x;
   const float* base = ws + ((int64_t)b * Hq + hq) * nsplit * (HD + 2);
+  // the loops are unrolled so that the loads of several splits are in flight
   float M = -INFINITY;
+#pragma unroll 8
   for (int s = 0; s < nsplit; ++s) M = fmaxf(M, base[s * (HD + 2)]);
   float l = 0.f, acc = 0.f;
+#pragma unroll 8
   for (int s = 0; s < nsplit; ++s) {
     const float m = base[s * (HD + 2)];
     const float f = (m == -INFINITY) ? 0.f : ex2_approx(m - M);
