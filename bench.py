@@ -66,6 +66,33 @@ def parse():
     return ap.parse_args()
 
 
+# ------------------------------------------------------------- ranks (N > 1)
+# Replicas only: every rank runs its own batch of the workload (its own seed),
+# no data crosses ranks, and the reported time is the max over ranks.
+def rank_workload(wl, rank):
+    """The workload of rank `rank`: same shapes, its own seeded inputs."""
+    from dataclasses import replace
+
+    return replace(wl, seed=wl.seed + 1000 * rank)
+
+
+def max_over_ranks(x, device):
+    """Max of the float x over all ranks (x itself without a process group)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Units per second of the whole job: every rank's units over the slowest rank's time."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -271,14 +298,13 @@ def run_decode(args, wl, lib, dev, rank, world):
     CUDA graphs of DECODE_GRAPH_STEPS steps; returns the JSON line."""
     import torch
     import torch.distributed as dist
-    from dataclasses import replace
 
     from hybrid_ssm_sliding_b200 import _lib as L
     from hybrid_ssm_sliding_b200 import build as B
     from hybrid_ssm_sliding_b200 import ops
     from hybrid_ssm_sliding_b200.workloads import make_decode_step_inputs, make_prefill_inputs
 
-    wl_rank = replace(wl, seed=wl.seed + 1000 * rank)
+    wl_rank = rank_workload(wl, rank)
     Bsz, D, N, K = wl.batch, wl.dim, wl.dstate, wl.dconv
     # state after a prefill of wl.seqlen tokens, through the library itself
     pre = make_prefill_inputs(wl_rank, device=dev)
@@ -342,15 +368,11 @@ def run_decode(args, wl, lib, dev, rank, world):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms_total = e0.elapsed_time(e1)
+    ms_total = max_over_ranks(e0.elapsed_time(e1), dev)
     clk = clocks.stop()
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
     n_steps = reps * G
     ms_step = ms_total / n_steps
-    value = world * Bsz / (ms_step / 1e3)
+    value = whole_job_rate(Bsz, world, ms_step)
 
     def time_graph(g, n=max(4, reps // 2)):
         g.replay()
@@ -408,12 +430,8 @@ def run_decode(args, wl, lib, dev, rank, world):
             e2e_step(host[i % G], layers[i % NLY])
         b.record(stream)
         torch.cuda.synchronize()
-        ms_e2e = a.elapsed_time(b) / n_e2e
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": world * Bsz / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        ms_e2e = max_over_ranks(a.elapsed_time(b) / n_e2e, dev)
+        e2e = {"value": whole_job_rate(Bsz, world, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
 
     cpu = None
@@ -509,8 +527,7 @@ def main():
             dist.barrier()
             dist.destroy_process_group()
         return
-    from dataclasses import replace
-    wl_rank = replace(wl, seed=wl.seed + 1000 * rank)   # each rank its own batch
+    wl_rank = rank_workload(wl, rank)   # each rank its own batch
     inp = make_prefill_inputs(wl_rank, device=dev)
     Bsz, Ln, D, N, K = wl.batch, wl.seqlen, wl.dim, wl.dstate, wl.dconv
     y = torch.empty((Bsz, Ln, D), dtype=torch.bfloat16, device=dev)
@@ -549,15 +566,10 @@ def main():
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms_total = e0.elapsed_time(e1)
+    ms_total = max_over_ranks(e0.elapsed_time(e1), dev)
     clk = clocks.stop()
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
     ms_step = ms_total / args.steps
-    tokens_all = world * Bsz * Ln
-    value = tokens_all / (ms_step / 1e3)
+    value = whole_job_rate(Bsz * Ln, world, ms_step)
     status = ops.get_status()
 
     # ---- per-kernel times (each kernel alone, back to back, same stream)
@@ -633,12 +645,8 @@ def main():
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        ms_e2e = a.elapsed_time(b) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": tokens_all / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        ms_e2e = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, dev)
+        e2e = {"value": whole_job_rate(Bsz * Ln, world, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
 
     cpu = None
