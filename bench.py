@@ -56,7 +56,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="samba", choices=["samba", "reference"])
     ap.add_argument("--workload", default="prefill_128k")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--kernel-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -327,13 +327,13 @@ def run_decode(args, wl, lib, dev, rank, world):
     ws = torch.empty((max(ops.swa_step_workspace_size(Bsz, wl.heads_q, wl.head_dim, wl.window), 16),),
                      dtype=torch.uint8, device=dev)
 
-    def scan_one(si, ly):
+    def scan_one(si, ly, y_out=None):
         ops.scan_step(ly["h"], ly["cs"], si["x"], si["delta"], A, si["B"], si["C"], D=Dsk, z_t=si["z"], conv_w=cw,
-                      conv_b=cb, y_t=y_t)
+                      conv_b=cb, y_t=y_t if y_out is None else y_out)
 
-    def swa_one(si, ly):
-        ops.swa_step(si["q"], si["k"], si["v"], ly["k_ring"], ly["v_ring"], ly["pos"], wl.window, o_t=o_t,
-                     workspace=ws)
+    def swa_one(si, ly, o_out=None):
+        ops.swa_step(si["q"], si["k"], si["v"], ly["k_ring"], ly["v_ring"], ly["pos"], wl.window,
+                     o_t=o_t if o_out is None else o_out, workspace=ws)
 
     def capture(body):
         for s_ in range(2):  # warm-up outside capture (first-call setup, attributes)
@@ -400,37 +400,62 @@ def run_decode(args, wl, lib, dev, rank, world):
     roofline = {k: kern[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
     roofline["kernel"] = dom
 
-    # end to end: per step, copy that step's inputs from pinned host memory
-    # and read y_t and o_t back, through the public API, outside graphs
+    # end to end: every step copies its inputs from pinned host memory (all of
+    # a step's inputs packed in one buffer, one copy) and reads y_t and o_t
+    # back (one copy), around the library calls; 32 steps in a CUDA graph
     e2e = None
     if not args.no_e2e:
-        host = [{k: v.to("cpu").pin_memory() for k, v in si.items()} for si in steps_in]
-        dev_in = {k: torch.empty_like(v) for k, v in steps_in[0].items()}
-        y_h = torch.empty(y_t.shape, dtype=y_t.dtype).pin_memory()
-        o_h = torch.empty(o_t.shape, dtype=o_t.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in host[0].values())
-        d2h = y_h.numel() * y_h.element_size() + o_h.numel() * o_h.element_size()
+        keys = list(steps_in[0].keys())
 
-        def e2e_step(hs, ly):
-            for kk in hs:
-                dev_in[kk].copy_(hs[kk], non_blocking=True)
-            scan_one(dev_in, ly)
-            swa_one(dev_in, ly)
-            y_h.copy_(y_t, non_blocking=True)
-            o_h.copy_(o_t, non_blocking=True)
+        def nbytes(t):
+            return t.numel() * t.element_size()
 
-        e2e_step(host[0], layers[0])
+        offs, off = {}, 0
+        for k in keys:
+            offs[k] = off
+            off += (nbytes(steps_in[0][k]) + 255) // 256 * 256
+        pack_bytes = off
+        host_packs = []
+        for si in steps_in:
+            hp = torch.zeros(pack_bytes, dtype=torch.uint8).pin_memory()
+            for k in keys:
+                hp[offs[k]:offs[k] + nbytes(si[k])].copy_(si[k].cpu().reshape(-1).view(torch.uint8))
+            host_packs.append(hp)
+        dev_pack = torch.empty(pack_bytes, dtype=torch.uint8, device=dev)
+        dev_in = {k: dev_pack[offs[k]:offs[k] + nbytes(steps_in[0][k])].view(steps_in[0][k].dtype)
+                  .view(steps_in[0][k].shape) for k in keys}
+        y_bytes = (nbytes(y_t) + 255) // 256 * 256
+        out_pack = torch.empty(y_bytes + nbytes(o_t), dtype=torch.uint8, device=dev)
+        y_view = out_pack[:nbytes(y_t)].view(y_t.dtype).view(y_t.shape)
+        o_view = out_pack[y_bytes:].view(o_t.dtype).view(o_t.shape)
+        host_out = torch.empty(out_pack.numel(), dtype=torch.uint8).pin_memory()
+        h2d, d2h = pack_bytes, out_pack.numel()
+
+        def e2e_one(s_, ly):
+            dev_pack.copy_(host_packs[s_], non_blocking=True)
+            scan_one(dev_in, ly, y_view)
+            swa_one(dev_in, ly, o_view)
+            host_out.copy_(out_pack, non_blocking=True)
+
+        for s_ in range(2):
+            e2e_one(s_, layers[s_ % NLY])
+        torch.cuda.synchronize()
+        g_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_e2e):
+            for s_ in range(G):
+                e2e_one(s_, layers[s_ % NLY])
+        g_e2e.replay()
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        n_e2e = 4 * G
+        n_rep = max(4, reps // 16)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for i in range(n_e2e):
-            e2e_step(host[i % G], layers[i % NLY])
+        for _ in range(n_rep):
+            g_e2e.replay()
         b.record(stream)
         torch.cuda.synchronize()
-        ms_e2e = max_over_ranks(a.elapsed_time(b) / n_e2e, dev)
+        ms_e2e = max_over_ranks(a.elapsed_time(b) / (n_rep * G), dev)
         e2e = {"value": whole_job_rate(Bsz, world, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
 
@@ -612,38 +637,63 @@ def main():
     roofline = {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
     roofline["kernel"] = "swa_fwd_kernel" if dominant is swa_roof else "scan_fwd_kernel"
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers.  Every step
+    # copies its inputs from pinned host memory and reads y and o back; the
+    # steps are pipelined over two device buffer sets and three streams
+    # (copy in, compute, copy out), as a serving loop would run them.
     e2e = None
     if not args.no_e2e:
         host = {k: v.to("cpu").pin_memory() for k, v in inp.items()}
-        dev_in = {k: torch.empty_like(v) for k, v in inp.items()}
         y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
         o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = y_h.numel() * y_h.element_size() + o_h.numel() * o_h.element_size()
-        skw = dict(scan_kw)
-        wkw = dict(swa_kw)
-        for kk in ("x", "delta", "A", "B", "C", "D", "z", "conv_w", "conv_b"):
-            skw[kk] = dev_in[kk]
-        for kk in ("q", "k", "v"):
-            wkw[kk] = dev_in[kk]
+        sets = []
+        for j in range(2):
+            dev_in = inp if j == 0 else {k: torch.empty_like(v) for k, v in inp.items()}
+            y_j = y if j == 0 else torch.empty_like(y)
+            o_j = o if j == 0 else torch.empty_like(o)
+            skw = dict(scan_kw, y=y_j)
+            wkw = dict(swa_kw, o=o_j)
+            for kk in ("x", "delta", "A", "B", "C", "D", "z", "conv_w", "conv_b"):
+                skw[kk] = dev_in[kk]
+            for kk in ("q", "k", "v"):
+                wkw[kk] = dev_in[kk]
+            sets.append({"in": dev_in, "y": y_j, "o": o_j, "skw": skw, "wkw": wkw,
+                         "in_done": torch.cuda.Event(), "comp_done": torch.cuda.Event(),
+                         "out_done": torch.cuda.Event()})
+        s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
-        def e2e_step():
-            for kk in host:
-                dev_in[kk].copy_(host[kk], non_blocking=True)
-            ops.mixer_prefill(skw, wkw)
-            y_h.copy_(y, non_blocking=True)
-            o_h.copy_(o, non_blocking=True)
+        def e2e_step(i):
+            st = sets[i % 2]
+            if i >= 2:
+                s_in.wait_event(st["comp_done"])     # compute of step i-2 has read these inputs
+            with torch.cuda.stream(s_in):
+                for kk in host:
+                    st["in"][kk].copy_(host[kk], non_blocking=True)
+                st["in_done"].record(s_in)
+            s_comp.wait_event(st["in_done"])
+            if i >= 2:
+                s_comp.wait_event(st["out_done"])    # y, o of step i-2 have been read back
+            with torch.cuda.stream(s_comp):
+                ops.mixer_prefill(st["skw"], st["wkw"])
+                st["comp_done"].record(s_comp)
+            s_out.wait_event(st["comp_done"])
+            with torch.cuda.stream(s_out):
+                y_h.copy_(st["y"], non_blocking=True)
+                o_h.copy_(st["o"], non_blocking=True)
+                st["out_done"].record(s_out)
 
-        e2e_step()
+        e2e_step(0)
+        e2e_step(1)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        b.record(stream)
+        a.record(s_in)
+        for i in range(args.e2e_steps):
+            e2e_step(i)
+        b.record(s_out)
         torch.cuda.synchronize()
         ms_e2e = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, dev)
         e2e = {"value": whole_job_rate(Bsz * Ln, world, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
