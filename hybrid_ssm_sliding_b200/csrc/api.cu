@@ -206,6 +206,7 @@ int samba_scan_step(float* h, float* conv_state, const void* x_t, int x_dtype, c
   if (!h || !x_t || !delta_t || !B_t || !C_t || !A || !y_t)
     return fail(SAMBA_ERR_INVALID_ARG, "%s: h, x_t, delta_t, B_t, C_t, A and y_t are required", who);
   if (batch < 1 || dim < 1) return fail(SAMBA_ERR_INVALID_ARG, "%s: bad shape", who);
+  if (batch > 65535) return fail(SAMBA_ERR_UNSUPPORTED, "%s: batch above 65535", who);
   if (dstate != 4 && dstate != 8 && dstate != 16) return fail(SAMBA_ERR_UNSUPPORTED, "%s: dstate", who);
   if (dconv < 2 || dconv > 4) return fail(SAMBA_ERR_UNSUPPORTED, "%s: dconv must be 2..4", who);
   if (!dtype_ok(x_dtype) || !dtype_ok(y_dtype) || (z_t && !dtype_ok(z_dtype)))

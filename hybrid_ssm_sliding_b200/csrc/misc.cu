@@ -93,27 +93,36 @@ int launch_conv1d(const void* x, int x_dtype, const float* w, const float* bias,
 }
 
 // -------------------------------------------------------------- scan step
-// One thread per (batch, channel) holding its N states.  Same arithmetic as
-// the prefill kernel with L = 1.
+// Four threads per (batch, channel), each holding N/4 of its states (one
+// channel per aligned group of four lanes); the C·h partials meet through two
+// shuffles.  Same arithmetic as the prefill kernel with L = 1.
 template <int N, typename XT, typename YT>
-__global__ void scan_step_kernel(float* __restrict__ h, float* __restrict__ cs, const XT* __restrict__ x_t,
-                                 const XT* __restrict__ z_t, const float* __restrict__ delta_t,
-                                 const float* __restrict__ B_t, const float* __restrict__ C_t,
-                                 const float* __restrict__ A, const float* __restrict__ Dskip,
-                                 const float* __restrict__ conv_w, const float* __restrict__ conv_b,
-                                 YT* __restrict__ y_t, int64_t Bsz, int64_t D, int K, uint32_t flags) {
-  const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (e >= Bsz * D) return;
-  const int64_t b = e / D, c = e % D;
+__global__ void __launch_bounds__(256) scan_step_kernel(
+    float* __restrict__ h, float* __restrict__ cs, const XT* __restrict__ x_t, const XT* __restrict__ z_t,
+    const float* __restrict__ delta_t, const float* __restrict__ B_t, const float* __restrict__ C_t,
+    const float* __restrict__ A, const float* __restrict__ Dskip, const float* __restrict__ conv_w,
+    const float* __restrict__ conv_b, YT* __restrict__ y_t, int64_t D, int K, uint32_t flags) {
+  constexpr int TPC = 4, NS = N / TPC;
+  const int64_t b = blockIdx.y;
+  const int64_t c = (int64_t)blockIdx.x * (blockDim.x / TPC) + threadIdx.x / TPC;
+  const int j = threadIdx.x % TPC;
+  if (c >= D) return;  // whole groups of four leave together
+  const unsigned gmask = 0xFu << (threadIdx.x & 28);
+  const int64_t e = b * D + c;
   const float xv = to_f32<XT>(x_t[e]);
   float u;
   if (flags & SAMBA_SCAN_FUSE_CONV) {
     float* st = cs + e * (K - 1);
+    float sv[8];
+    for (int k = 0; k < K - 1; ++k) sv[k] = st[k];
     float acc = conv_b ? conv_b[c] : 0.f;
-    for (int k = 0; k < K - 1; ++k) acc = fmaf(conv_w[c * K + k], st[k], acc);
+    for (int k = 0; k < K - 1; ++k) acc = fmaf(conv_w[c * K + k], sv[k], acc);
     acc = fmaf(conv_w[c * K + K - 1], xv, acc);
-    for (int k = 0; k + 1 < K - 1; ++k) st[k] = st[k + 1];
-    st[K - 2] = xv;
+    __syncwarp(gmask);  // every thread of the group has read the old state
+    if (j == 0) {
+      for (int k = 0; k + 1 < K - 1; ++k) st[k] = sv[k + 1];
+      st[K - 2] = xv;
+    }
     u = (flags & SAMBA_SCAN_CONV_SILU) ? silu_dev(acc) : acc;
   } else {
     u = xv;
@@ -121,31 +130,28 @@ __global__ void scan_step_kernel(float* __restrict__ h, float* __restrict__ cs, 
   const float wr = delta_t[e];
   const float dlt = (flags & SAMBA_SCAN_DELTA_SOFTPLUS) ? softplus_dev(wr) : wr;
   const float du = dlt * u;
-  float* hp = h + e * N;
-  const float* Ap = A + c * N;
-  const float* Bp = B_t + b * N;
-  const float* Cp = C_t + b * N;
-  float acc = 0.f;
+  float* hp = h + e * N + j * NS;
+  const float* Ap = A + c * N + j * NS;
+  const float* Bp = B_t + b * N + j * NS;
+  const float* Cp = C_t + b * N + j * NS;
+  constexpr float kLog2e = 1.4426950408889634f;
+  float hv[NS], acc = 0.f;
 #pragma unroll
-  for (int n = 0; n < N; n += 4) {
-    float4 hv = *reinterpret_cast<float4*>(hp + n);
-    const float4 av = *reinterpret_cast<const float4*>(Ap + n);
-    const float4 bv = *reinterpret_cast<const float4*>(Bp + n);
-    const float4 cv = *reinterpret_cast<const float4*>(Cp + n);
-    constexpr float kLog2e = 1.4426950408889634f;
-    hv.x = fmaf(ex2_approx(dlt * (av.x * kLog2e)), hv.x, du * bv.x);
-    hv.y = fmaf(ex2_approx(dlt * (av.y * kLog2e)), hv.y, du * bv.y);
-    hv.z = fmaf(ex2_approx(dlt * (av.z * kLog2e)), hv.z, du * bv.z);
-    hv.w = fmaf(ex2_approx(dlt * (av.w * kLog2e)), hv.w, du * bv.w);
-    acc = fmaf(cv.x, hv.x, acc);
-    acc = fmaf(cv.y, hv.y, acc);
-    acc = fmaf(cv.z, hv.z, acc);
-    acc = fmaf(cv.w, hv.w, acc);
-    *reinterpret_cast<float4*>(hp + n) = hv;
+  for (int n = 0; n < NS; ++n) hv[n] = hp[n];
+#pragma unroll
+  for (int n = 0; n < NS; ++n) {
+    hv[n] = fmaf(ex2_approx(dlt * (Ap[n] * kLog2e)), hv[n], du * Bp[n]);
+    acc = fmaf(Cp[n], hv[n], acc);
   }
-  float yv = acc + (Dskip ? Dskip[c] * u : 0.f);
-  if (z_t) yv *= silu_dev(to_f32<XT>(z_t[e]));
-  y_t[e] = from_f32<YT>(yv);
+#pragma unroll
+  for (int n = 0; n < NS; ++n) hp[n] = hv[n];
+  acc += __shfl_xor_sync(gmask, acc, 1);
+  acc += __shfl_xor_sync(gmask, acc, 2);
+  if (j == 0) {
+    float yv = acc + (Dskip ? Dskip[c] * u : 0.f);
+    if (z_t) yv *= silu_dev(to_f32<XT>(z_t[e]));
+    y_t[e] = from_f32<YT>(yv);
+  }
 }
 
 template <int N, typename XT, typename YT>
@@ -153,10 +159,10 @@ static void scan_step_go(float* h, float* cs, const void* x_t, const void* z_t, 
                          const float* C_t, const float* A, const float* Dskip, const float* conv_w,
                          const float* conv_b, void* y_t, int64_t B, int64_t D, int K, uint32_t flags,
                          cudaStream_t s) {
-  const int64_t n = B * D;
-  scan_step_kernel<N, XT, YT><<<(unsigned)((n + 127) / 128), 128, 0, s>>>(
+  const dim3 grid((unsigned)((D + 63) / 64), (unsigned)B);
+  scan_step_kernel<N, XT, YT><<<grid, 256, 0, s>>>(
       h, cs, reinterpret_cast<const XT*>(x_t), reinterpret_cast<const XT*>(z_t), delta_t, B_t, C_t, A, Dskip, conv_w,
-      conv_b, reinterpret_cast<YT*>(y_t), B, D, K, flags);
+      conv_b, reinterpret_cast<YT*>(y_t), D, K, flags);
 }
 
 template <int N>

@@ -193,6 +193,7 @@ int samba_mixer_prefill(const samba_scan_args* scan, const samba_swa_args* swa,
  *                          [D, K], conv_b [D] (or NULL) as in the prefill
  *   y_t        [B, D]      y_dtype
  * flags: as samba_scan_args.flags (FUSE_CONV requires conv_state and conv_w).
+ * B <= 65535 (SAMBA_ERR_UNSUPPORTED beyond); N in {4, 8, 16}; K in 2..4.
  */
 int samba_scan_step(float* h, float* conv_state, const void* x_t, int x_dtype, const void* z_t,
                     int z_dtype, const float* delta_t, const float* B_t, const float* C_t,

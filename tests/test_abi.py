@@ -115,6 +115,8 @@ def test_decode_rejects_bad_arguments_on_host(lib):
                                None) == L.SAMBA_ERR_INVALID_ARG
     assert lib.samba_scan_step(f, None, f, 1, None, 1, f, f, f, f, None, None, None, f, 1, 1, 8, 16, 4,
                                L.SCAN_FUSE_CONV, None) == L.SAMBA_ERR_INVALID_ARG
+    assert lib.samba_scan_step(f, None, f, 1, None, 1, f, f, f, f, None, None, None, f, 1, 70000, 8, 16, 4, 0,
+                               None) == L.SAMBA_ERR_UNSUPPORTED  # batch above 65535
     assert lib.samba_swa_ring_fill(f, f, 8, f, f, None, 1, 4, 64, 16, None) == L.SAMBA_ERR_INVALID_ARG
     assert lib.samba_swa_ring_fill(f, f, 8, f, f, f, 1, 4, 80, 16, None) == L.SAMBA_ERR_UNSUPPORTED
     need = lib.samba_swa_step_workspace_size(16, 32, 64, 2048)
