@@ -230,13 +230,31 @@ int launch_ring_fill(const void* k, const void* v, int64_t L, void* k_ring, void
 // (max, sum, unnormalised output) per head; a second kernel combines the
 // splits.  The newest position is read from k_t/v_t, which split 0 also
 // stores into its ring slot (that slot held a position outside the window, so
-// no other CTA reads it in this step).  Thread i of a CTA owns position i of
-// its chunk: it loads that position's K row into registers and its V row into
-// shared memory in one burst (all rows of the chunk in flight at once), so
-// the P·V loop runs from shared memory.
+// no other CTA reads it in this step).  Thread i of a CTA loads the K and V
+// rows of position i of its chunk into shared memory in one burst (all rows
+// of the chunk in flight at once); the scores K·qᵀ (positions x heads) and
+// the outputs P·V (heads x head dim) are bf16 tensor-core products
+// (mma m16n8k16, fp32 accumulate), P rounded to bf16 as in the prefill.
 template <int HD> struct StepCfg {
   static constexpr int CH = HD <= 64 ? 128 : 64;  // positions per CTA (= threads)
+  static constexpr int NWARP = CH / 32;
+  static constexpr int KP = HD + 8;                // row pitch of K, V, q in bf16 (conflict-free fragments)
+  static constexpr int PP = CH + 8;                // row pitch of P in bf16
+  // shared memory: V, then K + q during the scores, reused for scores + P
+  static constexpr int V_BYTES = CH * KP * 2;
+  static constexpr int KQ_BYTES = CH * KP * 2 + 16 * KP * 2;
+  static constexpr int SP_BYTES = 16 * CH * 4 + 16 * PP * 2;
+  static constexpr int SMEM = V_BYTES + (KQ_BYTES > SP_BYTES ? KQ_BYTES : SP_BYTES);
 };
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 
 template <int HD>
 __global__ void __launch_bounds__(StepCfg<HD>::CH) swa_step_split_kernel(
@@ -244,9 +262,8 @@ __global__ void __launch_bounds__(StepCfg<HD>::CH) swa_step_split_kernel(
     const __nv_bfloat16* __restrict__ v_t, __nv_bfloat16* __restrict__ k_ring, __nv_bfloat16* __restrict__ v_ring,
     const int64_t* __restrict__ pos, float* __restrict__ ws, int Hq, int Hkv, int64_t W, float scale_log2,
     int nsplit) {
-  constexpr int CH = StepCfg<HD>::CH;
-  constexpr int NW = CH / 32;       // warps
-  constexpr int PAIRS = HD / 2;
+  using Cfg = StepCfg<HD>;
+  constexpr int CH = Cfg::CH, NWARP = Cfg::NWARP, KP = Cfg::KP, PP = Cfg::PP;
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int group = Hq / Hkv;  // <= 16
   const int64_t p = pos[b];
@@ -257,14 +274,17 @@ __global__ void __launch_bounds__(StepCfg<HD>::CH) swa_step_split_kernel(
   const int n_here = (int)(p - a0 + 1 < CH ? (p - a0 + 1 > 0 ? p - a0 + 1 : 0) : CH);
   const int slot0 = (int)(a0 % W);
   const int Wi = (int)W;
-  __shared__ float qs[16][HD];
-  __shared__ float sc[16][CH];
-  __shared__ __align__(16) __nv_bfloat162 vs[CH][PAIRS];
+  __shared__ __align__(16) unsigned char sm[Cfg::SMEM];
+  __nv_bfloat16* Vs = reinterpret_cast<__nv_bfloat16*>(sm);                              // [CH][KP]
+  __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(sm + Cfg::V_BYTES);               // [CH][KP]
+  __nv_bfloat16* Qs = Ks + CH * KP;                                                       // [16][KP]
+  float* Sc = reinterpret_cast<float*>(sm + Cfg::V_BYTES);                                // [16][CH] (after K)
+  __nv_bfloat16* Ps = reinterpret_cast<__nv_bfloat16*>(sm + Cfg::V_BYTES + 16 * CH * 4);  // [16][PP]
   __shared__ float red_m[16], red_l[16];
 
-  const int tid = threadIdx.x;
-  // this thread's position: K row to registers, V row to shared memory
-  uint4 kraw[HD / 8];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gq = lane >> 2, tq = lane & 3;  // mma fragment coordinates
+  // this thread's position: K and V rows to shared memory (zeros past the window)
   {
     const bool valid = tid < n_here;
     int slot = slot0 + tid;
@@ -274,18 +294,22 @@ __global__ void __launch_bounds__(StepCfg<HD>::CH) swa_step_split_kernel(
     const int64_t noff = ((int64_t)b * Hkv + g) * HD;
     const uint4* krow = reinterpret_cast<const uint4*>(is_new ? k_t + noff : k_ring + roff);
     const uint4* vrow = reinterpret_cast<const uint4*>(is_new ? v_t + noff : v_ring + roff);
-    uint4 vraw[HD / 8];
+    uint4 kraw[HD / 8], vraw[HD / 8];
 #pragma unroll
     for (int c = 0; c < HD / 8; ++c) {
       kraw[c] = valid ? krow[c] : make_uint4(0u, 0u, 0u, 0u);
       vraw[c] = valid ? vrow[c] : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int c = 0; c < HD / 8; ++c) reinterpret_cast<uint4*>(&vs[tid][0])[c] = vraw[c];
+    for (int c = 0; c < HD / 8; ++c) {
+      reinterpret_cast<uint4*>(Ks + tid * KP)[c] = kraw[c];
+      reinterpret_cast<uint4*>(Vs + tid * KP)[c] = vraw[c];
+    }
   }
-  for (int i = tid; i < group * HD; i += CH) {
+  // the group's query rows (rows past the group are zero)
+  for (int i = tid; i < 16 * HD; i += CH) {
     const int hh = i / HD, dd = i % HD;
-    qs[hh][dd] = __bfloat162float(q_t[((int64_t)b * Hq + g * group + hh) * HD + dd]);
+    Qs[hh * KP + dd] = hh < group ? q_t[((int64_t)b * Hq + g * group + hh) * HD + dd] : __float2bfloat16_rn(0.f);
   }
   if (split == 0) {  // store the new key/value into its slot
     const int64_t slot = p % W;
@@ -296,42 +320,63 @@ __global__ void __launch_bounds__(StepCfg<HD>::CH) swa_step_split_kernel(
   }
   __syncthreads();
 
-  // scores of this thread's position for every head of the group
-  {
-    float kv[HD];
+  // scores: warp w takes positions [32w, 32w + 32) (two m16 tiles) against
+  // the 16 (zero-padded) head rows (two n8 tiles), k over the head dim
+  float sacc[2][2][4];
 #pragma unroll
-    for (int c = 0; c < HD / 8; ++c) {
-      const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&kraw[c]);
+  for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = __bfloat1622float2(pr[q]);
-        kv[8 * c + 2 * q] = f.x;
-        kv[8 * c + 2 * q + 1] = f.y;
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[mt][nt][e] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < HD / 16; ++ks) {
+    const int kc = 16 * ks + 2 * tq;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      const int r0 = 32 * warp + 16 * mt + gq;
+      const uint32_t a0r = *reinterpret_cast<const uint32_t*>(Ks + r0 * KP + kc);
+      const uint32_t a1r = *reinterpret_cast<const uint32_t*>(Ks + (r0 + 8) * KP + kc);
+      const uint32_t a2r = *reinterpret_cast<const uint32_t*>(Ks + r0 * KP + kc + 8);
+      const uint32_t a3r = *reinterpret_cast<const uint32_t*>(Ks + (r0 + 8) * KP + kc + 8);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int n = 8 * nt + gq;
+        const uint32_t b0r = *reinterpret_cast<const uint32_t*>(Qs + n * KP + kc);
+        const uint32_t b1r = *reinterpret_cast<const uint32_t*>(Qs + n * KP + kc + 8);
+        mma_bf16_16816(sacc[mt][nt], a0r, a1r, a2r, a3r, b0r, b1r);
       }
     }
-    const bool valid = tid < n_here;
-    for (int hh = 0; hh < group; ++hh) {
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};  // four short chains instead of one of length HD
-#pragma unroll
-      for (int dd = 0; dd < HD; ++dd) s4[dd & 3] = fmaf(qs[hh][dd], kv[dd], s4[dd & 3]);
-      const float s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      sc[hh][tid] = valid ? s * scale_log2 : -INFINITY;
-    }
   }
+  __syncthreads();  // K and q are read: their space now holds the scores and P
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int row = 32 * warp + 16 * mt + gq + (e >= 2 ? 8 : 0);  // position
+        const int col = 8 * nt + 2 * tq + (e & 1);                      // head
+        Sc[col * CH + row] = row < n_here ? sacc[mt][nt][e] * scale_log2 : -INFINITY;
+      }
   __syncthreads();
-  // per head max and exp-sum (one warp per head, heads strided over the warps)
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int hh = warp; hh < group; hh += NW) {
+  // per head max and exp-sum (one warp per head, heads strided over the
+  // warps); P in bf16, rows past the group zero
+  for (int hh = warp; hh < 16; hh += NWARP) {
+    if (hh >= group) {
+      for (int i = lane; i < CH; i += 32) Ps[hh * PP + i] = __float2bfloat16_rn(0.f);
+      continue;
+    }
     float m = -INFINITY;
-    for (int i = lane; i < CH; i += 32) m = fmaxf(m, sc[hh][i]);
+    for (int i = lane; i < CH; i += 32) m = fmaxf(m, Sc[hh * CH + i]);
 #pragma unroll
     for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     const float mu = (m == -INFINITY) ? 0.f : m;
     float l = 0.f;
     for (int i = lane; i < CH; i += 32) {
-      const float e = ex2_approx(sc[hh][i] - mu);
-      sc[hh][i] = e;
-      l += e;
+      const __nv_bfloat16 e = __float2bfloat16_rn(ex2_approx(Sc[hh * CH + i] - mu));
+      Ps[hh * PP + i] = e;
+      l += __bfloat162float(e);  // the sum of the probabilities P·V uses
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
@@ -341,28 +386,34 @@ __global__ void __launch_bounds__(StepCfg<HD>::CH) swa_step_split_kernel(
     }
   }
   __syncthreads();
-  // partial outputs: job = (head, dim pair); V from shared memory (invalid
-  // positions hold zeros and zero probabilities)
-  for (int job = tid; job < group * PAIRS; job += CH) {
-    const int hh = job / PAIRS, dp = job % PAIRS;
-    float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
-    const int n4 = (n_here + 3) & ~3;
-#pragma unroll 4
-    for (int i = 0; i < n4; i += 2) {
-      const float2 va = __bfloat1622float2(vs[i][dp]);
-      const float2 vb = __bfloat1622float2(vs[i + 1][dp]);
-      const float pa = sc[hh][i], pb = sc[hh][i + 1];
-      o0 = fmaf(pa, va.x, o0);
-      o1 = fmaf(pa, va.y, o1);
-      o2 = fmaf(pb, vb.x, o2);
-      o3 = fmaf(pb, vb.y, o3);
+  // outputs: heads (m16) x head dim (n8 tiles over the warps), k over positions
+  for (int nt = warp; nt < HD / 8; nt += NWARP) {
+    float oacc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int n = 8 * nt + gq;  // head-dim column of the B fragment
+#pragma unroll
+    for (int ks = 0; ks < CH / 16; ++ks) {
+      const int kc = 16 * ks + 2 * tq;
+      const uint32_t a0r = *reinterpret_cast<const uint32_t*>(Ps + gq * PP + kc);
+      const uint32_t a1r = *reinterpret_cast<const uint32_t*>(Ps + (gq + 8) * PP + kc);
+      const uint32_t a2r = *reinterpret_cast<const uint32_t*>(Ps + gq * PP + kc + 8);
+      const uint32_t a3r = *reinterpret_cast<const uint32_t*>(Ps + (gq + 8) * PP + kc + 8);
+      const unsigned short* vb = reinterpret_cast<const unsigned short*>(Vs);
+      const uint32_t b0r = (uint32_t)vb[kc * KP + n] | ((uint32_t)vb[(kc + 1) * KP + n] << 16);
+      const uint32_t b1r = (uint32_t)vb[(kc + 8) * KP + n] | ((uint32_t)vb[(kc + 9) * KP + n] << 16);
+      mma_bf16_16816(oacc, a0r, a1r, a2r, a3r, b0r, b1r);
     }
-    float* dst = ws + ((((int64_t)b * Hq + g * group + hh) * nsplit + split) * (HD + 2));
-    dst[2 + 2 * dp] = o0 + o2;
-    dst[2 + 2 * dp + 1] = o1 + o3;
-    if (dp == 0) {
-      dst[0] = red_m[hh];
-      dst[1] = red_l[hh];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int hh = gq + (e >= 2 ? 8 : 0);
+      const int dd = 8 * nt + 2 * tq + (e & 1);
+      if (hh < group) {
+        float* dst = ws + ((((int64_t)b * Hq + g * group + hh) * nsplit + split) * (HD + 2));
+        dst[2 + dd] = oacc[e];
+        if (dd == 0) {
+          dst[0] = red_m[hh];
+          dst[1] = red_l[hh];
+        }
+      }
     }
   }
 }

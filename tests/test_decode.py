@@ -77,7 +77,7 @@ def test_prefill_then_scan_steps_match_oracle(dt, N):
 
 # ------------------------------------------------------------------ SWA step
 @pytest.mark.parametrize("L1,W,Hq,Hkv,d", [(10, 16, 8, 2, 64), (40, 16, 4, 4, 32), (300, 256, 32, 4, 64),
-                                           (1, 700, 8, 1, 64), (600, 300, 16, 1, 16)])
+                                           (1, 700, 8, 1, 64), (600, 300, 16, 1, 16), (200, 150, 8, 2, 128)])
 def test_ring_fill_then_swa_steps_match_oracle(L1, W, Hq, Hkv, d):
     Bsz, steps = 2, 24
     g = torch.Generator(device="cuda")
