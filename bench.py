@@ -147,6 +147,33 @@ def swa_exact_band_flops(wl):
     return 4.0 * pairs * wl.head_dim * wl.batch * wl.heads_q
 
 
+# Special-function (MUFU) work.  The SM's MUFU pipe evaluates 16 ex2 / rcp /
+# lg2 per clock (measured on B200 with a dependent-free ex2 loop), so the peak
+# is 16 x SMs x the SM clock sampled during the run.
+MUFU_PER_CLK_SM = 16
+
+
+def scan_mufu_ops(wl):
+    """Special-function operations per (token, channel) of the fused scan:
+    one exp per state for exp(Δ A), exp and reciprocal for the conv SiLU,
+    exp and reciprocal for softplus(delta), exp and reciprocal for the silu(z)
+    gate."""
+    return wl.batch * wl.seqlen * wl.dim * (wl.dstate + 6)
+
+
+def swa_exps(wl):
+    """One exp per (query, key) pair of the band per query head."""
+    return swa_exact_band_flops(wl) / (4.0 * wl.head_dim)
+
+
+def mufu_roof(ops_count, ms, sms, sm_mhz):
+    """Special-function operations per second against the MUFU peak."""
+    achieved = ops_count / (ms / 1e3) / 1e12
+    peak = MUFU_PER_CLK_SM * sms * sm_mhz * 1e6 / 1e12
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tops/s", "frac": achieved / peak,
+            "ops": ops_count, "sms": sms, "sm_mhz": sm_mhz}
+
+
 # ----------------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples nvidia-smi clocks and throttle reasons while running."""
@@ -623,6 +650,10 @@ def main():
     swa_roof = {"bound": "tensor", "achieved": swa_tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": swa_tfs / peaks["bf16_tflops"], "traffic": None, "ms": ms_swa, "band_flops": sf,
                 "exact_band_flops": swa_exact_band_flops(wl), "peak_source": peaks["source"] + " burst"}
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = (clk or {}).get("sm_mhz") or (clk or {}).get("sm_max_mhz") or 1965.0
+    scan_roof["mufu"] = mufu_roof(scan_mufu_ops(wl), ms_scan, sms, mhz)
+    swa_roof["mufu"] = mufu_roof(swa_exps(wl), ms_swa, sms, mhz)
     traffic_file = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(traffic_file):
         try:

@@ -1,0 +1,52 @@
+"""The algorithmic work bench.py divides by: band pairs, exps, MUFU operations
+and bytes, counted here by brute force on small shapes (CPU only)."""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import bench
+from hybrid_ssm_sliding_b200.workloads import WORKLOADS
+
+
+def _band_pairs(L, W):
+    i = np.arange(L)[:, None]
+    j = np.arange(L)[None, :]
+    return int(((i - j >= 0) & (i - j < W)).sum())
+
+
+@pytest.mark.parametrize("L,W", [(64, 16), (10, 16), (16, 16), (33, 1), (200, 64)])
+def test_exact_band_flops_counts_the_causal_window(L, W):
+    wl = dataclasses.replace(WORKLOADS["tiny"], seqlen=L, window=W, batch=3, heads_q=5, head_dim=16)
+    pairs = _band_pairs(L, W)
+    assert bench.swa_exact_band_flops(wl) == 4.0 * pairs * 16 * 3 * 5
+    assert bench.swa_exps(wl) == pairs * 3 * 5
+
+
+def test_band_flops_upper_bound():
+    wl = WORKLOADS["prefill_128k"]
+    # 4·L·W·d per (batch, head) counts W keys for every query, including the
+    # first W-1 queries that see fewer; the exact band is W²/2-ish smaller.
+    exact = bench.swa_exact_band_flops(wl)
+    nominal = bench.swa_flops(wl)
+    W, L = wl.window, wl.seqlen
+    assert nominal - exact == 4.0 * (W * (W - 1) // 2) * wl.head_dim * wl.batch * wl.heads_q
+    assert exact < nominal
+
+
+def test_scan_counts():
+    wl = dataclasses.replace(WORKLOADS["tiny"], batch=2, seqlen=7, dim=5, dstate=4)
+    tc = 2 * 7 * 5
+    assert bench.scan_mufu_ops(wl) == tc * (4 + 6)
+    # 10 bytes per (token, channel), 2·N·4 per token for B and C, and the
+    # per-channel state and parameters
+    small = 2 * 5 * (4 + 3) * 4 + 5 * (4 + 4 + 2) * 4
+    assert bench.scan_bytes(wl) == tc * 10 + 2 * 7 * 2 * 4 * 4 + small
+
+
+def test_mufu_roof_arithmetic():
+    r = bench.mufu_roof(ops_count=2.0e12, ms=1000.0, sms=148, sm_mhz=1965.0)
+    assert r["achieved"] == pytest.approx(2.0)
+    assert r["peak"] == pytest.approx(16 * 148 * 1.965e9 / 1e12)
+    assert r["frac"] == pytest.approx(2.0 / r["peak"])
+    assert r["bound"] == "alu"
