@@ -78,8 +78,16 @@ constexpr int kScanCB = 32;     // channels in one TMA box (>= CU + alignment of
 #define SAMBA_SCAN_T 32
 #endif
 constexpr int kScanT = SAMBA_SCAN_T;  // tokens per tile
-constexpr int kScanPro = 8;     // prologue warps
-constexpr int kScanEpi = 4;     // epilogue warps
+// Prologue and epilogue warps (each a divisor of the tile's tokens).  Fixed by
+// measurement: 4 prologue or 2 epilogue warps were slower, and so were 16
+// prologue warps (fewer registers per thread).
+#ifndef SAMBA_SCAN_PRO
+#define SAMBA_SCAN_PRO 8
+#endif
+#ifndef SAMBA_SCAN_EPI
+#define SAMBA_SCAN_EPI 8
+#endif
+constexpr int kScanPro = SAMBA_SCAN_PRO;  // prologue warps
 // Upper bound on the block size (sets the register budget per thread).
 #ifndef SAMBA_SCAN_MAXTHREADS
 #define SAMBA_SCAN_MAXTHREADS 672
@@ -89,11 +97,17 @@ constexpr int kScanEpi = 4;     // epilogue warps
 #define SAMBA_SCAN_GROUP 4
 #endif
 #ifndef SAMBA_SCAN_SLOTS
-#define SAMBA_SCAN_SLOTS 3
+#define SAMBA_SCAN_SLOTS 4
 #endif
 
 constexpr int kScanSlots = SAMBA_SCAN_SLOTS;  // depth of the prologue -> scan -> epilogue hand-off
 constexpr int kScanSmemBudget = 227 * 1024;
+// Epilogue warps: SAMBA_SCAN_EPI, or 4 where that would take a block with gl
+// scan warps past SAMBA_SCAN_MAXTHREADS (8 scan warps at N = 8).
+__host__ __device__ constexpr int scan_epi_warps(int gl) {
+  return (gl + kScanPro + SAMBA_SCAN_EPI + 1) * 32 <= SAMBA_SCAN_MAXTHREADS ? SAMBA_SCAN_EPI : 4;
+}
+static_assert((8 + kScanPro + 4 + 1) * 32 <= SAMBA_SCAN_MAXTHREADS, "scan block exceeds SAMBA_SCAN_MAXTHREADS");
 
 template <int N, typename XT>
 struct ScanLayout {
@@ -190,7 +204,7 @@ __device__ __forceinline__ float softplus_fast(float w) {
 
 // ------------------------------------------------------------------ kernel
 // Warp roles (index ranges): [0, NSW) scan, then kScanPro prologue, then
-// kScanEpi epilogue, then one TMA producer.  Per tile i (slot k = i % SLOTS):
+// EPIW epilogue, then one TMA producer.  Per tile i (slot k = i % SLOTS):
 //   producer : full[s] <- TMA of x, z, delta, B, C          (waits empty[s])
 //   prologue : XCH[k], EPI[k] <- conv/softplus, D·u, z; arrives pro_full[k]
 //              (waits full[s]; scan_done[k] and epi_done[k] of tile i-SLOTS)
@@ -220,8 +234,8 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
   float* PART = reinterpret_cast<float*>(smem + Ly::PART_OFF);
 
   const int CU = p.CU;
-  constexpr int NSW = scan_warps(GL);
-  const int PRO0 = NSW, EPI0 = NSW + kScanPro, PROD = NSW + kScanPro + kScanEpi;
+  constexpr int NSW = scan_warps(GL), EPIW = scan_epi_warps(GL);
+  const int PRO0 = NSW, EPI0 = NSW + kScanPro, PROD = NSW + kScanPro + EPIW;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
   const int c_start = blockIdx.x * CU;
@@ -238,7 +252,7 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
     for (int k = 0; k < SLOTS; ++k) {
       mbar_init(&pro_full[k], kScanPro);
       mbar_init(&scan_done[k], NSW);
-      mbar_init(&epi_done[k], kScanEpi);
+      mbar_init(&epi_done[k], EPIW);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -279,7 +293,7 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
   if (warp >= EPI0) {
     // ============================================================ epilogue
     // Thread (eg, cl): channel cl (lane), tokens [eg·TPE, (eg+1)·TPE) of every tile.
-    constexpr int TPE = T / kScanEpi;
+    constexpr int TPE = T / EPIW;
     const int cl = lane, eg = warp - EPI0;
     const int64_t c = c_start + cl;
     const bool cval = cl < CU && c < p.D;
@@ -655,7 +669,10 @@ static int launch_scan_t(const samba_scan_args& a, cudaStream_t stream) {
   p.fuse_conv = (a.flags & SAMBA_SCAN_FUSE_CONV) != 0;
   p.conv_silu = (a.flags & SAMBA_SCAN_CONV_SILU) != 0;
   p.softplus = (a.flags & SAMBA_SCAN_DELTA_SOFTPLUS) != 0;
-  const int threads = (scan_warps(ScanShape<N>::GL) + kScanPro + kScanEpi + 1) * 32;
+  constexpr int GLN = ScanShape<N>::GL;
+  const int threads = (scan_warps(GLN) + kScanPro + scan_epi_warps(GLN) + 1) * 32;
+  static_assert((scan_warps(GLN) + kScanPro + scan_epi_warps(GLN) + 1) * 32 <= SAMBA_SCAN_MAXTHREADS,
+                "scan block exceeds SAMBA_SCAN_MAXTHREADS");
   dim3 grid((unsigned)((D + CU - 1) / CU), (unsigned)Bsz);
   kern<<<grid, threads, Ly::SMEM, stream>>>(mx, mz, mw, mb, mc, p);
   return check_launch("samba_selective_scan_fwd");
