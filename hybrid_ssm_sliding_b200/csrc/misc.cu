@@ -95,7 +95,35 @@ int launch_conv1d(const void* x, int x_dtype, const float* w, const float* bias,
 // -------------------------------------------------------------- scan step
 // Four threads per (batch, channel), each holding N/4 of its states (one
 // channel per aligned group of four lanes); the C·h partials meet through two
-// shuffles.  Same arithmetic as the prefill kernel with L = 1.
+// shuffles.  Same arithmetic as the prefill kernel with L = 1.  Every load
+// that does not depend on another is issued first (state, A, B, C as vectors;
+// conv taps and state for K <= 4 in registers), so that one round trip to
+// memory covers them all.
+template <int NS>
+__device__ __forceinline__ void ld_states(float (&v)[NS], const float* p) {
+  if constexpr (NS == 4) {
+    const float4 t = *reinterpret_cast<const float4*>(p);
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  } else if constexpr (NS == 2) {
+    const float2 t = *reinterpret_cast<const float2*>(p);
+    v[0] = t.x; v[1] = t.y;
+  } else {
+#pragma unroll
+    for (int n = 0; n < NS; ++n) v[n] = p[n];
+  }
+}
+template <int NS>
+__device__ __forceinline__ void st_states(float* p, const float (&v)[NS]) {
+  if constexpr (NS == 4) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  } else if constexpr (NS == 2) {
+    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  } else {
+#pragma unroll
+    for (int n = 0; n < NS; ++n) p[n] = v[n];
+  }
+}
+
 template <int N, typename XT, typename YT>
 __global__ void __launch_bounds__(256) scan_step_kernel(
     float* __restrict__ h, float* __restrict__ cs, const XT* __restrict__ x_t, const XT* __restrict__ z_t,
@@ -109,47 +137,64 @@ __global__ void __launch_bounds__(256) scan_step_kernel(
   if (c >= D) return;  // whole groups of four leave together
   const unsigned gmask = 0xFu << (threadIdx.x & 28);
   const int64_t e = b * D + c;
+  const bool fuse = (flags & SAMBA_SCAN_FUSE_CONV) != 0;
+  // ---- loads
   const float xv = to_f32<XT>(x_t[e]);
+  const float wr = delta_t[e];
+  float hv[NS], av[NS], bv[NS], cv[NS];
+  float* hp = h + e * N + j * NS;
+  ld_states<NS>(hv, hp);
+  ld_states<NS>(av, A + c * N + j * NS);
+  ld_states<NS>(bv, B_t + b * N + j * NS);
+  ld_states<NS>(cv, C_t + b * N + j * NS);
+  float* st = cs + e * (K - 1);
+  float sv[3] = {0.f, 0.f, 0.f}, cw[3] = {0.f, 0.f, 0.f}, wlast = 0.f, cbias = 0.f;
+  if (fuse) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+      if (k < K - 1) {
+        sv[k] = st[k];
+        cw[k] = conv_w[c * K + k];
+      }
+    wlast = conv_w[c * K + K - 1];
+    if (conv_b) cbias = conv_b[c];
+  }
+  const float zv = (z_t && j == 0) ? to_f32<XT>(z_t[e]) : 0.f;
+  const float dsk = (Dskip && j == 0) ? Dskip[c] : 0.f;
+  // ---- conv and the state shift
   float u;
-  if (flags & SAMBA_SCAN_FUSE_CONV) {
-    float* st = cs + e * (K - 1);
-    float sv[8];
-    for (int k = 0; k < K - 1; ++k) sv[k] = st[k];
-    float acc = conv_b ? conv_b[c] : 0.f;
-    for (int k = 0; k < K - 1; ++k) acc = fmaf(conv_w[c * K + k], sv[k], acc);
-    acc = fmaf(conv_w[c * K + K - 1], xv, acc);
+  if (fuse) {
+    float acc = cbias;
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+      if (k < K - 1) acc = fmaf(cw[k], sv[k], acc);
+    acc = fmaf(wlast, xv, acc);
     __syncwarp(gmask);  // every thread of the group has read the old state
     if (j == 0) {
-      for (int k = 0; k + 1 < K - 1; ++k) st[k] = sv[k + 1];
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        if (k + 1 < K - 1) st[k] = sv[k + 1];
       st[K - 2] = xv;
     }
     u = (flags & SAMBA_SCAN_CONV_SILU) ? silu_dev(acc) : acc;
   } else {
     u = xv;
   }
-  const float wr = delta_t[e];
   const float dlt = (flags & SAMBA_SCAN_DELTA_SOFTPLUS) ? softplus_dev(wr) : wr;
   const float du = dlt * u;
-  float* hp = h + e * N + j * NS;
-  const float* Ap = A + c * N + j * NS;
-  const float* Bp = B_t + b * N + j * NS;
-  const float* Cp = C_t + b * N + j * NS;
   constexpr float kLog2e = 1.4426950408889634f;
-  float hv[NS], acc = 0.f;
-#pragma unroll
-  for (int n = 0; n < NS; ++n) hv[n] = hp[n];
+  float acc = 0.f;
 #pragma unroll
   for (int n = 0; n < NS; ++n) {
-    hv[n] = fmaf(ex2_approx(dlt * (Ap[n] * kLog2e)), hv[n], du * Bp[n]);
-    acc = fmaf(Cp[n], hv[n], acc);
+    hv[n] = fmaf(ex2_approx(dlt * (av[n] * kLog2e)), hv[n], du * bv[n]);
+    acc = fmaf(cv[n], hv[n], acc);
   }
-#pragma unroll
-  for (int n = 0; n < NS; ++n) hp[n] = hv[n];
+  st_states<NS>(hp, hv);
   acc += __shfl_xor_sync(gmask, acc, 1);
   acc += __shfl_xor_sync(gmask, acc, 2);
   if (j == 0) {
-    float yv = acc + (Dskip ? Dskip[c] * u : 0.f);
-    if (z_t) yv *= silu_dev(to_f32<XT>(z_t[e]));
+    float yv = acc + (Dskip ? dsk * u : 0.f);
+    if (z_t) yv *= silu_dev(zv);
     y_t[e] = from_f32<YT>(yv);
   }
 }
@@ -266,6 +311,26 @@ __global__ void __launch_bounds__(StepCfg<HD>::CH) swa_step_split_kernel(
   constexpr int CH = Cfg::CH, NWARP = Cfg::NWARP, KP = Cfg::KP, PP = Cfg::PP;
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int group = Hq / Hkv;  // <= 16
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // Loads that do not depend on pos go first, so that they are in flight
+  // together with the read of pos: the group's query rows (16-byte chunks of
+  // the zero-padded 16-row tile) and, in split 0, the new key/value row.
+  constexpr int QCH = 16 * HD / 8, QPT = (QCH + CH - 1) / CH, RCH = HD / 8;
+  const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+  uint4 qraw[QPT];
+#pragma unroll
+  for (int j = 0; j < QPT; ++j) {
+    const int i = tid + j * CH, hh = i / RCH, c = i % RCH;
+    qraw[j] = (i < QCH && hh < group)
+                  ? reinterpret_cast<const uint4*>(q_t + ((int64_t)b * Hq + g * group + hh) * HD)[c]
+                  : zero4;
+  }
+  const int64_t noff = ((int64_t)b * Hkv + g) * HD;
+  uint4 knew = zero4, vnew = zero4;
+  if (split == 0 && tid < RCH) {
+    knew = reinterpret_cast<const uint4*>(k_t + noff)[tid];
+    vnew = reinterpret_cast<const uint4*>(v_t + noff)[tid];
+  }
   const int64_t p = pos[b];
   const int64_t lo = p - W + 1 > 0 ? p - W + 1 : 0;
   const int64_t a0 = lo + (int64_t)split * CH;
@@ -282,41 +347,42 @@ __global__ void __launch_bounds__(StepCfg<HD>::CH) swa_step_split_kernel(
   __nv_bfloat16* Ps = reinterpret_cast<__nv_bfloat16*>(sm + Cfg::V_BYTES + 16 * CH * 4);  // [16][PP]
   __shared__ float red_m[16], red_l[16];
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, tq = lane & 3;  // mma fragment coordinates
-  // this thread's position: K and V rows to shared memory (zeros past the window)
+  // K and V rows of the chunk to shared memory (zeros past the window), as
+  // 16-byte chunks: consecutive threads take consecutive chunks of a row, so
+  // a warp's load covers whole rows (RCH chunks each); the newest position
+  // comes from k_t / v_t.
   {
-    const bool valid = tid < n_here;
-    int slot = slot0 + tid;
-    slot = slot >= Wi ? slot - Wi : slot;
-    const bool is_new = a0 + tid == p;
-    const int64_t roff = (((int64_t)b * W + (valid ? slot : 0)) * Hkv + g) * HD;
-    const int64_t noff = ((int64_t)b * Hkv + g) * HD;
-    const uint4* krow = reinterpret_cast<const uint4*>(is_new ? k_t + noff : k_ring + roff);
-    const uint4* vrow = reinterpret_cast<const uint4*>(is_new ? v_t + noff : v_ring + roff);
-    uint4 kraw[HD / 8], vraw[HD / 8];
+    uint4 kraw[RCH], vraw[RCH];
 #pragma unroll
-    for (int c = 0; c < HD / 8; ++c) {
-      kraw[c] = valid ? krow[c] : make_uint4(0u, 0u, 0u, 0u);
-      vraw[c] = valid ? vrow[c] : make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < RCH; ++i) {
+      const int ig = tid + i * CH, r = ig / RCH, c = ig % RCH;
+      const bool valid = r < n_here;
+      int slot = slot0 + r;
+      slot = slot >= Wi ? slot - Wi : slot;
+      const bool is_new = a0 + r == p;
+      const int64_t roff = (((int64_t)b * W + (valid ? slot : 0)) * Hkv + g) * HD;
+      const uint4* krow = reinterpret_cast<const uint4*>(is_new ? k_t + noff : k_ring + roff);
+      const uint4* vrow = reinterpret_cast<const uint4*>(is_new ? v_t + noff : v_ring + roff);
+      kraw[i] = valid ? krow[c] : zero4;
+      vraw[i] = valid ? vrow[c] : zero4;
     }
 #pragma unroll
-    for (int c = 0; c < HD / 8; ++c) {
-      reinterpret_cast<uint4*>(Ks + tid * KP)[c] = kraw[c];
-      reinterpret_cast<uint4*>(Vs + tid * KP)[c] = vraw[c];
+    for (int i = 0; i < RCH; ++i) {
+      const int ig = tid + i * CH, r = ig / RCH, c = ig % RCH;
+      reinterpret_cast<uint4*>(Ks + r * KP)[c] = kraw[i];
+      reinterpret_cast<uint4*>(Vs + r * KP)[c] = vraw[i];
     }
   }
-  // the group's query rows (rows past the group are zero)
-  for (int i = tid; i < 16 * HD; i += CH) {
-    const int hh = i / HD, dd = i % HD;
-    Qs[hh * KP + dd] = hh < group ? q_t[((int64_t)b * Hq + g * group + hh) * HD + dd] : __float2bfloat16_rn(0.f);
+#pragma unroll
+  for (int j = 0; j < QPT; ++j) {
+    const int i = tid + j * CH;
+    if (i < QCH) reinterpret_cast<uint4*>(Qs + (i / RCH) * KP)[i % RCH] = qraw[j];
   }
-  if (split == 0) {  // store the new key/value into its slot
-    const int64_t slot = p % W;
-    for (int i = tid; i < HD; i += CH) {
-      k_ring[(((int64_t)b * W + slot) * Hkv + g) * HD + i] = k_t[((int64_t)b * Hkv + g) * HD + i];
-      v_ring[(((int64_t)b * W + slot) * Hkv + g) * HD + i] = v_t[((int64_t)b * Hkv + g) * HD + i];
-    }
+  if (split == 0 && tid < RCH) {  // the new key/value into its slot
+    const int64_t roff = (((int64_t)b * W + p % W) * Hkv + g) * HD;
+    reinterpret_cast<uint4*>(k_ring + roff)[tid] = knew;
+    reinterpret_cast<uint4*>(v_ring + roff)[tid] = vnew;
   }
   __syncthreads();
 

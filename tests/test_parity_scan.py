@@ -80,7 +80,7 @@ def test_tiny_workload_fp32():
     (2, 200, 48, 16, torch.bfloat16),   # ragged time tile and channel block
     (1, 64, 32, 16, torch.float32),
     (3, 131, 40, 8, torch.bfloat16),
-    (2, 150, 36, 8, torch.float32),     # N = 8 with fp32 x: two TMA stages, 4 epilogue warps
+    (2, 150, 48, 8, torch.float32),     # N = 8 with fp32 x: two TMA stages, 4 epilogue warps
     (2, 77, 24, 4, torch.float32),
     (1, 1, 16, 16, torch.bfloat16),     # L = 1
     (2, 2, 16, 16, torch.float32),      # L < K - 1
