@@ -275,9 +275,9 @@ int launch_ring_fill(const void* k, const void* v, int64_t L, void* k_ring, void
 // (max, sum, unnormalised output) per head; a second kernel combines the
 // splits.  The newest position is read from k_t/v_t, which split 0 also
 // stores into its ring slot (that slot held a position outside the window, so
-// no other CTA reads it in this step).  Thread i of a CTA loads the K and V
-// rows of position i of its chunk into shared memory in one burst (all rows
-// of the chunk in flight at once); the scores K·qᵀ (positions x heads) and
+// no other CTA reads it in this step).  The CTA loads its chunk's K and V
+// rows into shared memory in one burst of 16-byte chunks (all rows in flight
+// at once, a warp's load covering whole rows); the scores K·qᵀ (pos x heads) and
 // the outputs P·V (heads x head dim) are bf16 tensor-core products
 // (mma m16n8k16, fp32 accumulate), P rounded to bf16 as in the prefill.
 template <int HD> struct StepCfg {
