@@ -8,6 +8,7 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 #include <string>
 
 #include "../../include/samba.h"
@@ -30,6 +31,25 @@ int encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const vo
 
 // Number of SMs of the current device.
 int sm_count();
+
+// Per-device one-time setup (function attributes apply to the device that is
+// current when they are set).  once_per_device(o, f) runs f() unless it has
+// already succeeded for the current device; thread-safe.
+struct PerDeviceOnce {
+  std::mutex mu;
+  uint64_t done = 0;  // bit d: device d is set up
+};
+template <class F>
+int once_per_device(PerDeviceOnce& o, F&& f) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(SAMBA_ERR_CUDA, "cannot query the current device");
+  if (dev < 0 || dev >= 64) return f();  // no record past 64 devices: set up every time
+  std::lock_guard<std::mutex> lock(o.mu);
+  if ((o.done >> dev) & 1u) return SAMBA_OK;
+  const int rc = f();
+  if (rc == SAMBA_OK) o.done |= uint64_t(1) << dev;
+  return rc;
+}
 
 // Per-translation-unit status readers (each kernel file keeps its own word).
 int take_status_scan(cudaStream_t s);

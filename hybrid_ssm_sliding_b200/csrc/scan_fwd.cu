@@ -618,12 +618,13 @@ static int launch_scan_t(const samba_scan_args& a, cudaStream_t stream) {
   using Ly = ScanLayout<N, XT>;
   constexpr int POLY = SAMBA_SCAN_POLY;
   auto kern = scan_fwd_kernel<N, XT, YT, POLY>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::SMEM) != cudaSuccess)
-      return fail(SAMBA_ERR_CUDA, "scan: cannot set shared memory size");
-    attr_done = true;
-  }
+  static PerDeviceOnce attr;
+  const int arc = once_per_device(attr, [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::SMEM) == cudaSuccess
+               ? SAMBA_OK
+               : fail(SAMBA_ERR_CUDA, "scan: cannot set shared memory size");
+  });
+  if (arc != SAMBA_OK) return arc;
   const int CU = choose_cu(a.batch, a.dim);
   const uint64_t Bsz = a.batch, L = a.seqlen, D = a.dim;
   const uint32_t xs = sizeof(XT);

@@ -554,12 +554,13 @@ static int launch_swa_t(const samba_swa_args& a, cudaStream_t stream) {
   constexpr int STG = SWA_STAGES;
   using Cfg = SwaCfg<HD, GROUP, STG>;
   auto kern = swa_fwd_kernel<HD, GROUP, STG>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) != cudaSuccess)
-      return fail(SAMBA_ERR_CUDA, "swa: cannot set shared memory size");
-    attr_done = true;
-  }
+  static PerDeviceOnce attr;
+  const int arc = once_per_device(attr, [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) == cudaSuccess
+               ? SAMBA_OK
+               : fail(SAMBA_ERR_CUDA, "swa: cannot set shared memory size");
+  });
+  if (arc != SAMBA_OK) return arc;
   const uint64_t B = a.batch, L = a.seqlen, Hq = a.heads_q, Hkv = a.heads_kv;
   const CUtensorMapSwizzle swz =
       HD == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : (HD == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
