@@ -288,6 +288,12 @@ def swa(q, k, v, window, scale=None, block=64):
     return o, lse
 
 
+def _window_positions(p, window):
+    """Absolute positions a query at position p attends under the causal band
+    0 <= p - j < W: max(0, p - W + 1) .. p."""
+    return range(max(0, p - window + 1), p + 1)
+
+
 def ring_fill(k, v, window):
     """Decode state after a prefill of L tokens (the page's ``forward(prompt)``
     filling the cache): the last min(L, W) keys and values, key of absolute
@@ -300,7 +306,7 @@ def ring_fill(k, v, window):
     Bsz, L, Hkv, d = k.shape
     k_ring = np.zeros((Bsz, window, Hkv, d))
     v_ring = np.zeros((Bsz, window, Hkv, d))
-    for p in range(max(0, L - window), L):
+    for p in _window_positions(L - 1, window):  # the keys position L - 1 sees
         k_ring[:, p % window] = k[:, p]
         v_ring[:, p % window] = v[:, p]
     return k_ring, v_ring, np.full((Bsz,), L, dtype=np.int64)
@@ -332,7 +338,7 @@ def swa_step(q_t, k_t, v_t, k_ring, v_ring, pos, window, scale=None):
         p = int(pos[b])
         k_ring[b, p % window] = _f64(k_t)[b]
         v_ring[b, p % window] = _f64(v_t)[b]
-        slots = np.array([a % window for a in range(max(0, p - window + 1), p + 1)])
+        slots = np.array([a % window for a in _window_positions(p, window)])
         for h in range(Hq):
             kv = h // group
             s = k_ring[b, slots, kv, :] @ q_t[b, h] * scale

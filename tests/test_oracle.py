@@ -220,18 +220,25 @@ def test_scan_split_with_carry_equals_one_pass():
         np.testing.assert_allclose(b["conv_state"], full["conv_state"], atol=0)
 
 
-def test_scan_step_sequence_equals_prefill():
-    i = _tiny_scan_inputs(10, Bsz=2, L=40, D=8, N=4)
+def _scan_steps_match_prefill(L1=25, L=40):
+    """Prefill of L1 tokens, then L - L1 single-token steps, against one
+    prefill of L tokens: True when every step output and the final state
+    agree to 1e-12."""
+    i = _tiny_scan_inputs(10, Bsz=2, L=L, D=8, N=4)
     full = orc.selective_scan(**i)
-    L1 = 25
     pre = orc.selective_scan(**{k: (v[:, :L1] if k in ("x", "z", "delta", "Bm", "Cm") else v)
                                 for k, v in i.items()})
     h, cs = pre["h"], pre["conv_state"]
-    for t in range(L1, 40):
+    ok = True
+    for t in range(L1, L):
         y_t, h, cs = orc.scan_step(h, cs, i["x"][:, t], i["delta"][:, t], i["A"], i["Bm"][:, t],
                                    i["Cm"][:, t], i["Dskip"], i["z"][:, t], i["conv_w"], i["conv_b"])
-        np.testing.assert_allclose(y_t, full["y"][:, t], rtol=1e-12, atol=1e-12)
-    np.testing.assert_allclose(h, full["h"], rtol=1e-12, atol=1e-12)
+        ok = ok and np.allclose(y_t, full["y"][:, t], rtol=1e-12, atol=1e-12)
+    return ok and np.allclose(h, full["h"], rtol=1e-12, atol=1e-12)
+
+
+def test_scan_step_sequence_equals_prefill():
+    assert _scan_steps_match_prefill()
 
 
 # -------------------------------------------------------------------------- SWA
@@ -310,17 +317,24 @@ def test_swa_rows_equals_blocked():
     np.testing.assert_allclose(lse2, lse[:, :, rows], atol=1e-13)
 
 
-@pytest.mark.parametrize("L1,W", [(10, 16), (40, 16), (16, 16), (1, 4)])
-def test_swa_decode_steps_equal_prefill(L1, W):
+def _swa_steps_match_prefill(L1, W):
+    """Ring fill after L1 tokens, then 20 decode steps, against the banded
+    prefill of L1 + 20 tokens: True when every step output agrees to 1e-12
+    and pos ends at L1 + 20."""
     L = L1 + 20
     q, k, v = _attn_inputs(17, 2, L, 8, 2, 16)
     full, _ = orc.swa(q, k, v, W, block=16)
     kr, vr, pos = orc.ring_fill(k[:, :L1], v[:, :L1], W)
-    assert np.all(pos == L1)
+    ok = bool(np.all(pos == L1))
     for t in range(L1, L):
         o_t, kr, vr, pos = orc.swa_step(q[:, t], k[:, t], v[:, t], kr, vr, pos, W)
-        np.testing.assert_allclose(o_t, full[:, t], atol=1e-12)
-    assert np.all(pos == L)
+        ok = ok and np.allclose(o_t, full[:, t], atol=1e-12)
+    return ok and bool(np.all(pos == L))
+
+
+@pytest.mark.parametrize("L1,W", [(10, 16), (40, 16), (16, 16), (1, 4)])
+def test_swa_decode_steps_equal_prefill(L1, W):
+    assert _swa_steps_match_prefill(L1, W)
 
 
 # ----------------------------------------------- planted mistakes are caught
@@ -387,3 +401,37 @@ def test_scan_magnitudes_equal_outputs_when_no_term_is_negative():
     out = orc.selective_scan(x, dt, A, Bm, Cm, Ds, delta_softplus=False, magnitudes=True)
     np.testing.assert_allclose(out["y_mag"], out["y"], rtol=1e-13)
     np.testing.assert_allclose(out["h_mag"], out["h"], rtol=1e-13)
+
+
+# ------------------------------------------- planted mistakes in the decode steps
+def test_planted_decode_window_one_too_wide_is_caught(monkeypatch):
+    """W + 1 positions per query: the ring then hands the newest key twice."""
+    monkeypatch.setattr(orc, "_window_positions", lambda p, W: range(max(0, p - W), p + 1))
+    assert not _swa_steps_match_prefill(40, 16)
+
+
+def test_planted_decode_window_one_too_narrow_is_caught(monkeypatch):
+    monkeypatch.setattr(orc, "_window_positions", lambda p, W: range(max(0, p - W + 2), p + 1))
+    assert not _swa_steps_match_prefill(40, 16)
+
+
+def test_planted_scan_step_state_dropped_is_caught(monkeypatch):
+    """A step that restarts the SSM state (h0 = None) or the conv state."""
+    real = orc.selective_scan
+
+    def no_h(x, delta, A, Bm, Cm, Dskip=None, z=None, h0=None, *rest, **kw):
+        return real(x, delta, A, Bm, Cm, Dskip, z, None if x.shape[1] == 1 else h0, *rest, **kw)
+
+    monkeypatch.setattr(orc, "selective_scan", no_h)
+    assert not _scan_steps_match_prefill()
+    monkeypatch.undo()
+
+    def no_conv_state(x, delta, A, Bm, Cm, Dskip=None, z=None, h0=None, conv_w=None, conv_b=None,
+                      conv_state=None, *rest, **kw):
+        return real(x, delta, A, Bm, Cm, Dskip, z, h0, conv_w, conv_b,
+                    None if x.shape[1] == 1 else conv_state, *rest, **kw)
+
+    monkeypatch.setattr(orc, "selective_scan", no_conv_state)
+    assert not _scan_steps_match_prefill()
+    monkeypatch.undo()
+    assert _scan_steps_match_prefill()
