@@ -125,3 +125,51 @@ def test_decode_rejects_bad_arguments_on_host(lib):
         L.SAMBA_ERR_WORKSPACE
     assert lib.samba_swa_step(f, f, f, f, f, f, f, 16, 32, 4, 64, 2048, 0.0, None, 0, None) == \
         L.SAMBA_ERR_WORKSPACE
+
+
+def test_scan_step_argument_checks_on_host(lib):
+    f = 0x50000
+
+    def call(h=f, x_dtype=1, y_dtype=1, batch=1, dstate=16, dconv=4, flags=0):
+        return lib.samba_scan_step(h, None, f, x_dtype, None, 1, f, f, f, f, None, None, None, f, y_dtype,
+                                   batch, 8, dstate, dconv, flags, None)
+
+    assert call(batch=0) == L.SAMBA_ERR_INVALID_ARG
+    assert call(dstate=32) == L.SAMBA_ERR_UNSUPPORTED
+    assert call(dconv=1) == L.SAMBA_ERR_UNSUPPORTED
+    assert call(dconv=5) == L.SAMBA_ERR_UNSUPPORTED
+    assert call(x_dtype=7) == L.SAMBA_ERR_UNSUPPORTED
+    assert call(y_dtype=7) == L.SAMBA_ERR_UNSUPPORTED
+    assert call(flags=8) == L.SAMBA_ERR_INVALID_ARG
+    assert call(h=f + 4) == L.SAMBA_ERR_INVALID_ARG  # the state is read as 16-byte vectors
+
+
+def test_swa_step_argument_checks_on_host(lib):
+    f = 0x60000
+
+    def call(q=f, batch=16, hq=32, hkv=4, d=64, W=2048, ws=f, nbytes=None):
+        need = lib.samba_swa_step_workspace_size(max(batch, 1), max(hq, 1), max(d, 1), max(W, 1))
+        return lib.samba_swa_step(q, f, f, f, f, f, f, batch, hq, hkv, d, W, 0.0, ws,
+                                  need if nbytes is None else nbytes, None)
+
+    assert call(W=0) == L.SAMBA_ERR_INVALID_ARG
+    assert call(batch=0) == L.SAMBA_ERR_INVALID_ARG
+    assert call(d=80) == L.SAMBA_ERR_UNSUPPORTED
+    assert call(hq=33) == L.SAMBA_ERR_INVALID_ARG           # heads_q not a multiple of heads_kv
+    assert call(hq=68) == L.SAMBA_ERR_UNSUPPORTED           # 17 query heads per KV head
+    assert call(q=f + 8) == L.SAMBA_ERR_INVALID_ARG         # misaligned
+    assert call(ws=f + 4) == L.SAMBA_ERR_INVALID_ARG        # misaligned workspace
+    assert call(batch=70000) == L.SAMBA_ERR_UNSUPPORTED     # grid limit, refused before any launch
+
+
+def test_swa_step_noalloc_checks_on_host(lib):
+    f = 0x70000
+
+    def call(q=f, batch=16, hq=32, hkv=4, d=64, W=2048):
+        return lib.samba_swa_step_noalloc(q, f, f, f, f, f, f, batch, hq, hkv, d, W, 0.0, None)
+
+    assert call(hq=68) == L.SAMBA_ERR_UNSUPPORTED
+    assert call(q=f + 8) == L.SAMBA_ERR_INVALID_ARG
+    # 64 sequences x 32 heads x 16 splits x 66 floats = 8.6 MB: more than the built-in 4 MiB
+    assert lib.samba_swa_step_workspace_size(64, 32, 64, 2048) > 4 << 20
+    assert call(batch=64) == L.SAMBA_ERR_WORKSPACE
