@@ -125,6 +125,10 @@ int samba_conv1d_fwd(const void* x, int x_dtype, const float* w, const float* bi
  *   y_t    = (sum_n C_t[n] h_t[n] + Dskip[c] u_t) * silu(z_t)
  * for every batch b and channel c, t = 0..L-1, starting from h0 (zeros if
  * NULL).  B and C are shared by all channels (one group).
+ * Errors: SAMBA_ERR_INVALID_ARG for a missing x, delta, A, Bm, Cm, y (or
+ * conv_w with FUSE_CONV), D not a multiple of 8, unknown flag bits or a
+ * pointer not 16-byte aligned; SAMBA_ERR_UNSUPPORTED for B > 65535,
+ * L >= 2^31 - 1024, N or K outside the sets below, or z_dtype != x_dtype.
  */
 typedef struct samba_scan_args {
   const void* x;               /* [B, L, D]   x_dtype                         */
@@ -157,6 +161,10 @@ int samba_selective_scan_fwd(const samba_scan_args* args, samba_stream_t stream)
  * fp32 online softmax; o is rounded to bf16 once.  lse (optional) receives the
  * natural-log logsumexp of the scaled scores of every row.
  * W >= L gives plain causal attention.
+ * Errors: SAMBA_ERR_INVALID_ARG for a missing q, k, v or o, a non-positive
+ * size, Hq not a multiple of Hkv or a pointer not 16-byte aligned;
+ * SAMBA_ERR_UNSUPPORTED for Hq/Hkv outside {1, 2, 4, 8, 16}, d outside
+ * {16, 32, 64}, B > 65535 or L > 2^30.
  */
 typedef struct samba_swa_args {
   const void* q;      /* [B, L, Hq, d]   bf16 */
@@ -165,7 +173,7 @@ typedef struct samba_swa_args {
   void* o;            /* [B, L, Hq, d]   bf16 */
   float* lse;         /* [B, Hq, L]      fp32, or NULL */
   int64_t batch, seqlen, window;   /* B >= 1, L >= 1, W >= 1 */
-  int32_t heads_q, heads_kv, head_dim;  /* Hq % Hkv == 0, Hq/Hkv divides 128; d in {16, 32, 64} */
+  int32_t heads_q, heads_kv, head_dim;  /* Hq % Hkv == 0, Hq/Hkv in {1,2,4,8,16}; d in {16,32,64} */
   float scale;        /* softmax scale; <= 0 selects 1/sqrt(d) */
 } samba_swa_args;
 
@@ -193,7 +201,9 @@ int samba_mixer_prefill(const samba_scan_args* scan, const samba_swa_args* swa,
  *                          [D, K], conv_b [D] (or NULL) as in the prefill
  *   y_t        [B, D]      y_dtype
  * flags: as samba_scan_args.flags (FUSE_CONV requires conv_state and conv_w).
- * B <= 65535 (SAMBA_ERR_UNSUPPORTED beyond); N in {4, 8, 16}; K in 2..4.
+ * B <= 65535 (SAMBA_ERR_UNSUPPORTED beyond); N in {4, 8, 16}; K in 2..4;
+ * z_dtype == x_dtype.  h, A, B_t and C_t must be 16-byte aligned
+ * (SAMBA_ERR_INVALID_ARG otherwise): the states are read as vectors.
  */
 int samba_scan_step(float* h, float* conv_state, const void* x_t, int x_dtype, const void* z_t,
                     int z_dtype, const float* delta_t, const float* B_t, const float* C_t,
@@ -205,9 +215,12 @@ int samba_scan_step(float* h, float* conv_state, const void* x_t, int x_dtype, c
  * Ring-buffer KV window.  Slot p mod W of k_ring/v_ring holds the key/value
  * of absolute position p; pos[b] is the next position of sequence b.
  *
- * samba_swa_ring_fill: after a prefill of L tokens, copy the last min(L, W)
- * keys/values of k, v ([B, L, Hkv, d] bf16) into their slots and set
- * pos[b] = L.  Slots of positions < L - W are left untouched.
+ * k_ring, v_ring are [B, W, Hkv, d] bf16; head_dim d is 16, 32, 64 or 128
+ * (SAMBA_ERR_UNSUPPORTED otherwise).
+ *
+ * samba_swa_ring_fill: after a prefill of L tokens (L >= 0), copy the last
+ * min(L, W) keys/values of k, v ([B, L, Hkv, d] bf16) into their slots and
+ * set pos[b] = L.  Slots of positions < L - W are left untouched.
  */
 int samba_swa_ring_fill(const void* k, const void* v, int64_t seqlen, void* k_ring, void* v_ring,
                         int64_t* pos, int64_t batch, int heads_kv, int head_dim, int64_t window,
@@ -222,7 +235,12 @@ size_t samba_swa_step_workspace_size(int64_t batch, int heads_q, int head_dim, i
  * pos[b] += 1.  All of it happens on the device (pos is a device int64 [B]),
  * so consecutive steps can be captured in one CUDA graph.  `workspace` is
  * caller-owned device memory of at least samba_swa_step_workspace_size()
- * bytes (split partial results); it needs no initialisation.
+ * bytes (split partial results); it needs no initialisation.  scale <= 0
+ * selects 1/sqrt(d).
+ * Errors: SAMBA_ERR_INVALID_ARG for a null pointer, a non-positive size, Hq
+ * not a multiple of Hkv or a pointer (workspace included) not 16-byte
+ * aligned; SAMBA_ERR_UNSUPPORTED for Hq/Hkv > 16, d outside the set above
+ * or B > 65535; SAMBA_ERR_WORKSPACE for a missing or smaller workspace.
  */
 int samba_swa_step(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring,
                    int64_t* pos, void* o_t, int64_t batch, int heads_q, int heads_kv, int head_dim,
