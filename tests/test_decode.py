@@ -50,7 +50,7 @@ def test_conv1d_short_sequence_keeps_old_state():
 
 
 # ----------------------------------------------------------------- scan step
-@pytest.mark.parametrize("dt,N", [(torch.float32, 16), (torch.bfloat16, 16), (torch.float32, 4)])
+@pytest.mark.parametrize("dt,N", [(torch.float32, 16), (torch.bfloat16, 16), (torch.bfloat16, 8), (torch.float32, 4)])
 def test_prefill_then_scan_steps_match_oracle(dt, N):
     wl = Workload("d", 3, 40, 32, N, 4, 1, 1, 16, 16, 50 + N, act_dtype=dt)
     inp = make_prefill_inputs(wl, device="cuda", with_attention=False)
