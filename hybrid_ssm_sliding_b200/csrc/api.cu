@@ -183,19 +183,31 @@ int samba_mixer_prefill(const samba_scan_args* scan, const samba_swa_args* swa, 
     if (rc != SAMBA_OK) return rc;
     return launch_scan(*scan, s);
   }
-  cudaEvent_t fork, join;
-  if (cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess)
+  // Fork `aux` from `stream`, run the attention there and the scan on
+  // `stream`, then join `aux` back, so that the call as a whole stays ordered
+  // on `stream`.  The events are created per call and released at once (a
+  // recorded event may be destroyed while its work is pending).
+  cudaEvent_t fork = nullptr, join = nullptr;
+  if (cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess)
     return fail(SAMBA_ERR_CUDA, "samba_mixer_prefill: event creation failed");
-  cudaEventRecord(fork, s);
-  cudaStreamWaitEvent(a, fork, 0);
-  rc = launch_swa(*swa, a);
-  int rc2 = launch_scan(*scan, s);
-  cudaEventRecord(join, a);
-  cudaStreamWaitEvent(s, join, 0);
+  if (cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {
+    cudaEventDestroy(fork);
+    return fail(SAMBA_ERR_CUDA, "samba_mixer_prefill: event creation failed");
+  }
+  if (cudaEventRecord(fork, s) != cudaSuccess || cudaStreamWaitEvent(a, fork, 0) != cudaSuccess) {
+    rc = fail(SAMBA_ERR_CUDA, "samba_mixer_prefill: cannot fork the aux stream");
+  } else {
+    rc = launch_swa(*swa, a);
+    // After a failed attention launch the scan is not started; the join below
+    // still orders `stream` after whatever reached `aux`.
+    if (rc == SAMBA_OK) rc = launch_scan(*scan, s);
+    if ((cudaEventRecord(join, a) != cudaSuccess || cudaStreamWaitEvent(s, join, 0) != cudaSuccess) &&
+        rc == SAMBA_OK)
+      rc = fail(SAMBA_ERR_CUDA, "samba_mixer_prefill: cannot join the aux stream");
+  }
   cudaEventDestroy(fork);
   cudaEventDestroy(join);
-  return rc != SAMBA_OK ? rc : rc2;
+  return rc;
 }
 
 int samba_scan_step(float* h, float* conv_state, const void* x_t, int x_dtype, const void* z_t, int z_dtype,
@@ -222,6 +234,28 @@ static int check_ring(int64_t batch, int heads_kv, int head_dim, int64_t window,
   if (batch < 1 || heads_kv < 1 || window < 1) return fail(SAMBA_ERR_INVALID_ARG, "%s: bad shape", who);
   if (head_dim != 16 && head_dim != 32 && head_dim != 64 && head_dim != 128)
     return fail(SAMBA_ERR_UNSUPPORTED, "%s: head_dim must be 16, 32, 64 or 128", who);
+  // The decode kernels index ring slots with 32-bit ints and put the KV heads
+  // on a grid dimension of at most 65535 blocks.
+  if (window > (int64_t(1) << 30)) return fail(SAMBA_ERR_UNSUPPORTED, "%s: window above 2^30", who);
+  if (heads_kv > 65535) return fail(SAMBA_ERR_UNSUPPORTED, "%s: heads_kv above 65535", who);
+  return SAMBA_OK;
+}
+
+// Shared checks of samba_swa_step and samba_swa_step_noalloc, in the order
+// both report them.
+static int check_swa_step(const void* q_t, const void* k_t, const void* v_t, const void* k_ring, const void* v_ring,
+                          const int64_t* pos, const void* o_t, int64_t batch, int heads_q, int heads_kv,
+                          int head_dim, int64_t window, const char* who) {
+  if (!q_t || !k_t || !v_t || !k_ring || !v_ring || !pos || !o_t)
+    return fail(SAMBA_ERR_INVALID_ARG, "%s: null pointer", who);
+  int rc = check_ring(batch, heads_kv, head_dim, window, who);
+  if (rc != SAMBA_OK) return rc;
+  if (heads_q < 1 || heads_q % heads_kv != 0) return fail(SAMBA_ERR_INVALID_ARG, "%s: heads_q %% heads_kv", who);
+  if (heads_q / heads_kv > 16) return fail(SAMBA_ERR_UNSUPPORTED, "%s: heads_q / heads_kv must be <= 16", who);
+  if (batch > 65535) return fail(SAMBA_ERR_UNSUPPORTED, "%s: batch above 65535", who);
+  const void* ptrs[] = {q_t, k_t, v_t, k_ring, v_ring, o_t};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return fail(SAMBA_ERR_INVALID_ARG, "%s: misaligned pointer", who);
   return SAMBA_OK;
 }
 
@@ -248,18 +282,12 @@ int samba_swa_step(const void* q_t, const void* k_t, const void* v_t, void* k_ri
                    void* o_t, int64_t batch, int heads_q, int heads_kv, int head_dim, int64_t window, float scale,
                    void* workspace, size_t workspace_bytes, samba_stream_t stream) {
   const char* who = "samba_swa_step";
-  if (!q_t || !k_t || !v_t || !k_ring || !v_ring || !pos || !o_t)
-    return fail(SAMBA_ERR_INVALID_ARG, "%s: null pointer", who);
-  int rc = check_ring(batch, heads_kv, head_dim, window, who);
+  int rc = check_swa_step(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, batch, heads_q, heads_kv, head_dim, window, who);
   if (rc != SAMBA_OK) return rc;
-  if (heads_q < 1 || heads_q % heads_kv != 0) return fail(SAMBA_ERR_INVALID_ARG, "%s: heads_q %% heads_kv", who);
-  if (heads_q / heads_kv > 16) return fail(SAMBA_ERR_UNSUPPORTED, "%s: heads_q / heads_kv must be <= 16", who);
   const size_t need = swa_step_workspace(batch, heads_q, head_dim, window);
   if (need > 0 && (!workspace || workspace_bytes < need))
     return fail(SAMBA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", who, need, workspace_bytes);
-  const void* ptrs[] = {q_t, k_t, v_t, k_ring, v_ring, o_t, workspace};
-  for (const void* p : ptrs)
-    if (p && !aligned16(p)) return fail(SAMBA_ERR_INVALID_ARG, "%s: misaligned pointer", who);
+  if (workspace && !aligned16(workspace)) return fail(SAMBA_ERR_INVALID_ARG, "%s: misaligned workspace", who);
   if (!(scale > 0.f)) scale = 1.0f / std::sqrt(static_cast<float>(head_dim));
   return launch_swa_step(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, batch, heads_q, heads_kv, head_dim, window,
                          scale, workspace, reinterpret_cast<cudaStream_t>(stream));
@@ -269,15 +297,8 @@ int samba_swa_step_noalloc(const void* q_t, const void* k_t, const void* v_t, vo
                            int64_t* pos, void* o_t, int64_t batch, int heads_q, int heads_kv, int head_dim,
                            int64_t window, float scale, samba_stream_t stream) {
   const char* who = "samba_swa_step_noalloc";
-  if (!q_t || !k_t || !v_t || !k_ring || !v_ring || !pos || !o_t)
-    return fail(SAMBA_ERR_INVALID_ARG, "%s: null pointer", who);
-  int rc = check_ring(batch, heads_kv, head_dim, window, who);
+  int rc = check_swa_step(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, batch, heads_q, heads_kv, head_dim, window, who);
   if (rc != SAMBA_OK) return rc;
-  if (heads_q < 1 || heads_q % heads_kv != 0) return fail(SAMBA_ERR_INVALID_ARG, "%s: heads_q %% heads_kv", who);
-  if (heads_q / heads_kv > 16) return fail(SAMBA_ERR_UNSUPPORTED, "%s: heads_q / heads_kv must be <= 16", who);
-  const void* ptrs[] = {q_t, k_t, v_t, k_ring, v_ring, o_t};
-  for (const void* p : ptrs)
-    if (!aligned16(p)) return fail(SAMBA_ERR_INVALID_ARG, "%s: misaligned pointer", who);
   if (!(scale > 0.f)) scale = 1.0f / std::sqrt(static_cast<float>(head_dim));
   return launch_swa_step_noalloc(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, batch, heads_q, heads_kv, head_dim, window,
                                  scale, reinterpret_cast<cudaStream_t>(stream));

@@ -506,10 +506,18 @@ __global__ void swa_step_combine_kernel(const float* __restrict__ ws, __nv_bfloa
   if (hq == 0 && dd == 0) pos[b] += 1;
 }
 
+// Bytes of split partials: (max, sum, d outputs) per (batch, query head,
+// split).  SIZE_MAX when the product does not fit in size_t, so that no
+// workspace (and no built-in scratch) is ever taken as large enough.
 size_t swa_step_workspace(int64_t B, int Hq, int d, int64_t W) {
   const int ch = d <= 64 ? StepCfg<64>::CH : StepCfg<128>::CH;
-  const int64_t nsplit = (W + ch - 1) / ch;
-  return static_cast<size_t>(B * Hq * nsplit * (d + 2)) * sizeof(float);
+  const uint64_t nsplit = static_cast<uint64_t>((W + ch - 1) / ch);
+  uint64_t n = 0;
+  if (__builtin_mul_overflow(static_cast<uint64_t>(B), static_cast<uint64_t>(Hq), &n) ||
+      __builtin_mul_overflow(n, nsplit, &n) || __builtin_mul_overflow(n, static_cast<uint64_t>(d + 2), &n) ||
+      __builtin_mul_overflow(n, static_cast<uint64_t>(sizeof(float)), &n) || n > SIZE_MAX)
+    return SIZE_MAX;
+  return static_cast<size_t>(n);
 }
 
 template <int HD>
@@ -568,7 +576,6 @@ int launch_selftest_wait(cudaStream_t s) {
 // Scratch for samba_swa_step_noalloc: the split partials of swa_step live in
 // this file-scope device array instead of caller-provided workspace.  Every
 // GPU that loads the library holds it (4 MiB) until the process exits.
-#include <mutex>
 
 namespace samba {
 
@@ -576,24 +583,17 @@ constexpr size_t kSwaStepScratchBytes = size_t(4) << 20;
 static __device__ __align__(256) unsigned char g_swa_step_scratch[kSwaStepScratchBytes];
 
 // In host code g_swa_step_scratch names a host-side stand-in, not device
-// memory: the device address must be looked up once per device, with that
-// device current, and passed to the kernels.
-static std::mutex g_scratch_mu;
-static void* g_scratch_addr[128];
-
+// memory: its device address is looked up with cudaGetSymbolAddress, with
+// the calling device current, and passed to the kernels.  The lookup runs on
+// every call (it is a table lookup once the module is loaded), so that the
+// address stays right after cudaDeviceReset, which reloads the module and
+// may place the array elsewhere.
 static int scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128)
-    return fail(SAMBA_ERR_CUDA, "samba_swa_step_noalloc: no usable current device");
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_swa_step_scratch);
-    if (e != cudaSuccess || !p)
-      return fail(SAMBA_ERR_CUDA, "samba_swa_step_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_swa_step_scratch);
+  if (e != cudaSuccess || !p)
+    return fail(SAMBA_ERR_CUDA, "samba_swa_step_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+  *out = p;
   return SAMBA_OK;
 }
 

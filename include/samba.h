@@ -97,8 +97,12 @@ int samba_get_status(samba_stream_t stream);
 int samba_selftest_wait_timeout(samba_stream_t stream);
 
 /* ------------------------------------------------------------------ conv1d
- * Causal depthwise conv1d over time (the conv that Samba's Mamba layer puts in
- * front of its selective scan):
+ * Causal depthwise conv1d over time, the conv that a Mamba layer puts in front
+ * of its selective scan.  The pages do not print this step: their Mamba
+ * equations start from the scan input x_t.  It is part of the Mamba layer
+ * that Samba builds on, and this library runs it fused inside
+ * samba_selective_scan_fwd (SAMBA_SCAN_FUSE_CONV); this standalone form
+ * exists for callers that want u itself.
  *   u[b,t,c] = bias[c] + sum_{k<K} w[c,k] * xpad[b,t+k,c],  then SiLU if silu,
  * where xpad is x preceded by the K-1 inputs of conv_state_in (oldest first;
  * zeros when conv_state_in is NULL), so w[c,K-1] multiplies x_t.
@@ -220,13 +224,19 @@ int samba_scan_step(float* h, float* conv_state, const void* x_t, int x_dtype, c
  *
  * samba_swa_ring_fill: after a prefill of L tokens (L >= 0), copy the last
  * min(L, W) keys/values of k, v ([B, L, Hkv, d] bf16) into their slots and
- * set pos[b] = L.  Slots of positions < L - W are left untouched.
+ * set pos[b] = L.  Slots of positions < L - W are left untouched.  This is the
+ * hand-off of the page's inference pseudo-code (section 推理效率): its
+ * forward(prompt) leaves the window's keys and values in the cache that the
+ * following swa_step calls read.
+ * Limits of the ring (every decode SWA entry point): W <= 2^30 and
+ * Hkv <= 65535 (SAMBA_ERR_UNSUPPORTED beyond).
  */
 int samba_swa_ring_fill(const void* k, const void* v, int64_t seqlen, void* k_ring, void* v_ring,
                         int64_t* pos, int64_t batch, int heads_kv, int head_dim, int64_t window,
                         samba_stream_t stream);
 
-/* Bytes of device workspace samba_swa_step needs for these sizes. */
+/* Bytes of device workspace samba_swa_step needs for these sizes; 0 for a
+ * non-positive size, SIZE_MAX when the byte count does not fit in size_t. */
 size_t samba_swa_step_workspace_size(int64_t batch, int heads_q, int head_dim, int64_t window);
 
 /* samba_swa_step (swa_step): writes k_t, v_t ([B, Hkv, d]) into slot
@@ -260,10 +270,12 @@ int samba_swa_step(const void* q_t, const void* k_t, const void* v_t, void* k_ri
  * are rejected with SAMBA_ERR_WORKSPACE before anything is launched; the
  * 16 x 32-head, d = 64, W = 2048 decode needs 1.08 MB.
  *
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current, and keeps it; make that
- * first call before any stream capture.  The function calls no cudaMalloc,
- * cudaFree or other allocating routine.
+ * Every call looks up the array's device address (cudaGetSymbolAddress) on
+ * the current device; this is a table lookup once the library's device code
+ * is loaded there, and it keeps the address right after cudaDeviceReset.
+ * The first call on a device may load that code, so make it before any
+ * stream capture.  The function calls no cudaMalloc, cudaFree or other
+ * allocating routine.
  *
  * Every call shares the one array and finds the previous call's partials in
  * it.  That is harmless, because each step writes every partial it reads and
@@ -273,7 +285,8 @@ int samba_swa_step(const void* q_t, const void* k_t, const void* v_t, void* k_ri
  * samba_swa_step with separate workspaces.
  *
  * Arguments, layouts and errors are those of samba_swa_step without the
- * workspace.  The paper has no counterpart to this entry point; it exists
+ * workspace; the argument checks (SAMBA_ERR_UNSUPPORTED for B > 65535
+ * included) come before the size check.  The paper has no counterpart to this entry point; it exists
  * only for callers that cannot allocate.
  */
 int samba_swa_step_noalloc(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring,

@@ -160,6 +160,19 @@ def test_swa_step_argument_checks_on_host(lib):
     assert call(q=f + 8) == L.SAMBA_ERR_INVALID_ARG         # misaligned
     assert call(ws=f + 4) == L.SAMBA_ERR_INVALID_ARG        # misaligned workspace
     assert call(batch=70000) == L.SAMBA_ERR_UNSUPPORTED     # grid limit, refused before any launch
+    assert call(W=(1 << 30) + 1) == L.SAMBA_ERR_UNSUPPORTED  # ring slots are 32-bit indices
+    assert call(hq=70000, hkv=70000) == L.SAMBA_ERR_UNSUPPORTED  # KV heads on a 65535-block grid dimension
+
+
+def test_swa_step_workspace_size_saturates_instead_of_wrapping(lib):
+    size_max = ctypes.c_size_t(-1).value
+    # 65535 sequences x 2^20 query heads x 2^24 splits x 66 floats does not fit in 64 bits
+    assert lib.samba_swa_step_workspace_size(65535, 1 << 20, 64, 1 << 30) == size_max
+    assert lib.samba_swa_step_workspace_size(0, 32, 64, 2048) == 0
+    f = 0x68000
+    # no workspace can satisfy a saturated size, so the step refuses before any launch
+    assert lib.samba_swa_step(f, f, f, f, f, f, f, 65535, 1 << 20, 1 << 16, 64, 1 << 30, 0.0, f, size_max - 15,
+                              None) in (L.SAMBA_ERR_UNSUPPORTED, L.SAMBA_ERR_WORKSPACE)
 
 
 def test_swa_step_noalloc_checks_on_host(lib):
@@ -173,3 +186,6 @@ def test_swa_step_noalloc_checks_on_host(lib):
     # 64 sequences x 32 heads x 16 splits x 66 floats = 8.6 MB: more than the built-in 4 MiB
     assert lib.samba_swa_step_workspace_size(64, 32, 64, 2048) > 4 << 20
     assert call(batch=64) == L.SAMBA_ERR_WORKSPACE
+    # argument limits are reported as for samba_swa_step, before the scratch size
+    assert call(batch=70000) == L.SAMBA_ERR_UNSUPPORTED
+    assert call(W=(1 << 30) + 1) == L.SAMBA_ERR_UNSUPPORTED
