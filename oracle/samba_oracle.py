@@ -60,6 +60,7 @@ __all__ = [
     "selective_scan",
     "swa",
     "swa_rows",
+    "swa_blocks",
     "scan_step",
     "swa_step",
     "ring_fill",
@@ -129,7 +130,7 @@ def causal_conv1d(x, weight, bias=None, state=None, apply_silu=True):
 # ----------------------------------------------------------------------- scan
 def selective_scan(x, delta, A, Bm, Cm, Dskip=None, z=None, h0=None,
                    conv_w=None, conv_b=None, conv_state=None,
-                   delta_softplus=True, conv_silu=True, magnitudes=False):
+                   delta_softplus=True, conv_silu=True, magnitudes=False, h0_mag=None):
     """Selective SSM prefill, sequential in time.
 
     Page "SAMBA混合注意力状态空间模型", §数学框架 / Mamba层:
@@ -151,7 +152,9 @@ def selective_scan(x, delta, A, Bm, Cm, Dskip=None, z=None, h0=None,
     (Ā > 0), i.e. the size of the sums that produce y and h.  Rounding error
     of a finite-precision evaluation scales with these, not with |y|, which
     can be far smaller through cancellation; the tests measure relative
-    error against them.
+    error against them.  The magnitudes start from ``h0_mag`` (the h_mag of
+    an earlier segment, [B, D, N]) when it is given, else from |h0|, so that
+    a run split into segments carries its magnitudes like its state.
     """
     x = _f64(x)
     delta = _f64(delta)
@@ -170,7 +173,7 @@ def selective_scan(x, delta, A, Bm, Cm, Dskip=None, z=None, h0=None,
     h = np.zeros((Bsz, D, N)) if h0 is None else _f64(h0).copy()
     y = np.empty((Bsz, L, D))
     if magnitudes:
-        hm = np.abs(h)
+        hm = np.abs(h) if h0_mag is None else _f64(h0_mag).copy()
         ym = np.empty((Bsz, L, D))
     for t in range(L):
         dA = np.exp(dt[:, t, :, None] * A[None, :, :])                       # [B, D, N]
@@ -286,6 +289,50 @@ def swa(q, k, v, window, scale=None, block=64):
             o[:, i0:i1, h, :] = np.einsum("bij,bjd->bid", p / den, v[:, j0:i1, kv, :])
             lse[:, h, i0:i1] = (m + np.log(den))[:, :, 0]
     return o, lse
+
+
+def swa_blocks(q, k, v, window, starts, block=64, scale=None):
+    """Sliding-window attention for the query rows [s, s + block) of each
+    start s in ``starts`` (clipped at L), by the same definition as ``swa``:
+    the block's scores against the banded slice of keys it can see, the mask
+    0 <= i - j < W, and a max-subtracted softmax in float64.  The products
+    go through ``np.matmul``.
+
+    Returns (rows [R], o [B, R, Hq, d], lse [B, Hq, R]) with the rows of the
+    blocks in the order given.
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    Bsz, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    group = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    spans = [(int(s), min(L, int(s) + block)) for s in starts]
+    R = sum(i1 - i0 for i0, i1 in spans)
+    rows = np.empty(R, dtype=np.int64)
+    o = np.zeros((Bsz, R, Hq, d))
+    lse = np.zeros((Bsz, Hq, R))
+    r0 = 0
+    for i0, i1 in spans:
+        n = i1 - i0
+        j0 = max(0, i0 - window + 1)
+        mask = _visible(np.arange(i0, i1)[:, None], np.arange(j0, i1)[None, :], window)   # [I, J]
+        for h in range(Hq):
+            kv = h // group
+            qh = q[:, i0:i1, h, :]                                   # [B, I, d]
+            kh = k[:, j0:i1, kv, :]                                  # [B, J, d]
+            s = np.matmul(qh, np.swapaxes(kh, 1, 2)) * scale         # [B, I, J]
+            s = np.where(mask[None], s, -np.inf)
+            m = s.max(axis=2, keepdims=True)
+            p = np.exp(s - m)
+            den = p.sum(axis=2, keepdims=True)
+            o[:, r0:r0 + n, h, :] = np.matmul(p / den, v[:, j0:i1, kv, :])
+            lse[:, h, r0:r0 + n] = (m + np.log(den))[:, :, 0]
+        rows[r0:r0 + n] = np.arange(i0, i1)
+        r0 += n
+    return rows, o, lse
 
 
 def _window_positions(p, window):

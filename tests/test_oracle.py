@@ -220,6 +220,23 @@ def test_scan_split_with_carry_equals_one_pass():
         np.testing.assert_allclose(b["conv_state"], full["conv_state"], atol=0)
 
 
+def test_scan_magnitudes_carry_across_a_split():
+    """A run split in two, the second segment started from the first one's
+    state, conv state and h_mag, gives the magnitudes of one pass."""
+    i = _tiny_scan_inputs(24, Bsz=2, L=50, D=8, N=4)
+    full = orc.selective_scan(**i, magnitudes=True)
+    for cut in (1, 17, 49):
+        first = {k: (v[:, :cut] if k in ("x", "z", "delta", "Bm", "Cm") else v) for k, v in i.items()}
+        rest = {k: (v[:, cut:] if k in ("x", "z", "delta", "Bm", "Cm") else v) for k, v in i.items()}
+        a = orc.selective_scan(**first, magnitudes=True)
+        b = orc.selective_scan(**rest, h0=a["h"], conv_state=a["conv_state"], magnitudes=True, h0_mag=a["h_mag"])
+        np.testing.assert_allclose(np.concatenate([a["y_mag"], b["y_mag"]], 1), full["y_mag"], rtol=1e-12)
+        np.testing.assert_allclose(b["h_mag"], full["h_mag"], rtol=1e-12)
+        # without the carried magnitude the second segment restarts from |h|, which is smaller
+        c = orc.selective_scan(**rest, h0=a["h"], conv_state=a["conv_state"], magnitudes=True)
+        assert np.all(c["h_mag"] <= b["h_mag"] * (1 + 1e-12))
+
+
 def _scan_steps_match_prefill(L1=25, L=40):
     """Prefill of L1 tokens, then L - L1 single-token steps, against one
     prefill of L tokens: True when every step output and the final state
@@ -315,6 +332,40 @@ def test_swa_rows_equals_blocked():
     o2, lse2 = orc.swa_rows(q, k, v, 20, rows)
     np.testing.assert_allclose(o2, o[:, rows], atol=1e-13)
     np.testing.assert_allclose(lse2, lse[:, :, rows], atol=1e-13)
+
+
+@pytest.mark.parametrize("W", [1, 20, 200])
+def test_swa_blocks_match_full_masked_softmax_and_sdpa(W):
+    """The sampled-block form against a full L x L masked softmax (scipy) on
+    every requested row, and against torch's causal SDPA when W >= L."""
+    q, k, v = _attn_inputs(18, 2, 150, 8, 2, 16)
+    L, group = 150, 4
+    starts = [0, 37, 64, 140]           # the ramp, a ragged block, the tail clipped at L
+    rows, o, lse = orc.swa_blocks(q, k, v, W, starts, block=32)
+    np.testing.assert_array_equal(rows, np.concatenate([np.arange(s, min(L, s + 32)) for s in starts]))
+    i, j = np.meshgrid(np.arange(L), np.arange(L), indexing="ij")
+    visible = (j <= i) & (j > i - W)
+    for b in range(2):
+        for h in range(8):
+            sc = q[b, :, h, :] @ k[b, :, h // group, :].T / 4.0
+            sc = np.where(visible, sc, -np.inf)
+            p = scipy.special.softmax(sc, axis=1)
+            np.testing.assert_allclose(o[b, :, h, :], (p @ v[b, :, h // group, :])[rows], atol=1e-12)
+            np.testing.assert_allclose(lse[b, h], scipy.special.logsumexp(sc, axis=1)[rows], atol=1e-12)
+    if W >= L:
+        np.testing.assert_allclose(o, _sdpa_causal(q, k, v)[:, rows], atol=1e-12)
+
+
+def test_planted_swa_blocks_window_off_by_one_is_caught(monkeypatch):
+    q, k, v = _attn_inputs(19, 1, 80, 4, 2, 16)
+    _, good, _ = orc.swa_blocks(q, k, v, 16, [10, 50], block=16)
+    monkeypatch.setattr(orc, "_visible", lambda i, j, W: (i - j >= 0) & (i - j <= W))
+    _, bad, _ = orc.swa_blocks(q, k, v, 16, [10, 50], block=16)
+    assert not np.allclose(good, bad, atol=1e-6)
+    full = np.stack([scipy.special.softmax(np.where((np.arange(80)[None] <= r) & (np.arange(80)[None] > r - 16),
+                                                    q[0, r, 0] @ k[0, :, 0].T / 4.0, -np.inf), axis=1)[0]
+                     @ v[0, :, 0] for r in range(16, 26)])
+    assert not np.allclose(bad[0, 6:16, 0], full, atol=1e-6)
 
 
 def _swa_steps_match_prefill(L1, W):
