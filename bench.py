@@ -229,89 +229,196 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------- oracle leg
-def oracle_throughput(wl, n_chan=256, n_tok=2048, n_rows=64, seed=0):
-    """Times the float64 oracle, as it stands, on a bounded sample of the
-    workload and extrapolates to tokens/s of the whole mixer pair: the scan
-    on n_chan channels x n_tok tokens (cost scaled by D / n_chan), SWA on
-    n_rows query rows of every head (rows past the window's ramp)."""
+# The float64 oracle, as it stands, timed on the host cores: independent units
+# of the workload (blocks of channels for the scan; one KV head with its query
+# heads over blocks of query rows for SWA) run in a pool of one process per
+# core (spawn start method, NumPy single-threaded in each), and the throughput
+# of the whole pool is extrapolated to whole-workload tokens/s.
+
+def host_cores():
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:  # pragma: no cover
+        return max(1, os.cpu_count() or 1)
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+
+    return platform.processor() or "unknown"
+
+
+def _oracle_scan_unit(args):
+    """Oracle selective_scan on n_chan channels x n_tok tokens (one sequence)."""
+    n_chan, n_tok, N, K, seed = args
     import numpy as np
     from threadpoolctl import threadpool_limits
 
     import oracle.samba_oracle as orc
 
     rng = np.random.default_rng(seed)
-    N, K = wl.dstate, wl.dconv
     x = rng.standard_normal((1, n_tok, n_chan))
     z = rng.standard_normal((1, n_tok, n_chan))
     delta = np.log(np.expm1(np.exp(rng.uniform(math.log(1e-3), math.log(1e-1), (1, n_tok, n_chan)))))
     A = -np.tile(np.arange(1, N + 1, dtype=np.float64), (n_chan, 1))
     Bm = rng.standard_normal((1, n_tok, N))
     Cm = rng.standard_normal((1, n_tok, N))
-    Ds = rng.standard_normal(n_chan)
-    cw = rng.uniform(-0.5, 0.5, (n_chan, K))
-    cb = rng.uniform(-0.5, 0.5, n_chan)
-    span = wl.window + n_rows
-    q = rng.standard_normal((1, span, wl.heads_q, wl.head_dim))
-    k = rng.standard_normal((1, span, wl.heads_kv, wl.head_dim))
-    v = rng.standard_normal((1, span, wl.heads_kv, wl.head_dim))
-    rows = np.arange(span - n_rows, span)
     with threadpool_limits(1):
-        t0 = time.perf_counter()
-        orc.selective_scan(x, delta, A, Bm, Cm, Ds, z, conv_w=cw, conv_b=cb)
-        t_scan = time.perf_counter() - t0
-        t0 = time.perf_counter()
-        orc.swa_rows(q, k, v, wl.window, rows)
-        t_swa = time.perf_counter() - t0
-    per_token = t_scan / n_tok * (wl.dim / n_chan) + t_swa / n_rows
-    sample = (f"scan: {n_chan} of {wl.dim} channels x {n_tok} tokens ({t_scan:.1f} s, scaled by channels); "
-              f"swa: {n_rows} query rows x {wl.heads_q} heads at full window ({t_swa:.1f} s); "
-              f"float64 NumPy, extrapolated to whole-workload tokens/s")
-    return 1.0 / per_token, 1, sample
+        orc.selective_scan(x, delta, A, Bm, Cm, rng.standard_normal(n_chan), z,
+                           conv_w=rng.uniform(-0.5, 0.5, (n_chan, K)), conv_b=rng.uniform(-0.5, 0.5, n_chan))
+    return n_chan * n_tok
+
+
+def _oracle_swa_unit(args):
+    """Oracle swa_blocks: n_blocks blocks of 64 query rows of the `group`
+    query heads of one KV head, each block at a full window."""
+    group, d, W, n_blocks, seed = args
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    import oracle.samba_oracle as orc
+
+    rng = np.random.default_rng(seed)
+    span = W + 64 * n_blocks
+    q = rng.standard_normal((1, span, group, d))
+    k = rng.standard_normal((1, span, 1, d))
+    v = rng.standard_normal((1, span, 1, d))
+    with threadpool_limits(1):
+        rows, _, _ = orc.swa_blocks(q, k, v, W, [W + 64 * i for i in range(n_blocks)])
+    return len(rows)
+
+
+def _oracle_decode_unit(args):
+    """`reps` decode steps of one sequence with the oracle: scan_step on
+    n_chan channels (kind "scan") or swa_step of every head at a full ring
+    (kind "swa")."""
+    kind, n_chan, N, K, Hq, Hkv, d, W, reps, seed = args
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    import oracle.samba_oracle as orc
+
+    rng = np.random.default_rng(seed)
+    with threadpool_limits(1):
+        if kind == "scan":
+            h = rng.standard_normal((1, n_chan, N)) * 0.1
+            cs = rng.standard_normal((1, n_chan, K - 1))
+            A = -np.tile(np.arange(1, N + 1, dtype=np.float64), (n_chan, 1))
+            for _ in range(reps):
+                _, h, cs = orc.scan_step(h, cs, rng.standard_normal((1, n_chan)), rng.uniform(-6.9, -2.3, (1, n_chan)),
+                                         A, rng.standard_normal((1, N)), rng.standard_normal((1, N)),
+                                         rng.standard_normal(n_chan), rng.standard_normal((1, n_chan)),
+                                         conv_w=rng.uniform(-0.5, 0.5, (n_chan, K)),
+                                         conv_b=rng.uniform(-0.5, 0.5, n_chan))
+        else:
+            kr = rng.standard_normal((1, W, Hkv, d))
+            vr = rng.standard_normal((1, W, Hkv, d))
+            pos = np.full((1,), W + 7, dtype=np.int64)
+            for _ in range(reps):
+                _, kr, vr, pos = orc.swa_step(rng.standard_normal((1, Hq, d)), rng.standard_normal((1, Hkv, d)),
+                                              rng.standard_normal((1, Hkv, d)), kr, vr, pos, W)
+    return reps
+
+
+def oracle_pool():
+    """A pool of one oracle process per host core.  The spawn start method
+    gives every worker a fresh interpreter (no state inherited from a parent
+    that may already hold a CUDA context)."""
+    import multiprocessing as mp
+
+    return mp.get_context("spawn").Pool(host_cores())
+
+
+def _timed_map(pool, fn, units):
+    t0 = time.perf_counter()
+    done = sum(pool.map(fn, units, chunksize=1))
+    return done, time.perf_counter() - t0
+
+
+def oracle_throughput(wl, pool, scale=1.0, seed=0):
+    """Prefill tokens/s of the oracle on the host cores, from one timed
+    sample per mixer: the scan on 8 units of 32 channels x 16384 tokens per
+    core, SWA on 8 units per core of 4 blocks of 64 rows (a KV head with its
+    query heads, full window).  Returns (tokens/s, cores, sample text)."""
+    P = host_cores()
+    group = wl.heads_q // wl.heads_kv
+    n_tok = max(256, int(16384 * scale))
+    _timed_map(pool, _oracle_scan_unit, [(8, 64, wl.dstate, wl.dconv, seed)] * P)         # workers import
+    sc_units = [(32, n_tok, wl.dstate, wl.dconv, seed * 1000 + i) for i in range(8 * P)]
+    sw_units = [(group, wl.head_dim, wl.window, max(1, int(4 * scale)), seed * 1000 + i) for i in range(8 * P)]
+    sc_done, t_sc = _timed_map(pool, _oracle_scan_unit, sc_units)
+    sw_done, t_sw = _timed_map(pool, _oracle_swa_unit, sw_units)
+    per_token = t_sc / sc_done * wl.dim + t_sw / sw_done * wl.heads_kv
+    sample = (f"{P} processes on {cpu_model()}: scan {len(sc_units)} units of 32 channels x {n_tok} tokens "
+              f"({t_sc:.1f} s), SWA {len(sw_units)} units of {sw_units[0][3]} x 64 query rows x {group} heads "
+              f"at W = {wl.window} ({t_sw:.1f} s); float64 NumPy; extrapolated to whole-workload tokens/s "
+              f"(scan x {wl.dim} channels, SWA x {wl.heads_kv} KV heads per token)")
+    return 1.0 / per_token, P, sample
+
+
+def oracle_decode_throughput(wl, pool, scale=1.0, seed=0):
+    """Decode tokens/s of the oracle on the host cores: 4 units per core of
+    `reps` steps of one sequence, for the scan step (512 channels, scaled to
+    all of them) and for the SWA step (every head at a full ring)."""
+    P = host_cores()
+    reps = max(1, int(16 * scale))
+    n_chan = 512
+    dims = (wl.dstate, wl.dconv, wl.heads_q, wl.heads_kv, wl.head_dim)
+    _timed_map(pool, _oracle_decode_unit, [("scan", 8) + dims + (64, 1, 0)] * P)   # workers import
+    sc_steps, t_sc = _timed_map(pool, _oracle_decode_unit,
+                                [("scan", n_chan) + dims + (wl.window, reps, seed * 1000 + i) for i in range(4 * P)])
+    sw_steps, t_sw = _timed_map(pool, _oracle_decode_unit,
+                                [("swa", n_chan) + dims + (wl.window, reps, seed * 1000 + i) for i in range(4 * P)])
+    per_token = t_sc / sc_steps * (wl.dim / n_chan) + t_sw / sw_steps
+    sample = (f"{P} processes on {cpu_model()}: {4 * P} units of {reps} scan steps of one sequence on {n_chan} of "
+              f"{wl.dim} channels ({t_sc:.1f} s, scaled by channels) and {4 * P} units of {reps} SWA steps of "
+              f"{wl.heads_q} heads over a full {wl.window}-slot ring ({t_sw:.1f} s); float64 NumPy; extrapolated "
+              f"to tokens/s")
+    return 1.0 / per_token, P, sample
 
 
 def run_reference(args):
+    """The reference arm: the float64 oracle, as it stands, on the host cores.
+    Each step is one bounded parallel sample of the workload (a few seconds of
+    wall time); `value` is the median over the steps of the throughput
+    extrapolated to the whole workload, and `ms_per_step` the measured wall
+    time of one sampled step."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     from hybrid_ssm_sliding_b200.workloads import WORKLOADS
 
     wl = WORKLOADS[args.workload]
-    if wl.decode_steps > 0:
-        vals = []
-        t0 = time.perf_counter()
-        for s in range(max(1, args.steps)):
-            v, cores, sample = oracle_decode_throughput(wl, seed=s)
+    decode = wl.decode_steps > 0
+    measure = oracle_decode_throughput if decode else oracle_throughput
+    with oracle_pool() as pool:
+        for i in range(max(0, args.warmup)):
+            measure(wl, pool, scale=0.05, seed=1000 + i)
+        vals, walls, sample, cores = [], [], "", host_cores()
+        for i in range(max(1, args.steps)):
+            t0 = time.perf_counter()
+            v, cores, sample = measure(wl, pool, scale=0.25, seed=i)
+            walls.append(time.perf_counter() - t0)
             vals.append(v)
-        wall = time.perf_counter() - t0
-        value = statistics.median(vals)
-        print(json.dumps({
-            "impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.batch / value * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(wl),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": sample + f"; median of {args.steps} samples ({wall:.1f} s)"},
-            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-            "gpu_launches": 0}))
-        return 0
-    # Each step is a bounded sample (a few hundred ms), so K steps stay short.
-    for _ in range(max(0, args.warmup)):
-        oracle_throughput(wl, n_chan=64, n_tok=64, n_rows=1)
-    vals, samples = [], ""
-    t0 = time.perf_counter()
-    for s in range(args.steps):
-        v, cores, samples = oracle_throughput(wl, n_chan=256, n_tok=128, n_rows=2, seed=s)
-        vals.append(v)
-    wall = time.perf_counter() - t0
     value = statistics.median(vals)
-    tokens_per_step = wl.batch * wl.seqlen
+    tokens_per_step = wl.batch if decode else wl.batch * wl.seqlen
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": tokens_per_step / value * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference", "metric": DECODE_METRIC if decode else METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": len(vals), "warmup": args.warmup,
+        "ms_per_step": statistics.mean(walls) * 1e3,
+        "extrapolated_ms_per_workload_step": tokens_per_step / value * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(wl),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": samples + f"; median of {args.steps} samples ({wall:.1f} s)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample + f"; each step one such sample, median of {len(vals)} steps; value and "
+                                            f"extrapolated_ms_per_workload_step are extrapolated from the samples"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -488,7 +595,8 @@ def run_decode(args, wl, lib, dev, rank, world):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = oracle_decode_throughput(wl)
+        with oracle_pool() as pool:
+            v, cores, sample = oracle_decode_throughput(wl, pool)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
     cfg = workload_config(wl)
     sb_state = Bsz * D * N * 4 + Bsz * D * (K - 1) * 4
@@ -503,44 +611,6 @@ def run_decode(args, wl, lib, dev, rank, world):
         "kernels": kern, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
         "gpu_launches": n_steps * 3, "status": status,
     }
-
-
-def oracle_decode_throughput(wl, n_seq=2, n_chan=512, seed=0):
-    """Times the float64 oracle's decode step, as it stands, on n_seq
-    sequences (n_chan channels of the scan, every head of SWA at a full ring)
-    and extrapolates to tokens/s of the whole batch."""
-    import numpy as np
-    from threadpoolctl import threadpool_limits
-
-    import oracle.samba_oracle as orc
-
-    rng = np.random.default_rng(seed)
-    N, K, W = wl.dstate, wl.dconv, wl.window
-    h = rng.standard_normal((n_seq, n_chan, N)) * 0.1
-    cs = rng.standard_normal((n_seq, n_chan, K - 1))
-    A = -np.tile(np.arange(1, N + 1, dtype=np.float64), (n_chan, 1))
-    kr = rng.standard_normal((n_seq, W, wl.heads_kv, wl.head_dim))
-    vr = rng.standard_normal((n_seq, W, wl.heads_kv, wl.head_dim))
-    pos = np.full((n_seq,), W + 7, dtype=np.int64)
-    reps = 8
-    with threadpool_limits(1):
-        t0 = time.perf_counter()
-        for _ in range(reps):
-            orc.scan_step(h, cs, rng.standard_normal((n_seq, n_chan)), rng.uniform(-6.9, -2.3, (n_seq, n_chan)), A,
-                          rng.standard_normal((n_seq, N)), rng.standard_normal((n_seq, N)),
-                          rng.standard_normal(n_chan), rng.standard_normal((n_seq, n_chan)),
-                          conv_w=rng.uniform(-0.5, 0.5, (n_chan, K)), conv_b=rng.uniform(-0.5, 0.5, n_chan))
-        t_scan = (time.perf_counter() - t0) / reps
-        t0 = time.perf_counter()
-        for _ in range(reps):
-            orc.swa_step(rng.standard_normal((n_seq, wl.heads_q, wl.head_dim)),
-                         rng.standard_normal((n_seq, wl.heads_kv, wl.head_dim)),
-                         rng.standard_normal((n_seq, wl.heads_kv, wl.head_dim)), kr, vr, pos, W)
-        t_swa = (time.perf_counter() - t0) / reps
-    per_token = t_scan * (wl.dim / n_chan) / n_seq + t_swa / n_seq
-    sample = (f"{n_seq} sequences; scan step on {n_chan} of {wl.dim} channels ({t_scan * 1e3:.1f} ms, scaled by "
-              f"channels), SWA step over a full {W}-slot ring ({t_swa * 1e3:.1f} ms); float64 NumPy, {reps} reps")
-    return 1.0 / per_token, 1, sample
 
 
 # -------------------------------------------------------------------- GPU leg
@@ -732,7 +802,8 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = oracle_throughput(wl)
+        with oracle_pool() as pool:
+            v, cores, sample = oracle_throughput(wl, pool)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
 
     if rank == 0:
