@@ -1,5 +1,8 @@
 """Shared test helpers: error metrics and host copies of device tensors."""
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -44,3 +47,29 @@ def plain_rel_err(got, ref):
 SCAN_TOL = 1e-4          # max relative error of fp32 scan outputs and final states
 SWA_MAX_ABS = 2e-2       # bf16 attention output against the float64 oracle
 SWA_MEAN_ABS = 1e-2
+
+
+def scan_errors(got, ref, mag):
+    """The gated error (relative to the oracle's magnitudes) and the two
+    reported ones: relative to max(|r|, 1e-2 rms(r)), and plain relative
+    error over the entries with |r| >= rms(r)."""
+    return {"rel_to_mag": scan_rel_err(got, ref, mag), "rel_floor": scan_rel_err(got, ref),
+            "rel_plain": plain_rel_err(got, ref)}
+
+
+def record_margin(test, quantity, **values):
+    """Appends one measured error to the JSON-lines file named by the
+    SAMBA_MARGINS_FILE environment variable (nothing when it is unset)."""
+    path = os.environ.get("SAMBA_MARGINS_FILE")
+    if not path:
+        return
+    rec = {"test": test, "quantity": quantity}
+    rec.update({k: (float(v) if isinstance(v, (float, np.floating)) else v) for k, v in values.items()})
+    with open(path, "a") as f:
+        f.write(json.dumps(rec) + "\n")
+
+
+def nan_tensor(shape, dtype, device="cuda"):
+    """A tensor filled with NaN: outputs start poisoned, so that an element
+    the kernel never writes fails the comparison."""
+    return torch.full(shape, float("nan"), dtype=dtype, device=device)

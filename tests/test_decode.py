@@ -89,7 +89,7 @@ def test_ring_fill_then_swa_steps_match_oracle(L1, W, Hq, Hkv, d):
     kr, vr, pos = ops.swa_ring_fill(k[:, :L1].contiguous(), v[:, :L1].contiguous(), W)
     rk, rv, rpos = orc.ring_fill(host64(k[:, :L1]), host64(v[:, :L1]), W)
     full, _ = orc.swa(host64(q), host64(k), host64(v), W)
-    ws = torch.empty((ops.swa_step_workspace_size(Bsz, Hq, d, W),), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros((ops.swa_step_workspace_size(Bsz, Hq, d, W),), dtype=torch.uint8, device="cuda")
     for t in range(L1, Ln):
         o_t = ops.swa_step(q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(), kr, vr, pos, W,
                            workspace=ws)
