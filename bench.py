@@ -458,7 +458,7 @@ def run_decode(args, wl, lib, dev, rank, world):
     steps_in = [make_decode_step_inputs(wl_rank, s, device=dev) for s in range(G)]
     y_t = torch.empty((Bsz, D), dtype=torch.bfloat16, device=dev)
     o_t = torch.empty((Bsz, wl.heads_q, wl.head_dim), dtype=torch.bfloat16, device=dev)
-    ws = torch.empty((max(ops.swa_step_workspace_size(Bsz, wl.heads_q, wl.head_dim, wl.window), 16),),
+    ws = torch.zeros((max(ops.swa_step_workspace_size(Bsz, wl.heads_q, wl.head_dim, wl.window), 16),),
                      dtype=torch.uint8, device=dev)
 
     def scan_one(si, ly, y_out=None):
@@ -709,6 +709,12 @@ def main():
 
     ms_scan = time_kernel(lambda: L.check(lib.samba_selective_scan_fwd(ctypes.byref(sa), sh)), args.kernel_steps)
     ms_swa = time_kernel(lambda: L.check(lib.samba_swa_fwd(ctypes.byref(wa), sh)), args.kernel_steps)
+    # the same call with the attention forked onto a second stream (reported
+    # beside the headline, which runs both mixers on one stream)
+    aux = torch.cuda.Stream()
+    ms_two_stream = time_kernel(
+        lambda: L.check(lib.samba_mixer_prefill(ctypes.byref(sa), ctypes.byref(wa), sh, aux.cuda_stream)),
+        args.kernel_steps)
     peaks = load_peaks()
     sb = scan_bytes(wl)
     sf = swa_flops(wl)
@@ -812,6 +818,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(wl),
             "roofline": roofline, "kernels": {"scan": scan_roof, "swa": swa_roof},
+            "two_stream_ms_per_step": ms_two_stream,
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "gpu_launches": 2 * args.steps,
             "status": status,
         }
