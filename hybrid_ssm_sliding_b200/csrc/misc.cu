@@ -305,8 +305,8 @@ template <int HD>
 __global__ void __launch_bounds__(StepCfg<HD>::CH) swa_step_split_kernel(
     const __nv_bfloat16* __restrict__ q_t, const __nv_bfloat16* __restrict__ k_t,
     const __nv_bfloat16* __restrict__ v_t, __nv_bfloat16* __restrict__ k_ring, __nv_bfloat16* __restrict__ v_ring,
-    int64_t* __restrict__ pos, float* __restrict__ ws, unsigned* __restrict__ cnt, __nv_bfloat16* __restrict__ o_t,
-    int Hq, int Hkv, int64_t W, float scale_log2, int nsplit) {
+    const int64_t* __restrict__ pos, float* __restrict__ ws, int Hq, int Hkv, int64_t W, float scale_log2,
+    int nsplit) {
   using Cfg = StepCfg<HD>;
   constexpr int CH = Cfg::CH, NWARP = Cfg::NWARP, KP = Cfg::KP, PP = Cfg::PP;
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -482,101 +482,42 @@ __global__ void __launch_bounds__(StepCfg<HD>::CH) swa_step_split_kernel(
       }
     }
   }
-
-  // ---- the last CTA of (b, g) to finish combines the splits
-  // Every CTA publishes its partials (store, fence, then one count per CTA);
-  // the CTA that brings the count of (b, g) to nsplit reads all of them
-  // back from L2 and writes o_t for the group's heads, then resets the count.
-  // The last (b, g) of batch b to finish advances pos[b]: by then every CTA
-  // of batch b has read pos.  Nothing waits, so nothing can hang.
-  __shared__ unsigned s_last;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = atomicAdd(&cnt[(int64_t)b * Hkv + g], 1u) == (unsigned)nsplit - 1u;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  // Weights of the splits per head, 2^(m_s - M) / sum_s l_s 2^(m_s - M), one
-  // warp per head (lanes over the splits); kept in shared memory when they
-  // fit, so that the outputs below need one more round trip to L2 only.
-  constexpr int kMaxSplitW = 64;
-  __shared__ float s_f[16][kMaxSplitW];
-  const bool in_smem = nsplit <= kMaxSplitW;
-  __shared__ float s_M[16], s_inv[16];
-  for (int hh = warp; hh < group; hh += NWARP) {
-    const float* base = ws + (((int64_t)b * Hq + g * group + hh) * nsplit) * (HD + 2);
-    float M = -INFINITY;
-    for (int sp = lane; sp < nsplit; sp += 32) M = fmaxf(M, __ldcg(base + sp * (HD + 2)));
-#pragma unroll
-    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float l = 0.f;
-    for (int sp = lane; sp < nsplit; sp += 32) {
-      const float m = __ldcg(base + sp * (HD + 2));
-      const float f = (m == -INFINITY) ? 0.f : ex2_approx(m - M);
-      l = fmaf(__ldcg(base + sp * (HD + 2) + 1), f, l);
-      if (in_smem) s_f[hh][sp] = f;
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (lane == 0) {
-      s_M[hh] = M;
-      s_inv[hh] = 1.0f / l;
-    }
-  }
-  __syncthreads();
-  for (int e = tid; e < group * HD; e += CH) {
-    const int hh = e / HD, dd = e % HD;
-    const float* base = ws + (((int64_t)b * Hq + g * group + hh) * nsplit) * (HD + 2);
-    float acc = 0.f;
-    if (in_smem) {
-#pragma unroll 16
-      for (int sp = 0; sp < nsplit; ++sp) acc = fmaf(__ldcg(base + sp * (HD + 2) + 2 + dd), s_f[hh][sp], acc);
-    } else {
-      const float M = s_M[hh];
-#pragma unroll 8
-      for (int sp = 0; sp < nsplit; ++sp) {
-        const float m = __ldcg(base + sp * (HD + 2));
-        const float f = (m == -INFINITY) ? 0.f : ex2_approx(m - M);
-        acc = fmaf(__ldcg(base + sp * (HD + 2) + 2 + dd), f, acc);
-      }
-    }
-    o_t[((int64_t)b * Hq + g * group + hh) * HD + dd] = __float2bfloat16_rn(acc * s_inv[hh]);
-  }
-  if (tid == 0) {
-    cnt[(int64_t)b * Hkv + g] = 0u;
-    unsigned* cnt_b = cnt + (int64_t)gridDim.z * Hkv;
-    if (atomicAdd(&cnt_b[b], 1u) == (unsigned)Hkv - 1u) {
-      pos[b] += 1;
-      cnt_b[b] = 0u;
-    }
-  }
 }
 
-// Workspace of the decode SWA step: the split partials, (max, sum, d
-// outputs) per (batch, query head, split) as floats, then the completion
-// counts: one per (batch, KV head) followed by one per batch, in a region
-// sized B * (Hq + 1) (Hkv <= Hq, so the size needs only the query heads).
-// SIZE_MAX when the byte count does not fit in size_t, so that no workspace
-// (and no built-in scratch) is ever taken as large enough.
-static bool swa_step_layout(int64_t B, int Hq, int d, int64_t W, uint64_t* partial_bytes, uint64_t* total_bytes) {
+template <int HD>
+__global__ void swa_step_combine_kernel(const float* __restrict__ ws, __nv_bfloat16* __restrict__ o_t,
+                                        int64_t* __restrict__ pos, int Hq, int nsplit) {
+  const int hq = blockIdx.x, b = blockIdx.y;
+  const int dd = threadIdx.x;
+  const float* base = ws + ((int64_t)b * Hq + hq) * nsplit * (HD + 2);
+  // the loops are unrolled so that the loads of several splits are in flight
+  float M = -INFINITY;
+#pragma unroll 8
+  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, base[s * (HD + 2)]);
+  float l = 0.f, acc = 0.f;
+#pragma unroll 8
+  for (int s = 0; s < nsplit; ++s) {
+    const float m = base[s * (HD + 2)];
+    const float f = (m == -INFINITY) ? 0.f : ex2_approx(m - M);
+    l = fmaf(base[s * (HD + 2) + 1], f, l);
+    acc = fmaf(base[s * (HD + 2) + 2 + dd], f, acc);
+  }
+  o_t[((int64_t)b * Hq + hq) * HD + dd] = __float2bfloat16_rn(acc / l);
+  if (hq == 0 && dd == 0) pos[b] += 1;
+}
+
+// Bytes of split partials: (max, sum, d outputs) per (batch, query head,
+// split).  SIZE_MAX when the product does not fit in size_t, so that no
+// workspace (and no built-in scratch) is ever taken as large enough.
+size_t swa_step_workspace(int64_t B, int Hq, int d, int64_t W) {
   const int ch = d <= 64 ? StepCfg<64>::CH : StepCfg<128>::CH;
   const uint64_t nsplit = static_cast<uint64_t>((W + ch - 1) / ch);
-  uint64_t n = 0, c = 0;
+  uint64_t n = 0;
   if (__builtin_mul_overflow(static_cast<uint64_t>(B), static_cast<uint64_t>(Hq), &n) ||
       __builtin_mul_overflow(n, nsplit, &n) || __builtin_mul_overflow(n, static_cast<uint64_t>(d + 2), &n) ||
-      __builtin_mul_overflow(n, static_cast<uint64_t>(sizeof(float)), &n) ||
-      __builtin_mul_overflow(static_cast<uint64_t>(B), static_cast<uint64_t>(Hq) + 1u, &c) ||
-      __builtin_mul_overflow(c, static_cast<uint64_t>(sizeof(unsigned)), &c))
-    return false;
-  n = (n + 255) / 256 * 256;  // counters start on their own 256-byte line
-  if (__builtin_add_overflow(n, c, total_bytes) || *total_bytes > SIZE_MAX) return false;
-  *partial_bytes = n;
-  return true;
-}
-
-size_t swa_step_workspace(int64_t B, int Hq, int d, int64_t W) {
-  uint64_t part = 0, total = 0;
-  return swa_step_layout(B, Hq, d, W, &part, &total) ? static_cast<size_t>(total) : SIZE_MAX;
+      __builtin_mul_overflow(n, static_cast<uint64_t>(sizeof(float)), &n) || n > SIZE_MAX)
+    return SIZE_MAX;
+  return static_cast<size_t>(n);
 }
 
 template <int HD>
@@ -584,15 +525,15 @@ static void swa_step_go(const void* q_t, const void* k_t, const void* v_t, void*
                         void* o_t, int64_t B, int Hq, int Hkv, int64_t W, float scale, void* ws, cudaStream_t s) {
   constexpr int CH = StepCfg<HD>::CH;
   const int nsplit = (int)((W + CH - 1) / CH);
-  uint64_t part = 0, total = 0;
-  swa_step_layout(B, Hq, HD, W, &part, &total);  // checked by the caller
-  unsigned* cnt = reinterpret_cast<unsigned*>(reinterpret_cast<unsigned char*>(ws) + part);
   dim3 g1(nsplit, Hkv, (unsigned)B);
   swa_step_split_kernel<HD><<<g1, CH, 0, s>>>(
       reinterpret_cast<const __nv_bfloat16*>(q_t), reinterpret_cast<const __nv_bfloat16*>(k_t),
       reinterpret_cast<const __nv_bfloat16*>(v_t), reinterpret_cast<__nv_bfloat16*>(k_ring),
-      reinterpret_cast<__nv_bfloat16*>(v_ring), pos, reinterpret_cast<float*>(ws), cnt,
-      reinterpret_cast<__nv_bfloat16*>(o_t), Hq, Hkv, W, scale * 1.4426950408889634f, nsplit);
+      reinterpret_cast<__nv_bfloat16*>(v_ring), pos, reinterpret_cast<float*>(ws), Hq, Hkv, W,
+      scale * 1.4426950408889634f, nsplit);
+  dim3 g2(Hq, (unsigned)B);
+  swa_step_combine_kernel<HD><<<g2, HD, 0, s>>>(reinterpret_cast<const float*>(ws),
+                                                 reinterpret_cast<__nv_bfloat16*>(o_t), pos, Hq, nsplit);
 }
 
 int launch_swa_step(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring, int64_t* pos,

@@ -206,8 +206,8 @@ def swa_step(q_t, k_t, v_t, k_ring, v_ring, pos, window, scale=None, o_t=None, w
     if o_t is None:
         o_t = torch.empty_like(q_t)
     nbytes = swa_step_workspace_size(Bsz, Hq, d, window)
-    if workspace is None:  # zero-filled: the step's completion counters start at zero
-        workspace = torch.zeros((max(nbytes, 16),), dtype=torch.uint8, device=q_t.device)
+    if workspace is None:
+        workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=q_t.device)
     _need(workspace, "workspace", torch.uint8)
     L.check(L.load().samba_swa_step(L.ptr(q_t), L.ptr(k_t), L.ptr(v_t), L.ptr(k_ring), L.ptr(v_ring), L.ptr(pos),
                                     L.ptr(o_t), Bsz, Hq, Hkv, d, window, float(scale) if scale else 0.0,

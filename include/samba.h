@@ -243,15 +243,10 @@ size_t samba_swa_step_workspace_size(int64_t batch, int heads_q, int head_dim, i
  * pos[b] mod W, then each query q_t ([B, Hq, d]) attends the keys of
  * positions max(0, pos-W+1) .. pos and writes o_t ([B, Hq, d] bf16); finally
  * pos[b] += 1.  All of it happens on the device (pos is a device int64 [B]),
- * so consecutive steps can be captured in one CUDA graph.  The step is one
- * kernel: CTAs over (window chunk, KV head, sequence) write split partial
- * results, and the last CTA of each (sequence, KV head) to finish combines
- * them.  `workspace` is caller-owned device memory of at least
- * samba_swa_step_workspace_size() bytes: the split partials, then completion
- * counters.  It must be zero-filled before the first call that uses it (for
- * example with cudaMemsetAsync); every call leaves the counters at zero again,
- * so later calls need no initialisation.  Calls that may run at the same time
- * on the GPU need separate workspaces.  scale <= 0 selects 1/sqrt(d).
+ * so consecutive steps can be captured in one CUDA graph.  `workspace` is
+ * caller-owned device memory of at least samba_swa_step_workspace_size()
+ * bytes (split partial results); it needs no initialisation.  scale <= 0
+ * selects 1/sqrt(d).
  * Errors: SAMBA_ERR_INVALID_ARG for a null pointer, a non-positive size, Hq
  * not a multiple of Hkv or a pointer (workspace included) not 16-byte
  * aligned; SAMBA_ERR_UNSUPPORTED for Hq/Hkv > 16, d outside the set above
@@ -268,13 +263,12 @@ int samba_swa_step(const void* q_t, const void* k_t, const void* v_t, void* k_ri
  * running where a cudaMalloc would be refused or would synchronise the device.
  * Such a caller has no way to pass samba_swa_step a workspace.
  *
- * The split partials and the completion counters live in a 4 MiB array inside
- * the library (a file-scope __device__ array, zero-filled when the library's
- * device code is loaded), which every GPU that loads the library holds until
- * the process exits.  Calls that need more, that is
+ * The split partials live in a 4 MiB array inside the library (a file-scope
+ * __device__ array), which every GPU that loads the library holds until the
+ * process exits.  Calls whose partials do not fit, that is
  * samba_swa_step_workspace_size(batch, heads_q, head_dim, window) > 4 MiB,
  * are rejected with SAMBA_ERR_WORKSPACE before anything is launched; the
- * 16 x 32-head, d = 64, W = 2048 decode needs 2.17 MB.
+ * 16 x 32-head, d = 64, W = 2048 decode needs 1.08 MB.
  *
  * Every call looks up the array's device address (cudaGetSymbolAddress) on
  * the current device; this is a table lookup once the library's device code
@@ -283,11 +277,10 @@ int samba_swa_step(const void* q_t, const void* k_t, const void* v_t, void* k_ri
  * stream capture.  The function calls no cudaMalloc, cudaFree or other
  * allocating routine.
  *
- * Every call shares the one array and finds the previous call's contents in
- * it.  That is harmless: each step writes every partial it reads, and the
- * counters, which must start at zero, are zero when the array is loaded and
- * are left at zero by every call.  But two calls that may run at the same
- * time on the GPU (different streams, or different threads without ordering)
+ * Every call shares the one array and finds the previous call's partials in
+ * it.  That is harmless, because each step writes every partial it reads and
+ * nothing has to start at zero.  But two calls that may run at the same time
+ * on the GPU (different streams, or different threads without ordering)
  * race on the array and give wrong results; order them, or use
  * samba_swa_step with separate workspaces.
  *
