@@ -20,12 +20,17 @@
 //     masked element by element.
 //   * Warp 8 issues TMA: Q once per unit into one of two buffers (so the
 //     next unit's Q lands while this one is finishing), K and V per key tile
-//     into a STG-deep ring.  Warp 9 owns tensor memory and issues every
-//     tcgen05.mma, the whole warp in lock-step with one elected lane issuing:
-//     S = Q·Kᵀ (bf16, fp32 accumulate into TMEM) and O += P·V with P read
-//     straight from TMEM.  Over the flat sequence of key tiles (crossing
-//     unit boundaries) it issues S of tile t+1 into the columns of S(t) as
-//     soon as the softmax has read them, so Q·Kᵀ runs under the exps.
+//     into a STG-deep ring.  Warps 9 and 10 issue the tcgen05.mma of Q tiles
+//     A and B (warp 9 also owns the tensor memory), each whole warp in
+//     lock-step with one elected lane issuing: S = Q·Kᵀ (bf16, fp32
+//     accumulate into TMEM) and O += P·V with P read straight from TMEM.
+//     Over the flat sequence of key tiles (crossing unit boundaries) each
+//     issues S of tile t+1 into the columns of S(t) as soon as its softmax
+//     has read them, so Q·Kᵀ runs under the exps.  With one issuing warp per
+//     Q tile, neither tile's MMAs wait behind the other tile's softmax, and
+//     the softmax of B starts its first tile only once A has written its
+//     first P, so that the two softmax warpgroups do not reach their exp
+//     loops (the special-function unit) at the same time.
 //   * Warps 0-3 and 4-7 are the softmax warpgroups of Q tiles A and B:
 //     each thread owns one row, reads its S row from TMEM, keeps the running
 //     max and sum in fp32, writes P back to TMEM as bf16 (16 packed pairs at
@@ -62,24 +67,27 @@ struct SwaCfg {
   static constexpr int SMEM = BAR_OFF + 256 + 1024;        // + alignment slack
   static constexpr uint32_t SWZ = HD == 64 ? 2u : (HD == 32 ? 4u : 6u);  // descriptor swizzle code
   static constexpr uint32_t ATOM = 8 * ROW_BYTES;          // 8-row swizzle atom
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 352;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_P = 256, COL_O = 384;
 };
 
 // Warp roles: 0-3 softmax of Q tile A, 4-7 softmax of Q tile B (warp % 4 is
 // the TMEM lane quarter a warp may access; thread i of warp w owns row
-// 32 (w % 4) + i of its tile), 8 TMA producer, 9 MMA issuer.
-constexpr int kSoftmaxWarps = 8, kWarpTma = 8, kWarpMma = 9;
+// 32 (w % 4) + i of its tile), 8 TMA producer, 9 and 10 MMA issuers of Q
+// tiles A and B.
+constexpr int kSoftmaxWarps = 8, kWarpTma = 8, kWarpMma = 9, kWarpMmaB = 10;
 
 // Barrier indices inside the barrier block.  Per Q tile X in {A, B}:
 // BS_X  S_X of the next key tile is in TMEM          (tcgen05.commit)
 // BSF_X the softmax of X has read S_X into registers (one arrival per warp)
 // BP_X  P_X is in TMEM                               (one arrival per warp)
 // BO_X  O_X += P_X V has completed                   (tcgen05.commit)
+// BQ_EMPTY and the K/V stages' empty barriers take one commit from each of
+// the two MMA warps (count 2): a buffer is free once both tiles are done.
 enum : int {
   BQ_FULL0 = 0, BQ_FULL1, BQ_EMPTY0, BQ_EMPTY1, BS_A, BS_B, BSF_A, BSF_B, BP_A, BP_B, BO_A, BO_B,
-  BMMA_DONE, B_STAGE0
+  BMMA_DONE, BMMA_DONE_B, B_STAGE0
 };
 
 __device__ __forceinline__ float ex2f(float x) {
@@ -91,7 +99,7 @@ __device__ __forceinline__ float ex2f(float x) {
 // Every SWA_POLY-th pair of probabilities is evaluated on the FMA pipe
 // (0: never); the rest use the MUFU ex2.  Build-time, fixed by measurement.
 #ifndef SWA_POLY
-#define SWA_POLY 4
+#define SWA_POLY 8
 #endif
 
 // 2^x for a pair of arguments on the FMA pipe, accurate to ~1e-4 relative
@@ -183,7 +191,7 @@ __device__ __forceinline__ bool cursor_next(TileCursor& c, const SwaParams& p, i
 
 
 template <int HD, int GROUP, int STG>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     swa_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v, const SwaParams p) {
   using Cfg = SwaCfg<HD, GROUP, STG>;
@@ -202,7 +210,10 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = BQ_FULL0; i <= BQ_EMPTY1; ++i) mbar_init(&bars[i], 1);
+    mbar_init(&bars[BQ_FULL0], 1);
+    mbar_init(&bars[BQ_FULL1], 1);
+    mbar_init(&bars[BQ_EMPTY0], 2);
+    mbar_init(&bars[BQ_EMPTY1], 2);
     mbar_init(&bars[BS_A], 1);
     mbar_init(&bars[BS_B], 1);
     mbar_init(&bars[BSF_A], kSoftmaxWarps / 2);
@@ -212,9 +223,10 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(&bars[BO_A], 1);
     mbar_init(&bars[BO_B], 1);
     mbar_init(&bars[BMMA_DONE], 1);
+    mbar_init(&bars[BMMA_DONE + 1], 1);
     for (int s = 0; s < STG; ++s) {
       mbar_init(&kvfull[s], 1);
-      mbar_init(&kvempty[s], 1);
+      mbar_init(&kvempty[s], 2);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -265,13 +277,12 @@ __global__ void __launch_bounds__(320, 1)
         for (uint32_t n = (nu > 2 ? nu - 2 : 0); n < nu; ++n) mbar_wait(&bars[BQ_FULL0 + (n & 1)], (n >> 1) & 1, &never);
       }
     }
-  } else if (warp == kWarpMma) {
+  } else if (warp == kWarpMma || warp == kWarpMmaB) {
     // ================================================================ MMA
-    // The whole warp runs this loop in lock-step; each tcgen05 instruction
-    // is issued by one elected lane.  Over the flat sequence of key tiles t
-    // (crossing unit boundaries) the issue order is S_A(t+1) and S_B(t+1) as
-    // soon as the softmax has read S(t), then O_A += P_A(t) V(t) and
-    // O_B += P_B(t) V(t) as P arrives; the stage of tile t is then free.
+    // One warp per Q tile X: S_X(t+1) as soon as the softmax of X has read
+    // S_X(t), then O_X += P_X(t) V(t) once P_X(t) is in TMEM.  The stage of
+    // tile t is free when both warps have committed their P·V (count 2).
+    const int x = warp - kWarpMma;  // Q tile A (0) or B (1)
     constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
     constexpr uint32_t IDESC_O = idesc_bf16_f32(128, HD, 0, 1);
     const uint32_t q_base = smem_u32(smem + Cfg::Q_OFF);
@@ -293,7 +304,7 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lo_v0 = static_cast<uint32_t>(d_v0);
     constexpr uint32_t kTileDesc = Cfg::TILE_BYTES >> 4;
     auto desc64 = [](uint32_t lo, uint32_t hi) { return (static_cast<uint64_t>(hi) << 32) | lo; };
-    auto issue_s = [&](int x, uint32_t qb, uint32_t stage) {
+    auto issue_s = [&](uint32_t qb, uint32_t stage) {
       const uint32_t lq = lo_q0 + (2 * qb + x) * kTileDesc;
       const uint32_t lk = lo_k0 + stage * kTileDesc;
 #pragma unroll
@@ -301,14 +312,17 @@ __global__ void __launch_bounds__(320, 1)
         umma_ss_w(tmem + Cfg::COL_S + 128 * x, desc64(lq + 2 * k, hi_qk), desc64(lk + 2 * k, hi_qk), IDESC_S,
                   k > 0 ? 1u : 0u);
     };
-    auto issue_pv = [&](int x, uint32_t stage, bool first) {
+    auto issue_pv = [&](uint32_t stage, bool first) {
       const uint32_t lv = lo_v0 + stage * kTileDesc;
 #pragma unroll
       for (int k = 0; k < 8; ++k)  // 16 keys per step = two 8-row atoms of V
         umma_ts_w(tmem + Cfg::COL_O + 64 * x, tmem + Cfg::COL_P + 64 * x + 8 * k,
                   desc64(lv + k * (Cfg::ROW_BYTES), hi_v), IDESC_O, (first && k == 0) ? 0u : 1u);
     };
-
+    uint64_t* bar_s = &bars[BS_A + x];
+    uint64_t* bar_sf = &bars[BSF_A + x];
+    uint64_t* bar_p = &bars[BP_A + x];
+    uint64_t* bar_o = &bars[BO_A + x];
     TileCursor cs;  // tile t
     bool more = cursor_begin(cs, p, TOK2);
     bool first_cur = true;
@@ -316,10 +330,8 @@ __global__ void __launch_bounds__(320, 1)
       ok = wait(&bars[BQ_FULL0], 0) && wait(&kvfull[0], 0);
       if (ok) {
         tc_fence_after();
-        issue_s(0, 0, 0);
-        tc_commit_w(&bars[BS_A]);
-        issue_s(1, 0, 0);
-        tc_commit_w(&bars[BS_B]);
+        issue_s(0, 0);
+        tc_commit_w(bar_s);
         if (cs.nt == 1) tc_commit_w(&bars[BQ_EMPTY0]);
       }
     }
@@ -329,37 +341,36 @@ __global__ void __launch_bounds__(320, 1)
       const bool first_next = has_next && cn.jt == 0;
       const uint32_t s = t % STG, sn = (t + 1) % STG;
       const uint32_t qbn = cn.nu & 1;
-      if (has_next) {
-        if (first_next && !wait(&bars[BQ_FULL0 + qbn], (cn.nu >> 1) & 1)) { ok = false; break; }
-        if (!wait(&kvfull[sn], ((t + 1) / STG) & 1)) { ok = false; break; }
-        if (!wait(&bars[BSF_A], t & 1)) { ok = false; break; }
+      auto next_s = [&]() {  // S of tile t + 1, once its K/V (and Q) landed and S(t) was read
+        if (first_next && !wait(&bars[BQ_FULL0 + qbn], (cn.nu >> 1) & 1)) return false;
+        if (!wait(&kvfull[sn], ((t + 1) / STG) & 1)) return false;
+        if (!wait(bar_sf, t & 1)) return false;
         tc_fence_after();
-        issue_s(0, qbn, sn);
-        tc_commit_w(&bars[BS_A]);
-        if (!wait(&bars[BSF_B], t & 1)) { ok = false; break; }
-        tc_fence_after();
-        issue_s(1, qbn, sn);
-        tc_commit_w(&bars[BS_B]);
+        issue_s(qbn, sn);
+        tc_commit_w(bar_s);
         if (cn.jt == cn.nt - 1) tc_commit_w(&bars[BQ_EMPTY0 + qbn]);
-      }
-      if (!wait(&bars[BP_A], t & 1)) { ok = false; break; }
-      tc_fence_after();
-      issue_pv(0, s, first_cur);
-      tc_commit_w(&bars[BO_A]);
-      if (!wait(&bars[BP_B], t & 1)) { ok = false; break; }
-      tc_fence_after();
-      issue_pv(1, s, first_cur);
-      tc_commit_w(&bars[BO_B]);
-      tc_commit_w(&kvempty[s]);
+        return true;
+      };
+      auto this_pv = [&]() {  // O += P(t) V(t) once P(t) is in TMEM; then stage s is free
+        if (!wait(bar_p, t & 1)) return false;
+        tc_fence_after();
+        issue_pv(s, first_cur);
+        tc_commit_w(bar_o);
+        tc_commit_w(&kvempty[s]);
+        return true;
+      };
+      // S(t+1) goes first, so that Q·Kᵀ runs under the softmax of tile t.
+      ok = (!has_next || next_s()) && this_pv();
+      if (!ok) break;
       first_cur = first_next;
       cs = cn;
       more = has_next;
     }
     // Wait until every MMA issued by this warp has finished before the
     // tensor memory can be released.
-    tc_commit_w(&bars[BMMA_DONE]);
+    tc_commit_w(&bars[BMMA_DONE + x]);
     volatile int never = 0;
-    mbar_wait(&bars[BMMA_DONE], 0, &never);
+    mbar_wait(&bars[BMMA_DONE + x], 0, &never);
   } else if (warp < kSoftmaxWarps) {
     // ============================================================ softmax
     const int x = warp >> 2;                  // Q tile A or B
@@ -388,6 +399,8 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) mbar_arrive(bar);
     };
 
+    // Tile B starts once tile A has written its first P (see the header).
+    if (x == 1 && (int)blockIdx.x < p.total_units) ok = wait(&bars[BP_A], 0);
     for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
       int b, g;
       int64_t i0;
@@ -419,9 +432,15 @@ __global__ void __launch_bounds__(320, 1)
           const int64_t lw = irow - p.W + 1 - k0;
           const int lo = (int)(lo64 > lw ? lo64 : lw);
           const int hi = (int)(irow - k0);
+          // Branch-free: one unsigned compare and one select per column
+          // (c - lo wraps to a large value for c < lo).  A row that sees no
+          // key of this tile (hi < lo: the tile lies in its future, or below
+          // its window) gets an empty interval.
+          const int span_i = hi - lo;
+          const unsigned span = span_i < 0 ? 0u : static_cast<unsigned>(span_i);
+          const int lo_e = span_i < 0 ? (1 << 20) : lo;
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c < lo || c > hi) sc[c] = -INFINITY;
+          for (int c = 0; c < 128; ++c) sc[c] = ((unsigned)(c - lo_e) <= span) ? sc[c] : -INFINITY;
         }
         // Row max: eight chains of three-input maxima, chain q over the
         // columns c = q (mod 8).
