@@ -565,7 +565,7 @@ int take_status_swa(cudaStream_t s) { return take_status_word(s); }
 
 // K/V ring depth (stages of one K and one V tile each); build-time.
 #ifndef SWA_STAGES
-#define SWA_STAGES 4
+#define SWA_STAGES 5
 #endif
 
 template <int HD, int GROUP>
