@@ -61,6 +61,9 @@ __all__ = [
     "swa",
     "swa_rows",
     "swa_blocks",
+    "round_bf16",
+    "mamba_layer",
+    "swa_layer",
     "scan_step",
     "swa_step",
     "ring_fill",
@@ -333,6 +336,69 @@ def swa_blocks(q, k, v, window, starts, block=64, scale=None):
         rows[r0:r0 + n] = np.arange(i0, i1)
         r0 += n
     return rows, o, lse
+
+
+# --------------------------------------------------------------- layers
+def round_bf16(a):
+    """Rounds to bfloat16 (round to nearest, ties to even) and back to
+    float64: the value a bf16 activation holds.  The rounding goes through
+    float32 (as a kernel's fp32 result is stored as bf16)."""
+    f = np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+    bits = f.view(np.uint32).astype(np.uint64)
+    rounded = ((bits + 0x7FFF + ((bits >> 16) & 1)) & 0xFFFF0000).astype(np.uint32)
+    return rounded.view(np.float32).astype(np.float64)
+
+
+def mamba_layer(hidden, in_proj, conv_w, conv_b, x_proj, dt_proj, dt_bias, A, Dskip, out_proj,
+                bf16_activations=True):
+    """A Mamba layer around the selective scan (page "SAMBA混合注意力状态空间
+    模型", section 数学框架 / Mamba层: B_t = Linear_B(x_t), C_t = Linear_C(x_t),
+    Δ_t = τ_Δ(Linear_Δ(x_t))), with the readings of the layer the paper builds
+    on: [x, z] = hidden · in_projᵀ; u = SiLU(conv1d(x)); [δ_low, B, C] =
+    u · x_projᵀ; delta = δ_low · dt_projᵀ + dt_bias, Δ = softplus(delta);
+    y = scan(u, Δ, A, B, C, D, z); out = y · out_projᵀ.
+
+    hidden [B, L, d_model]; in_proj [2D, d_model]; conv_w [D, K]; conv_b [D];
+    x_proj [R + 2N, D]; dt_proj [D, R]; dt_bias [D]; A [D, N]; Dskip [D];
+    out_proj [d_model, D].  With ``bf16_activations`` the tensors a bf16
+    dataflow stores in bf16 (x, z, u, δ_low, y, out) are rounded to bf16.
+    Returns dict(out, h, conv_state).
+    """
+    rnd = round_bf16 if bf16_activations else (lambda t: t)
+    hidden = _f64(hidden)
+    D, N, R = _f64(A).shape[0], _f64(A).shape[1], _f64(dt_proj).shape[1]
+    xz = np.matmul(hidden, _f64(in_proj).T)
+    x, z = rnd(xz[..., :D]), rnd(xz[..., D:])
+    u, conv_state = causal_conv1d(x, conv_w, conv_b, None, apply_silu=True)
+    u = rnd(u)
+    dbc = np.matmul(u, _f64(x_proj).T)
+    dt_low = rnd(dbc[..., :R])
+    Bm, Cm = dbc[..., R:R + N], dbc[..., R + N:R + 2 * N]
+    delta = np.matmul(dt_low, _f64(dt_proj).T) + _f64(dt_bias)
+    sc = selective_scan(u, delta, A, Bm, Cm, Dskip, z)
+    y = rnd(sc["y"])
+    out = rnd(np.matmul(y, _f64(out_proj).T))
+    return {"out": out, "h": sc["h"], "conv_state": conv_state}
+
+
+def swa_layer(hidden, qkv_proj, o_proj, heads_q, heads_kv, head_dim, window, bf16_activations=True):
+    """A sliding-window attention layer around the banded attention: [q, k, v]
+    = hidden · qkv_projᵀ (column ranges H_q·d, H_kv·d, H_kv·d, each row of a
+    range laid out as heads × head_dim); o = SWA(q, k, v); out = o · o_projᵀ.
+    With ``bf16_activations`` q, k, v, o and out are rounded to bf16.
+    Returns dict(out, k, v)."""
+    rnd = round_bf16 if bf16_activations else (lambda t: t)
+    hidden = _f64(hidden)
+    Bsz, L, _ = hidden.shape
+    nq, nk = heads_q * head_dim, heads_kv * head_dim
+    qkv = np.matmul(hidden, _f64(qkv_proj).T)
+    q = rnd(qkv[..., :nq]).reshape(Bsz, L, heads_q, head_dim)
+    k = rnd(qkv[..., nq:nq + nk]).reshape(Bsz, L, heads_kv, head_dim)
+    v = rnd(qkv[..., nq + nk:nq + 2 * nk]).reshape(Bsz, L, heads_kv, head_dim)
+    o, _ = swa(q, k, v, window)
+    o = rnd(o)
+    out = rnd(np.matmul(o.reshape(Bsz, L, nq), _f64(o_proj).T))
+    return {"out": out, "k": k, "v": v}
 
 
 def _window_positions(p, window):

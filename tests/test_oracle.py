@@ -486,3 +486,79 @@ def test_planted_scan_step_state_dropped_is_caught(monkeypatch):
     assert not _scan_steps_match_prefill()
     monkeypatch.undo()
     assert _scan_steps_match_prefill()
+
+
+# ------------------------------------------------------------------ layers
+def test_round_bf16_matches_torch_conversion():
+    r = _rng(30)
+    vals = np.concatenate([r.standard_normal(4000) * 10.0 ** r.integers(-8, 8, 4000),
+                           1.0 + np.arange(64) * 2.0 ** -8])          # exact ties included
+    ref = torch.from_numpy(vals.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(orc.round_bf16(vals), ref)
+
+
+def _layer_weights(seed, dm=24, D=16, N=4, K=4, R=3):
+    r = _rng(seed)
+    return dict(in_proj=r.standard_normal((2 * D, dm)) / 5, conv_w=r.uniform(-0.5, 0.5, (D, K)),
+                conv_b=r.uniform(-0.5, 0.5, D), x_proj=r.standard_normal((R + 2 * N, D)) / 4,
+                dt_proj=r.standard_normal((D, R)) / 2, dt_bias=r.uniform(-6.9, -2.3, D),
+                A=-np.tile(np.arange(1, N + 1, dtype=np.float64), (D, 1)), Dskip=r.standard_normal(D),
+                out_proj=r.standard_normal((dm, D)) / 4)
+
+
+def _mamba_layer_by_torch(h, w):
+    """The same layer from torch.nn.functional (linear, conv1d) in float64 and
+    the oracle's scan: pins the weight layouts and the column ranges."""
+    F = torch.nn.functional
+    t = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))  # noqa: E731
+    D, N, R = w["A"].shape[0], w["A"].shape[1], w["dt_proj"].shape[1]
+    ht = t(h)
+    x = F.linear(ht, t(w["in_proj"][:D]))
+    z = F.linear(ht, t(w["in_proj"][D:]))
+    K = w["conv_w"].shape[1]
+    u = F.conv1d(x.transpose(1, 2), t(w["conv_w"])[:, None, :], t(w["conv_b"]), padding=K - 1, groups=D)
+    u = F.silu(u[..., :x.shape[1]]).transpose(1, 2)
+    dt_low = F.linear(u, t(w["x_proj"][:R]))
+    Bm = F.linear(u, t(w["x_proj"][R:R + N]))
+    Cm = F.linear(u, t(w["x_proj"][R + N:]))
+    delta = F.linear(dt_low, t(w["dt_proj"]), t(w["dt_bias"]))
+    sc = orc.selective_scan(u.numpy(), delta.numpy(), w["A"], Bm.numpy(), Cm.numpy(), w["Dskip"], z.numpy())
+    return F.linear(t(sc["y"]), t(w["out_proj"])).numpy()
+
+
+def test_mamba_layer_matches_torch_functional_composition():
+    w = _layer_weights(31)
+    h = _rng(32).standard_normal((2, 30, 24))
+    got = orc.mamba_layer(h, bf16_activations=False, **w)["out"]
+    np.testing.assert_allclose(got, _mamba_layer_by_torch(h, w), rtol=1e-11, atol=1e-11)
+
+
+def test_planted_swapped_b_and_c_ranges_are_caught(monkeypatch):
+    w = _layer_weights(33)
+    h = _rng(34).standard_normal((1, 20, 24))
+    real = orc.selective_scan
+
+    def swapped(x, delta, A, Bm, Cm, *a, **k):
+        return real(x, delta, A, Cm, Bm, *a, **k)
+
+    monkeypatch.setattr(orc, "selective_scan", swapped)
+    got = orc.mamba_layer(h, bf16_activations=False, **w)["out"]
+    monkeypatch.undo()
+    assert not np.allclose(got, _mamba_layer_by_torch(h, w), atol=1e-6)
+
+
+def test_swa_layer_matches_torch_functional_composition():
+    r = _rng(35)
+    dm, Hq, Hkv, d, L = 32, 4, 2, 8, 40
+    qkv = r.standard_normal(((Hq + 2 * Hkv) * d, dm)) / 5
+    o_proj = r.standard_normal((dm, Hq * d)) / 5
+    h = r.standard_normal((2, L, dm))
+    got = orc.swa_layer(h, qkv, o_proj, Hq, Hkv, d, L, bf16_activations=False)["out"]   # W = L: causal
+    F = torch.nn.functional
+    ht, W = torch.from_numpy(h), torch.from_numpy(qkv)
+    q = F.linear(ht, W[:Hq * d]).reshape(2, L, Hq, d).transpose(1, 2)
+    k = F.linear(ht, W[Hq * d:(Hq + Hkv) * d]).reshape(2, L, Hkv, d).repeat_interleave(Hq // Hkv, 2).transpose(1, 2)
+    v = F.linear(ht, W[(Hq + Hkv) * d:]).reshape(2, L, Hkv, d).repeat_interleave(Hq // Hkv, 2).transpose(1, 2)
+    o = F.scaled_dot_product_attention(q, k, v, is_causal=True).transpose(1, 2).reshape(2, L, Hq * d)
+    ref = F.linear(o, torch.from_numpy(o_proj)).numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-11)
