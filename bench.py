@@ -426,6 +426,93 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------ layers GPU leg
+LAYERS_METRIC = "Samba Mamba + SWA layer prefill tokens/s (projections, conv, scan, attention)"
+
+
+def layer_gemm_flops(wl):
+    """Dense FLOPs of the layers' projections for one step (2 per multiply-add)."""
+    M, dm, D, N, R = wl.batch * wl.seqlen, wl.d_model, wl.dim, wl.dstate, wl.dt_rank
+    nq, nk = wl.heads_q * wl.head_dim, wl.heads_kv * wl.head_dim
+    per_token = 2 * D * dm + (R + 2 * N) * D + D * R + dm * D + (nq + 2 * nk) * dm + dm * nq
+    return 2.0 * M * per_token
+
+
+def run_layers(args, wl, dev, rank, world):
+    """Times one Mamba layer and one SWA layer with their projections on the
+    same hidden state (random weights of the layer shapes)."""
+    import torch
+    import torch.distributed as dist
+
+    from hybrid_ssm_sliding_b200 import layers, ops
+
+    wl_rank = rank_workload(wl, rank)
+    mw = layers.random_mamba_weights(wl.d_model, wl.dim, wl.dstate, wl.dconv, wl.dt_rank, wl_rank.seed, dev)
+    sw = layers.random_swa_weights(wl.d_model, wl.heads_q, wl.heads_kv, wl.head_dim, wl.window, wl_rank.seed + 1,
+                                   dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl_rank.seed + 2)
+    hidden = torch.randn((wl.batch, wl.seqlen, wl.d_model), generator=g, device=dev).to(torch.bfloat16)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layers.mamba_layer_prefill(hidden, mw)
+        layers.swa_layer_prefill(hidden, sw)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = max_over_ranks(e0.elapsed_time(e1), dev)
+    clk = clocks.stop()
+    ms_step = ms_total / args.steps
+    # the largest projection alone, for the tensor roofline
+    M = wl.batch * wl.seqlen
+    h2 = hidden.view(M, wl.d_model)
+    xz = torch.empty((M, 2 * wl.dim), dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        ops.gemm(h2, mw.in_proj, outs=[(xz, 0, 2 * wl.dim, None)])
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    n = max(5, args.kernel_steps // 4)
+    for _ in range(n):
+        ops.gemm(h2, mw.in_proj, outs=[(xz, 0, 2 * wl.dim, None)])
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms_in = a.elapsed_time(b) / n
+    peaks = load_peaks()
+    fl_in = 2.0 * M * 2 * wl.dim * wl.d_model
+    tfs = fl_in / (ms_in / 1e3) / 1e12
+    roof = {"bound": "tensor", "achieved": tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": tfs / peaks["bf16_tflops"], "traffic": None, "kernel": "gemm_kernel (input projection)",
+            "ms": ms_in, "flops": fl_in, "peak_source": peaks["source"] + " burst"}
+    cfg = workload_config(wl)
+    cfg.update({"d_model": wl.d_model, "dt_rank": wl.dt_rank,
+                "layer_gemm_flops_per_step": layer_gemm_flops(wl)})
+    return {
+        "metric": LAYERS_METRIC, "value": whole_job_rate(wl.batch * wl.seqlen, world, ms_step), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (random weights of the layer shapes)", "config": cfg, "roofline": roof,
+        "cpu_baseline": None, "e2e": None, "clocks": clk, "gpu_launches": 11 * args.steps,
+        "status": ops.get_status(),
+    }
+
+
 # ------------------------------------------------------------ decode GPU leg
 def run_decode(args, wl, lib, dev, rank, world):
     """Times decode steps (scan step + SWA step over the whole batch) in
@@ -641,6 +728,14 @@ def main():
     lib = L.load()
 
     wl = WORKLOADS[args.workload]
+    if wl.d_model > 0:
+        line = run_layers(args, wl, dev, rank, world)
+        if rank == 0:
+            print(json.dumps(line))
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
     if wl.decode_steps > 0:
         line = run_decode(args, wl, lib, dev, rank, world)
         if rank == 0:

@@ -33,7 +33,7 @@ class ScanArgs(ctypes.Structure):
         ("conv_state_out", _vp), ("h0", _vp), ("h_final", _vp), ("y", _vp),
         ("batch", _i64), ("seqlen", _i64), ("dim", _i64),
         ("dstate", _i32), ("dconv", _i32), ("x_dtype", _i32), ("z_dtype", _i32), ("y_dtype", _i32),
-        ("flags", ctypes.c_uint32),
+        ("flags", ctypes.c_uint32), ("delta_sum", _vp),
     ]
 
 
@@ -43,6 +43,15 @@ class SwaArgs(ctypes.Structure):
         ("batch", _i64), ("seqlen", _i64), ("window", _i64),
         ("heads_q", _i32), ("heads_kv", _i32), ("head_dim", _i32), ("scale", ctypes.c_float),
     ]
+
+
+class GemmOut(ctypes.Structure):
+    _fields_ = [("ptr", _vp), ("bias", _vp), ("ld", _i64), ("col0", _i64), ("col1", _i64), ("dtype", _i32)]
+
+
+class GemmArgs(ctypes.Structure):
+    _fields_ = [("A", _vp), ("B", _vp), ("lda", _i64), ("ldb", _i64), ("M", _i64), ("N", _i64), ("K", _i64),
+                ("out", GemmOut * 3), ("nout", _i32)]
 
 
 class SambaError(RuntimeError):
@@ -82,8 +91,12 @@ def load() -> ctypes.CDLL:
                                    ctypes.c_int, _i64, ctypes.c_float, _vp, ctypes.c_size_t, _vp]
     lib.samba_swa_step_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, _i64, ctypes.c_float, _vp]
+    lib.samba_gemm.argtypes = [ctypes.POINTER(GemmArgs), _vp]
+    lib.samba_scan_carry.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, ctypes.c_int, _vp]
+    lib.samba_conv_state.argtypes = [_vp, ctypes.c_int, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp]
     for name in ("samba_conv1d_fwd", "samba_selective_scan_fwd", "samba_swa_fwd", "samba_mixer_prefill",
                  "samba_scan_step", "samba_swa_ring_fill", "samba_swa_step", "samba_get_status",
+                 "samba_scan_carry", "samba_conv_state", "samba_gemm",
                  "samba_selftest_wait_timeout", "samba_swa_step_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib

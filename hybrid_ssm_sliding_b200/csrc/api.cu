@@ -91,7 +91,7 @@ const char* samba_last_error(void) { return g_last_error.c_str(); }
 
 int samba_get_status(samba_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  int codes[3] = {take_status_scan(s), take_status_swa(s), take_status_misc(s)};
+  int codes[4] = {take_status_scan(s), take_status_swa(s), take_status_misc(s), take_status_gemm(s)};
   for (int c : codes)
     if (c == SAMBA_ERR_CUDA) return fail(SAMBA_ERR_CUDA, "samba_get_status: %s", cudaGetErrorString(cudaGetLastError()));
   for (int c : codes)
@@ -156,6 +156,27 @@ static int check_swa(const samba_swa_args* a, const char* who) {
   for (const void* p : ptrs)
     if (!aligned16(p)) return fail(SAMBA_ERR_INVALID_ARG, "%s: misaligned pointer", who);
   return SAMBA_OK;
+}
+
+int samba_gemm(const samba_gemm_args* a, samba_stream_t stream) {
+  const char* who = "samba_gemm";
+  if (!a || !a->A || !a->B) return fail(SAMBA_ERR_INVALID_ARG, "%s: A and B are required", who);
+  if (a->M < 1 || a->N < 1 || a->K < 1) return fail(SAMBA_ERR_INVALID_ARG, "%s: bad shape", who);
+  if (a->M > int64_t(65535) * 128 || a->N > INT32_MAX || a->K > INT32_MAX)
+    return fail(SAMBA_ERR_UNSUPPORTED, "%s: M, N or K too large", who);
+  if (a->lda < a->K || a->ldb < a->K || a->lda % 8 || a->ldb % 8)
+    return fail(SAMBA_ERR_INVALID_ARG, "%s: lda and ldb must be >= K and multiples of 8", who);
+  if (!aligned16(a->A) || !aligned16(a->B)) return fail(SAMBA_ERR_INVALID_ARG, "%s: misaligned operand", who);
+  if (a->nout < 1 || a->nout > 3) return fail(SAMBA_ERR_UNSUPPORTED, "%s: nout must be 1..3", who);
+  for (int o = 0; o < a->nout; ++o) {
+    const samba_gemm_out& out = a->out[o];
+    if (!out.ptr) return fail(SAMBA_ERR_INVALID_ARG, "%s: output %d is NULL", who, o);
+    if (!dtype_ok(out.dtype)) return fail(SAMBA_ERR_UNSUPPORTED, "%s: output %d dtype", who, o);
+    if (out.col0 < 0 || out.col1 <= out.col0 || out.col1 > a->N)
+      return fail(SAMBA_ERR_INVALID_ARG, "%s: output %d column range", who, o);
+    if (out.ld < out.col1 - out.col0) return fail(SAMBA_ERR_INVALID_ARG, "%s: output %d row stride", who, o);
+  }
+  return launch_gemm(*a, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int samba_selective_scan_fwd(const samba_scan_args* args, samba_stream_t stream) {
@@ -228,6 +249,28 @@ int samba_scan_step(float* h, float* conv_state, const void* x_t, int x_dtype, c
   if (flags & ~7u) return fail(SAMBA_ERR_INVALID_ARG, "%s: unknown flag bits", who);
   return launch_scan_step(h, conv_state, x_t, x_dtype, z_t, z_dtype, delta_t, B_t, C_t, A, Dskip, conv_w, conv_b,
                           y_t, y_dtype, batch, dim, dstate, dconv, flags, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int samba_scan_carry(const float* h_in, const float* dsum, const float* A, const float* h_local, float* h_out,
+                     int64_t batch, int64_t dim, int dstate, samba_stream_t stream) {
+  const char* who = "samba_scan_carry";
+  if (!dsum || !A || !h_local || !h_out) return fail(SAMBA_ERR_INVALID_ARG, "%s: dsum, A, h_local and h_out are required", who);
+  if (batch < 1 || dim < 1) return fail(SAMBA_ERR_INVALID_ARG, "%s: bad shape", who);
+  if (dstate != 4 && dstate != 8 && dstate != 16) return fail(SAMBA_ERR_UNSUPPORTED, "%s: dstate must be 4, 8 or 16", who);
+  return launch_scan_carry(h_in, dsum, A, h_local, h_out, batch, dim, dstate, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int samba_conv_state(const void* x, int x_dtype, const float* conv_state_in, float* conv_state_out, int64_t batch,
+                     int64_t seqlen, int64_t dim, int dconv, samba_stream_t stream) {
+  const char* who = "samba_conv_state";
+  if (!x || !conv_state_out) return fail(SAMBA_ERR_INVALID_ARG, "%s: x and conv_state_out are required", who);
+  if (batch < 1 || seqlen < 0 || dim < 1) return fail(SAMBA_ERR_INVALID_ARG, "%s: bad shape", who);
+  if (dconv < 2 || dconv > 4) return fail(SAMBA_ERR_UNSUPPORTED, "%s: dconv must be 2..4", who);
+  if (!dtype_ok(x_dtype)) return fail(SAMBA_ERR_UNSUPPORTED, "%s: dtype", who);
+  if (conv_state_in && conv_state_in == conv_state_out)
+    return fail(SAMBA_ERR_INVALID_ARG, "%s: conv_state_out may not alias conv_state_in", who);
+  return launch_conv_state(x, x_dtype, conv_state_in, conv_state_out, batch, seqlen, dim, dconv,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 static int check_ring(int64_t batch, int heads_kv, int head_dim, int64_t window, const char* who) {

@@ -1,0 +1,245 @@
+// Projection GEMM on the sm_100a tensor cores: C = A · Bᵀ with A [M, K] and
+// B [N, K] bf16 (both K-major, rows contiguous), fp32 accumulation in tensor
+// memory, and an epilogue that writes column ranges of C to up to three
+// outputs (each bf16 or fp32, with an optional per-column bias).
+//
+// Page "SAMBA混合注意力状态空间模型", section 数学框架 / Mamba层: the
+// selective parameters are linear maps of the layer input, B_t = Linear_B(x_t),
+// C_t = Linear_C(x_t), Δ_t = τ_Δ(Linear_Δ(x_t)); the layers around the two
+// mixers (the Mamba input and output projections, the attention's Q/K/V and
+// output projections) are linear maps of the same kind.  One GEMM with a
+// column-split epilogue produces such a map's outputs directly in the layouts
+// the mixers read: for instance x and z of the Mamba input projection in one
+// pass, or Δ-low-rank, B and C of the selective-parameter projection.
+//
+// Design: one CTA per 128 x BN tile of C (BN = 256 or 128), K in steps of 64
+// (128-byte rows, 128-byte swizzle).  Warp 4 streams A and B tiles into a
+// STG-deep shared-memory ring with TMA; warp 5 issues the tcgen05.mma
+// (kind::f16, M = 128, N = BN, K = 16 per instruction) into BN columns of
+// tensor memory; warps 0-3 (one TMEM lane quarter each, thread = row) read
+// the accumulator back and write the outputs.  Every wait is bounded.
+#include "common.cuh"
+#include "host.hpp"
+
+namespace samba {
+
+struct GemmOut {
+  void* ptr;          // row-major [M, col1 - col0] (leading dimension ld, in elements)
+  const float* bias;  // [col1 - col0] or null
+  int64_t ld;
+  int col0, col1;     // columns [col0, col1) of C
+  int dtype;          // SAMBA_BF16 or SAMBA_F32
+};
+
+struct GemmParams {
+  int64_t M, N, K;
+  GemmOut out[3];
+  int nout;
+};
+
+template <int BN, int STG>
+struct GemmCfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE = A_BYTES + B_BYTES;
+  static constexpr int BAR_OFF = STG * STAGE;
+  static constexpr int SMEM = BAR_OFF + 128 + 1024;  // barriers + alignment slack
+  static constexpr uint32_t TMEM_COLS = BN;
+  static constexpr int THREADS = 192;
+};
+
+template <int BN, int STG>
+__global__ void __launch_bounds__(192, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                const GemmParams p) {
+  using Cfg = GemmCfg<BN, STG>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::BAR_OFF);
+  uint64_t* empty = full + STG;
+  uint64_t* done = empty + STG;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * BN, m0 = static_cast<int64_t>(blockIdx.y) * Cfg::BM;
+  const int ktiles = static_cast<int>((p.K + Cfg::BK - 1) / Cfg::BK);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STG; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ================================================================ TMA
+    if (lane == 0) {
+      tma_prefetch_desc(&map_a);
+      tma_prefetch_desc(&map_b);
+      int issued = 0;
+      for (int i = 0; i < ktiles; ++i) {
+        const int s = i % STG;
+        if (i >= STG && !mbar_wait(&empty[s], ((i / STG) - 1) & 1, abort_flag)) break;
+        unsigned char* st = smem + s * Cfg::STAGE;
+        mbar_arrive_expect_tx(&full[s], Cfg::STAGE);
+        tma_load_2d(st, &map_a, &full[s], i * Cfg::BK, static_cast<int>(m0));
+        tma_load_2d(st + Cfg::A_BYTES, &map_b, &full[s], i * Cfg::BK, static_cast<int>(n0));
+        issued = i + 1;
+      }
+      // copies still in flight complete before the CTA can exit
+      volatile int never = 0;
+      for (int i = (issued > STG ? issued - STG : 0); i < issued; ++i) mbar_wait(&full[i % STG], (i / STG) & 1, &never);
+    }
+  } else if (warp == 5) {
+    // ================================================================ MMA
+    constexpr uint32_t IDESC = idesc_bf16_f32(Cfg::BM, BN, 0, 0);
+    const uint32_t base = smem_u32(smem);
+    const uint64_t d_a0 = smem_desc(base, 16, 1024, 2);
+    const uint32_t hi = static_cast<uint32_t>(d_a0 >> 32), lo0 = static_cast<uint32_t>(d_a0);
+    constexpr uint32_t kStageDesc = Cfg::STAGE >> 4, kBDesc = Cfg::A_BYTES >> 4;
+    auto desc64 = [&](uint32_t lo) { return (static_cast<uint64_t>(hi) << 32) | lo; };
+    bool ok = true;
+    for (int i = 0; i < ktiles && ok; ++i) {
+      const int s = i % STG;
+      ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (i / STG) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t la = lo0 + s * kStageDesc, lb = la + kBDesc;
+#pragma unroll
+      for (int k = 0; k < Cfg::BK / 16; ++k)  // 16 K-elements = 32 bytes = 2 descriptor units
+        umma_ss_w(tmem, desc64(la + 2 * k), desc64(lb + 2 * k), IDESC, (i > 0 || k > 0) ? 1u : 0u);
+      tc_commit_w(&empty[s]);
+    }
+    tc_commit_w(done);  // every MMA of this tile has completed
+  } else {
+    // ============================================================ epilogue
+    const int row_local = warp * 32 + lane;
+    const int64_t row = m0 + row_local;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag));
+    if (ok && ktiles > 0) {
+      tc_fence_after();
+      const uint32_t t_row = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(t_row + c0, r);
+        tc_wait_ld();
+        if (row >= p.M) continue;
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          const int64_t col = n0 + c0 + j;  // 8 consecutive columns
+#pragma unroll
+          for (int o = 0; o < 3; ++o) {
+            if (o >= p.nout) break;
+            const GemmOut& out = p.out[o];
+            if (col + 8 <= out.col0 || col >= out.col1) continue;
+            const bool whole = col >= out.col0 && col + 8 <= out.col1 && col + 8 <= p.N;
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              v[e] = __uint_as_float(r[j + e]);
+              const int64_t cc = col + e - out.col0;
+              if (out.bias && cc >= 0 && cc < out.col1 - out.col0) v[e] += out.bias[cc];
+            }
+            const int64_t base_idx = row * out.ld + (col - out.col0);
+            if (out.dtype == SAMBA_BF16) {
+              __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(out.ptr) + base_idx;
+              if (whole && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+                uint4 pk;
+                pk.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[0])) |
+                       ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[1])) << 16);
+                pk.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[2])) |
+                       ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[3])) << 16);
+                pk.z = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[4])) |
+                       ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[5])) << 16);
+                pk.w = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[6])) |
+                       ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[7])) << 16);
+                *reinterpret_cast<uint4*>(dst) = pk;
+              } else {
+                for (int e = 0; e < 8; ++e) {
+                  const int64_t cc = col + e;
+                  if (cc >= out.col0 && cc < out.col1 && cc < p.N) dst[e] = __float2bfloat16_rn(v[e]);
+                }
+              }
+            } else {
+              float* dst = reinterpret_cast<float*>(out.ptr) + base_idx;
+              if (whole && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+                reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
+                reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+              } else {
+                for (int e = 0; e < 8; ++e) {
+                  const int64_t cc = col + e;
+                  if (cc >= out.col0 && cc < out.col1 && cc < p.N) dst[e] = v[e];
+                }
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::TMEM_COLS);
+  }
+}
+
+int take_status_gemm(cudaStream_t s) { return take_status_word(s); }
+
+template <int BN>
+static int launch_gemm_t(const samba_gemm_args& a, cudaStream_t stream) {
+  constexpr int STG = BN == 256 ? 4 : 6;
+  using Cfg = GemmCfg<BN, STG>;
+  auto kern = gemm_kernel<BN, STG>;
+  static PerDeviceOnce attr;
+  const int arc = once_per_device(attr, [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) == cudaSuccess
+               ? SAMBA_OK
+               : fail(SAMBA_ERR_CUDA, "gemm: cannot set shared memory size");
+  });
+  if (arc != SAMBA_OK) return arc;
+  CUtensorMap ma, mb;
+  const uint32_t box_a[2] = {(uint32_t)Cfg::BK, (uint32_t)Cfg::BM};
+  const uint32_t box_b[2] = {(uint32_t)Cfg::BK, (uint32_t)BN};
+  const uint64_t da[2] = {(uint64_t)a.K, (uint64_t)a.M}, sa[1] = {(uint64_t)a.lda * 2};
+  const uint64_t db[2] = {(uint64_t)a.K, (uint64_t)a.N}, sb[1] = {(uint64_t)a.ldb * 2};
+  int rc = encode_tiled(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.A, da, sa, box_a, CU_TENSOR_MAP_SWIZZLE_128B,
+                        "gemm A");
+  if (rc) return rc;
+  rc = encode_tiled(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.B, db, sb, box_b, CU_TENSOR_MAP_SWIZZLE_128B, "gemm B");
+  if (rc) return rc;
+  GemmParams p;
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  p.nout = a.nout;
+  for (int o = 0; o < a.nout; ++o) {
+    p.out[o].ptr = a.out[o].ptr;
+    p.out[o].bias = a.out[o].bias;
+    p.out[o].ld = a.out[o].ld;
+    p.out[o].col0 = static_cast<int>(a.out[o].col0);
+    p.out[o].col1 = static_cast<int>(a.out[o].col1);
+    p.out[o].dtype = a.out[o].dtype;
+  }
+  const dim3 grid((unsigned)((a.N + BN - 1) / BN), (unsigned)((a.M + Cfg::BM - 1) / Cfg::BM));
+  kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(ma, mb, p);
+  return check_launch("samba_gemm");
+}
+
+int launch_gemm(const samba_gemm_args& a, cudaStream_t s) {
+  return a.N >= 256 ? launch_gemm_t<256>(a, s) : launch_gemm_t<128>(a, s);
+}
+
+}  // namespace samba

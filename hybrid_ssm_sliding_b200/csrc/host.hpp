@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include <cstdarg>
+#include <algorithm>
 #include <cstdio>
 #include <mutex>
 #include <string>
@@ -55,6 +56,8 @@ int once_per_device(PerDeviceOnce& o, F&& f) {
 int take_status_scan(cudaStream_t s);
 int take_status_swa(cudaStream_t s);
 int take_status_misc(cudaStream_t s);
+int take_status_gemm(cudaStream_t s);
+int launch_gemm(const samba_gemm_args& a, cudaStream_t stream);
 int launch_selftest_wait(cudaStream_t s);
 
 // Launchers (validated arguments only).
@@ -70,6 +73,10 @@ int launch_scan_step(float* h, float* conv_state, const void* x_t, int x_dtype, 
 int launch_ring_fill(const void* k, const void* v, int64_t L, void* k_ring, void* v_ring, int64_t* pos, int64_t B,
                      int Hkv, int d, int64_t W, cudaStream_t stream);
 size_t swa_step_workspace(int64_t B, int Hq, int d, int64_t W);
+int launch_scan_carry(const float* h_in, const float* dsum, const float* A, const float* h_local, float* h_out,
+                      int64_t B, int64_t D, int N, cudaStream_t stream);
+int launch_conv_state(const void* x, int x_dtype, const float* cs_in, float* cs_out, int64_t B, int64_t L, int64_t D,
+                      int K, cudaStream_t stream);
 int launch_swa_step_noalloc(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring,
                             int64_t* pos, void* o_t, int64_t B, int Hq, int Hkv, int d, int64_t W, float scale,
                             cudaStream_t stream);

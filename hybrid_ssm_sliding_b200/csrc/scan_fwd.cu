@@ -60,6 +60,7 @@ struct ScanParams {
   float* conv_state_out;
   const float* h0;
   float* h_final;
+  float* delta_sum;  // [B, D] sum over t of Δ, or null
   const void* x;  // for the conv state at the end
   void* y;
   int64_t L, D;
@@ -124,7 +125,9 @@ struct ScanLayout {
   static constexpr int XCH_BYTES = SLOTS * T * CB * 8;       // float2 [SLOTS][T][CB] (Δ, Δu)
   static constexpr int EPI_BYTES = SLOTS * T * CB * 8;       // float2 [SLOTS][T][CB] (D·u, z)
   static constexpr int PART_BYTES = SLOTS * T * CB * GL * 4; // float  [SLOTS][T][GL][CB]
-  static constexpr int FIXED = XCH_BYTES + EPI_BYTES + PART_BYTES + 512;
+  // barriers (256 B), then the prologue's partial sums of Δ ([kScanPro][CB] floats)
+  static constexpr int BAR_BYTES = 512 + kScanPro * CB * 4;
+  static constexpr int FIXED = XCH_BYTES + EPI_BYTES + PART_BYTES + BAR_BYTES;
   // TMA ring: as many stages (up to 6) as fit next to the hand-off buffers
   static constexpr int STAGES_FIT = (kScanSmemBudget - FIXED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
@@ -133,7 +136,7 @@ struct ScanLayout {
   static constexpr int EPI_OFF = XCH_OFF + XCH_BYTES;
   static constexpr int PART_OFF = EPI_OFF + EPI_BYTES;
   static constexpr int BAR_OFF = PART_OFF + PART_BYTES;
-  static constexpr int SMEM = BAR_OFF + 512;
+  static constexpr int SMEM = BAR_OFF + BAR_BYTES;
 };
 
 // Scan warps: one per group of NS states (GL of them); lane = channel (CU <= 32).
@@ -229,6 +232,8 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
   uint64_t* scan_done = pro_full + SLOTS;   // [SLOTS]
   uint64_t* epi_done = scan_done + SLOTS;   // [SLOTS]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(epi_done + SLOTS);
+  uint64_t* dsum_bar = reinterpret_cast<uint64_t*>(smem + Ly::BAR_OFF + 256);  // partial Δ sums written
+  float* DSUM = reinterpret_cast<float*>(smem + Ly::BAR_OFF + 512);            // [kScanPro][CB]
   float2* XCH = reinterpret_cast<float2*>(smem + Ly::XCH_OFF);
   float2* EPI = reinterpret_cast<float2*>(smem + Ly::EPI_OFF);
   float* PART = reinterpret_cast<float*>(smem + Ly::PART_OFF);
@@ -254,6 +259,7 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
       mbar_init(&scan_done[k], NSW);
       mbar_init(&epi_done[k], EPIW);
     }
+    mbar_init(dsum_bar, kScanPro - 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -347,6 +353,7 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
     float cw[4] = {0.f, 0.f, 0.f, 0.f};
     float cbias = 0.f, dsk = 0.f;
     float hist[3] = {0.f, 0.f, 0.f};  // x of the 3 tokens before the first tile (conv state)
+    float dsum = 0.f;                 // sum of Δ over this thread's tokens (0 for padding tokens)
     if (cval) {
       if (p.fuse_conv) {
         // tap k (0..3) multiplies x_{t-3+k}: weight k - (4 - K), if any
@@ -414,6 +421,7 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
         float dlt = p.softplus ? softplus_fast(wr) : wr;
         if (tok >= L || !cact) dlt = 0.f;  // padding tokens leave the state untouched
         const float du = dlt * u;
+        dsum += dlt;
         // z itself goes to the epilogue warps, which wait on the scan most
         // of the time and evaluate the gate silu(z) there
         const float g = p.has_z ? zv[q] : 1.f;
@@ -426,6 +434,23 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
       if (lane == 0) mbar_arrive(&pro_full[k]);
     }
     if (*abort_flag) return;
+    // Σ_t Δ per channel: each prologue warp holds the sums of its tokens; the
+    // first one adds them in warp order once the others have written theirs.
+    if (p.delta_sum) {
+      DSUM[tg * CB + cl] = dsum;
+      if (tg != 0) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dsum_bar);
+      } else {
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(dsum_bar, 0, abort_flag));
+        if (ok && cval) {
+          float sum = 0.f;
+#pragma unroll
+          for (int w = 0; w < kScanPro; ++w) sum += DSUM[w * CB + cl];
+          p.delta_sum[(int64_t)b * p.D + c] = sum;
+        }
+      }
+    }
     // final conv state: the last K-1 entries of (old state, x)
     if (p.conv_state_out && cval && tg == 0) {
       for (int jj = 0; jj < K - 1; ++jj) {
@@ -660,6 +685,7 @@ static int launch_scan_t(const samba_scan_args& a, cudaStream_t stream) {
   p.conv_state_out = a.conv_state_out;
   p.h0 = a.h0;
   p.h_final = a.h_final;
+  p.delta_sum = a.delta_sum;
   p.x = a.x;
   p.y = a.y;
   p.L = a.seqlen;

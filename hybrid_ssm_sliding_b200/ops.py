@@ -65,7 +65,7 @@ def conv1d_fwd(x, w, bias=None, conv_state_in=None, silu=True, u=None, u_dtype=N
 
 def _scan_struct(x, delta, A, B, C, D=None, z=None, conv_w=None, conv_b=None, conv_state_in=None,
                  h0=None, y=None, y_dtype=None, h_final=None, conv_state_out=None,
-                 delta_softplus=True, conv_silu=True, fuse_conv=None):
+                 delta_softplus=True, conv_silu=True, fuse_conv=None, delta_sum=None):
     _need(x, "x")
     Bsz, Ln, Dm = x.shape
     N = A.shape[1]
@@ -84,6 +84,7 @@ def _scan_struct(x, delta, A, B, C, D=None, z=None, conv_w=None, conv_b=None, co
     _opt(conv_state_out, "conv_state_out", torch.float32, (Bsz, Dm, K - 1))
     _opt(h0, "h0", torch.float32, (Bsz, Dm, N))
     _opt(h_final, "h_final", torch.float32, (Bsz, Dm, N))
+    _opt(delta_sum, "delta_sum", torch.float32, (Bsz, Dm))
     if y is None:
         y = torch.empty_like(x, dtype=y_dtype or x.dtype)
     _need(y, "y", None, x.shape)
@@ -92,16 +93,16 @@ def _scan_struct(x, delta, A, B, C, D=None, z=None, conv_w=None, conv_b=None, co
     a = L.ScanArgs(L.ptr(x), L.ptr(z), L.ptr(delta), L.ptr(A), L.ptr(B), L.ptr(C), L.ptr(D), L.ptr(conv_w),
                    L.ptr(conv_b), L.ptr(conv_state_in), L.ptr(conv_state_out), L.ptr(h0), L.ptr(h_final),
                    L.ptr(y), Bsz, Ln, Dm, N, K, L.dtype_code(x), L.dtype_code(z) if z is not None else 0,
-                   L.dtype_code(y), flags)
+                   L.dtype_code(y), flags, L.ptr(delta_sum))
     return a, y
 
 
 def selective_scan_fwd(x, delta, A, B, C, D=None, z=None, conv_w=None, conv_b=None, conv_state_in=None,
                        h0=None, y=None, y_dtype=None, h_final=None, conv_state_out=None,
-                       delta_softplus=True, conv_silu=True, fuse_conv=None, stream=None):
+                       delta_softplus=True, conv_silu=True, fuse_conv=None, delta_sum=None, stream=None):
     """Fused selective-scan prefill (see samba_selective_scan_fwd).  Returns y."""
     a, y = _scan_struct(x, delta, A, B, C, D, z, conv_w, conv_b, conv_state_in, h0, y, y_dtype, h_final,
-                        conv_state_out, delta_softplus, conv_silu, fuse_conv)
+                        conv_state_out, delta_softplus, conv_silu, fuse_conv, delta_sum)
     L.check(L.load().samba_selective_scan_fwd(ctypes.byref(a), L.stream_handle(stream)))
     return y
 
@@ -166,6 +167,74 @@ def scan_step(h, conv_state, x_t, delta_t, A, B_t, C_t, D=None, z_t=None, conv_w
                                      L.ptr(C_t), L.ptr(A), L.ptr(D), L.ptr(conv_w), L.ptr(conv_b), L.ptr(y_t),
                                      L.dtype_code(y_t), Bsz, Dm, N, K, flags, L.stream_handle(stream)))
     return y_t
+
+
+def gemm(a, w, outs=None, out_dtype=torch.bfloat16, bias=None, stream=None):
+    """C = a @ w.T on the tensor cores (see samba_gemm): a [M, K] bf16 (rows
+    may be strided), w [N, K] bf16.  ``outs`` is a list of up to three
+    (tensor, col0, col1, bias) entries that receive columns [col0, col1) of C
+    (tensors 2-D [M, col1 - col0], row stride any, bf16 or fp32); by default
+    one new [M, N] tensor of out_dtype (with ``bias``) is returned."""
+    if a.dim() != 2 or w.dim() != 2:
+        raise ValueError("a and w must be 2-D")
+    if a.dtype != torch.bfloat16 or w.dtype != torch.bfloat16:
+        raise TypeError("a and w must be bfloat16")
+    if not (a.is_cuda and w.is_cuda):
+        raise ValueError("a and w must be CUDA tensors")
+    if a.stride(1) != 1 or w.stride(1) != 1:
+        raise ValueError("a and w need contiguous rows")
+    M, K = a.shape
+    N = w.shape[0]
+    if w.shape[1] != K:
+        raise ValueError("a and w disagree on K")
+    ret = None
+    if outs is None:
+        ret = torch.empty((M, N), dtype=out_dtype, device=a.device)
+        outs = [(ret, 0, N, bias)]
+    args = L.GemmArgs()
+    args.A, args.B = L.ptr(a), L.ptr(w)
+    args.lda, args.ldb = a.stride(0), w.stride(0)
+    args.M, args.N, args.K = M, N, K
+    if not 1 <= len(outs) <= 3:
+        raise ValueError("one to three outputs")
+    for i, (t, c0, c1, b) in enumerate(outs):
+        if t.dim() != 2 or t.shape[0] != M or t.shape[1] != c1 - c0 or t.stride(1) != 1:
+            raise ValueError(f"output {i} must be a [M, {c1 - c0}] matrix with contiguous rows")
+        _opt(b, f"bias {i}", torch.float32, (c1 - c0,))
+        o = args.out[i]
+        o.ptr, o.bias, o.ld, o.col0, o.col1, o.dtype = L.ptr(t), L.ptr(b), t.stride(0), c0, c1, L.dtype_code(t)
+    args.nout = len(outs)
+    L.check(L.load().samba_gemm(ctypes.byref(args), L.stream_handle(stream)))
+    return ret if ret is not None else [o[0] for o in outs]
+
+
+def scan_carry(h_in, dsum, A, h_local, h_out=None, stream=None):
+    """Joins a scan segment to its predecessor (see samba_scan_carry):
+    h_out = exp(A * dsum) * h_in + h_local.  h_in may be None (zero state)."""
+    _need(h_local, "h_local", torch.float32)
+    Bsz, Dm, N = h_local.shape
+    _need(dsum, "dsum", torch.float32, (Bsz, Dm))
+    _need(A, "A", torch.float32, (Dm, N))
+    _opt(h_in, "h_in", torch.float32, (Bsz, Dm, N))
+    if h_out is None:
+        h_out = torch.empty_like(h_local)
+    _need(h_out, "h_out", torch.float32, (Bsz, Dm, N))
+    L.check(L.load().samba_scan_carry(L.ptr(h_in), L.ptr(dsum), L.ptr(A), L.ptr(h_local), L.ptr(h_out), Bsz, Dm,
+                                      N, L.stream_handle(stream)))
+    return h_out
+
+
+def conv_state(x, dconv, conv_state_in=None, conv_state_out=None, stream=None):
+    """The conv state after x (see samba_conv_state): [B, D, K-1] fp32."""
+    _need(x, "x")
+    Bsz, Ln, Dm = x.shape
+    _opt(conv_state_in, "conv_state_in", torch.float32, (Bsz, Dm, dconv - 1))
+    if conv_state_out is None:
+        conv_state_out = torch.empty((Bsz, Dm, dconv - 1), dtype=torch.float32, device=x.device)
+    _need(conv_state_out, "conv_state_out", torch.float32, (Bsz, Dm, dconv - 1))
+    L.check(L.load().samba_conv_state(L.ptr(x), L.dtype_code(x), L.ptr(conv_state_in), L.ptr(conv_state_out), Bsz,
+                                      Ln, Dm, dconv, L.stream_handle(stream)))
+    return conv_state_out
 
 
 def swa_ring_fill(k, v, window, k_ring=None, v_ring=None, pos=None, stream=None):

@@ -48,6 +48,8 @@ class Workload:
     act_dtype: torch.dtype = torch.bfloat16     # x, z, y (timing) dtype
     attn_dtype: torch.dtype = torch.bfloat16    # q, k, v, o
     decode_steps: int = 0
+    d_model: int = 0      # layer workloads: model width around the mixers (0: mixers only)
+    dt_rank: int = 0      # layer workloads: rank of the step-size projection
     notes: str = field(default="", compare=False)
 
     @property
@@ -66,6 +68,11 @@ WORKLOADS = {
     # one 32K-token prompt at the same widths: every input still exceeds L2,
     # but the whole problem holds ~1.5 GB, small enough for profiler captures
     "prefill_32k": Workload("prefill_32k", 1, 32768, 4096, 16, 4, 32, 4, 64, 2048, 5),
+    # a Mamba layer and an SWA layer with their projections (d_model 2048,
+    # d_inner 4096, step-size rank 128) on the 4K and 128K prompts
+    "layers_4k": Workload("layers_4k", 1, 4096, 4096, 16, 4, 32, 4, 64, 2048, 6, d_model=2048, dt_rank=128),
+    "layers_128k": Workload("layers_128k", 1, 131072, 4096, 16, 4, 32, 4, 64, 2048, 7, d_model=2048,
+                            dt_rank=128),
 }
 
 

@@ -129,6 +129,10 @@ int samba_conv1d_fwd(const void* x, int x_dtype, const float* w, const float* bi
  *   y_t    = (sum_n C_t[n] h_t[n] + Dskip[c] u_t) * silu(z_t)
  * for every batch b and channel c, t = 0..L-1, starting from h0 (zeros if
  * NULL).  B and C are shared by all channels (one group).
+ * With delta_sum, the call also writes sum_t Δ_t per (b, c): the decay of
+ * state n over the whole call is exp(A[c,n] * delta_sum[b,c]), which is what
+ * samba_scan_carry needs to join this segment of a longer sequence to the
+ * segment before it (see there).
  * Errors: SAMBA_ERR_INVALID_ARG for a missing x, delta, A, Bm, Cm, y (or
  * conv_w with FUSE_CONV), D not a multiple of 8, unknown flag bits or a
  * pointer not 16-byte aligned; SAMBA_ERR_UNSUPPORTED for B > 65535,
@@ -153,9 +157,43 @@ typedef struct samba_scan_args {
   int32_t dstate, dconv;       /* N in {4, 8, 16}; K in 2..4                  */
   int32_t x_dtype, z_dtype, y_dtype;
   uint32_t flags;
+  float* delta_sum;            /* [B, D] fp32, or NULL: sum over t of Δ_t     */
 } samba_scan_args;
 
 int samba_selective_scan_fwd(const samba_scan_args* args, samba_stream_t stream);
+
+/* ------------------------------------------------------ sequence segments
+ * A sequence split into consecutive segments (for example one per GPU) can be
+ * scanned segment by segment with exactly the result of one pass, because the
+ * recurrence is linear in its state: over a segment s, the final state is
+ *   h_end(s) = exp(A * dsum(s)) ⊙ h_start(s) + h_local(s),
+ * where h_local(s) is the final state of the segment scanned from zero and
+ * dsum(s) = sum_t Δ_t over the segment (samba_scan_args.delta_sum).  So every
+ * segment can first be scanned from zero (giving h_local and dsum), the
+ * segments' start states follow by folding this carry from the first segment
+ * on, and a second pass from the right start state gives the outputs.  The
+ * page's recurrence (section 数学框架 / Mamba层) is the same in every segment;
+ * the split is only an order of evaluation.
+ *
+ * samba_scan_carry: h_out = exp(A ⊙ dsum) ⊙ h_in + h_local, elementwise over
+ * [B, D, N] (A [D, N] fp32, dsum [B, D] fp32, h_in, h_local, h_out
+ * [B, D, N] fp32; h_in may be NULL for a zero start state; h_out may alias
+ * h_in or h_local).  exp is evaluated as the scan evaluates its decays.
+ * Errors: SAMBA_ERR_INVALID_ARG for a missing A, dsum, h_local or h_out or a
+ * non-positive size; SAMBA_ERR_UNSUPPORTED for N outside {4, 8, 16}.
+ */
+int samba_scan_carry(const float* h_in, const float* dsum, const float* A, const float* h_local, float* h_out,
+                     int64_t batch, int64_t dim, int dstate, samba_stream_t stream);
+
+/* samba_conv_state: the conv state a segment hands to the next one, the last
+ * K-1 inputs of (conv_state_in, x) ([B, D, K-1] fp32, oldest first), without
+ * computing the conv.  x is [B, L, D] x_dtype (L >= 0); conv_state_in is
+ * [B, D, K-1] fp32 or NULL (zeros); conv_state_out may not alias it.  Equals
+ * the conv_state_out of samba_selective_scan_fwd and samba_conv1d_fwd.
+ * Errors: SAMBA_ERR_INVALID_ARG for a missing x or conv_state_out, aliasing,
+ * or a bad shape; SAMBA_ERR_UNSUPPORTED for K outside 2..4 or a dtype. */
+int samba_conv_state(const void* x, int x_dtype, const float* conv_state_in, float* conv_state_out,
+                     int64_t batch, int64_t seqlen, int64_t dim, int dconv, samba_stream_t stream);
 
 /* -------------------------------------------------------------------- SWA
  * Causal sliding-window attention prefill with grouped KV heads:
@@ -182,6 +220,46 @@ typedef struct samba_swa_args {
 } samba_swa_args;
 
 int samba_swa_fwd(const samba_swa_args* args, samba_stream_t stream);
+
+/* ------------------------------------------------------------- projections
+ * The linear maps around the two mixers (a Mamba layer's input projection to
+ * x and z, its selective-parameter projection to the low-rank Δ, B and C, the
+ * Δ up-projection, its output projection; the attention's Q/K/V and output
+ * projections: page "SAMBA混合注意力状态空间模型", section 数学框架 /
+ * Mamba层, B_t = Linear_B(x_t), C_t = Linear_C(x_t), Δ_t = τ_Δ(Linear_Δ(x_t)))
+ * as one GEMM on the tensor cores:
+ *   C[m, n] = sum_k A[m, k] * B[n, k]     (bf16 inputs, fp32 accumulation)
+ * A is [M, K] with row stride lda, B is [N, K] with row stride ldb (a
+ * weight in the usual [out_features, in_features] layout), both bf16,
+ * 16-byte aligned, lda and ldb multiples of 8.  The columns of C go to up to
+ * three outputs: out[i] receives columns [col0, col1) as a row-major
+ * [M, col1 - col0] matrix with row stride ld (elements), in bf16 or fp32,
+ * plus bias[col - col0] when bias is not NULL.  Columns outside every range
+ * are dropped.
+ * Errors: SAMBA_ERR_INVALID_ARG for a missing operand or output, a
+ * non-positive size, a stride below its row length or not a multiple of 8, an
+ * empty or out-of-range column range or a misaligned pointer;
+ * SAMBA_ERR_UNSUPPORTED for M above 65535 * 128, N or K above 2^31 - 1, an
+ * output dtype other than SAMBA_F32 / SAMBA_BF16, or nout outside 1..3.
+ */
+typedef struct samba_gemm_out {
+  void* ptr;          /* [M, col1 - col0] row-major, row stride ld        */
+  const float* bias;  /* [col1 - col0] fp32, or NULL                      */
+  int64_t ld;
+  int64_t col0, col1;
+  int32_t dtype;      /* SAMBA_F32 or SAMBA_BF16                          */
+} samba_gemm_out;
+
+typedef struct samba_gemm_args {
+  const void* A;      /* [M, K] bf16, row stride lda                      */
+  const void* B;      /* [N, K] bf16, row stride ldb                      */
+  int64_t lda, ldb;
+  int64_t M, N, K;
+  samba_gemm_out out[3];
+  int32_t nout;
+} samba_gemm_args;
+
+int samba_gemm(const samba_gemm_args* args, samba_stream_t stream);
 
 /* ------------------------------------------------------------ mixer prefill
  * One Mamba mixer (scan) and one SWA mixer on their own inputs (the two token

@@ -189,3 +189,29 @@ def test_swa_step_noalloc_checks_on_host(lib):
     # argument limits are reported as for samba_swa_step, before the scratch size
     assert call(batch=70000) == L.SAMBA_ERR_UNSUPPORTED
     assert call(W=(1 << 30) + 1) == L.SAMBA_ERR_UNSUPPORTED
+
+
+def test_gemm_rejects_bad_arguments_on_host(lib):
+    f = 0x80000
+
+    def call(M=128, N=256, K=64, lda=64, ldb=64, nout=1, ptr=f, col0=0, col1=256, ld=256, dtype=1, A=f):
+        a = L.GemmArgs()
+        a.A, a.B, a.lda, a.ldb, a.M, a.N, a.K = A, f, lda, ldb, M, N, K
+        o = a.out[0]
+        o.ptr, o.bias, o.ld, o.col0, o.col1, o.dtype = ptr, None, ld, col0, col1, dtype
+        a.nout = nout
+        return lib.samba_gemm(ctypes.byref(a), None)
+
+    assert call(A=None) == L.SAMBA_ERR_INVALID_ARG
+    assert call(K=0) == L.SAMBA_ERR_INVALID_ARG
+    assert call(lda=60) == L.SAMBA_ERR_INVALID_ARG          # below K
+    assert call(lda=68, K=64) == L.SAMBA_ERR_INVALID_ARG    # not a multiple of 8
+    assert call(A=f + 8) == L.SAMBA_ERR_INVALID_ARG         # misaligned
+    assert call(nout=0) == L.SAMBA_ERR_UNSUPPORTED
+    assert call(nout=4) == L.SAMBA_ERR_UNSUPPORTED
+    assert call(ptr=None) == L.SAMBA_ERR_INVALID_ARG
+    assert call(col1=300) == L.SAMBA_ERR_INVALID_ARG        # past N
+    assert call(col0=10, col1=10) == L.SAMBA_ERR_INVALID_ARG
+    assert call(ld=100) == L.SAMBA_ERR_INVALID_ARG          # row stride below the range
+    assert call(dtype=7) == L.SAMBA_ERR_UNSUPPORTED
+    assert call(M=65535 * 128 + 1) == L.SAMBA_ERR_UNSUPPORTED
