@@ -61,6 +61,8 @@ __all__ = [
     "swa",
     "swa_rows",
     "swa_blocks",
+    "selective_scan_bwd",
+    "swa_bwd",
     "round_bf16",
     "mamba_layer",
     "swa_layer",
@@ -336,6 +338,168 @@ def swa_blocks(q, k, v, window, starts, block=64, scale=None):
         rows[r0:r0 + n] = np.arange(i0, i1)
         r0 += n
     return rows, o, lse
+
+
+# ------------------------------------------------------------- backward
+def _sigmoid(x):
+    x = _f64(x)
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def _silu_grad(x):
+    """d silu(x) / dx = σ(x) (1 + x (1 - σ(x)))."""
+    sg = _sigmoid(x)
+    return sg * (1.0 + x * (1.0 - sg))
+
+
+def selective_scan_bwd(dy, x, delta, A, Bm, Cm, Dskip=None, z=None, h0=None,
+                       conv_w=None, conv_b=None, conv_state=None,
+                       delta_softplus=True, conv_silu=True):
+    """Reverse-mode gradients of ``selective_scan``'s output y.
+
+    The forward is the recurrence of page "SAMBA混合注意力状态空间模型",
+    §数学框架 / Mamba层, with the readings of ``selective_scan``.  Given
+    dy = ∂L/∂y [B, L, D], the chain rule taken step by step through that
+    definition (the forward states recomputed and kept, then one sequential
+    walk from t = L-1 down to 0):
+
+        g_y   = dy ⊙ silu(z)                       (gradient of C·h + D u)
+        dz    = dy ⊙ (C·h + D u) ⊙ silu'(z)
+        G_t   = ∂L/∂h_t = C_t g_y,t + Ā_{t+1} ⊙ G_{t+1}
+        dC_t  = Σ_c g_y,t,c h_t,c              dB_t = Σ_c G_t,c Δ_t,c u_t,c
+        dΔ_t  = Σ_n G_t (A Ā_t h_{t-1} + B_t u_t)
+        dA    = Σ_t Δ_t Ā_t G_t h_{t-1}        du_t = D g_y,t + Δ_t Σ_n G_t B_t
+        dD    = Σ_t g_y,t u_t                  dh0  = Ā_0 ⊙ G_0
+    then through softplus (dδ = dΔ σ(δ)), the SiLU after the conv and the
+    depthwise causal conv (a correlation, so its input gradient is the
+    transposed correlation and its weight gradient a correlation of the
+    output gradient with the padded input).
+
+    Arguments as ``selective_scan``.  Returns dict(dx, ddelta, dA, dB, dC,
+    dD, dz, dh0, dconv_w, dconv_b, dconv_state); entries whose input was
+    None are None.
+    """
+    x = _f64(x)
+    delta = _f64(delta)
+    A = _f64(A)
+    Bm = _f64(Bm)
+    Cm = _f64(Cm)
+    dy = _f64(dy)
+    Bsz, L, D = x.shape
+    N = A.shape[1]
+
+    # forward recompute, keeping every state
+    if conv_w is not None:
+        conv_w = _f64(conv_w)
+        K = conv_w.shape[1]
+        st = np.zeros((Bsz, D, K - 1)) if conv_state is None else _f64(conv_state)
+        xpad = np.concatenate([np.transpose(st, (0, 2, 1)), x], axis=1)      # [B, L+K-1, D]
+        pre = np.zeros((Bsz, L, D))
+        for k in range(K):
+            pre += conv_w[None, None, :, k] * xpad[:, k:k + L, :]
+        if conv_b is not None:
+            pre += _f64(conv_b)[None, None, :]
+        u = silu(pre) if conv_silu else pre
+    else:
+        u = x
+    dt = softplus(delta) if delta_softplus else delta
+    hs = np.empty((L + 1, Bsz, D, N))
+    hs[0] = np.zeros((Bsz, D, N)) if h0 is None else _f64(h0)
+    for t in range(L):
+        hs[t + 1] = np.exp(dt[:, t, :, None] * A[None]) * hs[t] + (dt[:, t, :] * u[:, t, :])[:, :, None] * Bm[:, t, None, :]
+    ypre = np.einsum("lbdn,bln->bld", hs[1:], Cm)
+    if Dskip is not None:
+        ypre = ypre + _f64(Dskip)[None, None, :] * u
+
+    # output gate
+    if z is not None:
+        z = _f64(z)
+        gy = dy * silu(z)
+        dz = dy * ypre * _silu_grad(z)
+    else:
+        gy = dy
+        dz = None
+    dD = None if Dskip is None else np.einsum("bld,bld->d", gy, u)
+    du = np.zeros((Bsz, L, D)) if Dskip is None else gy * _f64(Dskip)[None, None, :]
+
+    # reverse walk
+    G = np.zeros((Bsz, D, N))
+    dB = np.zeros((Bsz, L, N))
+    dC = np.zeros((Bsz, L, N))
+    ddt = np.zeros((Bsz, L, D))
+    dA = np.zeros((D, N))
+    for t in range(L - 1, -1, -1):
+        G = G + gy[:, t, :, None] * Cm[:, t, None, :]
+        dC[:, t, :] = np.einsum("bd,bdn->bn", gy[:, t, :], hs[t + 1])
+        decay = np.exp(dt[:, t, :, None] * A[None])                            # Ā_t [B, D, N]
+        hprev = hs[t]
+        dB[:, t, :] = np.einsum("bdn,bd->bn", G, dt[:, t, :] * u[:, t, :])
+        ddt[:, t, :] = np.einsum("bdn,bdn->bd", G, A[None] * decay * hprev) + \
+            u[:, t, :] * np.einsum("bdn,bn->bd", G, Bm[:, t, :])
+        dA += np.einsum("bdn,bd->dn", G * decay * hprev, dt[:, t, :])
+        du[:, t, :] += dt[:, t, :] * np.einsum("bdn,bn->bd", G, Bm[:, t, :])
+        G = G * decay
+    dh0 = G
+    ddelta = ddt * _sigmoid(delta) if delta_softplus else ddt
+
+    # conv and its SiLU
+    if conv_w is not None:
+        dpre = du * _silu_grad(pre) if conv_silu else du
+        dxpad = np.zeros((Bsz, L + K - 1, D))
+        dconv_w = np.zeros((D, K))
+        for k in range(K):
+            dxpad[:, k:k + L, :] += conv_w[None, None, :, k] * dpre
+            dconv_w[:, k] = np.einsum("bld,bld->d", dpre, xpad[:, k:k + L, :])
+        dconv_b = dpre.sum(axis=(0, 1)) if conv_b is not None else None
+        dx = dxpad[:, K - 1:, :]
+        dconv_state = np.transpose(dxpad[:, :K - 1, :], (0, 2, 1)).copy()
+    else:
+        dx, dconv_w, dconv_b, dconv_state = du, None, None, None
+    return {"dx": dx, "ddelta": ddelta, "dA": dA, "dB": dB, "dC": dC, "dD": dD, "dz": dz, "dh0": dh0,
+            "dconv_w": dconv_w, "dconv_b": dconv_b, "dconv_state": dconv_state}
+
+
+def swa_bwd(do, q, k, v, window, scale=None, block=64):
+    """Reverse-mode gradients of ``swa`` (the banded attention of page
+    "SAMBA混合注意力状态空间模型", §滑动窗口注意力, read as the causal band
+    0 <= i - j < W with grouped kv heads).
+
+    Per query row i and head h, with P the row's softmax over its visible
+    keys and dO = ∂L/∂o:  dV_j += P_ij dO_i,  dP_ij = dO_i · v_j,
+    dS_ij = P_ij (dP_ij - Σ_j' P_ij' dP_ij'),  dq_i = scale Σ_j dS_ij k_j,
+    dk_j += scale dS_ij q_i; the gradients of a kv head sum over the query
+    heads that read it.  Processed per query block over the banded keys.
+
+    Returns (dq [B, L, Hq, d], dk, dv [B, L, Hkv, d]).
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    do = _f64(do)
+    Bsz, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    group = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for i0 in range(0, L, block):
+        i1 = min(L, i0 + block)
+        j0 = max(0, i0 - window + 1)
+        mask = _visible(np.arange(i0, i1)[:, None], np.arange(j0, i1)[None, :], window)
+        for h in range(Hq):
+            kv = h // group
+            s = np.einsum("bid,bjd->bij", q[:, i0:i1, h, :], k[:, j0:i1, kv, :]) * scale
+            s = np.where(mask[None], s, -np.inf)
+            e = np.exp(s - s.max(axis=2, keepdims=True))
+            p = e / e.sum(axis=2, keepdims=True)
+            dv[:, j0:i1, kv, :] += np.einsum("bij,bid->bjd", p, do[:, i0:i1, h, :])
+            dp = np.einsum("bid,bjd->bij", do[:, i0:i1, h, :], v[:, j0:i1, kv, :])
+            ds = p * (dp - (p * dp).sum(axis=2, keepdims=True))
+            dq[:, i0:i1, h, :] += scale * np.einsum("bij,bjd->bid", ds, k[:, j0:i1, kv, :])
+            dk[:, j0:i1, kv, :] += scale * np.einsum("bij,bid->bjd", ds, q[:, i0:i1, h, :])
+    return dq, dk, dv
 
 
 # --------------------------------------------------------------- layers

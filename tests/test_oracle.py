@@ -562,3 +562,184 @@ def test_swa_layer_matches_torch_functional_composition():
     o = F.scaled_dot_product_attention(q, k, v, is_causal=True).transpose(1, 2).reshape(2, L, Hq * d)
     ref = F.linear(o, torch.from_numpy(o_proj)).numpy()
     np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-11)
+
+
+# ----------------------------------------------------------------- backward
+def _scan_bwd_inputs(seed, Bsz=2, L=7, D=3, N=2, K=4):
+    r = _rng(seed)
+    return {
+        "x": r.standard_normal((Bsz, L, D)), "delta": r.standard_normal((Bsz, L, D)) * 0.7 - 1.0,
+        "A": -r.uniform(0.2, 2.0, (D, N)), "Bm": r.standard_normal((Bsz, L, N)), "Cm": r.standard_normal((Bsz, L, N)),
+        "Dskip": r.standard_normal(D), "z": r.standard_normal((Bsz, L, D)), "h0": r.standard_normal((Bsz, D, N)),
+        "conv_w": r.standard_normal((D, K)) * 0.5, "conv_b": r.standard_normal(D) * 0.3,
+        "conv_state": r.standard_normal((Bsz, D, K - 1)),
+    }
+
+
+_SCAN_GRAD_OF = {"x": "dx", "delta": "ddelta", "A": "dA", "Bm": "dB", "Cm": "dC", "Dskip": "dD", "z": "dz",
+                 "h0": "dh0", "conv_w": "dconv_w", "conv_b": "dconv_b", "conv_state": "dconv_state"}
+
+
+@pytest.mark.parametrize("name", list(_SCAN_GRAD_OF))
+def test_scan_bwd_matches_central_differences(name):
+    """Directional derivative of <dy, y> along a random direction, by central
+    differences in float64, equals <gradient, direction> (brute force, no
+    shared derivation)."""
+    inp = _scan_bwd_inputs(40)
+    r = _rng(41)
+    dy = r.standard_normal(inp["x"].shape)
+    g = orc.selective_scan_bwd(dy, **inp)[_SCAN_GRAD_OF[name]]
+    direction = r.standard_normal(np.shape(inp[name]))
+    eps = 1e-6
+
+    def f(sign):
+        args = dict(inp)
+        args[name] = inp[name] + sign * eps * direction
+        return float(np.sum(dy * orc.selective_scan(**args)["y"]))
+
+    fd = (f(1) - f(-1)) / (2 * eps)
+    an = float(np.sum(g * direction))
+    assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), (name, fd, an)
+
+
+def test_scan_bwd_matches_torch_autograd():
+    """All gradients against torch autograd of the same recurrence written
+    with plain torch operations in float64."""
+    inp = _scan_bwd_inputs(42, Bsz=2, L=12, D=5, N=3)
+    dy = _rng(43).standard_normal(inp["x"].shape)
+    got = orc.selective_scan_bwd(dy, **inp)
+    t = {k: torch.tensor(v, requires_grad=True) for k, v in inp.items()}
+    F = torch.nn.functional
+    Bsz, L, D = inp["x"].shape
+    K = inp["conv_w"].shape[1]
+    xpad = torch.cat([t["conv_state"].transpose(1, 2), t["x"]], dim=1)
+    pre = F.conv1d(xpad.transpose(1, 2), t["conv_w"][:, None, :], t["conv_b"], groups=D).transpose(1, 2)
+    u = F.silu(pre)
+    dt = F.softplus(t["delta"])
+    h = t["h0"]
+    ys = []
+    for s in range(L):
+        h = torch.exp(dt[:, s, :, None] * t["A"]) * h + (dt[:, s] * u[:, s])[:, :, None] * t["Bm"][:, s, None, :]
+        ys.append((h * t["Cm"][:, s, None, :]).sum(-1))
+    y = (torch.stack(ys, 1) + t["Dskip"] * u) * F.silu(t["z"])
+    y.backward(torch.from_numpy(dy))
+    for name, key in _SCAN_GRAD_OF.items():
+        np.testing.assert_allclose(got[key], t[name].grad.numpy(), rtol=1e-10, atol=1e-12, err_msg=name)
+
+
+def test_scan_bwd_without_conv_gate_or_skip():
+    """Optional parts absent: the gradient of y = C·h alone, against autograd."""
+    inp = _scan_bwd_inputs(44, Bsz=1, L=9, D=4, N=3)
+    dy = _rng(45).standard_normal(inp["x"].shape)
+    got = orc.selective_scan_bwd(dy, inp["x"], inp["delta"], inp["A"], inp["Bm"], inp["Cm"], delta_softplus=False)
+    assert got["dz"] is None and got["dD"] is None and got["dconv_w"] is None
+    t = {k: torch.tensor(inp[k], requires_grad=True) for k in ("x", "delta", "A", "Bm", "Cm")}
+    h = torch.zeros((1, 4, 3), dtype=torch.float64)
+    ys = []
+    for s in range(9):
+        h = torch.exp(t["delta"][:, s, :, None] * t["A"]) * h + (t["delta"][:, s] * t["x"][:, s])[:, :, None] * t["Bm"][:, s, None, :]
+        ys.append((h * t["Cm"][:, s, None, :]).sum(-1))
+    torch.stack(ys, 1).backward(torch.from_numpy(dy))
+    for name, key in (("x", "dx"), ("delta", "ddelta"), ("A", "dA"), ("Bm", "dB"), ("Cm", "dC")):
+        np.testing.assert_allclose(got[key], t[name].grad.numpy(), rtol=1e-10, atol=1e-12, err_msg=name)
+
+
+def test_scan_bwd_zero_step_closed_form():
+    """Δ = 0 (no softplus): the state never changes and y_t = C_t·h0, so
+    dC_t = Σ_c dy_t,c h0_c, dh0 = Σ_t dy_t ⊗ C_t, dA = 0, dB = 0 and dx = 0."""
+    r = _rng(46)
+    Bsz, L, D, N = 2, 6, 3, 4
+    h0 = r.standard_normal((Bsz, D, N))
+    Bm, Cm, dy = r.standard_normal((Bsz, L, N)), r.standard_normal((Bsz, L, N)), r.standard_normal((Bsz, L, D))
+    got = orc.selective_scan_bwd(dy, r.standard_normal((Bsz, L, D)), np.zeros((Bsz, L, D)), -np.ones((D, N)), Bm, Cm,
+                                 h0=h0, delta_softplus=False)
+    np.testing.assert_allclose(got["dC"], np.einsum("bld,bdn->bln", dy, h0), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(got["dh0"], np.einsum("bld,bln->bdn", dy, Cm), rtol=1e-12, atol=1e-12)
+    for key in ("dA", "dB", "dx"):
+        assert np.all(got[key] == 0), key
+
+
+def _swa_bwd_inputs(seed, Bsz=1, L=11, Hq=4, Hkv=2, d=3):
+    r = _rng(seed)
+    return (r.standard_normal((Bsz, L, Hq, d)), r.standard_normal((Bsz, L, Hkv, d)),
+            r.standard_normal((Bsz, L, Hkv, d)), r.standard_normal((Bsz, L, Hq, d)))
+
+
+@pytest.mark.parametrize("W", [1, 3, 5, 100])
+@pytest.mark.parametrize("which", [0, 1, 2])
+def test_swa_bwd_matches_central_differences(W, which):
+    q, k, v, do = _swa_bwd_inputs(50 + W)
+    grads = orc.swa_bwd(do, q, k, v, W, block=4)
+    args = [q, k, v]
+    direction = _rng(60 + which).standard_normal(args[which].shape)
+    eps = 1e-6
+
+    def f(sign):
+        a = list(args)
+        a[which] = args[which] + sign * eps * direction
+        return float(np.sum(do * orc.swa(a[0], a[1], a[2], W)[0]))
+
+    fd = (f(1) - f(-1)) / (2 * eps)
+    an = float(np.sum(grads[which] * direction))
+    assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), (W, which, fd, an)
+
+
+@pytest.mark.parametrize("W", [1, 4, 17, 64])
+def test_swa_bwd_matches_torch_autograd_of_masked_softmax(W):
+    q, k, v, do = _swa_bwd_inputs(70 + W, Bsz=2, L=40, Hq=6, Hkv=2, d=8)
+    dq, dk, dv = orc.swa_bwd(do, q, k, v, W, block=16)
+    tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+    g = 3
+    i = torch.arange(40)[:, None]
+    j = torch.arange(40)[None, :]
+    mask = (i - j >= 0) & (i - j < W)
+    s = torch.einsum("bihd,bjhd->bhij", tq, tk.repeat_interleave(g, 2)) / math.sqrt(8)
+    p = torch.softmax(s.masked_fill(~mask, float("-inf")), dim=-1)
+    o = torch.einsum("bhij,bjhd->bihd", p, tv.repeat_interleave(g, 2))
+    o.backward(torch.from_numpy(do))
+    for got, ref in ((dq, tq), (dk, tk), (dv, tv)):
+        np.testing.assert_allclose(got, ref.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_swa_bwd_window_one_closed_form():
+    """W = 1: o_i = v_i, so dv = the dO of the query heads that read each kv
+    head summed, and dq = dk = 0."""
+    q, k, v, do = _swa_bwd_inputs(80, Bsz=2, L=9, Hq=6, Hkv=3, d=4)
+    dq, dk, dv = orc.swa_bwd(do, q, k, v, 1)
+    np.testing.assert_allclose(dv, do.reshape(2, 9, 3, 2, 4).sum(axis=3), rtol=1e-12, atol=1e-12)
+    assert np.all(dq == 0) and np.all(dk == 0)
+
+
+def test_planted_swa_bwd_without_row_correction_is_caught():
+    """A backward that drops the Σ P dP term of dS fails the same
+    central-difference check that the oracle passes."""
+    q, k, v, do = _swa_bwd_inputs(81)
+    W = 5
+    direction = _rng(82).standard_normal(q.shape)
+    eps = 1e-6
+    fd = (np.sum(do * orc.swa(q + eps * direction, k, v, W)[0]) -
+          np.sum(do * orc.swa(q - eps * direction, k, v, W)[0])) / (2 * eps)
+    good = orc.swa_bwd(do, q, k, v, W)[0]
+    bad = _swa_bwd_dq_without_correction(do, q, k, v, W)
+    assert abs(fd - np.sum(good * direction)) <= 1e-7 * max(1.0, abs(fd))
+    assert abs(fd - np.sum(bad * direction)) > 1e-3 * max(1.0, abs(fd))
+
+
+def _swa_bwd_dq_without_correction(do, q, k, v, W):
+    """dq of a backward with dS = P ⊙ dP (the Σ P dP term dropped): the
+    planted mistake for the test above, written out here so the oracle itself
+    is not modified."""
+    Bsz, L, Hq, d = q.shape
+    group = Hq // k.shape[2]
+    scale = 1.0 / math.sqrt(d)
+    dq = np.zeros_like(q)
+    i = np.arange(L)[:, None]
+    j = np.arange(L)[None, :]
+    mask = (i - j >= 0) & (i - j < W)
+    for h in range(Hq):
+        s = np.where(mask, np.einsum("bid,bjd->bij", q[:, :, h], k[:, :, h // group]) * scale, -np.inf)
+        p = np.exp(s - s.max(axis=2, keepdims=True))
+        p /= p.sum(axis=2, keepdims=True)
+        dp = np.einsum("bid,bjd->bij", do[:, :, h], v[:, :, h // group])
+        dq[:, :, h] = scale * np.einsum("bij,bjd->bid", p * dp, k[:, :, h // group])
+    return dq
