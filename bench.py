@@ -829,9 +829,9 @@ def main():
     if os.path.exists(traffic_file):
         try:
             tr = json.load(open(traffic_file))
-            for name, roof in (("scan", scan_roof), ("swa", swa_roof)):
+            for name, src, roof in (("scan", "scan_fwd", scan_roof), ("swa", "swa_fwd", swa_roof)):
                 ent = tr.get(name, {}).get(wl.name)
-                if ent and ent.get("source_hash") == B.source_hash():
+                if ent and ent.get("kernel_hash") == B.kernel_hash(src):
                     roof["traffic"] = ent["bytes_per_launch"]
         except Exception:
             pass

@@ -52,6 +52,20 @@ def source_hash() -> str:
     return h.hexdigest()[:12]
 
 
+def kernel_hash(name: str) -> str:
+    """Short hash of one kernel file (``csrc/<name>.cu``) and the shared device
+    header it includes: the sources that fix that kernel's device code, so a
+    recorded profile of it stays valid while other files change."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for d in (os.path.join(CSRC, name + ".cu"), os.path.join(CSRC, "common.cuh")):
+        h.update(os.path.basename(d).encode())
+        with open(d, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
 def up_to_date() -> bool:
     if not os.path.exists(LIB):
         return False
