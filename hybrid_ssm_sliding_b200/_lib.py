@@ -37,6 +37,19 @@ class ScanArgs(ctypes.Structure):
     ]
 
 
+class ScanBwdArgs(ctypes.Structure):
+    _fields_ = [
+        ("x", _vp), ("z", _vp), ("delta", _vp), ("A", _vp), ("Bm", _vp), ("Cm", _vp), ("Dskip", _vp),
+        ("conv_w", _vp), ("conv_b", _vp), ("conv_state_in", _vp), ("h0", _vp), ("dy", _vp),
+        ("dx", _vp), ("ddelta", _vp), ("dz", _vp), ("dA", _vp), ("dB", _vp), ("dC", _vp), ("dD", _vp),
+        ("dconv_w", _vp), ("dconv_b", _vp), ("dh0", _vp), ("dconv_state", _vp),
+        ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
+        ("batch", _i64), ("seqlen", _i64), ("dim", _i64),
+        ("dstate", _i32), ("dconv", _i32), ("x_dtype", _i32), ("z_dtype", _i32), ("y_dtype", _i32),
+        ("flags", ctypes.c_uint32),
+    ]
+
+
 class SwaArgs(ctypes.Structure):
     _fields_ = [
         ("q", _vp), ("k", _vp), ("v", _vp), ("o", _vp), ("lse", _vp),
@@ -93,10 +106,13 @@ def load() -> ctypes.CDLL:
                                            ctypes.c_int, _i64, ctypes.c_float, _vp]
     lib.samba_gemm.argtypes = [ctypes.POINTER(GemmArgs), _vp]
     lib.samba_scan_carry.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, ctypes.c_int, _vp]
+    lib.samba_scan_bwd_workspace_size.argtypes = [_i64, _i64, _i64, _i32]
+    lib.samba_scan_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.samba_selective_scan_bwd.argtypes = [ctypes.POINTER(ScanBwdArgs), _vp]
     lib.samba_conv_state.argtypes = [_vp, ctypes.c_int, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp]
     for name in ("samba_conv1d_fwd", "samba_selective_scan_fwd", "samba_swa_fwd", "samba_mixer_prefill",
                  "samba_scan_step", "samba_swa_ring_fill", "samba_swa_step", "samba_get_status",
-                 "samba_scan_carry", "samba_conv_state", "samba_gemm",
+                 "samba_scan_carry", "samba_conv_state", "samba_gemm", "samba_selective_scan_bwd",
                  "samba_selftest_wait_timeout", "samba_swa_step_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib

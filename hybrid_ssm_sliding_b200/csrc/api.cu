@@ -158,6 +158,54 @@ static int check_swa(const samba_swa_args* a, const char* who) {
   return SAMBA_OK;
 }
 
+size_t samba_scan_bwd_workspace_size(int64_t batch, int64_t seqlen, int64_t dim, int32_t dstate) {
+  if (batch < 1 || seqlen < 1 || dim < 1 || dstate < 1) return 0;
+  return scan_bwd_workspace(batch, seqlen, dim, dstate);
+}
+
+int samba_selective_scan_bwd(const samba_scan_bwd_args* a, samba_stream_t stream) {
+  const char* who = "samba_selective_scan_bwd";
+  if (!a) return fail(SAMBA_ERR_INVALID_ARG, "%s: null args", who);
+  // the forward's checks on the shared fields
+  samba_scan_args f = {};
+  f.x = a->x;
+  f.z = a->z;
+  f.delta = a->delta;
+  f.A = a->A;
+  f.Bm = a->Bm;
+  f.Cm = a->Cm;
+  f.Dskip = a->Dskip;
+  f.conv_w = a->conv_w;
+  f.conv_b = a->conv_b;
+  f.y = const_cast<void*>(a->dy);  // read only: checked like the forward output
+  f.batch = a->batch;
+  f.seqlen = a->seqlen;
+  f.dim = a->dim;
+  f.dstate = a->dstate;
+  f.dconv = a->dconv;
+  f.x_dtype = a->x_dtype;
+  f.z_dtype = a->z_dtype;
+  f.y_dtype = a->y_dtype;
+  f.flags = a->flags;
+  int rc = check_scan(&f, who);
+  if (rc != SAMBA_OK) return rc;
+  if (a->z && a->z_dtype != a->x_dtype) return fail(SAMBA_ERR_UNSUPPORTED, "%s: z dtype must equal x dtype", who);
+  if (!a->dx || !a->ddelta || !a->dA || !a->dB || !a->dC)
+    return fail(SAMBA_ERR_INVALID_ARG, "%s: dy, dx, ddelta, dA, dB and dC are required", who);
+  if ((a->z && !a->dz) || (a->Dskip && !a->dD))
+    return fail(SAMBA_ERR_INVALID_ARG, "%s: dz is required with z and dD with Dskip", who);
+  const bool fuse = (a->flags & SAMBA_SCAN_FUSE_CONV) != 0;
+  if (fuse && (!a->dconv_w || (a->conv_b && !a->dconv_b)))
+    return fail(SAMBA_ERR_INVALID_ARG, "%s: dconv_w (and dconv_b with conv_b) are required with FUSE_CONV", who);
+  const void* ptrs[] = {a->dx, a->dz, a->ddelta, a->dB, a->dC, a->workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SAMBA_ERR_INVALID_ARG, "%s: misaligned pointer", who);
+  const size_t need = scan_bwd_workspace(a->batch, a->seqlen, a->dim, a->dstate);
+  if (!a->workspace || need == SIZE_MAX || a->workspace_bytes < need)
+    return fail(SAMBA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed", who, need);
+  return launch_scan_bwd(*a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int samba_gemm(const samba_gemm_args* a, samba_stream_t stream) {
   const char* who = "samba_gemm";
   if (!a || !a->A || !a->B) return fail(SAMBA_ERR_INVALID_ARG, "%s: A and B are required", who);

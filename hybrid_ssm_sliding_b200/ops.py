@@ -107,6 +107,60 @@ def selective_scan_fwd(x, delta, A, B, C, D=None, z=None, conv_w=None, conv_b=No
     return y
 
 
+def scan_bwd_workspace_size(batch, seqlen, dim, dstate):
+    return int(L.load().samba_scan_bwd_workspace_size(batch, seqlen, dim, dstate))
+
+
+def selective_scan_bwd(dy, x, delta, A, B, C, D=None, z=None, conv_w=None, conv_b=None, conv_state_in=None,
+                       h0=None, delta_softplus=True, conv_silu=True, fuse_conv=None, want_dh0=False,
+                       want_dconv_state=False, workspace=None, stream=None):
+    """Gradients of selective_scan_fwd's y given dy (see
+    samba_selective_scan_bwd).  Returns a dict with dx, ddelta, dA, dB, dC
+    and, where the forward input exists, dz, dD, dconv_w, dconv_b, plus dh0 /
+    dconv_state when asked for."""
+    _need(x, "x")
+    Bsz, Ln, Dm = x.shape
+    N = A.shape[1]
+    _need(dy, "dy", None, x.shape)
+    _need(delta, "delta", torch.float32, x.shape)
+    _need(A, "A", torch.float32, (Dm, N))
+    _need(B, "B", torch.float32, (Bsz, Ln, N))
+    _need(C, "C", torch.float32, (Bsz, Ln, N))
+    _opt(D, "D", torch.float32, (Dm,))
+    _opt(z, "z", x.dtype, x.shape)
+    if fuse_conv is None:
+        fuse_conv = conv_w is not None
+    K = conv_w.shape[1] if conv_w is not None else 4
+    _opt(conv_w, "conv_w", torch.float32, (Dm, K))
+    _opt(conv_b, "conv_b", torch.float32, (Dm,))
+    _opt(conv_state_in, "conv_state_in", torch.float32, (Bsz, Dm, K - 1))
+    _opt(h0, "h0", torch.float32, (Bsz, Dm, N))
+    dev = x.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"dx": torch.empty_like(x), "ddelta": torch.empty((Bsz, Ln, Dm), **f32), "dA": torch.empty((Dm, N), **f32),
+           "dB": torch.empty((Bsz, Ln, N), **f32), "dC": torch.empty((Bsz, Ln, N), **f32),
+           "dz": torch.empty_like(x) if z is not None else None,
+           "dD": torch.empty((Dm,), **f32) if D is not None else None,
+           "dconv_w": torch.empty((Dm, K), **f32) if fuse_conv else None,
+           "dconv_b": torch.empty((Dm,), **f32) if fuse_conv and conv_b is not None else None,
+           "dh0": torch.empty((Bsz, Dm, N), **f32) if want_dh0 else None,
+           "dconv_state": torch.empty((Bsz, Dm, K - 1), **f32) if want_dconv_state else None}
+    need = scan_bwd_workspace_size(Bsz, Ln, Dm, N)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=dev)
+    flags = ((L.SCAN_FUSE_CONV if fuse_conv else 0) | (L.SCAN_DELTA_SOFTPLUS if delta_softplus else 0)
+             | (L.SCAN_CONV_SILU if conv_silu else 0))
+    a = L.ScanBwdArgs(L.ptr(x), L.ptr(z), L.ptr(delta), L.ptr(A), L.ptr(B), L.ptr(C), L.ptr(D), L.ptr(conv_w),
+                      L.ptr(conv_b), L.ptr(conv_state_in), L.ptr(h0), L.ptr(dy),
+                      L.ptr(out["dx"]), L.ptr(out["ddelta"]), L.ptr(out["dz"]), L.ptr(out["dA"]), L.ptr(out["dB"]),
+                      L.ptr(out["dC"]), L.ptr(out["dD"]), L.ptr(out["dconv_w"]), L.ptr(out["dconv_b"]),
+                      L.ptr(out["dh0"]), L.ptr(out["dconv_state"]), L.ptr(workspace),
+                      workspace.numel() * workspace.element_size(), Bsz, Ln, Dm, N, K, L.dtype_code(x),
+                      L.dtype_code(z) if z is not None else 0, L.dtype_code(dy), flags)
+    L.check(L.load().samba_selective_scan_bwd(ctypes.byref(a), L.stream_handle(stream)))
+    return out
+
+
 def _swa_struct(q, k, v, window, scale=None, o=None, lse=None):
     _need(q, "q", torch.bfloat16)
     Bsz, Ln, Hq, d = q.shape

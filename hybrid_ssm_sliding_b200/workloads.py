@@ -73,6 +73,9 @@ WORKLOADS = {
     "layers_4k": Workload("layers_4k", 1, 4096, 4096, 16, 4, 32, 4, 64, 2048, 6, d_model=2048, dt_rank=128),
     "layers_128k": Workload("layers_128k", 1, 131072, 4096, 16, 4, 32, 4, 64, 2048, 7, d_model=2048,
                             dt_rank=128),
+    # forward + backward of both mixers at the pages' 4K training context,
+    # 8 sequences per step
+    "train_4k": Workload("train_4k", 8, 4096, 4096, 16, 4, 32, 4, 64, 2048, 8),
 }
 
 
@@ -141,3 +144,20 @@ def make_decode_step_inputs(wl: Workload, step: int, device="cpu"):
         "k": _normal((Bsz, wl.heads_kv, wl.head_dim), gen, device, wl.attn_dtype),
         "v": _normal((Bsz, wl.heads_kv, wl.head_dim), gen, device, wl.attn_dtype),
     }
+
+
+def make_output_grads(wl: Workload, device="cpu", y_dtype=None, with_attention=True, with_scan=True):
+    """Seeded gradients of a loss with respect to the mixers' outputs, for the
+    backward: dy [B, L, D] (y_dtype, default the activation dtype) and dO
+    [B, L, Hq, d] bf16, N(0, 1), from a generator of their own (seed + 1000)
+    so that the forward inputs do not depend on them."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(wl.seed + 1000)
+    out = {}
+    dy = _normal((wl.batch, wl.seqlen, wl.dim), gen, device, y_dtype or wl.act_dtype)
+    do = _normal((wl.batch, wl.seqlen, wl.heads_q, wl.head_dim), gen, device, wl.attn_dtype)
+    if with_scan:
+        out["dy"] = dy
+    if with_attention:
+        out["do"] = do
+    return out

@@ -162,6 +162,79 @@ typedef struct samba_scan_args {
 
 int samba_selective_scan_fwd(const samba_scan_args* args, samba_stream_t stream);
 
+/* --------------------------------------------------------- scan backward
+ * Reverse-mode gradients of samba_selective_scan_fwd's output y (the
+ * recurrence of page "SAMBA混合注意力状态空间模型", section 数学框架 /
+ * Mamba层, with the forward's readings): given dy = ∂L/∂y, the call writes
+ * ∂L/∂ of every input.  With G_t = ∂L/∂h_t = C_t g_t + exp(Δ_{t+1} A) G_{t+1}
+ * and g_t = dy_t silu(z_t):
+ *   dC_t = Σ_c g_t h_t      dB_t = Σ_c G_t Δ_t u_t     dA = Σ_{b,t} G_t Δ_t Ā_t h_{t-1}
+ *   dΔ_t = Σ_n G_t (A Ā_t h_{t-1} + B_t u_t)          du_t = D g_t + Δ_t Σ_n G_t B_t
+ *   dD = Σ_{b,t} g_t u_t    dz_t = dy_t (C_t·h_t + D u_t) silu'(z_t)   dh0 = Ā_0 G_0
+ * then ddelta = dΔ σ(delta) (with DELTA_SOFTPLUS) and, with FUSE_CONV, the
+ * gradients through the conv's SiLU and the depthwise conv (dx, dconv_w,
+ * dconv_b, dconv_state).  The forward states are recomputed: a first pass
+ * stores the state at the start of every 16-token chunk in the workspace,
+ * then every chunk is recomputed and walked from its last token to its first.
+ *
+ * Inputs are those of the forward (same shapes, dtypes and flags; y_dtype is
+ * the dtype of dy).  Outputs:
+ *   dx      [B, L, D]  x_dtype          ddelta [B, L, D] fp32
+ *   dz      [B, L, D]  x_dtype, required iff z is given
+ *   dA      [D, N]     fp32 (summed over the batch)
+ *   dB, dC  [B, L, N]  fp32 (summed over the channels)
+ *   dD      [D]        fp32, required iff Dskip is given
+ *   dconv_w [D, K], dconv_b [D] fp32, required with FUSE_CONV (dconv_b iff conv_b)
+ *   dh0     [B, D, N]  fp32, or NULL
+ *   dconv_state [B, D, K-1] fp32, or NULL (meaningful with FUSE_CONV)
+ * dA, dB, dC, dD, dconv_w and dconv_b are sums of contributions added with
+ * atomics: the call clears them on the stream first, and their summation
+ * order (hence the last bits) varies between runs.  The workspace is
+ * caller-owned device memory of samba_scan_bwd_workspace_size() bytes,
+ * 16-byte aligned; nothing else is allocated.
+ * Errors: as samba_selective_scan_fwd for the inputs, plus
+ * SAMBA_ERR_INVALID_ARG for a missing dy, dx, ddelta, dA, dB or dC, a missing
+ * dz / dD / dconv_w / dconv_b where the forward input exists, or a misaligned
+ * pointer; SAMBA_ERR_WORKSPACE for a missing or short workspace.
+ */
+typedef struct samba_scan_bwd_args {
+  const void* x;               /* forward inputs, as samba_scan_args           */
+  const void* z;
+  const float* delta;
+  const float* A;
+  const float* Bm;
+  const float* Cm;
+  const float* Dskip;
+  const float* conv_w;
+  const float* conv_b;
+  const float* conv_state_in;
+  const float* h0;
+  const void* dy;              /* [B, L, D]   y_dtype                          */
+  void* dx;                    /* [B, L, D]   x_dtype                          */
+  float* ddelta;               /* [B, L, D]                                    */
+  void* dz;                    /* [B, L, D]   x_dtype, iff z                   */
+  float* dA;                   /* [D, N]                                       */
+  float* dB;                   /* [B, L, N]                                    */
+  float* dC;                   /* [B, L, N]                                    */
+  float* dD;                   /* [D], iff Dskip                               */
+  float* dconv_w;              /* [D, K], with FUSE_CONV                       */
+  float* dconv_b;              /* [D], with FUSE_CONV and conv_b               */
+  float* dh0;                  /* [B, D, N] or NULL                            */
+  float* dconv_state;          /* [B, D, K-1] or NULL                          */
+  void* workspace;             /* samba_scan_bwd_workspace_size() bytes        */
+  size_t workspace_bytes;
+  int64_t batch, seqlen, dim;  /* as the forward                               */
+  int32_t dstate, dconv;
+  int32_t x_dtype, z_dtype, y_dtype;
+  uint32_t flags;
+} samba_scan_bwd_args;
+
+/* Bytes of workspace samba_selective_scan_bwd needs (the chunk checkpoints,
+ * B * ceil(L/16) * N * D fp32); SIZE_MAX if that overflows. */
+size_t samba_scan_bwd_workspace_size(int64_t batch, int64_t seqlen, int64_t dim, int32_t dstate);
+
+int samba_selective_scan_bwd(const samba_scan_bwd_args* args, samba_stream_t stream);
+
 /* ------------------------------------------------------ sequence segments
  * A sequence split into consecutive segments (for example one per GPU) can be
  * scanned segment by segment with exactly the result of one pass, because the

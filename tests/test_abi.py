@@ -215,3 +215,34 @@ def test_gemm_rejects_bad_arguments_on_host(lib):
     assert call(ld=100) == L.SAMBA_ERR_INVALID_ARG          # row stride below the range
     assert call(dtype=7) == L.SAMBA_ERR_UNSUPPORTED
     assert call(M=65535 * 128 + 1) == L.SAMBA_ERR_UNSUPPORTED
+
+
+def test_scan_bwd_rejects_bad_arguments_on_host(lib):
+    f = 0x80000
+    need = lib.samba_scan_bwd_workspace_size(2, 100, 64, 16)
+    # ceil(100 / 16) chunk checkpoints, then per-32-channel-block partials of dB and dC
+    assert need == 2 * 7 * 16 * 64 * 4 + (64 // 32) * 2 * 2 * 100 * 16 * 4
+    assert lib.samba_scan_bwd_workspace_size(0, 100, 64, 16) == 0
+    assert lib.samba_scan_bwd_workspace_size(2**40, 2**40, 2**20, 16) == 2**64 - 1   # saturates
+
+    def call(**over):
+        a = L.ScanBwdArgs()
+        for k in ("x", "delta", "A", "Bm", "Cm", "dy", "dx", "ddelta", "dA", "dB", "dC", "workspace"):
+            setattr(a, k, f)
+        a.batch, a.seqlen, a.dim, a.dstate, a.dconv = 2, 100, 64, 16, 4
+        a.workspace_bytes = need
+        a.x_dtype = a.y_dtype = 1
+        for k, v in over.items():
+            setattr(a, k, v)
+        return lib.samba_selective_scan_bwd(ctypes.byref(a), None)
+
+    assert lib.samba_selective_scan_bwd(None, None) == L.SAMBA_ERR_INVALID_ARG
+    assert call(dy=None) == L.SAMBA_ERR_INVALID_ARG
+    assert call(dB=None) == L.SAMBA_ERR_INVALID_ARG
+    assert call(z=f, z_dtype=1) == L.SAMBA_ERR_INVALID_ARG              # z without dz
+    assert call(Dskip=f) == L.SAMBA_ERR_INVALID_ARG                     # Dskip without dD
+    assert call(flags=L.SCAN_FUSE_CONV, conv_w=f) == L.SAMBA_ERR_INVALID_ARG   # no dconv_w
+    assert call(dx=f + 4) == L.SAMBA_ERR_INVALID_ARG                     # misaligned
+    assert call(dstate=12) == L.SAMBA_ERR_UNSUPPORTED
+    assert call(workspace=None) == L.SAMBA_ERR_WORKSPACE
+    assert call(workspace_bytes=need - 1) == L.SAMBA_ERR_WORKSPACE
