@@ -459,7 +459,7 @@ def selective_scan_bwd(dy, x, delta, A, Bm, Cm, Dskip=None, z=None, h0=None,
             "dconv_w": dconv_w, "dconv_b": dconv_b, "dconv_state": dconv_state}
 
 
-def swa_bwd(do, q, k, v, window, scale=None, block=64):
+def swa_bwd(do, q, k, v, window, scale=None, block=64, magnitudes=False):
     """Reverse-mode gradients of ``swa`` (the banded attention of page
     "SAMBA混合注意力状态空间模型", §滑动窗口注意力, read as the causal band
     0 <= i - j < W with grouped kv heads).
@@ -470,7 +470,15 @@ def swa_bwd(do, q, k, v, window, scale=None, block=64):
     dk_j += scale dS_ij q_i; the gradients of a kv head sum over the query
     heads that read it.  Processed per query block over the banded keys.
 
-    Returns (dq [B, L, Hq, d], dk, dv [B, L, Hkv, d]).
+    Returns (dq [B, L, Hq, d], dk, dv [B, L, Hkv, d]).  With ``magnitudes``
+    also a dict of the sizes of the sums that produce them, the same sums over
+    the absolute values of their terms (what rounding error of a finite-
+    precision evaluation scales with):
+        dv_mag = Σ_i P |dO_i|,  dq_mag = scale Σ_j (|dS| + P Dm_i) |k_j|,
+        dk_mag = scale Σ_i (|dS| + P Dm_i) |q_i|,  Dm_i = Σ_d |dO_id| Σ_j P_ij |v_jd|,
+    where the P Dm term sizes D_i = dO_i · o_i, which an implementation takes
+    from its stored o (itself a sum of size Σ_j P |v_j|) rather than as
+    Σ_j P dP.
     """
     q = _f64(q)
     k = _f64(k)
@@ -484,6 +492,8 @@ def swa_bwd(do, q, k, v, window, scale=None, block=64):
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
+    if magnitudes:
+        mq, mk, mv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     for i0 in range(0, L, block):
         i1 = min(L, i0 + block)
         j0 = max(0, i0 - window + 1)
@@ -499,6 +509,15 @@ def swa_bwd(do, q, k, v, window, scale=None, block=64):
             ds = p * (dp - (p * dp).sum(axis=2, keepdims=True))
             dq[:, i0:i1, h, :] += scale * np.einsum("bij,bjd->bid", ds, k[:, j0:i1, kv, :])
             dk[:, j0:i1, kv, :] += scale * np.einsum("bij,bid->bjd", ds, q[:, i0:i1, h, :])
+            if magnitudes:
+                omag = np.einsum("bij,bjd->bid", p, np.abs(v[:, j0:i1, kv, :]))
+                dmag = np.einsum("bid,bid->bi", np.abs(do[:, i0:i1, h, :]), omag)[:, :, None]
+                w = np.abs(ds) + p * dmag
+                mv[:, j0:i1, kv, :] += np.einsum("bij,bid->bjd", p, np.abs(do[:, i0:i1, h, :]))
+                mq[:, i0:i1, h, :] += scale * np.einsum("bij,bjd->bid", w, np.abs(k[:, j0:i1, kv, :]))
+                mk[:, j0:i1, kv, :] += scale * np.einsum("bij,bid->bjd", w, np.abs(q[:, i0:i1, h, :]))
+    if magnitudes:
+        return dq, dk, dv, {"dq": mq, "dk": mk, "dv": mv}
     return dq, dk, dv
 
 

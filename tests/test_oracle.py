@@ -743,3 +743,41 @@ def _swa_bwd_dq_without_correction(do, q, k, v, W):
         dp = np.einsum("bid,bjd->bij", do[:, :, h], v[:, :, h // group])
         dq[:, :, h] = scale * np.einsum("bij,bjd->bid", p * dp, k[:, :, h // group])
     return dq
+
+
+def test_swa_bwd_magnitudes_bound_the_gradients():
+    """The magnitudes are sums of absolute values of the terms of each
+    gradient, so they bound it (triangle inequality), and the gradients they
+    come with are unchanged."""
+    q, k, v, do = _swa_bwd_inputs(90, Bsz=2, L=30, Hq=4, Hkv=2, d=5)
+    plain = orc.swa_bwd(do, q, k, v, 7, block=8)
+    dq, dk, dv, mag = orc.swa_bwd(do, q, k, v, 7, block=8, magnitudes=True)
+    for g, p_, key in ((dq, plain[0], "dq"), (dk, plain[1], "dk"), (dv, plain[2], "dv")):
+        np.testing.assert_array_equal(g, p_)
+        assert np.all(mag[key] >= np.abs(g) * (1 - 1e-12)), key
+
+
+def test_swa_bwd_magnitudes_by_brute_force():
+    """Each magnitude against explicit loops over (query, key) pairs on a tiny
+    case, with P, dS and the size of o written out from their definitions."""
+    q, k, v, do = _swa_bwd_inputs(91, Bsz=1, L=6, Hq=2, Hkv=1, d=3)
+    W, sc = 3, 1.0 / math.sqrt(3)
+    _, _, _, mag = orc.swa_bwd(do, q, k, v, W, magnitudes=True)
+    mq, mk, mv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for h in range(2):
+        for i in range(6):
+            js = [j for j in range(6) if 0 <= i - j < W]
+            s = np.array([q[0, i, h] @ k[0, j, 0] * sc for j in js])
+            p = np.exp(s - s.max())
+            p /= p.sum()
+            omag = sum(pj * np.abs(v[0, j, 0]) for pj, j in zip(p, js))
+            dmag = float(np.abs(do[0, i, h]) @ omag)
+            dp = np.array([do[0, i, h] @ v[0, j, 0] for j in js])
+            ds = p * (dp - p @ dp)
+            for a, j in enumerate(js):
+                mv[0, j, 0] += p[a] * np.abs(do[0, i, h])
+                w = abs(ds[a]) + p[a] * dmag
+                mq[0, i, h] += sc * w * np.abs(k[0, j, 0])
+                mk[0, j, 0] += sc * w * np.abs(q[0, i, h])
+    for key, ref in (("dq", mq), ("dk", mk), ("dv", mv)):
+        np.testing.assert_allclose(mag[key], ref, rtol=1e-12, atol=1e-14, err_msg=key)
