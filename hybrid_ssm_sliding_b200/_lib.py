@@ -58,6 +58,15 @@ class SwaArgs(ctypes.Structure):
     ]
 
 
+class SwaBwdArgs(ctypes.Structure):
+    _fields_ = [
+        ("q", _vp), ("k", _vp), ("v", _vp), ("o", _vp), ("lse", _vp), ("dO", _vp), ("dq", _vp), ("dk", _vp),
+        ("dv", _vp), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
+        ("batch", _i64), ("seqlen", _i64), ("window", _i64),
+        ("heads_q", _i32), ("heads_kv", _i32), ("head_dim", _i32), ("scale", ctypes.c_float),
+    ]
+
+
 class GemmOut(ctypes.Structure):
     _fields_ = [("ptr", _vp), ("bias", _vp), ("ld", _i64), ("col0", _i64), ("col1", _i64), ("dtype", _i32)]
 
@@ -109,10 +118,13 @@ def load() -> ctypes.CDLL:
     lib.samba_scan_bwd_workspace_size.argtypes = [_i64, _i64, _i64, _i32]
     lib.samba_scan_bwd_workspace_size.restype = ctypes.c_size_t
     lib.samba_selective_scan_bwd.argtypes = [ctypes.POINTER(ScanBwdArgs), _vp]
+    lib.samba_swa_bwd_workspace_size.argtypes = [_i64, _i64, _i32]
+    lib.samba_swa_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.samba_swa_bwd.argtypes = [ctypes.POINTER(SwaBwdArgs), _vp]
     lib.samba_conv_state.argtypes = [_vp, ctypes.c_int, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp]
     for name in ("samba_conv1d_fwd", "samba_selective_scan_fwd", "samba_swa_fwd", "samba_mixer_prefill",
                  "samba_scan_step", "samba_swa_ring_fill", "samba_swa_step", "samba_get_status",
-                 "samba_scan_carry", "samba_conv_state", "samba_gemm", "samba_selective_scan_bwd",
+                 "samba_scan_carry", "samba_conv_state", "samba_gemm", "samba_selective_scan_bwd", "samba_swa_bwd",
                  "samba_selftest_wait_timeout", "samba_swa_step_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib

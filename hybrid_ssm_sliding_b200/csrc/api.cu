@@ -91,7 +91,8 @@ const char* samba_last_error(void) { return g_last_error.c_str(); }
 
 int samba_get_status(samba_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  int codes[4] = {take_status_scan(s), take_status_swa(s), take_status_misc(s), take_status_gemm(s)};
+  int codes[5] = {take_status_scan(s), take_status_swa(s), take_status_misc(s), take_status_gemm(s),
+                  take_status_swa_bwd(s)};
   for (int c : codes)
     if (c == SAMBA_ERR_CUDA) return fail(SAMBA_ERR_CUDA, "samba_get_status: %s", cudaGetErrorString(cudaGetLastError()));
   for (int c : codes)
@@ -204,6 +205,39 @@ int samba_selective_scan_bwd(const samba_scan_bwd_args* a, samba_stream_t stream
   if (!a->workspace || need == SIZE_MAX || a->workspace_bytes < need)
     return fail(SAMBA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed", who, need);
   return launch_scan_bwd(*a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t samba_swa_bwd_workspace_size(int64_t batch, int64_t seqlen, int32_t heads_q) {
+  if (batch < 1 || seqlen < 1 || heads_q < 1) return 0;
+  return swa_bwd_workspace(batch, seqlen, heads_q);
+}
+
+int samba_swa_bwd(const samba_swa_bwd_args* a, samba_stream_t stream) {
+  const char* who = "samba_swa_bwd";
+  if (!a) return fail(SAMBA_ERR_INVALID_ARG, "%s: null args", who);
+  samba_swa_args f = {};
+  f.q = a->q;
+  f.k = a->k;
+  f.v = a->v;
+  f.o = const_cast<void*>(a->o);  // read only: checked like the forward output
+  f.batch = a->batch;
+  f.seqlen = a->seqlen;
+  f.window = a->window;
+  f.heads_q = a->heads_q;
+  f.heads_kv = a->heads_kv;
+  f.head_dim = a->head_dim;
+  f.scale = a->scale;
+  int rc = check_swa(&f, who);
+  if (rc != SAMBA_OK) return rc;
+  if (!a->lse || !a->dO || !a->dq || !a->dk || !a->dv)
+    return fail(SAMBA_ERR_INVALID_ARG, "%s: o, lse, dO, dq, dk and dv are required", who);
+  const void* ptrs[] = {a->lse, a->dO, a->dq, a->dk, a->dv, a->workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SAMBA_ERR_INVALID_ARG, "%s: misaligned pointer", who);
+  const size_t need = swa_bwd_workspace(a->batch, a->seqlen, a->heads_q);
+  if (!a->workspace || need == SIZE_MAX || a->workspace_bytes < need)
+    return fail(SAMBA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed", who, need);
+  return launch_swa_bwd(*a, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int samba_gemm(const samba_gemm_args* a, samba_stream_t stream) {

@@ -60,6 +60,9 @@ int take_status_gemm(cudaStream_t s);
 int launch_gemm(const samba_gemm_args& a, cudaStream_t stream);
 size_t scan_bwd_workspace(int64_t B, int64_t L, int64_t D, int N);
 int launch_scan_bwd(const samba_scan_bwd_args& a, cudaStream_t stream);
+size_t swa_bwd_workspace(int64_t B, int64_t L, int Hq);
+int launch_swa_bwd(const samba_swa_bwd_args& a, cudaStream_t stream);
+int take_status_swa_bwd(cudaStream_t s);
 int launch_selftest_wait(cudaStream_t s);
 
 // Launchers (validated arguments only).

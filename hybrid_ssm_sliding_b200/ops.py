@@ -183,6 +183,37 @@ def swa_fwd(q, k, v, window, scale=None, o=None, lse=None, stream=None):
     return o
 
 
+def swa_bwd_workspace_size(batch, seqlen, heads_q):
+    return int(L.load().samba_swa_bwd_workspace_size(batch, seqlen, heads_q))
+
+
+def swa_bwd(do, q, k, v, o, lse, window, scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients of swa_fwd given dO (see samba_swa_bwd): o and lse are the
+    forward's outputs for the same q, k, v.  Returns (dq, dk, dv)."""
+    _need(q, "q", torch.bfloat16)
+    Bsz, Ln, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _need(k, "k", torch.bfloat16, (Bsz, Ln, Hkv, d))
+    _need(v, "v", torch.bfloat16, (Bsz, Ln, Hkv, d))
+    _need(o, "o", torch.bfloat16, q.shape)
+    _need(do, "dO", torch.bfloat16, q.shape)
+    _need(lse, "lse", torch.float32, (Bsz, Hq, Ln))
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _need(dq, "dq", torch.bfloat16, q.shape)
+    _need(dk, "dk", torch.bfloat16, k.shape)
+    _need(dv, "dv", torch.bfloat16, v.shape)
+    need = swa_bwd_workspace_size(Bsz, Ln, Hq)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=q.device)
+    a = L.SwaBwdArgs(L.ptr(q), L.ptr(k), L.ptr(v), L.ptr(o), L.ptr(lse), L.ptr(do), L.ptr(dq), L.ptr(dk), L.ptr(dv),
+                     L.ptr(workspace), workspace.numel() * workspace.element_size(), Bsz, Ln, int(window), Hq, Hkv, d,
+                     float(scale) if scale else 0.0)
+    L.check(L.load().samba_swa_bwd(ctypes.byref(a), L.stream_handle(stream)))
+    return dq, dk, dv
+
+
 def mixer_prefill(scan: dict, swa: dict, stream=None, aux_stream=None):
     """One Mamba mixer and one SWA mixer (see samba_mixer_prefill).
     ``scan`` / ``swa`` hold the keyword arguments of selective_scan_fwd /

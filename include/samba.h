@@ -235,6 +235,49 @@ size_t samba_scan_bwd_workspace_size(int64_t batch, int64_t seqlen, int64_t dim,
 
 int samba_selective_scan_bwd(const samba_scan_bwd_args* args, samba_stream_t stream);
 
+/* ---------------------------------------------------------- SWA backward
+ * Reverse-mode gradients of samba_swa_fwd (the banded attention of page
+ * "SAMBA混合注意力状态空间模型", section 滑动窗口注意力, causal band
+ * 0 <= i - j < W, grouped kv heads).  With P the softmax, dO = ∂L/∂o and
+ * D_i = dO_i · o_i:  dv_j = Σ_i P_ij dO_i,  dS_ij = P_ij (dO_i · v_j - D_i),
+ * dq_i = scale Σ_j dS_ij k_j,  dk_j = scale Σ_i dS_ij q_i, the kv gradients
+ * summed over the query heads that read the kv head.  P is recomputed from
+ * q, k and the forward's log-sum-exp (samba_swa_args.lse).
+ *
+ *   q, dO, o   [B, L, Hq, d]   bf16  (o and lse: the forward's outputs)
+ *   k, v       [B, L, Hkv, d]  bf16
+ *   lse        [B, Hq, L]      fp32, natural log
+ *   dq         [B, L, Hq, d]   bf16, written
+ *   dk, dv     [B, L, Hkv, d]  bf16, written
+ * Shapes, scale and limits as samba_swa_fwd.  The workspace is caller-owned
+ * device memory of samba_swa_bwd_workspace_size() bytes, 16-byte aligned
+ * (per row: the base-2 log-sum-exp and D).  Three kernels run on the stream:
+ * the per-row terms, then dk/dv (one CTA per 128-key tile), then dq.
+ * Errors: as samba_swa_fwd, plus SAMBA_ERR_INVALID_ARG for a missing o,
+ * lse, dO, dq, dk or dv or a misaligned pointer, SAMBA_ERR_WORKSPACE for a
+ * missing or short workspace.
+ */
+typedef struct samba_swa_bwd_args {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const float* lse;
+  const void* dO;
+  void* dq;
+  void* dk;
+  void* dv;
+  void* workspace;
+  size_t workspace_bytes;
+  int64_t batch, seqlen, window;
+  int32_t heads_q, heads_kv, head_dim;
+  float scale;                 /* 0: 1/sqrt(d)                                 */
+} samba_swa_bwd_args;
+
+size_t samba_swa_bwd_workspace_size(int64_t batch, int64_t seqlen, int32_t heads_q);
+
+int samba_swa_bwd(const samba_swa_bwd_args* args, samba_stream_t stream);
+
 /* ------------------------------------------------------ sequence segments
  * A sequence split into consecutive segments (for example one per GPU) can be
  * scanned segment by segment with exactly the result of one pass, because the

@@ -246,3 +246,29 @@ def test_scan_bwd_rejects_bad_arguments_on_host(lib):
     assert call(dstate=12) == L.SAMBA_ERR_UNSUPPORTED
     assert call(workspace=None) == L.SAMBA_ERR_WORKSPACE
     assert call(workspace_bytes=need - 1) == L.SAMBA_ERR_WORKSPACE
+
+
+def test_swa_bwd_rejects_bad_arguments_on_host(lib):
+    f = 0x80000
+    need = lib.samba_swa_bwd_workspace_size(2, 100, 8)
+    assert need == 2 * 128 * 8 * 2 * 4          # per row: base-2 lse and D, rows padded to 128
+    assert lib.samba_swa_bwd_workspace_size(2**40, 2**40, 2**20) == 2**64 - 1
+
+    def call(**over):
+        a = L.SwaBwdArgs()
+        for key in ("q", "k", "v", "o", "lse", "dO", "dq", "dk", "dv", "workspace"):
+            setattr(a, key, f)
+        a.workspace_bytes = need
+        a.batch, a.seqlen, a.window, a.heads_q, a.heads_kv, a.head_dim = 2, 100, 16, 8, 2, 64
+        for key, val in over.items():
+            setattr(a, key, val)
+        return lib.samba_swa_bwd(ctypes.byref(a), None)
+
+    assert lib.samba_swa_bwd(None, None) == L.SAMBA_ERR_INVALID_ARG
+    assert call(lse=None) == L.SAMBA_ERR_INVALID_ARG
+    assert call(dO=None) == L.SAMBA_ERR_INVALID_ARG
+    assert call(dk=f + 8) == L.SAMBA_ERR_INVALID_ARG
+    assert call(head_dim=48) == L.SAMBA_ERR_UNSUPPORTED
+    assert call(heads_kv=3) == L.SAMBA_ERR_INVALID_ARG
+    assert call(workspace=None) == L.SAMBA_ERR_WORKSPACE
+    assert call(workspace_bytes=need - 4) == L.SAMBA_ERR_WORKSPACE
