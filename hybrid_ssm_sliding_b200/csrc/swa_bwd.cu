@@ -108,7 +108,14 @@ struct BwdCfg {
   static constexpr int TILE_BYTES = 128 * ROW_BYTES;
   static constexpr uint32_t SWZ = HD == 64 ? 2u : (HD == 32 ? 4u : 6u);
   static constexpr uint32_t ATOM = 8 * ROW_BYTES;
-  static constexpr int THREADS = 192;  // 4 compute warps, TMA warp 4, MMA warp 5
+  // NCW compute warps per tensor-memory lane quarter (warp w reads lanes
+  // 32 (w % 4) ..), each taking 128 / NCW of the tile's columns, so that
+  // every sub-partition runs NCW independent exp chains.
+  static constexpr int NCW = 4;
+  static constexpr int CWARPS = 4 * NCW;
+  static constexpr int CW = 128 / NCW;             // columns per compute warp
+  static constexpr int WARP_TMA = CWARPS, WARP_MMA = CWARPS + 1;
+  static constexpr int THREADS = 32 * (CWARPS + 2);
 };
 
 // dK/dV kernel shared memory: K, V; STG stages of (Q, dO, lse2[128], D[128]).
@@ -145,7 +152,7 @@ __device__ __forceinline__ bool visible(int64_t i, int64_t j, int64_t W, int64_t
 
 // ------------------------------------------------------------ dK / dV
 template <int HD, int GROUP, int STG>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
     swa_bwd_kv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_do,
                       const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                       const SwaBwdParams p) {
@@ -172,7 +179,7 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars[BB_KV], 1);
     mbar_init(&bars[BB_S], 1);
-    mbar_init(&bars[BB_P], 4);
+    mbar_init(&bars[BB_P], Cfg::CWARPS);
     mbar_init(&bars[BB_O], 1);
     mbar_init(&bars[BB_DONE], 1);
     for (int s = 0; s < STG; ++s) {
@@ -182,7 +189,7 @@ __global__ void __launch_bounds__(192, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == Cfg::WARP_MMA) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -191,7 +198,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == Cfg::WARP_TMA) {
     // ================================================================ TMA
     if (lane == 0) {
       tma_prefetch_desc(&map_q);
@@ -221,7 +228,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int m = (issued > STG ? issued - STG : 0); m < issued; ++m)
         mbar_wait(&st_full[m % STG], (m / STG) & 1, &never);
     }
-  } else if (warp == 5) {
+  } else if (warp == Cfg::WARP_MMA) {
     // ================================================================ MMA
     constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
     constexpr uint32_t IDESC_G = idesc_bf16_f32(128, HD, 0, 1);
@@ -296,9 +303,10 @@ __global__ void __launch_bounds__(192, 1)
     mbar_wait(&bars[BB_DONE], 0, &never);
   } else {
     // ============================================================ compute
-    const int r = warp * 32 + lane;  // key row of the tile
+    const int quarter = warp & 3, part = warp >> 2;
+    const int r = quarter * 32 + lane;  // key row of the tile
     const int64_t j = k0 + r;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
     };
@@ -319,7 +327,7 @@ __global__ void __launch_bounds__(192, 1)
       // key and its last query still sees the first key
       const bool full = (i0 >= k0 + 127) && (i0 + TOK - 1 - k0 < p.W) && (i0 + TOK - 1 < p.L);
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = part * (Cfg::CW / 32); cc < (part + 1) * (Cfg::CW / 32); ++cc) {
         uint32_t sr[32], dr[32];
         tmem_ld32(tmem + lane_off + Cfg::COL_S + 32 * cc, sr);
         tmem_ld32(tmem + lane_off + Cfg::COL_DP + 32 * cc, dr);
@@ -358,6 +366,7 @@ __global__ void __launch_bounds__(192, 1)
         __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + ((static_cast<int64_t>(b) * p.L + j) * p.Hkv + g) * HD;
 #pragma unroll
         for (int q = 0; q < HD / 16; ++q) {
+          if (q % Cfg::NCW != part) continue;  // the parts of a quarter share the columns
           uint32_t t16[16];
           if (nq > 0) {
             tmem_ld16(tmem + lane_off + col + 16 * q, t16);
@@ -385,7 +394,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == Cfg::WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -393,7 +402,7 @@ __global__ void __launch_bounds__(192, 1)
 
 // ----------------------------------------------------------------- dQ
 template <int HD, int GROUP, int STG>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
     swa_bwd_q_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_do,
                      const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                      const SwaBwdParams p) {
@@ -420,7 +429,7 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars[BB_KV], 1);  // here: Q and dO landed
     mbar_init(&bars[BB_S], 1);
-    mbar_init(&bars[BB_P], 4);
+    mbar_init(&bars[BB_P], Cfg::CWARPS);
     mbar_init(&bars[BB_O], 1);
     mbar_init(&bars[BB_DONE], 1);
     for (int s = 0; s < STG; ++s) {
@@ -430,7 +439,7 @@ __global__ void __launch_bounds__(192, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == Cfg::WARP_MMA) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -439,7 +448,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == Cfg::WARP_TMA) {
     // ================================================================ TMA
     if (lane == 0) {
       tma_prefetch_desc(&map_q);
@@ -465,7 +474,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int t = (issued > STG ? issued - STG : 0); t < issued; ++t)
         mbar_wait(&st_full[t % STG], (t / STG) & 1, &never);
     }
-  } else if (warp == 5) {
+  } else if (warp == Cfg::WARP_MMA) {
     // ================================================================ MMA
     constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
     constexpr uint32_t IDESC_G = idesc_bf16_f32(128, HD, 0, 1);
@@ -528,10 +537,11 @@ __global__ void __launch_bounds__(192, 1)
     mbar_wait(&bars[BB_DONE], 0, &never);
   } else {
     // ============================================================ compute
-    const int r = warp * 32 + lane;  // query row: token r / GROUP, head r % GROUP
+    const int quarter = warp & 3, part = warp >> 2;
+    const int r = quarter * 32 + lane;  // query row: token r / GROUP, head r % GROUP
     const int tok = r / GROUP, hh = r % GROUP;
     const int64_t irow = i0 + tok;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int64_t rix = ((static_cast<int64_t>(b) * p.Hkv + g) * p.Lp + i0) * GROUP + r;
     const float lse2 = p.lse2s[rix], Dr = p.Ds[rix];
     auto wait = [&](uint64_t* bar, uint32_t parity) {
@@ -546,7 +556,7 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const bool full = (kk0 + 127 <= i0) && (i0 + TOK - 1 - kk0 < p.W) && (kk0 >= 0) && (i0 + TOK - 1 < p.L);
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = part * (Cfg::CW / 32); cc < (part + 1) * (Cfg::CW / 32); ++cc) {
         uint32_t sr[32], dr[32];
         tmem_ld32(tmem + lane_off + Cfg::COL_S + 32 * cc, sr);
         tmem_ld32(tmem + lane_off + Cfg::COL_DP + 32 * cc, dr);
@@ -579,6 +589,7 @@ __global__ void __launch_bounds__(192, 1)
       __nv_bfloat16* dst = p.dq + ((static_cast<int64_t>(b) * p.L + irow) * p.Hq + g * GROUP + hh) * HD;
 #pragma unroll
       for (int q = 0; q < HD / 16; ++q) {
+        if (q % Cfg::NCW != part) continue;  // the parts of a quarter share the columns
         uint32_t t16[16];
         tmem_ld16(tmem + lane_off + Cfg::COL_DQ + 16 * q, t16);
         tc_wait_ld();
@@ -600,7 +611,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == Cfg::WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -675,10 +686,10 @@ int launch_swa_bwd_t(const samba_swa_bwd_args& a, cudaStream_t stream) {
     int rc = check_launch("samba_swa_bwd (prep)");
     if (rc) return rc;
   }
-  kkv<<<(unsigned)nkv, 192, smem_kv, stream>>>(mq, mdo, mk, mv, p);
+  kkv<<<(unsigned)nkv, KC::THREADS, smem_kv, stream>>>(mq, mdo, mk, mv, p);
   int rc = check_launch("samba_swa_bwd (dk, dv)");
   if (rc) return rc;
-  kq<<<(unsigned)nq, 192, smem_q, stream>>>(mq, mdo, mk, mv, p);
+  kq<<<(unsigned)nq, QC::THREADS, smem_q, stream>>>(mq, mdo, mk, mv, p);
   return check_launch("samba_swa_bwd (dq)");
 }
 
