@@ -114,6 +114,7 @@ struct BwdCfg {
   static constexpr int NCW = 4;
   static constexpr int CWARPS = 4 * NCW;
   static constexpr int CW = 128 / NCW;             // columns per compute warp
+  static_assert(CW == 32, "one 32-column chunk per compute warp");
   static constexpr int WARP_TMA = CWARPS, WARP_MMA = CWARPS + 1;
   static constexpr int THREADS = 32 * (CWARPS + 2);
 };
@@ -143,7 +144,10 @@ struct QCfg : BwdCfg<HD, GROUP> {
 };
 
 // Barrier block (indices into uint64 slots).
-enum : int { BB_KV = 0, BB_S, BB_P, BB_O, BB_DONE, BB_STAGE0 };
+// BB_S: S/dP of a tile in tensor memory; BB_SF: every compute warp has read
+// them (the columns may take the next tile's); BB_P: P/dS (dS) written;
+// BB_O: the gradient MMAs that read them have completed.
+enum : int { BB_KV = 0, BB_S, BB_SF, BB_P, BB_O, BB_DONE, BB_STAGE0 };
 
 // Band test for a (key j, query i) pair: 0 <= i - j < W and i < L.
 __device__ __forceinline__ bool visible(int64_t i, int64_t j, int64_t W, int64_t L) {
@@ -180,6 +184,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
     mbar_init(&bars[BB_KV], 1);
     mbar_init(&bars[BB_S], 1);
     mbar_init(&bars[BB_P], Cfg::CWARPS);
+    mbar_init(&bars[BB_SF], Cfg::CWARPS);
     mbar_init(&bars[BB_O], 1);
     mbar_init(&bars[BB_DONE], 1);
     for (int s = 0; s < STG; ++s) {
@@ -274,29 +279,30 @@ __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
                   (first && k == 0) ? 0u : 1u);
       }
     };
-    bool ok = wait(&bars[BB_KV], 0);
+    // S/dP of tile m+1 go in as soon as the compute warps have read those of
+    // tile m, so Sᵀ and dPᵀ run under tile m's exps; the gradient MMAs of
+    // tile m follow once its P and dS are written.
+    bool ok = wait(&bars[BB_KV], 0) && wait(&st_full[0], 0);
+    if (ok) {
+      tc_fence_after();
+      issue_sdp(0);
+      tc_commit_w(&bars[BB_S]);
+    }
     for (int m = 0; m < nq && ok; ++m) {
-      const int s = m % STG;
-      ok = wait(&st_full[s], (m / STG) & 1);
-      if (ok && m > 0) ok = wait(&bars[BB_P], (m - 1) & 1);  // S/dP of tile m-1 read, P/dS of it written
+      if (m + 1 < nq) {
+        const int sn = (m + 1) % STG;
+        ok = wait(&st_full[sn], ((m + 1) / STG) & 1) && wait(&bars[BB_SF], m & 1);
+        if (!ok) break;
+        tc_fence_after();
+        issue_sdp(sn);
+        tc_commit_w(&bars[BB_S]);
+      }
+      ok = wait(&bars[BB_P], m & 1);
       if (!ok) break;
       tc_fence_after();
-      issue_sdp(s);
-      tc_commit_w(&bars[BB_S]);
-      if (m > 0) {
-        issue_grad((m - 1) % STG, m == 1);
-        tc_commit_w(&bars[BB_O]);
-        tc_commit_w(&st_empty[(m - 1) % STG]);
-      }
-    }
-    if (ok && nq > 0) {
-      ok = wait(&bars[BB_P], (nq - 1) & 1);
-      if (ok) {
-        tc_fence_after();
-        issue_grad((nq - 1) % STG, nq == 1);
-        tc_commit_w(&bars[BB_O]);
-        tc_commit_w(&st_empty[(nq - 1) % STG]);
-      }
+      issue_grad(m % STG, m == 0);
+      tc_commit_w(&bars[BB_O]);
+      tc_commit_w(&st_empty[m % STG]);
     }
     tc_commit_w(&bars[BB_DONE]);
     volatile int never = 0;
@@ -317,8 +323,6 @@ __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
       ok = wait(&bars[BB_S], m & 1);
       // the stage's lse2 / D columns (written by the copy engine) are read below
       if (ok) ok = wait(&st_full[s], (m / STG) & 1);
-      // P/dS of tile m-1 are still read by its gradient MMAs until BB_O
-      if (ok && m > 0) ok = wait(&bars[BB_O], (m - 1) & 1);
       if (!ok) break;
       tc_fence_after();
       const float* lse2 = reinterpret_cast<const float*>(smem + Cfg::STAGE_OFF + s * Cfg::STAGE + 2 * Cfg::TILE_BYTES);
@@ -326,12 +330,15 @@ __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
       // the whole tile is inside the band when its first query sees the last
       // key and its last query still sees the first key
       const bool full = (i0 >= k0 + 127) && (i0 + TOK - 1 - k0 < p.W) && (i0 + TOK - 1 < p.L);
-#pragma unroll 1
-      for (int cc = part * (Cfg::CW / 32); cc < (part + 1) * (Cfg::CW / 32); ++cc) {
+      {
+        const int cc = part;  // this warp's 32 columns
         uint32_t sr[32], dr[32];
         tmem_ld32(tmem + lane_off + Cfg::COL_S + 32 * cc, sr);
         tmem_ld32(tmem + lane_off + Cfg::COL_DP + 32 * cc, dr);
         tc_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[BB_SF]);  // the next tile's Sᵀ, dPᵀ may take these columns
         uint32_t pk[16], dk[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
@@ -346,6 +353,12 @@ __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
           }
           pk[q] = pack_bf16x2(pv[0], pv[1]);
           dk[q] = pack_bf16x2(dsv[0], dsv[1]);
+        }
+        // P/dS of tile m-1 are read by its gradient MMAs until BB_O
+        if (m > 0) {
+          ok = wait(&bars[BB_O], (m - 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
         }
         tmem_st16(tmem + lane_off + Cfg::COL_P + 16 * cc, pk);
         tmem_st16(tmem + lane_off + Cfg::COL_DS + 16 * cc, dk);
@@ -430,6 +443,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
     mbar_init(&bars[BB_KV], 1);  // here: Q and dO landed
     mbar_init(&bars[BB_S], 1);
     mbar_init(&bars[BB_P], Cfg::CWARPS);
+    mbar_init(&bars[BB_SF], Cfg::CWARPS);
     mbar_init(&bars[BB_O], 1);
     mbar_init(&bars[BB_DONE], 1);
     for (int s = 0; s < STG; ++s) {
@@ -508,29 +522,29 @@ __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
         umma_ts_w(tmem + Cfg::COL_DQ, tmem + Cfg::COL_DS + 8 * k, d64(lk + k * Cfg::ROW_BYTES, hi_mn), IDESC_G,
                   (first && k == 0) ? 0u : 1u);
     };
-    bool ok = wait(&bars[BB_KV], 0);
+    // S/dP of key tile t+1 go in as soon as the compute warps have read
+    // those of tile t; dQ of tile t follows once its dS is written.
+    bool ok = wait(&bars[BB_KV], 0) && wait(&st_full[0], 0);
+    if (ok) {
+      tc_fence_after();
+      issue_sdp(0);
+      tc_commit_w(&bars[BB_S]);
+    }
     for (int t = 0; t < nt && ok; ++t) {
-      const int s = t % STG;
-      ok = wait(&st_full[s], (t / STG) & 1);
-      if (ok && t > 0) ok = wait(&bars[BB_P], (t - 1) & 1);
+      if (t + 1 < nt) {
+        const int sn = (t + 1) % STG;
+        ok = wait(&st_full[sn], ((t + 1) / STG) & 1) && wait(&bars[BB_SF], t & 1);
+        if (!ok) break;
+        tc_fence_after();
+        issue_sdp(sn);
+        tc_commit_w(&bars[BB_S]);
+      }
+      ok = wait(&bars[BB_P], t & 1);
       if (!ok) break;
       tc_fence_after();
-      issue_sdp(s);
-      tc_commit_w(&bars[BB_S]);
-      if (t > 0) {
-        issue_dq((t - 1) % STG, t == 1);
-        tc_commit_w(&bars[BB_O]);
-        tc_commit_w(&st_empty[(t - 1) % STG]);
-      }
-    }
-    if (ok && nt > 0) {
-      ok = wait(&bars[BB_P], (nt - 1) & 1);
-      if (ok) {
-        tc_fence_after();
-        issue_dq((nt - 1) % STG, nt == 1);
-        tc_commit_w(&bars[BB_O]);
-        tc_commit_w(&st_empty[(nt - 1) % STG]);
-      }
+      issue_dq(t % STG, t == 0);
+      tc_commit_w(&bars[BB_O]);
+      tc_commit_w(&st_empty[t % STG]);
     }
     tc_commit_w(&bars[BB_DONE]);
     volatile int never = 0;
@@ -551,16 +565,18 @@ __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
     for (int t = 0; t < nt && ok; ++t) {
       const int64_t kk0 = top - 128 * (t + 1);
       ok = wait(&bars[BB_S], t & 1);
-      if (ok && t > 0) ok = wait(&bars[BB_O], (t - 1) & 1);
       if (!ok) break;
       tc_fence_after();
       const bool full = (kk0 + 127 <= i0) && (i0 + TOK - 1 - kk0 < p.W) && (kk0 >= 0) && (i0 + TOK - 1 < p.L);
-#pragma unroll 1
-      for (int cc = part * (Cfg::CW / 32); cc < (part + 1) * (Cfg::CW / 32); ++cc) {
+      {
+        const int cc = part;  // this warp's 32 columns
         uint32_t sr[32], dr[32];
         tmem_ld32(tmem + lane_off + Cfg::COL_S + 32 * cc, sr);
         tmem_ld32(tmem + lane_off + Cfg::COL_DP + 32 * cc, dr);
         tc_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[BB_SF]);  // the next key tile's S, dP may take these columns
         uint32_t dk[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
@@ -573,6 +589,12 @@ __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
             dsv[e] = pr * (__uint_as_float(dr[2 * q + e]) - Dr);
           }
           dk[q] = pack_bf16x2(dsv[0], dsv[1]);
+        }
+        // dS of key tile t-1 is read by its dQ MMAs until BB_O
+        if (t > 0) {
+          ok = wait(&bars[BB_O], (t - 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
         }
         tmem_st16(tmem + lane_off + Cfg::COL_DS + 16 * cc, dk);
       }
