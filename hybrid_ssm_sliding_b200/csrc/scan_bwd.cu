@@ -39,7 +39,9 @@ namespace {
 
 constexpr int kCh = 32;      // channels per CTA (one per lane)
 constexpr int kTc = 16;      // tokens per chunk
-constexpr int kThreads = 128;
+// Warps per CTA: one per group of N / warps states (8 warps of 2 states at
+// N = 16), so that every SM holds three CTAs of 8 warps.
+constexpr int nwarps(int N) { return N >= 8 ? 8 : 4; }
 constexpr int kHalo = 3;     // earlier inputs the conv needs (K <= 4)
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -154,9 +156,9 @@ struct ScanBwdSmem {
   float Bv[kTc][N];
   float Cv[kTc][N];
   float H[kTc][N][kCh];        // h_t of the chunk
-  float part[2][4][kTc][kCh];  // per-warp partials: [0] y (forward) / dΔ (reverse), [1] du
+  float part[2][kTc][kCh];     // sums over the warps' states: [0] C·h (forward) / dΔ (reverse), [1] du
   float dc[kTc + kHalo][kCh];  // conv-output gradient, rows kTc.. = first rows of the later chunk
-  float red[3 + 4][4][kCh];    // per-channel sums of the 4 token lanes (dD, dconv_b, dconv_w[K])
+  float red[3 + 4][nwarps(N)][kCh];  // per-channel sums of the token lanes (dD, dconv_b, dconv_w[K])
   float dbc[2][kTc][N];        // this block's dB, dC of the chunk (summed over its channels)
 };
 
@@ -164,15 +166,20 @@ struct ScanBwdSmem {
 // registers so that their latency hides behind the work on the chunk before.
 template <int N>
 struct ChunkRegs {
+  static constexpr int NW = nwarps(N), kThreads = 32 * NW;
+  static constexpr int XR = (kTc + kHalo + NW - 1) / NW, TR = kTc / NW;
   static constexpr int kBC = (kTc * N + kThreads - 1) / kThreads;
-  float x[5];        // rows pt, pt+4, ... of [3 earlier tokens ; the chunk]
-  float delta[4], z[4], dy[4];
+  float x[XR];       // rows pt, pt+NW, ... of [3 earlier tokens ; the chunk]
+  float delta[TR], z[TR], dy[TR];
   float Bv[kBC], Cv[kBC];
 };
 
 template <int N, typename XT, typename YT>
-__global__ void __launch_bounds__(kThreads) scan_bwd_kernel(const ScanBwdParams p) {
-  constexpr int SPL = N / 4;   // states per lane
+__global__ void __launch_bounds__(32 * nwarps(N), 3) scan_bwd_kernel(const ScanBwdParams p) {
+  constexpr int NW = nwarps(N);
+  constexpr int kThreads = 32 * NW;
+  constexpr int SPL = N / NW;  // states per lane
+  using CR = ChunkRegs<N>;
   constexpr int G4 = 4;        // tokens per reduction group
   constexpr int NV = G4 * 2 * SPL;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -220,8 +227,8 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(const ScanBwdParams 
     const int64_t t0 = static_cast<int64_t>(c) * kTc;
     const int nv = chunk_len(c);
 #pragma unroll
-    for (int i = 0; i < 5; ++i) {
-      const int r = pt + 4 * i;
+    for (int i = 0; i < CR::XR; ++i) {
+      const int r = pt + NW * i;
       const int64_t tau = t0 - kHalo + r;
       float v = 0.f;
       if (r < kTc + kHalo && ch_ok) {
@@ -235,8 +242,8 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(const ScanBwdParams 
       R.x[i] = v;
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int t = pt + 4 * i;
+    for (int i = 0; i < CR::TR; ++i) {
+      const int t = pt + NW * i;
       const bool ok = ch_ok && t < nv;
       const int64_t e = (b * L + t0 + t) * D + ch_p;
       R.delta[i] = ok ? p.delta[e] : 0.f;
@@ -257,8 +264,8 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(const ScanBwdParams 
   auto stage = [&](int c, bool full, const ChunkRegs<N>& R) {
     const int nv = chunk_len(c);
 #pragma unroll
-    for (int i = 0; i < 5; ++i) {
-      const int r = pt + 4 * i;
+    for (int i = 0; i < CR::XR; ++i) {
+      const int r = pt + NW * i;
       if (r < kTc + kHalo) S.x[r][pc] = R.x[i];
     }
 #pragma unroll
@@ -271,9 +278,11 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(const ScanBwdParams 
     }
     __syncthreads();  // the conv below reads rows that other warps stored
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int t = pt + 4 * i;
+    for (int i = 0; i < CR::TR; ++i) {
+      const int t = pt + NW * i;
       const bool ok = ch_ok && t < nv;
+      S.part[0][t][pc] = 0.f;  // the sums the warps add into start from zero
+      S.part[1][t][pc] = 0.f;
       float u = 0.f, pre = 0.f, dt = 0.f, sg = 0.f;
       if (ok) {
         if (fuse) {
@@ -326,7 +335,10 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(const ScanBwdParams 
 #pragma unroll
       for (int j = 0; j < SPL; ++j) p.ckpt[((b * p.nchunks + c) * N + warp * SPL + j) * D + ch_l] = h[j];
     }
-    for (int t = 0; t < nv; ++t) {
+    // All kTc tokens, unrolled: past nv the staged Δ and u are zero, so
+    // those steps leave h unchanged (exp(0) = 1, no input).
+#pragma unroll
+    for (int t = 0; t < kTc; ++t) {
       const float dt = S.dt[t][lane], du = dt * S.u[t][lane];
 #pragma unroll
       for (int j = 0; j < SPL; ++j) h[j] = fmaf(ex2_fast(dt * Al[j]), h[j], du * S.Bv[t][warp * SPL + j]);
@@ -339,21 +351,32 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(const ScanBwdParams 
 #pragma unroll
   for (int j = 0; j < SPL; ++j) g[j] = dAacc[j] = 0.f;
   float accD = 0.f, accB = 0.f, accW[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int r = pt; r < kHalo; r += 4) S.dc[kTc + r][pc] = 0.f;  // nothing after the last token
+  for (int r = pt; r < kHalo; r += NW) S.dc[kTc + r][pc] = 0.f;  // nothing after the last token
+  // the checkpoint a chunk starts from is fetched with its inputs, a chunk ahead
+  auto fetch_ckpt = [&](int c, float (&dst)[SPL]) {
+#pragma unroll
+    for (int j = 0; j < SPL; ++j) dst[j] = lane_ok ? p.ckpt[((b * p.nchunks + c) * N + warp * SPL + j) * D + ch_l] : 0.f;
+  };
+  float hs_next[SPL];
   fetch(p.nchunks - 1, true, R);
+  fetch_ckpt(p.nchunks - 1, hs_next);
   for (int c = p.nchunks - 1; c >= 0; --c) {
     const int64_t t0 = static_cast<int64_t>(c) * kTc;
     const int nv = chunk_len(c);
-    stage(c, true, R);
-    if (c > 0) fetch(c - 1, true, R);
-    // (a) states of the chunk, forward from its checkpoint; partial readout
     float hs[SPL];
 #pragma unroll
-    for (int j = 0; j < SPL; ++j) {
-      hs[j] = lane_ok ? p.ckpt[((b * p.nchunks + c) * N + warp * SPL + j) * D + ch_l] : 0.f;
-      h[j] = hs[j];
+    for (int j = 0; j < SPL; ++j) hs[j] = hs_next[j];
+    stage(c, true, R);
+    if (c > 0) {
+      fetch(c - 1, true, R);
+      fetch_ckpt(c - 1, hs_next);
     }
-    for (int t = 0; t < nv; ++t) {
+    // (a) states of the chunk, forward from its checkpoint; partial readout.
+    // All kTc tokens, unrolled (past nv: no change, C = 0).
+#pragma unroll
+    for (int j = 0; j < SPL; ++j) h[j] = hs[j];
+#pragma unroll
+    for (int t = 0; t < kTc; ++t) {
       const float dt = S.dt[t][lane], du = dt * S.u[t][lane];
       float yp = 0.f;
 #pragma unroll
@@ -363,22 +386,24 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(const ScanBwdParams 
         S.H[t][n][lane] = h[j];
         yp = fmaf(S.Cv[t][n], h[j], yp);
       }
-      S.part[0][warp][t][lane] = yp;
+      atomicAdd(&S.part[0][t][lane], yp);
     }
     __syncthreads();
-    // (b) the gate's gradient dz = dy · (C·h + D u) · silu'(z)
-    if (z) {
-      for (int t = pt; t < nv; t += 4) {
-        const float ypre = S.part[0][0][t][pc] + S.part[0][1][t][pc] + S.part[0][2][t][pc] + S.part[0][3][t][pc] +
-                           dsk * S.u[t][pc];
-        if (ch_ok) stv<XT>(p.dz, (b * L + t0 + t) * D + ch_p, ypre * S.dydsz[t][pc]);
+    // (b) the gate's gradient dz = dy · (C·h + D u) · silu'(z); the sums are
+    // then cleared for the reverse walk's dΔ
+    for (int t = pt; t < kTc; t += NW) {
+      if (z && t < nv && ch_ok) {
+        const float ypre = S.part[0][t][pc] + dsk * S.u[t][pc];
+        stv<XT>(p.dz, (b * L + t0 + t) * D + ch_p, ypre * S.dydsz[t][pc]);
       }
+      S.part[0][t][pc] = 0.f;
     }
     __syncthreads();
     // (c) the adjoint recurrence, last token first, in groups of G4 tokens
     // whose 2·SPL channel sums each are reduced together.  Tokens past nv
     // (a partial last chunk) contribute nothing and leave g unchanged.
-    for (int tg = (nv - 1) / G4; tg >= 0; --tg) {
+#pragma unroll
+    for (int tg = kTc / G4 - 1; tg >= 0; --tg) {
       float q[NV];
 #pragma unroll
       for (int i = 0; i < G4; ++i) {
@@ -404,8 +429,8 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(const ScanBwdParams 
           g[j] *= decay;
         }
         if (valid) {
-          S.part[0][warp][t][lane] = fmaf(uv, gB, ddt);
-          S.part[1][warp][t][lane] = dt * gB;
+          atomicAdd(&S.part[0][t][lane], fmaf(uv, gB, ddt));
+          atomicAdd(&S.part[1][t][lane], dt * gB);
         }
       }
       int which = 0;
@@ -427,12 +452,11 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(const ScanBwdParams 
       }
     }
     // (d) du, dΔ, the conv's SiLU; accumulate dD and the conv parameter sums
-    for (int t = pt; t < kTc; t += 4) {
+    for (int t = pt; t < kTc; t += NW) {
       float dcv = 0.f;
       if (t < nv) {
-        const float du = dsk * S.gy[t][pc] + S.part[1][0][t][pc] + S.part[1][1][t][pc] + S.part[1][2][t][pc] +
-                         S.part[1][3][t][pc];
-        const float ddt = S.part[0][0][t][pc] + S.part[0][1][t][pc] + S.part[0][2][t][pc] + S.part[0][3][t][pc];
+        const float du = dsk * S.gy[t][pc] + S.part[1][t][pc];
+        const float ddt = S.part[0][t][pc];
         const int64_t e = (b * L + t0 + t) * D + ch_p;
         if (ch_ok) p.ddelta[e] = ddt * S.sg[t][pc];
         accD = fmaf(S.gy[t][pc], S.u[t][pc], accD);
@@ -457,7 +481,7 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(const ScanBwdParams 
     __syncthreads();
     // (e) the conv's input gradient: dx_t = Σ_k w_k dc_{t + K-1-k}
     if (fuse) {
-      for (int t = pt; t < nv; t += 4) {
+      for (int t = pt; t < nv; t += NW) {
         float v = 0.f;
         #pragma unroll
         for (int k = 0; k < 4; ++k)
@@ -467,7 +491,7 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(const ScanBwdParams 
     }
     __syncthreads();
     // the first rows of this chunk become the halo of the chunk before it
-    for (int r = pt; r < kHalo; r += 4) S.dc[kTc + r][pc] = S.dc[r][pc];
+    for (int r = pt; r < kHalo; r += NW) S.dc[kTc + r][pc] = S.dc[r][pc];
     __syncthreads();
   }
 
@@ -496,7 +520,12 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(const ScanBwdParams 
   for (int k = 0; k < 4; ++k) S.red[2 + k][pt][pc] = accW[k];
   __syncthreads();
   if (pt == 0 && ch_ok) {
-    auto tot = [&](int i) { return S.red[i][0][pc] + S.red[i][1][pc] + S.red[i][2][pc] + S.red[i][3][pc]; };
+    auto tot = [&](int i) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) acc += S.red[i][w][pc];
+      return acc;
+    };
     if (p.dD) atomicAdd(p.dD + ch_p, tot(0));
     if (fuse) {
       if (p.dconv_b) atomicAdd(p.dconv_b + ch_p, tot(1));
@@ -538,7 +567,7 @@ int scan_bwd_go(const ScanBwdParams& p, int64_t B, cudaStream_t s) {
   });
   if (rc != SAMBA_OK) return rc;
   const dim3 grid((unsigned)((p.D + kCh - 1) / kCh), (unsigned)B);
-  kern<<<grid, kThreads, smem, s>>>(p);
+  kern<<<grid, ChunkRegs<N>::kThreads, smem, s>>>(p);
   const int rc2 = check_launch("samba_selective_scan_bwd");
   if (rc2 != SAMBA_OK) return rc2;
   const int64_t bln4 = B * p.L * N / 4;
