@@ -50,6 +50,7 @@ class Workload:
     decode_steps: int = 0
     d_model: int = 0      # layer workloads: model width around the mixers (0: mixers only)
     dt_rank: int = 0      # layer workloads: rank of the step-size projection
+    train: bool = False   # forward + backward of both mixers
     notes: str = field(default="", compare=False)
 
     @property
@@ -75,7 +76,9 @@ WORKLOADS = {
                             dt_rank=128),
     # forward + backward of both mixers at the pages' 4K training context,
     # 8 sequences per step
-    "train_4k": Workload("train_4k", 8, 4096, 4096, 16, 4, 32, 4, 64, 2048, 8),
+    "train_4k": Workload("train_4k", 8, 4096, 4096, 16, 4, 32, 4, 64, 2048, 8, train=True),
+    # two sequences of the same shape: a small case for profiler captures
+    "train_4k_b2": Workload("train_4k_b2", 2, 4096, 4096, 16, 4, 32, 4, 64, 2048, 9, train=True),
 }
 
 
