@@ -12,12 +12,16 @@
 // the mixers read: for instance x and z of the Mamba input projection in one
 // pass, or Δ-low-rank, B and C of the selective-parameter projection.
 //
-// Design: one CTA per 128 x BN tile of C (BN = 256 or 128), K in steps of 64
-// (128-byte rows, 128-byte swizzle).  Warp 4 streams A and B tiles into a
-// STG-deep shared-memory ring with TMA; warp 5 issues the tcgen05.mma
-// (kind::f16, M = 128, N = BN, K = 16 per instruction) into BN columns of
-// tensor memory; warps 0-3 (one TMEM lane quarter each, thread = row) read
-// the accumulator back and write the outputs.  Every wait is bounded.
+// Design: persistent CTAs, one per SM, walking the 128 x BN tiles of C
+// (BN = 256 or 128) with the N tile fastest; K in steps of 64 (128-byte
+// rows, 128-byte swizzle).  Warp 4 streams A and B tiles into a STG-deep
+// shared-memory ring with TMA, continuously across tiles; warp 5 issues the
+// tcgen05.mma (kind::f16, M = 128, N = BN, K = 16 per instruction) into one of
+// two BN-column accumulators in tensor memory, alternating per tile; warps
+// 0-3 (one TMEM lane quarter each, thread = row) read a finished accumulator
+// back and write the outputs while the next tile accumulates into the other,
+// so the epilogue runs under the next tile's main loop.  Every wait is
+// bounded.
 #include "common.cuh"
 #include "host.hpp"
 
@@ -42,8 +46,8 @@ struct GemmCfg {
   static constexpr int BM = 128, BK = 64;
   static constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE = A_BYTES + B_BYTES;
   static constexpr int BAR_OFF = STG * STAGE;
-  static constexpr int SMEM = BAR_OFF + 128 + 1024;  // barriers + alignment slack
-  static constexpr uint32_t TMEM_COLS = BN;
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;  // barriers + alignment slack
+  static constexpr uint32_t TMEM_COLS = 2 * BN;      // two accumulators
   static constexpr int THREADS = 192;
 };
 
@@ -56,17 +60,25 @@ __global__ void __launch_bounds__(192, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::BAR_OFF);
   uint64_t* empty = full + STG;
-  uint64_t* done = empty + STG;
+  uint64_t* acc_full = empty + STG;   // [2] an accumulator holds a finished tile
+  uint64_t* acc_empty = acc_full + 2; // [2] the epilogue has read it (4 warps)
+  uint64_t* done = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  static_assert((2 * STG + 5) * 8 + 8 <= 256, "barrier block");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * BN, m0 = static_cast<int64_t>(blockIdx.y) * Cfg::BM;
   const int ktiles = static_cast<int>((p.K + Cfg::BK - 1) / Cfg::BK);
+  const int64_t n_tiles_n = (p.N + BN - 1) / BN;
+  const int64_t n_tiles = n_tiles_n * ((p.M + Cfg::BM - 1) / Cfg::BM);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STG; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -86,19 +98,22 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       tma_prefetch_desc(&map_a);
       tma_prefetch_desc(&map_b);
-      int issued = 0;
-      for (int i = 0; i < ktiles; ++i) {
-        const int s = i % STG;
-        if (i >= STG && !mbar_wait(&empty[s], ((i / STG) - 1) & 1, abort_flag)) break;
-        unsigned char* st = smem + s * Cfg::STAGE;
-        mbar_arrive_expect_tx(&full[s], Cfg::STAGE);
-        tma_load_2d(st, &map_a, &full[s], i * Cfg::BK, static_cast<int>(m0));
-        tma_load_2d(st + Cfg::A_BYTES, &map_b, &full[s], i * Cfg::BK, static_cast<int>(n0));
-        issued = i + 1;
+      uint32_t it = 0;  // k-steps issued so far, over all tiles of this CTA
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+        const int64_t n0 = (tile % n_tiles_n) * BN, m0 = (tile / n_tiles_n) * Cfg::BM;
+        for (int i = 0; i < ktiles; ++i, ++it) {
+          const int s = it % STG;
+          if (it >= STG && !mbar_wait(&empty[s], ((it / STG) - 1) & 1, abort_flag)) { ok = false; break; }
+          unsigned char* st = smem + s * Cfg::STAGE;
+          mbar_arrive_expect_tx(&full[s], Cfg::STAGE);
+          tma_load_2d(st, &map_a, &full[s], i * Cfg::BK, static_cast<int>(m0));
+          tma_load_2d(st + Cfg::A_BYTES, &map_b, &full[s], i * Cfg::BK, static_cast<int>(n0));
+        }
       }
       // copies still in flight complete before the CTA can exit
       volatile int never = 0;
-      for (int i = (issued > STG ? issued - STG : 0); i < issued; ++i) mbar_wait(&full[i % STG], (i / STG) & 1, &never);
+      for (uint32_t i = (it > STG ? it - STG : 0); i < it; ++i) mbar_wait(&full[i % STG], (i / STG) & 1, &never);
     }
   } else if (warp == 5) {
     // ================================================================ MMA
@@ -108,31 +123,52 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t hi = static_cast<uint32_t>(d_a0 >> 32), lo0 = static_cast<uint32_t>(d_a0);
     constexpr uint32_t kStageDesc = Cfg::STAGE >> 4, kBDesc = Cfg::A_BYTES >> 4;
     auto desc64 = [&](uint32_t lo) { return (static_cast<uint64_t>(hi) << 32) | lo; };
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
     bool ok = true;
-    for (int i = 0; i < ktiles && ok; ++i) {
-      const int s = i % STG;
-      ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (i / STG) & 1, abort_flag));
-      if (!ok) break;
+    uint32_t it = 0, lt = 0;
+    for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++lt) {
+      const uint32_t acc = lt & 1;
+      // the accumulator's previous tile (two tiles back) must have been read out
+      if (lt >= 2 && !(ok = wait(&acc_empty[acc], ((lt >> 1) - 1) & 1))) break;
       tc_fence_after();
-      const uint32_t la = lo0 + s * kStageDesc, lb = la + kBDesc;
+      const uint32_t d_tmem = tmem + acc * BN;
+      for (int i = 0; i < ktiles; ++i, ++it) {
+        const int s = it % STG;
+        ok = wait(&full[s], (it / STG) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t la = lo0 + s * kStageDesc, lb = la + kBDesc;
 #pragma unroll
-      for (int k = 0; k < Cfg::BK / 16; ++k)  // 16 K-elements = 32 bytes = 2 descriptor units
-        umma_ss_w(tmem, desc64(la + 2 * k), desc64(lb + 2 * k), IDESC, (i > 0 || k > 0) ? 1u : 0u);
-      tc_commit_w(&empty[s]);
+        for (int k = 0; k < Cfg::BK / 16; ++k)  // 16 K-elements = 32 bytes = 2 descriptor units
+          umma_ss_w(d_tmem, desc64(la + 2 * k), desc64(lb + 2 * k), IDESC, (i > 0 || k > 0) ? 1u : 0u);
+        tc_commit_w(&empty[s]);
+      }
+      if (!ok) break;
+      tc_commit_w(&acc_full[acc]);  // every MMA of this tile has completed
     }
-    tc_commit_w(done);  // every MMA of this tile has completed
+    tc_commit_w(done);
+    volatile int never = 0;
+    mbar_wait(done, 0, &never);
   } else {
     // ============================================================ epilogue
     const int row_local = warp * 32 + lane;
-    const int64_t row = m0 + row_local;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag));
-    if (ok && ktiles > 0) {
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    uint32_t lt = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++lt) {
+      const int64_t n0 = (tile % n_tiles_n) * BN, m0 = (tile / n_tiles_n) * Cfg::BM;
+      const int64_t row = m0 + row_local;
+      const uint32_t acc = lt & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], (lt >> 1) & 1, abort_flag));
+      if (!ok) break;
       tc_fence_after();
-      const uint32_t t_row = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+      const uint32_t t_row = tmem + lane_off + acc * BN;
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t r[32];
-        tmem_ld32(t_row + c0, r);
+        tmem_ld32(t_row + c0, r);  // warp-collective: every lane, whatever its row
         tc_wait_ld();
         if (row >= p.M) continue;
 #pragma unroll
@@ -186,6 +222,10 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       }
+      // this accumulator may take the tile after next
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
     }
   }
   tc_fence_before();
@@ -233,7 +273,8 @@ static int launch_gemm_t(const samba_gemm_args& a, cudaStream_t stream) {
     p.out[o].col1 = static_cast<int>(a.out[o].col1);
     p.out[o].dtype = a.out[o].dtype;
   }
-  const dim3 grid((unsigned)((a.N + BN - 1) / BN), (unsigned)((a.M + Cfg::BM - 1) / Cfg::BM));
+  const int64_t tiles = ((a.N + BN - 1) / BN) * ((a.M + Cfg::BM - 1) / Cfg::BM);
+  const unsigned grid = (unsigned)std::min<int64_t>(tiles, sm_count());
   kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(ma, mb, p);
   return check_launch("samba_gemm");
 }
