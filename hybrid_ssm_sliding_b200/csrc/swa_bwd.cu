@@ -149,11 +149,6 @@ struct QCfg : BwdCfg<HD, GROUP> {
 // BB_O: the gradient MMAs that read them have completed.
 enum : int { BB_KV = 0, BB_S, BB_SF, BB_P, BB_O, BB_DONE, BB_STAGE0 };
 
-// Band test for a (key j, query i) pair: 0 <= i - j < W and i < L.
-__device__ __forceinline__ bool visible(int64_t i, int64_t j, int64_t W, int64_t L) {
-  return i < L && i >= j && i - j < W;
-}
-
 // ------------------------------------------------------------ dK / dV
 template <int HD, int GROUP, int STG>
 __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
@@ -330,6 +325,23 @@ __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
       // the whole tile is inside the band when its first query sees the last
       // key and its last query still sees the first key
       const bool full = (i0 >= k0 + 127) && (i0 + TOK - 1 - k0 < p.W) && (i0 + TOK - 1 < p.L);
+      // Key j sees the query tokens [j, min(j + W, L)): in this tile the
+      // columns [clo, chi] (token (c / GROUP) + i0); an empty row gets an
+      // interval no column falls in.  One unsigned compare per column.
+      int clo = 0;
+      unsigned cspan = 127u;
+      if (!full) {
+        const int64_t tlo = j > i0 ? j : i0;
+        const int64_t thi_x = (j + p.W < p.L ? j + p.W : p.L);  // exclusive
+        const int64_t thi = (thi_x < i0 + TOK ? thi_x : i0 + TOK) - 1;
+        if (thi < tlo) {
+          clo = 1 << 20;
+          cspan = 0u;
+        } else {
+          clo = static_cast<int>(tlo - i0) * GROUP;
+          cspan = static_cast<unsigned>((static_cast<int>(thi - i0) + 1) * GROUP - 1 - clo);
+        }
+      }
       {
         const int cc = part;  // this warp's 32 columns
         uint32_t sr[32], dr[32];
@@ -347,7 +359,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
           for (int e = 0; e < 2; ++e) {
             const int c = 32 * cc + 2 * q + e;  // query row of the tile: token c / GROUP, head c % GROUP
             float pr = ex2b(fmaf(__uint_as_float(sr[2 * q + e]), p.scale_log2, -lse2[c]));
-            if (!full && !visible(i0 + c / GROUP, j, p.W, p.L)) pr = 0.f;
+            pr = (static_cast<unsigned>(c - clo) <= cspan) ? pr : 0.f;
             pv[e] = pr;
             dsv[e] = pr * (__uint_as_float(dr[2 * q + e]) - Dv[c]);
           }
@@ -568,6 +580,22 @@ __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const bool full = (kk0 + 127 <= i0) && (i0 + TOK - 1 - kk0 < p.W) && (kk0 >= 0) && (i0 + TOK - 1 < p.L);
+      // Row irow sees the keys [max(0, irow - W + 1), irow] (none past L):
+      // the columns [clo, clo + cspan] of this key tile.
+      int clo = 0;
+      unsigned cspan = 127u;
+      if (!full) {
+        const int64_t jlo = irow - p.W + 1 > 0 ? irow - p.W + 1 : 0;
+        const int64_t lo = jlo - kk0 > 0 ? jlo - kk0 : 0;
+        const int64_t hi = irow - kk0 < 127 ? irow - kk0 : 127;
+        if (irow >= p.L || hi < lo) {
+          clo = 1 << 20;
+          cspan = 0u;
+        } else {
+          clo = static_cast<int>(lo);
+          cspan = static_cast<unsigned>(hi - lo);
+        }
+      }
       {
         const int cc = part;  // this warp's 32 columns
         uint32_t sr[32], dr[32];
@@ -585,7 +613,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
           for (int e = 0; e < 2; ++e) {
             const int c = 32 * cc + 2 * q + e;
             float pr = ex2b(fmaf(__uint_as_float(sr[2 * q + e]), p.scale_log2, -lse2));
-            if (!full && !(kk0 + c >= 0 && visible(irow, kk0 + c, p.W, p.L))) pr = 0.f;
+            pr = (static_cast<unsigned>(c - clo) <= cspan) ? pr : 0.f;
             dsv[e] = pr * (__uint_as_float(dr[2 * q + e]) - Dr);
           }
           dk[q] = pack_bf16x2(dsv[0], dsv[1]);
