@@ -50,3 +50,17 @@ def test_mufu_roof_arithmetic():
     assert r["peak"] == pytest.approx(16 * 148 * 1.965e9 / 1e12)
     assert r["frac"] == pytest.approx(2.0 / r["peak"])
     assert r["bound"] == "alu"
+
+
+def test_backward_counts():
+    """The attention backward's five band products and the scan backward's
+    bytes, written out term by term."""
+    wl = dataclasses.replace(WORKLOADS["tiny"], batch=2, seqlen=7, dim=5, dstate=4, heads_q=3, window=4,
+                             head_dim=16, dconv=4)
+    assert bench.swa_bwd_flops(wl) == 5 * 2.0 * 2 * 3 * 7 * 4 * 16
+    assert bench.swa_bwd_flops(wl) == 2.5 * bench.swa_flops(wl)
+    tc = 2 * 7 * 5
+    per_tc = 2 + 2 + 2 + 4 + 2 + 2 + 4          # x, z, dy, delta in; dx, dz, ddelta out
+    per_token = 4 * 4 * 4                       # B, C in; dB, dC out (fp32, N = 4)
+    small = 5 * (4 + 4 + 2) * 4 * 2             # A, conv w/b, D and their gradients
+    assert bench.scan_bwd_bytes(wl) == tc * per_tc + 2 * 7 * per_token + small
