@@ -47,6 +47,9 @@ UNIT = "tokens/s"
 DECODE_METRIC = "Samba mixer decode tokens/s (16 sequences, one token each per step; SWA ring W = 2048)"
 DECODE_GRAPH_STEPS = 32
 DECODE_LAYERS = 4
+SERVE_PAIRS = 4
+SERVE_METRIC = ("Samba layer-stack decode tokens/s (16 sequences after 4096-token prompts, one token each per step "
+                "through 4 Mamba + SWA layer pairs with their projections; SWA ring W = 2048)")
 
 
 def parse():
@@ -384,6 +387,60 @@ def oracle_decode_throughput(wl, pool, scale=1.0, seed=0):
     return 1.0 / per_token, P, sample
 
 
+def _oracle_serve_unit(args):
+    """`reps` decode steps of one sequence through one Mamba + SWA layer pair
+    with the oracle's layer steps, at the workload's widths (random float64
+    weights of the layer shapes, a full ring).  Returns (reps, seconds the
+    steps took)."""
+    dm, D, N, K, R, Hq, Hkv, d, W, reps, seed = args
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    import oracle.samba_oracle as orc
+
+    rng = np.random.default_rng(seed)
+    mw = dict(in_proj=rng.standard_normal((2 * D, dm)) / dm ** 0.5, conv_w=rng.uniform(-0.5, 0.5, (D, K)),
+              conv_b=rng.uniform(-0.5, 0.5, D), x_proj=rng.standard_normal((R + 2 * N, D)) / D ** 0.5,
+              dt_proj=rng.standard_normal((D, R)) / R ** 0.5, dt_bias=rng.uniform(-6.9, -2.3, D),
+              A=-np.tile(np.arange(1, N + 1, dtype=np.float64), (D, 1)), Dskip=rng.standard_normal(D),
+              out_proj=rng.standard_normal((dm, D)) / D ** 0.5)
+    qkv = rng.standard_normal(((Hq + 2 * Hkv) * d, dm)) / dm ** 0.5
+    o_proj = rng.standard_normal((dm, Hq * d)) / (Hq * d) ** 0.5
+    h = rng.standard_normal((1, D, N)) * 0.1
+    cs = rng.standard_normal((1, D, K - 1))
+    kr = rng.standard_normal((1, W, Hkv, d))
+    vr = rng.standard_normal((1, W, Hkv, d))
+    pos = np.full((1,), W + 7, dtype=np.int64)
+    xs = rng.standard_normal((reps, 1, dm))
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        for r in range(reps):
+            x, h, cs = orc.mamba_layer_step(xs[r], h=h, conv_state=cs, **mw)
+            _, kr, vr, pos = orc.swa_layer_step(x, qkv, o_proj, Hq, Hkv, d, kr, vr, pos, W)
+        return reps, time.perf_counter() - t0
+
+
+def oracle_serve_throughput(wl, pool, scale=1.0, seed=0, pairs=None):
+    """Decode tokens/s of the oracle's layer steps on the host cores: one unit
+    per core of `reps` steps of one sequence through one layer pair (the steps
+    timed inside the unit), scaled to the stack's pairs."""
+    P = host_cores()
+    pairs = pairs or SERVE_PAIRS
+    reps = max(2, int(128 * scale))
+    dims = (wl.d_model, wl.dim, wl.dstate, wl.dconv, wl.dt_rank, wl.heads_q, wl.heads_kv, wl.head_dim, wl.window)
+    pool.map(_oracle_serve_unit, [(64, 64, 4, 4, 8, 2, 1, 16, 16, 1, 0)] * P, chunksize=1)   # workers import
+    res = pool.map(_oracle_serve_unit, [dims + (reps, seed * 1000 + i) for i in range(P)], chunksize=1)
+    done, t = sum(r[0] for r in res), sum(r[1] for r in res)
+    # the P units run at the same time, one per core: the pool decodes P
+    # token-pairs in the time one unit takes for one
+    per_token = t / done / P * pairs
+    sample = (f"{P} processes on {cpu_model()}, at the same time: each {reps} decode steps of one sequence through "
+              f"one Mamba + SWA layer pair at d_model {wl.d_model}, d_inner {wl.dim}, {wl.heads_q}/{wl.heads_kv} "
+              f"heads, a full {wl.window}-slot ring ({t / P:.1f} s of steps per process, weight setup untimed); "
+              f"float64 NumPy; scaled to {pairs} pairs and extrapolated to tokens/s")
+    return 1.0 / per_token, P, sample
+
+
 def run_reference(args):
     """The reference arm: the float64 oracle, as it stands, on the host cores.
     Each step is one bounded parallel sample of the workload (a few seconds of
@@ -397,7 +454,8 @@ def run_reference(args):
 
     wl = WORKLOADS[args.workload]
     decode = wl.decode_steps > 0
-    measure = oracle_decode_throughput if decode else oracle_throughput
+    serve = decode and wl.d_model > 0
+    measure = oracle_serve_throughput if serve else (oracle_decode_throughput if decode else oracle_throughput)
     with oracle_pool() as pool:
         for i in range(max(0, args.warmup)):
             measure(wl, pool, scale=0.05, seed=1000 + i)
@@ -410,7 +468,8 @@ def run_reference(args):
     value = statistics.median(vals)
     tokens_per_step = wl.batch if decode else wl.batch * wl.seqlen
     line = {
-        "impl": "reference", "metric": DECODE_METRIC if decode else METRIC, "value": value, "unit": UNIT,
+        "impl": "reference", "metric": SERVE_METRIC if serve else (DECODE_METRIC if decode else METRIC),
+        "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": len(vals), "warmup": args.warmup,
         "ms_per_step": statistics.mean(walls) * 1e3,
         "extrapolated_ms_per_workload_step": tokens_per_step / value * 1e3,
@@ -509,6 +568,390 @@ def run_layers(args, wl, dev, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (random weights of the layer shapes)", "config": cfg, "roofline": roof,
         "cpu_baseline": None, "e2e": None, "clocks": clk, "gpu_launches": 11 * args.steps,
+        "status": ops.get_status(),
+    }
+
+
+# ------------------------------------------------------------ serving GPU leg
+def serve_gemm_shapes(wl):
+    """(name, N, K, output bytes per element; 0 for mixed outputs) of every
+    projection of one layer pair, in the order a decode step runs them."""
+    D, N, R, dm = wl.dim, wl.dstate, wl.dt_rank, wl.d_model
+    nq, nk = wl.heads_q * wl.head_dim, wl.heads_kv * wl.head_dim
+    return [("in_proj", 2 * D, dm, 2), ("x_proj", R + 2 * N, D, 0), ("dt_proj", D, R, 4), ("out_proj", dm, D, 2),
+            ("qkv_proj", nq + 2 * nk, dm, 2), ("o_proj", dm, nq, 2)]
+
+
+def serve_step_bytes(wl):
+    """Algorithmic HBM bytes of one decode step of the stack for the whole
+    batch, per kernel class summed over the pairs: each projection reads its
+    weights once and its [B, K] bf16 input and writes its [B, N] output (x_proj
+    writes the rank-R part in bf16 and B, C in fp32; dt_proj writes fp32 and
+    reads its bias); the conv step reads x and writes u (bf16), reads and
+    writes the conv state and reads its weights and bias; the scan step is the
+    mixer's decode step without the conv (u in instead of x, no conv state or
+    conv weights, the dt bias not read); the SWA step as the mixer's."""
+    Bsz, D, N, K, R = wl.batch, wl.dim, wl.dstate, wl.dconv, wl.dt_rank
+    out = {}
+    for name, n, k, ob in serve_gemm_shapes(wl):
+        if name == "x_proj":
+            wr = Bsz * (R * 2 + 2 * N * 4)
+        elif name == "dt_proj":
+            wr = Bsz * n * 4 + n * 4
+        else:
+            wr = Bsz * n * ob
+        out[name] = SERVE_PAIRS * (n * k * 2 + Bsz * k * 2 + wr)
+    out["conv"] = SERVE_PAIRS * (2 * Bsz * D * (K - 1) * 4 + Bsz * D * 2 * 2 + D * (K + 1) * 4)
+    sb, wb = decode_bytes(wl)
+    # the layer's scan step takes u (bf16) instead of x and fuses no conv
+    out["scan_step"] = SERVE_PAIRS * (sb - 2 * Bsz * D * (K - 1) * 4 - D * (K + 2) * 4 + D * 4)
+    # (decode_bytes counts D (K + 2) fp32 for the conv weights, the conv bias
+    # and the skip D; the layer's scan step reads only the skip)
+    out["swa_step"] = SERVE_PAIRS * wb
+    return out
+
+
+def run_serve(args, wl, dev, rank, world):
+    """The prefill-to-decode serving loop of a layer stack: SERVE_PAIRS Mamba
+    + SWA layer pairs (random weights of the layer shapes), a 4096-token
+    prompt per sequence through every layer's prefill, then decode steps of
+    one token per sequence through the whole stack (each layer's output the
+    next layer's input; the tokens' input rows are seeded, as the embeddings
+    of a given continuation would be), 32 steps per CUDA graph."""
+    import torch
+    import torch.distributed as dist
+
+    from hybrid_ssm_sliding_b200 import layers, ops
+
+    wl_rank = rank_workload(wl, rank)
+    Bsz, dm, W = wl.batch, wl.d_model, wl.window
+    stack = []
+    for i in range(SERVE_PAIRS):
+        stack.append(("mamba", layers.random_mamba_weights(dm, wl.dim, wl.dstate, wl.dconv, wl.dt_rank,
+                                                           wl_rank.seed + 10 * i, dev)))
+        stack.append(("swa", layers.random_swa_weights(dm, wl.heads_q, wl.heads_kv, wl.head_dim, W,
+                                                       wl_rank.seed + 10 * i + 1, dev)))
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl_rank.seed + 2)
+    prompt = torch.randn((Bsz, wl.seqlen, dm), generator=g, device=dev).to(torch.bfloat16)
+    G = DECODE_GRAPH_STEPS
+    tokens = torch.randn((G, Bsz, dm), generator=g, device=dev).to(torch.bfloat16)
+    stream = torch.cuda.current_stream()
+
+    def prefill():
+        states, h = [], prompt
+        for kind, w in stack:
+            if kind == "mamba":
+                h, hf, cs = layers.mamba_layer_prefill(h, w)
+                states.append(layers.mamba_decode_state(hf, cs))
+            else:
+                h, k, v = layers.swa_layer_prefill(h, w)
+                states.append(layers.swa_decode_state(k, v, W, wl.heads_q))
+        return states, h
+
+    prefill()
+    torch.cuda.synchronize()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    states, _ = prefill()
+    p1.record(stream)
+    torch.cuda.synchronize()
+    ms_prefill = p0.elapsed_time(p1)
+    del prompt
+
+    def decode_step(x, st=states):
+        for (kind, w), s_ in zip(stack, st):
+            x = (layers.mamba_layer_step if kind == "mamba" else layers.swa_layer_step)(x, w, s_)
+        return x
+
+    # warm-up outside capture (first-call setup)
+    for j in range(2):
+        decode_step(tokens[j])
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        outs = [decode_step(tokens[j]) for j in range(G)]
+    reps = args.graphs if args.graphs > 0 else max(4, min(64, wl.decode_steps // G // 32))
+    for _ in range(max(1, args.warmup)):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = max_over_ranks(e0.elapsed_time(e1), dev)
+    clk = clocks.stop()
+    n_steps = reps * G
+    ms_step = ms_total / n_steps
+    value = whole_job_rate(Bsz, world, ms_step)
+    status = ops.get_status()
+
+    # each kernel class alone: the same calls as one decode step makes, over
+    # every pair, G steps per graph
+    mam = [w for kind, w in stack if kind == "mamba"]
+    swl = [w for kind, w in stack if kind == "swa"]
+    mst = [s_ for (kind, _), s_ in zip(stack, states) if kind == "mamba"]
+    sst = [s_ for (kind, _), s_ in zip(stack, states) if kind == "swa"]
+    D, N, R = wl.dim, wl.dstate, wl.dt_rank
+    nq, nk = wl.heads_q * wl.head_dim, wl.heads_kv * wl.head_dim
+
+    def bf(*shape):
+        return torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+
+    x_in, u_in, dtl_in, y_in, o_in = bf(Bsz, dm), bf(Bsz, D), bf(Bsz, R), bf(Bsz, D), bf(Bsz, nq)
+    xz_out = torch.empty((Bsz, 2 * D), dtype=torch.bfloat16, device=dev)
+    dl_out = torch.empty((Bsz, R), dtype=torch.bfloat16, device=dev)
+    bc_out = torch.empty((Bsz, 2 * N), dtype=torch.float32, device=dev)
+    delta_out = torch.empty((Bsz, D), dtype=torch.float32, device=dev)
+    dm_out = torch.empty((Bsz, dm), dtype=torch.bfloat16, device=dev)
+    qkv_out = torch.empty((Bsz, nq + 2 * nk), dtype=torch.bfloat16, device=dev)
+    u_out = torch.empty((Bsz, D), dtype=torch.bfloat16, device=dev)
+    y_out = torch.empty((Bsz, D), dtype=torch.bfloat16, device=dev)
+    o_out = torch.empty((Bsz, wl.heads_q, wl.head_dim), dtype=torch.bfloat16, device=dev)
+    delta_in = torch.full((Bsz, D), -3.0, device=dev)
+    bc_in = torch.randn((Bsz, 2 * N), generator=g, device=dev)
+    q_in, kv_in = bf(Bsz, wl.heads_q, wl.head_dim), bf(Bsz, wl.heads_kv, wl.head_dim)
+    kernels = {
+        "in_proj": lambda i: ops.gemm(x_in, mam[i].in_proj, outs=[(xz_out, 0, 2 * D, None)]),
+        "x_proj": lambda i: ops.gemm(u_in, mam[i].x_proj, outs=[(dl_out, 0, R, None),
+                                                                 (bc_out, R, R + 2 * N, None)]),
+        "dt_proj": lambda i: ops.gemm(dtl_in, mam[i].dt_proj, outs=[(delta_out, 0, D, mam[i].dt_bias)]),
+        "out_proj": lambda i: ops.gemm(y_in, mam[i].out_proj, outs=[(dm_out, 0, dm, None)]),
+        "qkv_proj": lambda i: ops.gemm(x_in, swl[i].qkv_proj, outs=[(qkv_out, 0, nq + 2 * nk, None)]),
+        "o_proj": lambda i: ops.gemm(o_in, swl[i].o_proj, outs=[(dm_out, 0, dm, None)]),
+        "conv": lambda i: ops.conv1d_fwd(u_in.view(Bsz, 1, D), mam[i].conv_w, mam[i].conv_b,
+                                         conv_state_in=mst[i].conv, conv_state_out=mst[i].conv,
+                                         u=u_out.view(Bsz, 1, D)),
+        "scan_step": lambda i: ops.scan_step(mst[i].h, None, u_in, delta_in, mam[i].A, bc_in[:, :N].contiguous(),
+                                             bc_in[:, N:].contiguous(), D=mam[i].D, z_t=y_in, y_t=y_out),
+        "swa_step": lambda i: ops.swa_step(q_in, kv_in, kv_in, sst[i].k_ring, sst[i].v_ring, sst[i].pos, W,
+                                           o_t=o_out, workspace=sst[i].workspace),
+    }
+    nbytes = serve_step_bytes(wl)
+    peaks = load_peaks()
+    kern = {}
+    for name, fn in kernels.items():
+        for i in range(SERVE_PAIRS):
+            fn(i)
+        torch.cuda.synchronize()
+        kg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(kg):
+            for _ in range(G):
+                for i in range(SERVE_PAIRS):
+                    fn(i)
+        kg.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = max(4, reps // 2)
+        a.record(stream)
+        for _ in range(n):
+            kg.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / (n * G)            # per decode step, all pairs
+        gbs = nbytes[name] / (ms / 1e3) / 1e9
+        kern[name] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                      "frac": gbs / peaks["hbm_gbs"], "traffic": None, "ms_per_step": ms,
+                      "algorithmic_bytes_per_step": nbytes[name], "peak_source": peaks["source"]}
+        del kg
+    dom = max(kern, key=lambda k: kern[k]["ms_per_step"])
+    roofline = {k: kern[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+    roofline["kernel"] = dom
+    total_bytes = sum(nbytes.values())
+    step_gbs = total_bytes / (ms_step / 1e3) / 1e9
+    whole = {"achieved": step_gbs, "frac": step_gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_step": total_bytes}
+
+    # end to end through the layer API: every step copies its token rows from
+    # pinned host memory and reads the stack's output back, 32 steps per graph
+    e2e = None
+    if not args.no_e2e:
+        host_in = [tokens[j].cpu().pin_memory() for j in range(G)]
+        host_out = [torch.empty((Bsz, dm), dtype=torch.bfloat16).pin_memory() for _ in range(G)]
+        dev_in = torch.empty((Bsz, dm), dtype=torch.bfloat16, device=dev)
+
+        def e2e_one(j):
+            dev_in.copy_(host_in[j], non_blocking=True)
+            host_out[j].copy_(decode_step(dev_in), non_blocking=True)
+
+        for j in range(2):
+            e2e_one(j)
+        torch.cuda.synchronize()
+        g_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_e2e):
+            for j in range(G):
+                e2e_one(j)
+        g_e2e.replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        n_rep = max(4, reps // 4)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_rep):
+            g_e2e.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = max_over_ranks(a.elapsed_time(b) / (n_rep * G), dev)
+        e2e = {"value": whole_job_rate(Bsz, world, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": Bsz * dm * 2,
+               "d2h_bytes_per_step": Bsz * dm * 2, "ms_per_step": ms_e2e}
+        del g_e2e
+    del graph, outs
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        with oracle_pool() as pool:
+            v, cores, sample = oracle_serve_throughput(wl, pool)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+    cfg = workload_config(wl)
+    state_bytes = SERVE_PAIRS * (Bsz * D * N * 4 + 2 * Bsz * D * (wl.dconv - 1) * 4
+                                 + 2 * Bsz * W * wl.heads_kv * wl.head_dim * 2)
+    weight_bytes = SERVE_PAIRS * sum(n * k * 2 for _, n, k, _ in serve_gemm_shapes(wl))
+    cfg.update({"d_model": dm, "dt_rank": R, "layer_pairs": SERVE_PAIRS, "prompt_tokens": wl.seqlen,
+                "graph_steps": G, "prefill_ms": ms_prefill,
+                "prefill_tokens_per_s": whole_job_rate(Bsz * wl.seqlen, 1, ms_prefill),
+                "l2": f"inputs larger than L2: every step reads the stack's weights ({weight_bytes / 1e6:.0f} MB) "
+                      f"and states ({state_bytes / 1e6:.0f} MB)"})
+    per_pair_launches = 6 + 4       # Mamba: 4 GEMMs, the conv step, the scan step; SWA: 2 GEMMs, the 2-kernel SWA step
+    return {
+        "metric": SERVE_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": n_steps,
+        "warmup": max(1, args.warmup) * G, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (random weights of the layer shapes)",
+        "config": cfg, "roofline": roofline, "step_roofline": whole, "kernels": kern, "cpu_baseline": cpu,
+        "e2e": e2e, "clocks": clk, "gpu_launches": n_steps * SERVE_PAIRS * per_pair_launches, "status": status,
+    }
+
+
+TRAIN_METRIC = "Samba mixer training step tokens/s (forward + backward of the selective scan and SWA)"
+
+
+def swa_bwd_flops(wl):
+    """Band FLOPs of the attention backward: the five products of the chain
+    rule (S recomputed, dP, dV, dK, dQ), each 2·L·W·d per (batch, query head)
+    on the band, i.e. 10·L·W·d (the forward's 4·L·W·d is two of them)."""
+    return 10.0 * wl.batch * wl.heads_q * wl.seqlen * wl.window * wl.head_dim
+
+
+def scan_bwd_bytes(wl):
+    """HBM bytes the scan backward must move once: x, z, dy (bf16) and delta
+    (fp32) in, dx, dz (bf16) and ddelta (fp32) out per (token, channel); B, C
+    in and dB, dC out per token; the per-channel parameters and gradients."""
+    tc = wl.batch * wl.seqlen * wl.dim
+    per_token = 4 * wl.dstate * 4
+    small = wl.dim * (wl.dstate + wl.dconv + 2) * 4 * 2
+    return tc * (2 + 2 + 2 + 4 + 2 + 2 + 4) + wl.batch * wl.seqlen * per_token + small
+
+
+def run_train(args, wl, dev, rank, world):
+    """Times one training step of the two mixers: the fused scan and SWA
+    forwards (with the attention's log-sum-exp) and both backwards from
+    seeded output gradients."""
+    import torch
+    import torch.distributed as dist
+
+    from hybrid_ssm_sliding_b200 import ops
+    from hybrid_ssm_sliding_b200.workloads import make_output_grads, make_prefill_inputs
+
+    wl_rank = rank_workload(wl, rank)
+    inp = make_prefill_inputs(wl_rank, device=dev)
+    grads = make_output_grads(wl_rank, device=dev)
+    Bsz, Ln, D, N, K = wl.batch, wl.seqlen, wl.dim, wl.dstate, wl.dconv
+    y = torch.empty((Bsz, Ln, D), dtype=torch.bfloat16, device=dev)
+    o = torch.empty_like(inp["q"])
+    lse = torch.empty((Bsz, wl.heads_q, Ln), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(inp["q"]), torch.empty_like(inp["k"]), torch.empty_like(inp["v"])
+    ws_scan = torch.empty((ops.scan_bwd_workspace_size(Bsz, Ln, D, N),), dtype=torch.uint8, device=dev)
+    ws_swa = torch.empty((ops.swa_bwd_workspace_size(Bsz, Ln, wl.heads_q),), dtype=torch.uint8, device=dev)
+    scan_in = dict(D=inp["D"], z=inp["z"], conv_w=inp["conv_w"], conv_b=inp["conv_b"])
+    stream = torch.cuda.current_stream()
+
+    def fwd():
+        ops.selective_scan_fwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], y=y, **scan_in)
+        ops.swa_fwd(inp["q"], inp["k"], inp["v"], wl.window, o=o, lse=lse)
+
+    def bwd_scan():
+        return ops.selective_scan_bwd(grads["dy"], inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"],
+                                      workspace=ws_scan, **scan_in)
+
+    def bwd_swa():
+        ops.swa_bwd(grads["do"], inp["q"], inp["k"], inp["v"], o, lse, wl.window, dq=dq, dk=dk, dv=dv,
+                    workspace=ws_swa)
+
+    def step():
+        fwd()
+        bwd_scan()
+        bwd_swa()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = max_over_ranks(e0.elapsed_time(e1), dev)
+    clk = clocks.stop()
+    ms_step = ms_total / args.steps
+
+    def timed(fn, n):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    n = max(5, args.kernel_steps // 5)
+    ms_fwd, ms_bscan, ms_bswa = timed(fwd, n), timed(bwd_scan, n), timed(bwd_swa, n)
+    peaks = load_peaks()
+    fl = swa_bwd_flops(wl)
+    swa_tfs = fl / (ms_bswa / 1e3) / 1e12
+    sb = scan_bwd_bytes(wl)
+    scan_gbs = sb / (ms_bscan / 1e3) / 1e9
+    kernels = {
+        "swa_bwd": {"bound": "tensor", "achieved": swa_tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": swa_tfs / peaks["bf16_tflops"], "traffic": None, "ms": ms_bswa, "band_flops": fl,
+                    "peak_source": peaks["source"] + " burst"},
+        "scan_bwd": {"bound": "hbm", "achieved": scan_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": scan_gbs / peaks["hbm_gbs"], "traffic": None, "ms": ms_bscan, "algorithmic_bytes": sb,
+                     "peak_source": peaks["source"]},
+    }
+    dom = "scan_bwd" if ms_bscan >= ms_bswa else "swa_bwd"
+    roof = {k: kernels[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+    roof["kernel"] = "scan_bwd_kernel" if dom == "scan_bwd" else "swa_bwd_kv_kernel + swa_bwd_q_kernel"
+    cfg = workload_config(wl)
+    cfg["step"] = "scan and SWA forward (with log-sum-exp), then scan and SWA backward from seeded dy, dO"
+    return {
+        "metric": TRAIN_METRIC, "value": whole_job_rate(wl.batch * wl.seqlen, world, ms_step), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": cfg, "roofline": roof, "kernels": kernels,
+        "phases_ms": {"forward": ms_fwd, "scan_backward": ms_bscan, "swa_backward": ms_bswa},
+        "cpu_baseline": None, "e2e": None, "clocks": clk, "gpu_launches": 7 * args.steps,
         "status": ops.get_status(),
     }
 
@@ -728,8 +1171,16 @@ def main():
     lib = L.load()
 
     wl = WORKLOADS[args.workload]
+    if wl.train:
+        line = run_train(args, wl, dev, rank, world)
+        if rank == 0:
+            print(json.dumps(line))
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
     if wl.d_model > 0:
-        line = run_layers(args, wl, dev, rank, world)
+        line = (run_serve if wl.decode_steps > 0 else run_layers)(args, wl, dev, rank, world)
         if rank == 0:
             print(json.dumps(line))
         if world > 1:

@@ -111,8 +111,8 @@ int samba_conv1d_fwd(const void* x, int x_dtype, const float* w, const float* bi
   if (batch < 1 || seqlen < 1 || dim < 1) return fail(SAMBA_ERR_INVALID_ARG, "samba_conv1d_fwd: bad shape");
   if (dconv < 2 || dconv > 4) return fail(SAMBA_ERR_UNSUPPORTED, "samba_conv1d_fwd: dconv must be 2..4");
   if (!dtype_ok(x_dtype) || !dtype_ok(u_dtype)) return fail(SAMBA_ERR_UNSUPPORTED, "samba_conv1d_fwd: dtype");
-  if (conv_state_in && conv_state_in == conv_state_out)
-    return fail(SAMBA_ERR_INVALID_ARG, "samba_conv1d_fwd: conv_state_out may not alias conv_state_in");
+  if (seqlen > 1 && conv_state_in && conv_state_in == conv_state_out)
+    return fail(SAMBA_ERR_INVALID_ARG, "samba_conv1d_fwd: conv_state_out may alias conv_state_in only for L = 1");
   if (!aligned16(x) || !aligned16(u)) return fail(SAMBA_ERR_INVALID_ARG, "samba_conv1d_fwd: misaligned pointer");
   return launch_conv1d(x, x_dtype, w, bias, conv_state_in, u, u_dtype, conv_state_out, batch, seqlen, dim, dconv,
                        silu, reinterpret_cast<cudaStream_t>(stream));

@@ -13,7 +13,8 @@
 // pass, or Δ-low-rank, B and C of the selective-parameter projection.
 //
 // Design: persistent CTAs, one per SM, walking the 128 x BN tiles of C
-// (BN = 256 or 128) with the N tile fastest; K in steps of 64 (128-byte
+// (BN = 256, 128 when N < 256, 64 when M <= 128) with the N tile fastest;
+// K in steps of 64 (128-byte
 // rows, 128-byte swizzle).  Warp 4 streams A and B tiles into a STG-deep
 // shared-memory ring with TMA, continuously across tiles; warp 5 issues the
 // tcgen05.mma (kind::f16, M = 128, N = BN, K = 16 per instruction) into one of
@@ -240,7 +241,7 @@ int take_status_gemm(cudaStream_t s) { return take_status_word(s); }
 
 template <int BN>
 static int launch_gemm_t(const samba_gemm_args& a, cudaStream_t stream) {
-  constexpr int STG = BN == 256 ? 4 : 6;
+  constexpr int STG = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
   using Cfg = GemmCfg<BN, STG>;
   auto kern = gemm_kernel<BN, STG>;
   static PerDeviceOnce attr;
@@ -279,7 +280,11 @@ static int launch_gemm_t(const samba_gemm_args& a, cudaStream_t stream) {
   return check_launch("samba_gemm");
 }
 
+// Tile width: 256 columns for large problems; with at most one 128-row block
+// (decode-sized M) 64 columns, so that the weight matrix is streamed by as
+// many SMs as possible.
 int launch_gemm(const samba_gemm_args& a, cudaStream_t s) {
+  if (a.M <= 128) return launch_gemm_t<64>(a, s);
   return a.N >= 256 ? launch_gemm_t<256>(a, s) : launch_gemm_t<128>(a, s);
 }
 

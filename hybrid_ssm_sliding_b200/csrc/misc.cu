@@ -67,12 +67,39 @@ __global__ void conv_state_kernel(const XT* __restrict__ x, const float* __restr
   }
 }
 
+// One position (L = 1) with the conv state carried: one thread per (b, c)
+// reads the channel's K-1 earlier inputs and x, writes u and the shifted
+// state.  A thread reads everything it needs before it writes, and no other
+// thread touches that channel's state, so cs_out may be cs_in.
+template <typename XT, typename UT>
+__global__ void conv1d_step_kernel(const XT* __restrict__ x, const float* __restrict__ w,
+                                   const float* __restrict__ bias, const float* cs_in, UT* __restrict__ u,
+                                   float* cs_out, int64_t B, int64_t D, int K, int silu) {
+  const int64_t n = B * D;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t c = e % D;
+    float xp[4];
+    for (int k = 0; k < K - 1; ++k) xp[k] = cs_in ? cs_in[e * (K - 1) + k] : 0.f;
+    xp[K - 1] = to_f32<XT>(x[e]);
+    float acc = bias ? bias[c] : 0.f;
+    for (int k = 0; k < K; ++k) acc = fmaf(w[c * K + k], xp[k], acc);
+    if (silu) acc = silu_dev(acc);
+    u[e] = from_f32<UT>(acc);
+    for (int k = 0; k < K - 1; ++k) cs_out[e * (K - 1) + k] = xp[k + 1];
+  }
+}
+
 template <typename XT, typename UT>
 static void conv1d_go(const void* x, const float* w, const float* bias, const float* cs_in, void* u, float* cs_out,
                       int64_t B, int64_t L, int64_t D, int K, int silu, cudaStream_t s) {
   const int64_t n = B * L * D;
   const int threads = 256;
   const int blocks = (int)std::min<int64_t>((n + threads - 1) / threads, (int64_t)sm_count() * 16);
+  if (L == 1 && cs_out) {
+    conv1d_step_kernel<XT, UT><<<blocks, threads, 0, s>>>(reinterpret_cast<const XT*>(x), w, bias, cs_in,
+                                                           reinterpret_cast<UT*>(u), cs_out, B, D, K, silu);
+    return;
+  }
   conv1d_kernel<XT, UT><<<blocks, threads, 0, s>>>(reinterpret_cast<const XT*>(x), w, bias, cs_in,
                                                     reinterpret_cast<UT*>(u), B, L, D, K, silu);
   if (cs_out) {

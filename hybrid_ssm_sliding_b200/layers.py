@@ -24,7 +24,7 @@ MLP: these are the two token-mixing layers only.
 
 from __future__ import annotations
 
-from dataclasses import dataclass
+from dataclasses import dataclass, field
 
 import torch
 
@@ -61,9 +61,10 @@ class SwaLayerWeights:
     window: int
 
 
-def mamba_layer_prefill(hidden, w: MambaLayerWeights, stream=None):
+def mamba_layer_prefill(hidden, w: MambaLayerWeights, stream=None, taps=None):
     """hidden [B, L, d_model] bf16 -> (out [B, L, d_model] bf16, h_final
-    [B, D, N] fp32, conv_state [B, D, K-1] fp32)."""
+    [B, D, N] fp32, conv_state [B, D, K-1] fp32).  A dict passed as ``taps``
+    receives the intermediate activations (x, z, u, delta, B, C, y)."""
     Bsz, Ln, dm = hidden.shape
     D, N, K, R = w.dims
     M = Bsz * Ln
@@ -85,6 +86,8 @@ def mamba_layer_prefill(hidden, w: MambaLayerWeights, stream=None):
     y = ops.selective_scan_fwd(u, delta, w.A, Bm, Cm, D=w.D, z=z, fuse_conv=False, h_final=h_final,
                                y_dtype=torch.bfloat16, stream=stream)
     out = ops.gemm(y.view(M, D), w.out_proj, stream=stream).view(Bsz, Ln, dm)
+    if taps is not None:
+        taps.update(x=x, z=z, u=u, delta=delta, B=Bm, C=Cm, y=y)
     return out, h_final, cs
 
 
@@ -146,3 +149,82 @@ def random_swa_weights(d_model, Hq, Hkv, d, window, seed, device="cuda"):
         qkv_proj=(torch.randn((n, d_model), generator=g, device=device) / math.sqrt(d_model)).to(torch.bfloat16),
         o_proj=(torch.randn((d_model, Hq * d), generator=g, device=device) / math.sqrt(Hq * d)).to(torch.bfloat16),
         heads_q=Hq, heads_kv=Hkv, head_dim=d, window=window)
+
+
+# ----------------------------------------------------------------- decode
+@dataclass
+class MambaDecodeState:
+    """Decode state of a Mamba layer: the SSM state and the conv state (the
+    conv of one position updates its state in place)."""
+    h: torch.Tensor                      # [B, D, N] fp32
+    conv: torch.Tensor                   # [B, D, K-1] fp32
+
+
+@dataclass
+class SwaDecodeState:
+    """Decode state of an SWA layer: the K/V ring and the next position."""
+    k_ring: torch.Tensor                 # [B, W, Hkv, d] bf16
+    v_ring: torch.Tensor
+    pos: torch.Tensor                    # [B] int64
+    workspace: torch.Tensor = field(default=None)
+
+
+def mamba_decode_state(h_final, conv_state):
+    """The decode state after a prefill (mamba_layer_prefill's h_final and
+    conv state)."""
+    return MambaDecodeState(h=h_final.clone(), conv=conv_state.clone())
+
+
+def swa_decode_state(k, v, window, heads_q):
+    """The decode state after a prefill (swa_layer_prefill's k, v): the ring
+    of the last W positions."""
+    k_ring, v_ring, pos = ops.swa_ring_fill(k, v, window)
+    Bsz, _, _, d = k.shape
+    ws = torch.empty((max(ops.swa_step_workspace_size(Bsz, heads_q, d, window), 16),), dtype=torch.uint8,
+                     device=k.device)
+    return SwaDecodeState(k_ring, v_ring, pos, ws)
+
+
+def mamba_layer_step(hidden_t, w: MambaLayerWeights, st: MambaDecodeState, stream=None, taps=None):
+    """One token per sequence through the Mamba layer: hidden_t [B, d_model]
+    bf16 -> out_t [B, d_model] bf16, the state advanced in place.  The same
+    steps as mamba_layer_prefill at L = 1: in_proj -> (x, z); the conv over
+    the carried inputs -> u; x_proj -> (rank-R input, B, C); dt_proj + bias ->
+    delta; one scan step (samba_scan_step, conv not fused: u is its input);
+    out_proj.  A dict passed as ``taps`` receives the step's activations
+    (x, z, u, delta, B, C, y; [B, ...] each)."""
+    Bsz, dm = hidden_t.shape
+    D, N, K, R = w.dims
+    dev = hidden_t.device
+    x = torch.empty((Bsz, D), dtype=torch.bfloat16, device=dev)
+    z = torch.empty_like(x)
+    ops.gemm(hidden_t, w.in_proj, outs=[(x, 0, D, None), (z, D, 2 * D, None)], stream=stream)
+    u = ops.conv1d_fwd(x.view(Bsz, 1, D), w.conv_w, w.conv_b, conv_state_in=st.conv, silu=True,
+                       conv_state_out=st.conv, stream=stream).view(Bsz, D)
+    dt_low = torch.empty((Bsz, R), dtype=torch.bfloat16, device=dev)
+    Bt = torch.empty((Bsz, N), dtype=torch.float32, device=dev)
+    Ct = torch.empty_like(Bt)
+    ops.gemm(u, w.x_proj, outs=[(dt_low, 0, R, None), (Bt, R, R + N, None), (Ct, R + N, R + 2 * N, None)],
+             stream=stream)
+    delta = torch.empty((Bsz, D), dtype=torch.float32, device=dev)
+    ops.gemm(dt_low, w.dt_proj, outs=[(delta, 0, D, w.dt_bias)], stream=stream)
+    y = ops.scan_step(st.h, None, u, delta, w.A, Bt, Ct, D=w.D, z_t=z, y_dtype=torch.bfloat16, stream=stream)
+    if taps is not None:
+        taps.update(x=x, z=z, u=u, delta=delta, B=Bt, C=Ct, y=y)
+    return ops.gemm(y, w.out_proj, stream=stream)
+
+
+def swa_layer_step(hidden_t, w: SwaLayerWeights, st: SwaDecodeState, stream=None):
+    """One token per sequence through the SWA layer: qkv projection, one SWA
+    step on the ring (samba_swa_step, pos advanced), output projection."""
+    Bsz, dm = hidden_t.shape
+    Hq, Hkv, d = w.heads_q, w.heads_kv, w.head_dim
+    dev = hidden_t.device
+    q = torch.empty((Bsz, Hq, d), dtype=torch.bfloat16, device=dev)
+    k = torch.empty((Bsz, Hkv, d), dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+    nq, nk = Hq * d, Hkv * d
+    ops.gemm(hidden_t, w.qkv_proj, outs=[(q.view(Bsz, nq), 0, nq, None), (k.view(Bsz, nk), nq, nq + nk, None),
+                                        (v.view(Bsz, nk), nq + nk, nq + 2 * nk, None)], stream=stream)
+    o = ops.swa_step(q, k, v, st.k_ring, st.v_ring, st.pos, w.window, workspace=st.workspace, stream=stream)
+    return ops.gemm(o.view(Bsz, nq), w.o_proj, stream=stream)

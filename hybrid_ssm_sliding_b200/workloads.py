@@ -74,6 +74,11 @@ WORKLOADS = {
     "layers_4k": Workload("layers_4k", 1, 4096, 4096, 16, 4, 32, 4, 64, 2048, 6, d_model=2048, dt_rank=128),
     "layers_128k": Workload("layers_128k", 1, 131072, 4096, 16, 4, 32, 4, 64, 2048, 7, d_model=2048,
                             dt_rank=128),
+    # the serving loop of a layer stack: 16 sequences after 4096-token
+    # prompts decode one token each per step through Mamba + SWA layer pairs
+    # with their projections (d_model 2048, step-size rank 128)
+    "serve_64k": Workload("serve_64k", 16, 4096, 4096, 16, 4, 32, 4, 64, 2048, 10, decode_steps=65536,
+                          d_model=2048, dt_rank=128),
     # forward + backward of both mixers at the pages' 4K training context,
     # 8 sequences per step
     "train_4k": Workload("train_4k", 8, 4096, 4096, 16, 4, 32, 4, 64, 2048, 8, train=True),

@@ -113,8 +113,13 @@ int samba_selftest_wait_timeout(samba_stream_t stream);
  *   conv_state_in  [B, D, K-1] fp32, or NULL (zeros)
  *   u              [B, L, D]   u_dtype
  *   conv_state_out [B, D, K-1] fp32, or NULL: the last K-1 entries of xpad.
- *                  May not alias conv_state_in.
+ *                  May be conv_state_in itself only when L = 1 (a decode
+ *                  step: one launch then updates the state in place);
+ *                  otherwise it may not alias conv_state_in.
  * K must be 2..4; B, L >= 1; D >= 1.  L may be smaller than K-1.
+ * Errors: SAMBA_ERR_INVALID_ARG for a missing x, w or u, a bad shape, a
+ * misaligned x or u, or conv_state_out == conv_state_in with L > 1;
+ * SAMBA_ERR_UNSUPPORTED for K outside 2..4 or another dtype.
  */
 int samba_conv1d_fwd(const void* x, int x_dtype, const float* w, const float* bias,
                      const float* conv_state_in, void* u, int u_dtype, float* conv_state_out,

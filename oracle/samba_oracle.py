@@ -69,6 +69,8 @@ __all__ = [
     "scan_step",
     "swa_step",
     "ring_fill",
+    "mamba_layer_step",
+    "swa_layer_step",
 ]
 
 
@@ -642,3 +644,50 @@ def swa_step(q_t, k_t, v_t, k_ring, v_ring, pos, window, scale=None):
             o[b, h] = (e / e.sum()) @ v_ring[b, slots, kv, :]
         pos[b] = p + 1
     return o, k_ring, v_ring, pos
+
+
+# ------------------------------------------------------------ layer decode
+def mamba_layer_step(hidden_t, in_proj, conv_w, conv_b, x_proj, dt_proj, dt_bias, A, Dskip, out_proj, h, conv_state,
+                     bf16_activations=True):
+    """One decoding step of the Mamba layer (the layer of ``mamba_layer``
+    with ``mamba_step`` of the page's §推理效率 pseudo-code as its mixer):
+    the same projections, roundings and conv as the prefill on one position,
+    the conv continuing from ``conv_state`` and the scan from ``h``.
+
+    hidden_t [B, d_model]; h [B, D, N]; conv_state [B, D, K-1].  Returns
+    (out_t [B, d_model], h, conv_state) (new arrays).
+    """
+    rnd = round_bf16 if bf16_activations else (lambda t: t)
+    hidden_t = _f64(hidden_t)
+    D, N, R = _f64(A).shape[0], _f64(A).shape[1], _f64(dt_proj).shape[1]
+    xz = hidden_t @ _f64(in_proj).T
+    x, z = rnd(xz[:, :D]), rnd(xz[:, D:])
+    u, conv_state = causal_conv1d(x[:, None, :], conv_w, conv_b, conv_state, apply_silu=True)
+    u = rnd(u[:, 0, :])
+    dbc = u @ _f64(x_proj).T
+    dt_low = rnd(dbc[:, :R])
+    B_t, C_t = dbc[:, R:R + N], dbc[:, R + N:R + 2 * N]
+    delta_t = dt_low @ _f64(dt_proj).T + _f64(dt_bias)
+    y, h, _ = scan_step(h, None, u, delta_t, A, B_t, C_t, Dskip, z)
+    out = rnd(rnd(y) @ _f64(out_proj).T)
+    return out, h, conv_state
+
+
+def swa_layer_step(hidden_t, qkv_proj, o_proj, heads_q, heads_kv, head_dim, k_ring, v_ring, pos, window,
+                   bf16_activations=True):
+    """One decoding step of the SWA layer: the projections of ``swa_layer``
+    on one position around ``swa_step`` on the ring.
+
+    hidden_t [B, d_model]; rings [B, W, Hkv, d]; pos [B].  Returns (out_t
+    [B, d_model], k_ring, v_ring, pos) (new arrays)."""
+    rnd = round_bf16 if bf16_activations else (lambda t: t)
+    hidden_t = _f64(hidden_t)
+    Bsz = hidden_t.shape[0]
+    nq, nk = heads_q * head_dim, heads_kv * head_dim
+    qkv = hidden_t @ _f64(qkv_proj).T
+    q = rnd(qkv[:, :nq]).reshape(Bsz, heads_q, head_dim)
+    k = rnd(qkv[:, nq:nq + nk]).reshape(Bsz, heads_kv, head_dim)
+    v = rnd(qkv[:, nq + nk:nq + 2 * nk]).reshape(Bsz, heads_kv, head_dim)
+    o, k_ring, v_ring, pos = swa_step(q, k, v, k_ring, v_ring, pos, window)
+    out = rnd(rnd(o).reshape(Bsz, nq) @ _f64(o_proj).T)
+    return out, k_ring, v_ring, pos

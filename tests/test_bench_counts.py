@@ -64,3 +64,31 @@ def test_backward_counts():
     per_token = 4 * 4 * 4                       # B, C in; dB, dC out (fp32, N = 4)
     small = 5 * (4 + 4 + 2) * 4 * 2             # A, conv w/b, D and their gradients
     assert bench.scan_bwd_bytes(wl) == tc * per_tc + 2 * 7 * per_token + small
+
+
+def test_serve_step_bytes_term_by_term():
+    """The serving loop's bytes per decode step, listed tensor by tensor for
+    one layer pair (times the pairs)."""
+    wl = dataclasses.replace(WORKLOADS["serve_64k"], batch=3, dim=40, dstate=8, d_model=24, dt_rank=4, heads_q=4,
+                             heads_kv=2, head_dim=16, window=32, seqlen=100)
+    B, D, N, K, R, dm = 3, 40, 8, 4, 4, 24
+    nq, nk = 4 * 16, 2 * 16
+    bf, f4 = 2, 4
+    want = {
+        "in_proj": 2 * D * dm * bf + B * dm * bf + B * 2 * D * bf,
+        "x_proj": (R + 2 * N) * D * bf + B * D * bf + B * R * bf + B * 2 * N * f4,
+        "dt_proj": D * R * bf + B * R * bf + B * D * f4 + D * f4,
+        "out_proj": dm * D * bf + B * D * bf + B * dm * bf,
+        "qkv_proj": (nq + 2 * nk) * dm * bf + B * dm * bf + B * (nq + 2 * nk) * bf,
+        "o_proj": dm * nq * bf + B * nq * bf + B * dm * bf,
+        # x in, u out; conv state in and out; weights and bias
+        "conv": B * D * bf * 2 + 2 * B * D * (K - 1) * f4 + D * (K + 1) * f4,
+        # h in and out; u, z in, y out (bf16); delta in (fp32); B, C; A; skip D
+        "scan_step": 2 * B * D * N * f4 + B * D * (bf + bf + bf) + B * D * f4 + 2 * B * N * f4 + D * N * f4 + D * f4,
+        # the W ring slots of K and V read, k_t, v_t written, q_t in, o_t out
+        "swa_step": 2 * 32 * B * nk * bf + 2 * B * nk * bf + 2 * B * nq * bf,
+    }
+    got = bench.serve_step_bytes(wl)
+    assert set(got) == set(want)
+    for k in want:
+        assert got[k] == bench.SERVE_PAIRS * want[k], k

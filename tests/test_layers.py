@@ -44,17 +44,28 @@ def test_mamba_layer_matches_oracle(Bsz, Ln, dm, D, N, R):
     g = torch.Generator(device="cuda")
     g.manual_seed(Ln + 1)
     hidden = torch.randn((Bsz, Ln, dm), generator=g, device="cuda").to(torch.bfloat16)
-    out, h_final, cs = layers.mamba_layer_prefill(hidden, w)
+    taps = {}
+    out, h_final, cs = layers.mamba_layer_prefill(hidden, w, taps=taps)
     torch.cuda.synchronize()
     assert ops.get_status() == 0
     ref = orc.mamba_layer(host64(hidden), host64(w.in_proj), host64(w.conv_w), host64(w.conv_b), host64(w.x_proj),
                           host64(w.dt_proj), host64(w.dt_bias), host64(w.A), host64(w.D), host64(w.out_proj))
     _bound_check(out, ref["out"], f"mamba layer B{Bsz} L{Ln} d_model {dm} D {D}", 1e-2)
-    np.testing.assert_array_equal(host64(cs), ref["conv_state"])
-    # the final state passes through the same bf16 roundings; compare it at
-    # the scan's tolerance against the oracle's state of that dataflow
-    eh = scan_errors(host64(h_final), ref["h"], np.abs(ref["h"]) + 1e-2 * np.sqrt(np.mean(ref["h"] ** 2)))
-    assert eh["rel_to_mag"] <= 1e-2, f"h rel err {eh['rel_to_mag']:.3e}"
+    # the conv state holds x, the bf16 of a GEMM output: its fp32 accumulation
+    # and the oracle's float64 sum may round one bf16 unit apart
+    cs_err = np.abs(host64(cs) - ref["conv_state"])
+    assert np.all(cs_err <= 2.0 ** -7 * np.abs(ref["conv_state"])), f"conv state off by {cs_err.max():.3e}"
+    # The final state: an activation that rounds to the other bf16 neighbour
+    # than the oracle's moves h by a few units in the third digit where h is
+    # small, so h is checked against the oracle's scan over the activations
+    # the layer actually used (its taps), at the scan's own tolerance.
+    sc = orc.selective_scan(host64(taps["u"]), host64(taps["delta"]), host64(w.A), host64(taps["B"]),
+                            host64(taps["C"]), host64(w.D), host64(taps["z"]), magnitudes=True)
+    eh = scan_errors(host64(h_final), sc["h"], sc["h_mag"])
+    record_margin(f"mamba layer B{Bsz} L{Ln} d_model {dm} D {D}", "h", tol=SCAN_TOL, **eh)
+    assert eh["rel_to_mag"] <= SCAN_TOL, f"h rel err {eh['rel_to_mag']:.3e}"
+    y_err = np.abs(host64(taps["y"]) - sc["y"]) / (SCAN_TOL * sc["y_mag"] + 2.0 ** -8 * np.abs(sc["y"]))
+    assert y_err.max() <= 1.0, f"y off by {y_err.max():.2f} x its bound"
 
 
 @pytest.mark.parametrize("Bsz,Ln,dm,Hq,Hkv,d,W", [(1, 300, 256, 8, 2, 64, 128), (2, 200, 128, 4, 4, 32, 1000)])

@@ -1,0 +1,211 @@
+"""GPU parity of the layers' decode steps: a prompt of L tokens through the
+layer prefill, then s tokens one at a time through the layer step
+(samba_gemm at M = batch, samba_conv1d_fwd on one position with the carried
+conv state, samba_scan_step, samba_swa_step on the ring).  The step outputs
+must equal the float64 layer oracle run over all L + s tokens at positions
+L .. L + s - 1: decoding a token is the prefill of one more position.
+
+Bounds are those of the layer prefill tests (2^-7 |ref| plus 1e-2 of the
+output rms for the Mamba layer, 5e-2 for the SWA layer); the carried states
+after the last step are checked against the oracle's states after L + s
+tokens.  The stack test runs two Mamba + SWA pairs as a serving loop does
+(each layer's output is the next layer's input) and checks every layer
+against the oracle over the input that layer actually received."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.samba_oracle as orc
+from hybrid_ssm_sliding_b200 import build as B
+from hybrid_ssm_sliding_b200 import layers, ops
+from tests._helpers import SCAN_TOL, host64, record_margin, scan_errors
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    B.build()
+
+
+def _bound_check(got, ref, name, share):
+    got = host64(got)
+    assert np.all(np.isfinite(got)), "unwritten or non-finite output"
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    worst = float(np.max(np.abs(got - ref) / (2.0 ** -7 * np.abs(ref) + share * rms)))
+    record_margin(name, "out", worst_over_bound=worst, max_abs=float(np.max(np.abs(got - ref))), rms=rms)
+    assert worst <= 1.0, f"{name}: error {worst:.2f} x the bound"
+
+
+def _hidden(Bsz, Ln, dm, seed):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    return torch.randn((Bsz, Ln, dm), generator=g, device="cuda").to(torch.bfloat16)
+
+
+def _mamba_ref(hidden, w):
+    return orc.mamba_layer(host64(hidden), host64(w.in_proj), host64(w.conv_w), host64(w.conv_b), host64(w.x_proj),
+                           host64(w.dt_proj), host64(w.dt_bias), host64(w.A), host64(w.D), host64(w.out_proj))
+
+
+def _swa_ref(hidden, w):
+    return orc.swa_layer(host64(hidden), host64(w.qkv_proj), host64(w.o_proj), w.heads_q, w.heads_kv, w.head_dim,
+                         w.window)
+
+
+@pytest.mark.parametrize("Bsz,Ln,s,dm,D,N,R", [
+    (2, 100, 6, 256, 512, 16, 32),     # batch 2, a ragged prompt
+    (16, 33, 4, 128, 256, 8, 16),      # the decode batch width of the serving workload
+    (1, 1, 5, 128, 256, 16, 16),       # a one-token prompt: the conv state is mostly the zero start
+    (3, 64, 130, 64, 128, 16, 8),      # more steps than prompt tokens
+])
+def test_mamba_layer_step_continues_the_prefill(Bsz, Ln, s, dm, D, N, R):
+    w = layers.random_mamba_weights(dm, D, N, 4, R, seed=7 * Ln + s)
+    hidden = _hidden(Bsz, Ln + s, dm, Ln + s)
+    out_p, h_final, cs = layers.mamba_layer_prefill(hidden[:, :Ln].contiguous(), w)
+    h_pre = h_final.clone()
+    st = layers.mamba_decode_state(h_final, cs)
+    outs, taps = [], []
+    for j in range(s):
+        taps.append({})
+        outs.append(layers.mamba_layer_step(hidden[:, Ln + j].contiguous(), w, st, taps=taps[-1]))
+    torch.cuda.synchronize()
+    assert ops.get_status() == 0
+    ref = _mamba_ref(hidden, w)
+    name = f"mamba layer decode B{Bsz} L{Ln}+{s} d_model {dm} D {D}"
+    _bound_check(torch.stack(outs, dim=1), ref["out"][:, Ln:], name, 1e-2)
+    _bound_check(out_p, ref["out"][:, :Ln], name + " (prefill part)", 1e-2)
+    # the conv state holds x, the bf16 of a GEMM output: its fp32 accumulation
+    # and the oracle's float64 sum may round one bf16 unit apart
+    cs_err = np.abs(host64(st.conv) - ref["conv_state"])
+    assert np.all(cs_err <= 2.0 ** -7 * np.abs(ref["conv_state"])), f"conv state off by {cs_err.max():.3e}"
+    # The state: an activation that rounds to the other bf16 neighbour than
+    # the oracle's moves h by a few units in the third digit where h is
+    # small, so h is checked against the oracle's scan over the activations
+    # the steps actually used (their taps), from the prefill's state, at the
+    # scan's own tolerance.
+    cat = lambda k: np.stack([host64(t[k]) for t in taps], axis=1)   # noqa: E731
+    sc = orc.selective_scan(cat("u"), cat("delta"), host64(w.A), cat("B"), cat("C"), host64(w.D), cat("z"),
+                            h0=host64(h_pre), magnitudes=True, h0_mag=np.abs(host64(h_pre)))
+    eh = scan_errors(host64(st.h), sc["h"], sc["h_mag"])
+    record_margin(name, "h", tol=SCAN_TOL, **eh)
+    assert eh["rel_to_mag"] <= SCAN_TOL, f"h rel err {eh['rel_to_mag']:.3e}"
+    # y is that scan's output rounded to bf16 (half a unit: 2^-8 |y|)
+    y_err = np.abs(cat("y") - sc["y"]) / (SCAN_TOL * sc["y_mag"] + 2.0 ** -8 * np.abs(sc["y"]))
+    assert y_err.max() <= 1.0, f"y off by {y_err.max():.2f} x its bound"
+
+
+@pytest.mark.parametrize("Bsz,Ln,s,dm,Hq,Hkv,d,W", [
+    (2, 300, 5, 256, 8, 2, 64, 128),    # ring full and wrapping
+    (16, 40, 3, 128, 4, 1, 64, 64),     # the serving batch width, GQA 4:1
+    (1, 20, 50, 128, 4, 4, 32, 64),     # the ring fills up during the steps
+    (2, 7, 4, 64, 2, 2, 64, 1),         # a window of one key: o_t = v_t
+])
+def test_swa_layer_step_continues_the_prefill(Bsz, Ln, s, dm, Hq, Hkv, d, W):
+    w = layers.random_swa_weights(dm, Hq, Hkv, d, W, seed=Ln + W + s)
+    hidden = _hidden(Bsz, Ln + s, dm, Ln + 3 * s)
+    out_p, k, v = layers.swa_layer_prefill(hidden[:, :Ln].contiguous(), w)
+    st = layers.swa_decode_state(k, v, W, Hq)
+    outs = [layers.swa_layer_step(hidden[:, Ln + j].contiguous(), w, st) for j in range(s)]
+    torch.cuda.synchronize()
+    assert ops.get_status() == 0
+    ref = _swa_ref(hidden, w)
+    name = f"swa layer decode B{Bsz} L{Ln}+{s} {Hq}/{Hkv}x{d} W{W}"
+    _bound_check(torch.stack(outs, dim=1), ref["out"][:, Ln:], name, 5e-2)
+    assert np.all(host64(st.pos) == Ln + s)
+    # the ring after the steps holds the oracle's keys of the last W
+    # positions (the projections' bf16 k, v), each in slot p mod W
+    k_ring, v_ring, _ = orc.ring_fill(ref["k"], ref["v"], W)
+    filled = [p % W for p in range(max(0, Ln + s - W), Ln + s)]
+    for got, want in ((st.k_ring, k_ring), (st.v_ring, v_ring)):
+        g = host64(got)[:, filled]
+        r = want[:, filled]
+        assert np.max(np.abs(g - r) / (2.0 ** -7 * np.abs(r) + 1e-3)) <= 1.0
+
+
+def test_layer_stack_serving_loop():
+    """Two Mamba + SWA pairs: the prompt through every layer's prefill (each
+    layer's output the next one's input), then decode steps through the whole
+    stack.  Every layer's prefill and step outputs must match the oracle run
+    over the inputs that layer received, concatenated over time."""
+    Bsz, Ln, s, dm, D, N, R = 4, 70, 5, 128, 256, 16, 16
+    Hq, Hkv, d, W = 4, 2, 32, 48
+    stack = []
+    for i in range(2):
+        stack.append(("mamba", layers.random_mamba_weights(dm, D, N, 4, R, seed=100 + i)))
+        stack.append(("swa", layers.random_swa_weights(dm, Hq, Hkv, d, W, seed=200 + i)))
+    tokens = _hidden(Bsz, Ln + s, dm, 300)
+    seen = [[] for _ in stack]       # per layer: its input, prompt then each step
+    got = [[] for _ in stack]
+    states = []
+    h = tokens[:, :Ln].contiguous()
+    for i, (kind, w) in enumerate(stack):
+        seen[i].append(h)
+        if kind == "mamba":
+            out, hf, cs = layers.mamba_layer_prefill(h, w)
+            states.append(layers.mamba_decode_state(hf, cs))
+        else:
+            out, k, v = layers.swa_layer_prefill(h, w)
+            states.append(layers.swa_decode_state(k, v, W, Hq))
+        got[i].append(out)
+        h = out
+    for j in range(s):
+        h = tokens[:, Ln + j].contiguous()
+        for i, (kind, w) in enumerate(stack):
+            seen[i].append(h[:, None])
+            step = layers.mamba_layer_step if kind == "mamba" else layers.swa_layer_step
+            h = step(h, w, states[i])
+            got[i].append(h[:, None])
+    torch.cuda.synchronize()
+    assert ops.get_status() == 0
+    for i, (kind, w) in enumerate(stack):
+        inp = torch.cat(seen[i], dim=1)
+        ref = _mamba_ref(inp, w) if kind == "mamba" else _swa_ref(inp, w)
+        _bound_check(torch.cat(got[i], dim=1), ref["out"], f"stack layer {i} ({kind}) B{Bsz} L{Ln}+{s}",
+                     1e-2 if kind == "mamba" else 5e-2)
+
+
+def test_decode_steps_replay_in_a_cuda_graph():
+    """The steps of one Mamba + SWA pair captured in a CUDA graph of four
+    steps and replayed twice give the outputs of the same eight steps run
+    eagerly (state buffers stay in place, so the capture is valid)."""
+    Bsz, Ln, dm, D, N, R = 16, 64, 128, 256, 16, 16
+    Hq, Hkv, d, W = 4, 1, 64, 32
+    mw = layers.random_mamba_weights(dm, D, N, 4, R, seed=11)
+    sw = layers.random_swa_weights(dm, Hq, Hkv, d, W, seed=12)
+    tokens = _hidden(Bsz, Ln + 8, dm, 13)
+
+    def fresh():
+        out, hf, cs = layers.mamba_layer_prefill(tokens[:, :Ln].contiguous(), mw)
+        _, k, v = layers.swa_layer_prefill(out, sw)
+        return layers.mamba_decode_state(hf, cs), layers.swa_decode_state(k, v, W, Hq)
+
+    ms, ss = fresh()
+    eager = []
+    for j in range(8):
+        eager.append(layers.swa_layer_step(layers.mamba_layer_step(tokens[:, Ln + j].contiguous(), mw, ms), sw, ss))
+    ms, ss = fresh()
+    inp = torch.empty((Bsz, dm), dtype=torch.bfloat16, device="cuda")
+    outs = [torch.empty((Bsz, dm), dtype=torch.bfloat16, device="cuda") for _ in range(4)]
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    inputs = [torch.empty_like(inp) for _ in range(4)]
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            for j in range(4):
+                outs[j].copy_(layers.swa_layer_step(layers.mamba_layer_step(inputs[j], mw, ms, stream=side), sw, ss,
+                                                    stream=side))
+    torch.cuda.current_stream().wait_stream(side)
+    graphed = []
+    for rep in range(2):
+        for j in range(4):
+            inputs[j].copy_(tokens[:, Ln + 4 * rep + j])
+        g.replay()
+        graphed += [o.clone() for o in outs]
+    torch.cuda.synchronize()
+    assert ops.get_status() == 0
+    for a, b in zip(eager, graphed):
+        assert torch.equal(a, b)

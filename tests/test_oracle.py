@@ -564,6 +564,52 @@ def test_swa_layer_matches_torch_functional_composition():
     np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-11)
 
 
+@pytest.mark.parametrize("bf16", [False, True])
+def test_mamba_layer_step_continues_the_layer_prefill(bf16):
+    """Decoding one token is the prefill of one more position: the layer
+    prefill over L tokens, then s steps from its final states, reproduce the
+    prefill over L + s tokens (a prefill pinned above against torch's
+    functional layers)."""
+    w = _layer_weights(41)
+    h = _rng(42).standard_normal((2, 13, 24))
+    L0 = 9
+    pre = orc.mamba_layer(h[:, :L0], bf16_activations=bf16, **w)
+    full = orc.mamba_layer(h, bf16_activations=bf16, **w)
+    hs, cs = pre["h"], pre["conv_state"]
+    for t in range(L0, h.shape[1]):
+        out, hs, cs = orc.mamba_layer_step(h[:, t], h=hs, conv_state=cs, bf16_activations=bf16, **w)
+        np.testing.assert_allclose(out, full["out"][:, t], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(hs, full["h"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(cs, full["conv_state"])
+
+
+def test_planted_step_without_conv_state_is_caught():
+    w = _layer_weights(43)
+    h = _rng(44).standard_normal((1, 6, 24))
+    pre = orc.mamba_layer(h[:, :5], bf16_activations=False, **w)
+    full = orc.mamba_layer(h, bf16_activations=False, **w)
+    out, _, _ = orc.mamba_layer_step(h[:, 5], h=pre["h"], conv_state=np.zeros_like(pre["conv_state"]),
+                                     bf16_activations=False, **w)
+    assert not np.allclose(out, full["out"][:, 5], atol=1e-6)
+
+
+@pytest.mark.parametrize("W", [1, 5, 40])
+def test_swa_layer_step_continues_the_layer_prefill(W):
+    r = _rng(45 + W)
+    dm, Hq, Hkv, d, L = 32, 4, 2, 8, 17
+    qkv = r.standard_normal(((Hq + 2 * Hkv) * d, dm)) / 5
+    o_proj = r.standard_normal((dm, Hq * d)) / 5
+    h = r.standard_normal((2, L, dm))
+    L0 = 11
+    pre = orc.swa_layer(h[:, :L0], qkv, o_proj, Hq, Hkv, d, W)
+    full = orc.swa_layer(h, qkv, o_proj, Hq, Hkv, d, W)
+    kr, vr, pos = orc.ring_fill(pre["k"], pre["v"], W)
+    for t in range(L0, L):
+        out, kr, vr, pos = orc.swa_layer_step(h[:, t], qkv, o_proj, Hq, Hkv, d, kr, vr, pos, W)
+        np.testing.assert_allclose(out, full["out"][:, t], rtol=1e-12, atol=1e-12)
+    assert np.all(pos == L)
+
+
 # ----------------------------------------------------------------- backward
 def _scan_bwd_inputs(seed, Bsz=2, L=7, D=3, N=2, K=4):
     r = _rng(seed)
