@@ -643,10 +643,10 @@ def run_serve(args, wl, dev, rank, world):
         for kind, w in stack:
             if kind == "mamba":
                 h, hf, cs = layers.mamba_layer_prefill(h, w)
-                states.append(layers.mamba_decode_state(hf, cs))
+                states.append(layers.mamba_decode_state(hf, cs, w))
             else:
                 h, k, v = layers.swa_layer_prefill(h, w)
-                states.append(layers.swa_decode_state(k, v, W, wl.heads_q))
+                states.append(layers.swa_decode_state(k, v, w))
         return states, h
 
     prefill()
@@ -723,13 +723,18 @@ def run_serve(args, wl, dev, rank, world):
     bc_in = torch.randn((Bsz, 2 * N), generator=g, device=dev)
     q_in, kv_in = bf(Bsz, wl.heads_q, wl.head_dim), bf(Bsz, wl.heads_kv, wl.head_dim)
     kernels = {
-        "in_proj": lambda i: ops.gemm(x_in, mam[i].in_proj, outs=[(xz_out, 0, 2 * D, None)]),
+        "in_proj": lambda i: ops.gemm(x_in, mam[i].in_proj, outs=[(xz_out, 0, 2 * D, None)],
+                                      workspace=mst[i].gemm_ws),
         "x_proj": lambda i: ops.gemm(u_in, mam[i].x_proj, outs=[(dl_out, 0, R, None),
-                                                                 (bc_out, R, R + 2 * N, None)]),
-        "dt_proj": lambda i: ops.gemm(dtl_in, mam[i].dt_proj, outs=[(delta_out, 0, D, mam[i].dt_bias)]),
-        "out_proj": lambda i: ops.gemm(y_in, mam[i].out_proj, outs=[(dm_out, 0, dm, None)]),
-        "qkv_proj": lambda i: ops.gemm(x_in, swl[i].qkv_proj, outs=[(qkv_out, 0, nq + 2 * nk, None)]),
-        "o_proj": lambda i: ops.gemm(o_in, swl[i].o_proj, outs=[(dm_out, 0, dm, None)]),
+                                                                 (bc_out, R, R + 2 * N, None)],
+                                     workspace=mst[i].gemm_ws),
+        "dt_proj": lambda i: ops.gemm(dtl_in, mam[i].dt_proj, outs=[(delta_out, 0, D, mam[i].dt_bias)],
+                                      workspace=mst[i].gemm_ws),
+        "out_proj": lambda i: ops.gemm(y_in, mam[i].out_proj, outs=[(dm_out, 0, dm, None)],
+                                       workspace=mst[i].gemm_ws),
+        "qkv_proj": lambda i: ops.gemm(x_in, swl[i].qkv_proj, outs=[(qkv_out, 0, nq + 2 * nk, None)],
+                                       workspace=sst[i].gemm_ws),
+        "o_proj": lambda i: ops.gemm(o_in, swl[i].o_proj, outs=[(dm_out, 0, dm, None)], workspace=sst[i].gemm_ws),
         "conv": lambda i: ops.conv1d_fwd(u_in.view(Bsz, 1, D), mam[i].conv_w, mam[i].conv_b,
                                          conv_state_in=mst[i].conv, conv_state_out=mst[i].conv,
                                          u=u_out.view(Bsz, 1, D)),

@@ -73,7 +73,7 @@ class GemmOut(ctypes.Structure):
 
 class GemmArgs(ctypes.Structure):
     _fields_ = [("A", _vp), ("B", _vp), ("lda", _i64), ("ldb", _i64), ("M", _i64), ("N", _i64), ("K", _i64),
-                ("out", GemmOut * 3), ("nout", _i32)]
+                ("out", GemmOut * 3), ("nout", _i32), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
 
 
 class SambaError(RuntimeError):
@@ -114,6 +114,8 @@ def load() -> ctypes.CDLL:
     lib.samba_swa_step_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, _i64, ctypes.c_float, _vp]
     lib.samba_gemm.argtypes = [ctypes.POINTER(GemmArgs), _vp]
+    lib.samba_gemm_workspace_size.argtypes = [_i64, _i64]
+    lib.samba_gemm_workspace_size.restype = ctypes.c_size_t
     lib.samba_scan_carry.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, ctypes.c_int, _vp]
     lib.samba_scan_bwd_workspace_size.argtypes = [_i64, _i64, _i64, _i32]
     lib.samba_scan_bwd_workspace_size.restype = ctypes.c_size_t

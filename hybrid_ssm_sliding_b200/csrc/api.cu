@@ -258,8 +258,11 @@ int samba_gemm(const samba_gemm_args* a, samba_stream_t stream) {
       return fail(SAMBA_ERR_INVALID_ARG, "%s: output %d column range", who, o);
     if (out.ld < out.col1 - out.col0) return fail(SAMBA_ERR_INVALID_ARG, "%s: output %d row stride", who, o);
   }
+  if (a->workspace && !aligned16(a->workspace)) return fail(SAMBA_ERR_INVALID_ARG, "%s: misaligned workspace", who);
   return launch_gemm(*a, reinterpret_cast<cudaStream_t>(stream));
 }
+
+size_t samba_gemm_workspace_size(int64_t M, int64_t N) { return gemm_workspace_size(M, N); }
 
 int samba_selective_scan_fwd(const samba_scan_args* args, samba_stream_t stream) {
   int rc = check_scan(args, "samba_selective_scan_fwd");

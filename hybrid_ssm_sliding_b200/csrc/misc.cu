@@ -6,6 +6,7 @@
 
 #include "common.cuh"
 #include "host.hpp"
+#include "pdl.cuh"
 
 namespace samba {
 
@@ -75,6 +76,8 @@ template <typename XT, typename UT>
 __global__ void conv1d_step_kernel(const XT* __restrict__ x, const float* __restrict__ w,
                                    const float* __restrict__ bias, const float* cs_in, UT* __restrict__ u,
                                    float* cs_out, int64_t B, int64_t D, int K, int silu) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int64_t n = B * D;
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
     const int64_t c = e % D;
@@ -95,9 +98,9 @@ static void conv1d_go(const void* x, const float* w, const float* bias, const fl
   const int64_t n = B * L * D;
   const int threads = 256;
   const int blocks = (int)std::min<int64_t>((n + threads - 1) / threads, (int64_t)sm_count() * 16);
-  if (L == 1 && cs_out) {
-    conv1d_step_kernel<XT, UT><<<blocks, threads, 0, s>>>(reinterpret_cast<const XT*>(x), w, bias, cs_in,
-                                                           reinterpret_cast<UT*>(u), cs_out, B, D, K, silu);
+  if (L == 1 && cs_out) {  // a decode step: launched as a programmatic dependent (pdl.cuh)
+    launch_pdl(conv1d_step_kernel<XT, UT>, dim3(blocks), dim3(threads), 0, s, reinterpret_cast<const XT*>(x), w,
+               bias, cs_in, reinterpret_cast<UT*>(u), cs_out, B, D, K, silu);
     return;
   }
   conv1d_kernel<XT, UT><<<blocks, threads, 0, s>>>(reinterpret_cast<const XT*>(x), w, bias, cs_in,
@@ -158,6 +161,8 @@ __global__ void __launch_bounds__(256) scan_step_kernel(
     const float* __restrict__ A, const float* __restrict__ Dskip, const float* __restrict__ conv_w,
     const float* __restrict__ conv_b, YT* __restrict__ y_t, int64_t D, int K, uint32_t flags) {
   constexpr int TPC = 4, NS = N / TPC;
+  pdl_launch_dependents();
+  pdl_wait();  // every input and the state come from earlier kernels
   const int64_t b = blockIdx.y;
   const int64_t c = (int64_t)blockIdx.x * (blockDim.x / TPC) + threadIdx.x / TPC;
   const int j = threadIdx.x % TPC;
@@ -232,9 +237,9 @@ static void scan_step_go(float* h, float* cs, const void* x_t, const void* z_t, 
                          const float* conv_b, void* y_t, int64_t B, int64_t D, int K, uint32_t flags,
                          cudaStream_t s) {
   const dim3 grid((unsigned)((D + 63) / 64), (unsigned)B);
-  scan_step_kernel<N, XT, YT><<<grid, 256, 0, s>>>(
-      h, cs, reinterpret_cast<const XT*>(x_t), reinterpret_cast<const XT*>(z_t), delta_t, B_t, C_t, A, Dskip, conv_w,
-      conv_b, reinterpret_cast<YT*>(y_t), D, K, flags);
+  launch_pdl(scan_step_kernel<N, XT, YT>, grid, dim3(256), 0, s, h, cs, reinterpret_cast<const XT*>(x_t),
+             reinterpret_cast<const XT*>(z_t), delta_t, B_t, C_t, A, Dskip, conv_w, conv_b,
+             reinterpret_cast<YT*>(y_t), D, K, flags);
 }
 
 template <int N>
@@ -297,27 +302,66 @@ int launch_ring_fill(const void* k, const void* v, int64_t L, void* k_ring, void
 }
 
 // --------------------------------------------------------------- SWA step
-// Split over the window: CTA (split, kv head g, batch b) handles CH consecutive
-// positions of the window for the `group` query heads of g, writing a partial
-// (max, sum, unnormalised output) per head; a second kernel combines the
-// splits.  The newest position is read from k_t/v_t, which split 0 also
-// stores into its ring slot (that slot held a position outside the window, so
-// no other CTA reads it in this step).  The CTA loads its chunk's K and V
-// rows into shared memory in one burst of 16-byte chunks (all rows in flight
-// at once, a warp's load covering whole rows); the scores K·qᵀ (pos x heads) and
-// the outputs P·V (heads x head dim) are bf16 tensor-core products
-// (mma m16n8k16, fp32 accumulate), P rounded to bf16 as in the prefill.
+// Split over the ring: CTA (split, kv head g, batch b) takes the ring slots
+// [split * chunk, min(W, (split + 1) * chunk)) for the `group` query heads of
+// g and writes one partial (max, sum, unnormalised output) per head; a second
+// kernel, launched as its programmatic dependent, combines the splits and
+// advances pos once every split CTA has read it.  Softmax does not depend on
+// the order of the keys, so a CTA works on slots, not positions: slot j holds
+// a position of the window exactly when j <= p (p = pos[b], the position of
+// the new token; for p >= W every slot does), and the new key and value (slot
+// p mod W) come from k_t / v_t, which the CTA owning that slot also stores
+// into the ring (no CTA of this step reads that slot from the ring).
+//
+// K and V stream through shared memory in sub-chunks of 64 slots, one tensor
+// TMA copy per matrix (and 64-wide column panel), STG - 1 sub-chunks in
+// flight.  The slot ranges do not depend on p, so the first copies go out
+// before pos is read; rows past p or past the CTA's range (which hold no
+// position of this CTA's window and may hold anything) and the new slot's row
+// are put right in shared memory once their sub-chunk has landed.  Each of
+// the 4 warps takes 16 slots of a sub-chunk and keeps its own running max,
+// sum and output for the (up to 16, zero-padded) query heads in registers,
+// flash-attention style: scores q·Kᵀ and outputs P·V are bf16 tensor-core
+// products (mma m16n8k16 with fp32 accumulation, fragments through ldmatrix
+// from the swizzled tiles), P rounded to bf16 as in the prefill.  The sum of
+// P comes out of the same product, from a column of ones beside V, so it adds
+// exactly the rounded values that P·V adds.  The warps' states merge through
+// shared memory at the end.
 template <int HD> struct StepCfg {
-  static constexpr int CH = HD <= 64 ? 128 : 64;  // positions per CTA (= threads)
-  static constexpr int NWARP = CH / 32;
-  static constexpr int KP = HD + 8;                // row pitch of K, V, q in bf16 (conflict-free fragments)
-  static constexpr int PP = CH + 8;                // row pitch of P in bf16
-  // shared memory: V, then K + q during the scores, reused for scores + P
-  static constexpr int V_BYTES = CH * KP * 2;
-  static constexpr int KQ_BYTES = CH * KP * 2 + 16 * KP * 2;
-  static constexpr int SP_BYTES = 16 * CH * 4 + 16 * PP * 2;
-  static constexpr int SMEM = V_BYTES + (KQ_BYTES > SP_BYTES ? KQ_BYTES : SP_BYTES);
+  static constexpr int CH = HD <= 64 ? 128 : 64;   // smallest chunk (sizes the workspace)
+  static constexpr int SC = 64;                    // slots per sub-chunk
+  static constexpr int PW = HD < 64 ? HD : 64;     // panel width (elements): one TMA box row
+  static constexpr int NPANEL = HD / PW;
+  static constexpr int RB = PW * 2;                // bytes per panel row = swizzle span
+  static constexpr int MAT_BYTES = SC * HD * 2;    // one matrix (K or V) of a sub-chunk
+  static constexpr int STAGE_BYTES = 2 * MAT_BYTES;
+  static constexpr int STG = HD <= 64 ? 4 : 2;
+  static constexpr int KP = HD + 8;                // q tile pitch in bf16 (conflict-free ldmatrix)
+  static constexpr int Q_OFF = STG * STAGE_BYTES;
+  static constexpr int BAR_OFF = Q_OFF + 16 * KP * 2;
+  static constexpr int SMEM = BAR_OFF + 64 + 1024;  // barriers, abort flag; 1024-byte alignment slack
+  // after the main loop the stage buffers hold the merge: each warp's O
+  // [4][16][HD] fp32, then the warps' max and sum [4][16] each
+  static constexpr int WM_OFF = 4 * 16 * HD * 4;
+  static_assert(WM_OFF + 2 * 4 * 16 * 4 <= Q_OFF, "merge fits the stage buffers");
+  static_assert(STG * 8 + 8 <= 64, "barrier block");
+  static constexpr int THREADS = 128;
 };
+
+// Byte offset of 16-byte chunk c (of HD / 8) in row r of a sub-chunk matrix
+// as the tensor copy lays it out: NPANEL panels of [SC][RB], each row's
+// chunks permuted by the swizzle of its span (128, 64 or 32 bytes).
+template <int HD>
+__device__ __forceinline__ uint32_t step_tile_off(int r, int c) {
+  using Cfg = StepCfg<HD>;
+  constexpr int CPR = Cfg::RB / 16;  // chunks per panel row
+  const int panel = c / CPR, ci = c % CPR;
+  int x;
+  if constexpr (Cfg::RB == 128) x = ci ^ (r & 7);
+  else if constexpr (Cfg::RB == 64) x = ci ^ ((r >> 1) & 3);
+  else x = ci ^ ((r >> 2) & 1);
+  return static_cast<uint32_t>(panel * Cfg::SC * Cfg::RB + r * Cfg::RB + x * 16);
+}
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
@@ -328,185 +372,242 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t saddr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(saddr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t saddr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(saddr));
+}
+
 template <int HD>
-__global__ void __launch_bounds__(StepCfg<HD>::CH) swa_step_split_kernel(
+__global__ void __launch_bounds__(128) swa_step_split_kernel(
+    const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
     const __nv_bfloat16* __restrict__ q_t, const __nv_bfloat16* __restrict__ k_t,
     const __nv_bfloat16* __restrict__ v_t, __nv_bfloat16* __restrict__ k_ring, __nv_bfloat16* __restrict__ v_ring,
-    const int64_t* __restrict__ pos, float* __restrict__ ws, int Hq, int Hkv, int64_t W, float scale_log2,
-    int nsplit) {
+    const int64_t* __restrict__ pos, float* __restrict__ ws, int Hq, int Hkv, int W, float scale_log2, int nsplit,
+    int chunk) {
   using Cfg = StepCfg<HD>;
-  constexpr int CH = Cfg::CH, NWARP = Cfg::NWARP, KP = Cfg::KP, PP = Cfg::PP;
+  constexpr int SC = Cfg::SC, KP = Cfg::KP, STG = Cfg::STG, RCH = HD / 8;
+  extern __shared__ unsigned char sm_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+  __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(sm + Cfg::Q_OFF);     // [16][KP]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + Cfg::BAR_OFF);            // [STG]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + STG);
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int group = Hq / Hkv;  // <= 16
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // Loads that do not depend on pos go first, so that they are in flight
-  // together with the read of pos: the group's query rows (16-byte chunks of
-  // the zero-padded 16-row tile) and, in split 0, the new key/value row.
-  constexpr int QCH = 16 * HD / 8, QPT = (QCH + CH - 1) / CH, RCH = HD / 8;
-  const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
-  uint4 qraw[QPT];
-#pragma unroll
-  for (int j = 0; j < QPT; ++j) {
-    const int i = tid + j * CH, hh = i / RCH, c = i % RCH;
-    qraw[j] = (i < QCH && hh < group)
-                  ? reinterpret_cast<const uint4*>(q_t + ((int64_t)b * Hq + g * group + hh) * HD)[c]
-                  : zero4;
-  }
+  const int gq = lane >> 2, tq = lane & 3;
+  const int j_lo = split * chunk;
+  const int j_hi = static_cast<int64_t>(j_lo) + chunk < W ? j_lo + chunk : W;
+  const int nsub = (j_hi - j_lo + SC - 1) / SC;
+  const int64_t row_stride = static_cast<int64_t>(Hkv) * HD;           // elements between ring slots
   const int64_t noff = ((int64_t)b * Hkv + g) * HD;
-  uint4 knew = zero4, vnew = zero4;
-  if (split == 0 && tid < RCH) {
-    knew = reinterpret_cast<const uint4*>(k_t + noff)[tid];
-    vnew = reinterpret_cast<const uint4*>(v_t + noff)[tid];
-  }
-  const int64_t p = pos[b];
-  const int64_t lo = p - W + 1 > 0 ? p - W + 1 : 0;
-  const int64_t a0 = lo + (int64_t)split * CH;
-  // positions a0 .. a0 + n_here - 1 of this chunk are valid; their ring slots
-  // are consecutive modulo W, starting at slot0 (one 64-bit remainder per CTA)
-  const int n_here = (int)(p - a0 + 1 < CH ? (p - a0 + 1 > 0 ? p - a0 + 1 : 0) : CH);
-  const int slot0 = (int)(a0 % W);
-  const int Wi = (int)W;
-  __shared__ __align__(16) unsigned char sm[Cfg::SMEM];
-  __nv_bfloat16* Vs = reinterpret_cast<__nv_bfloat16*>(sm);                              // [CH][KP]
-  __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(sm + Cfg::V_BYTES);               // [CH][KP]
-  __nv_bfloat16* Qs = Ks + CH * KP;                                                       // [16][KP]
-  float* Sc = reinterpret_cast<float*>(sm + Cfg::V_BYTES);                                // [16][CH] (after K)
-  __nv_bfloat16* Ps = reinterpret_cast<__nv_bfloat16*>(sm + Cfg::V_BYTES + 16 * CH * 4);  // [16][PP]
-  __shared__ float red_m[16], red_l[16];
+  const uint32_t sm_base = smem_u32(sm);
 
-  const int gq = lane >> 2, tq = lane & 3;  // mma fragment coordinates
-  // K and V rows of the chunk to shared memory (zeros past the window), as
-  // 16-byte chunks: consecutive threads take consecutive chunks of a row, so
-  // a warp's load covers whole rows (RCH chunks each); the newest position
-  // comes from k_t / v_t.
-  {
-    uint4 kraw[RCH], vraw[RCH];
-#pragma unroll
-    for (int i = 0; i < RCH; ++i) {
-      const int ig = tid + i * CH, r = ig / RCH, c = ig % RCH;
-      const bool valid = r < n_here;
-      int slot = slot0 + r;
-      slot = slot >= Wi ? slot - Wi : slot;
-      const bool is_new = a0 + r == p;
-      const int64_t roff = (((int64_t)b * W + (valid ? slot : 0)) * Hkv + g) * HD;
-      const uint4* krow = reinterpret_cast<const uint4*>(is_new ? k_t + noff : k_ring + roff);
-      const uint4* vrow = reinterpret_cast<const uint4*>(is_new ? v_t + noff : v_ring + roff);
-      kraw[i] = valid ? krow[c] : zero4;
-      vraw[i] = valid ? vrow[c] : zero4;
-    }
-#pragma unroll
-    for (int i = 0; i < RCH; ++i) {
-      const int ig = tid + i * CH, r = ig / RCH, c = ig % RCH;
-      reinterpret_cast<uint4*>(Ks + r * KP)[c] = kraw[i];
-      reinterpret_cast<uint4*>(Vs + r * KP)[c] = vraw[i];
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < QPT; ++j) {
-    const int i = tid + j * CH;
-    if (i < QCH) reinterpret_cast<uint4*>(Qs + (i / RCH) * KP)[i % RCH] = qraw[j];
-  }
-  if (split == 0 && tid < RCH) {  // the new key/value into its slot
-    const int64_t roff = (((int64_t)b * W + p % W) * Hkv + g) * HD;
-    reinterpret_cast<uint4*>(k_ring + roff)[tid] = knew;
-    reinterpret_cast<uint4*>(v_ring + roff)[tid] = vnew;
+  if (tid == 0) {
+    for (int s = 0; s < STG; ++s) mbar_init(&full[s], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
   }
   __syncthreads();
+  pdl_launch_dependents();
+  pdl_wait();  // q, k, v, the ring and pos all come from earlier kernels
 
-  // scores: warp w takes positions [32w, 32w + 32) (two m16 tiles) against
-  // the 16 (zero-padded) head rows (two n8 tiles), k over the head dim
-  float sacc[2][2][4];
+  auto issue = [&](int stage, int sub) {  // one thread
+    unsigned char* Ks = sm + stage * Cfg::STAGE_BYTES;
+    unsigned char* Vs = Ks + Cfg::MAT_BYTES;
+    const int j = j_lo + sub * SC;   // slots past W read as zeros
+    mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[mt][nt][e] = 0.f;
-#pragma unroll
-  for (int ks = 0; ks < HD / 16; ++ks) {
-    const int kc = 16 * ks + 2 * tq;
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      const int r0 = 32 * warp + 16 * mt + gq;
-      const uint32_t a0r = *reinterpret_cast<const uint32_t*>(Ks + r0 * KP + kc);
-      const uint32_t a1r = *reinterpret_cast<const uint32_t*>(Ks + (r0 + 8) * KP + kc);
-      const uint32_t a2r = *reinterpret_cast<const uint32_t*>(Ks + r0 * KP + kc + 8);
-      const uint32_t a3r = *reinterpret_cast<const uint32_t*>(Ks + (r0 + 8) * KP + kc + 8);
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int n = 8 * nt + gq;
-        const uint32_t b0r = *reinterpret_cast<const uint32_t*>(Qs + n * KP + kc);
-        const uint32_t b1r = *reinterpret_cast<const uint32_t*>(Qs + n * KP + kc + 8);
-        mma_bf16_16816(sacc[mt][nt], a0r, a1r, a2r, a3r, b0r, b1r);
-      }
+    for (int pn = 0; pn < Cfg::NPANEL; ++pn) {
+      tma_load_4d(Ks + pn * SC * Cfg::RB, &map_k, &full[stage], pn * Cfg::PW, g, j, b);
+      tma_load_4d(Vs + pn * SC * Cfg::RB, &map_v, &full[stage], pn * Cfg::PW, g, j, b);
     }
+  };
+  if (tid == 0) {
+    tma_prefetch_desc(&map_k);
+    tma_prefetch_desc(&map_v);
+    for (int st = 0; st < STG - 1 && st < nsub; ++st) issue(st, st);
   }
-  __syncthreads();  // K and q are read: their space now holds the scores and P
+
+  const int64_t p = pos[b];
+  const int jnew = static_cast<int>(p % W);
+  // slots [j_lo, lim) of this CTA hold positions of the window
+  const int lim = p + 1 < j_hi ? static_cast<int>(p + 1) : j_hi;
+  for (int i = tid; i < 16 * RCH; i += 128) {
+    const int hh = i / RCH, c = i % RCH;
+    const uint4 v = hh < group ? reinterpret_cast<const uint4*>(q_t + ((int64_t)b * Hq + g * group + hh) * HD)[c]
+                               : make_uint4(0u, 0u, 0u, 0u);
+    reinterpret_cast<uint4*>(Qs + hh * KP)[c] = v;
+  }
+  if (jnew >= j_lo && jnew < j_hi && tid < RCH) {  // the new key and value into their slot
+    const int64_t roff = ((int64_t)b * W + jnew) * row_stride + (int64_t)g * HD;
+    reinterpret_cast<uint4*>(k_ring + roff)[tid] = reinterpret_cast<const uint4*>(k_t + noff)[tid];
+    reinterpret_cast<uint4*>(v_ring + roff)[tid] = reinterpret_cast<const uint4*>(v_t + noff)[tid];
+  }
+
+  uint32_t qa[HD / 16][4];
+  float o[HD / 8][4], ol[4] = {0.f, 0.f, 0.f, 0.f};  // ol: P times a column of ones (the sums)
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
+  for (int nt = 0; nt < HD / 8; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY;  // running max of rows gq and gq + 8, in log2 units
+  constexpr uint32_t kOnes = 0x3F803F80u;  // two bf16 1.0
+  bool ok = true;
+  const int mi = lane >> 3, l7 = lane & 7;
+
+  for (int sub = 0; sub < nsub; ++sub) {
+    const int stage = sub % STG;
+    ok = mbar_wait(&full[stage], (sub / STG) & 1, abort_flag) && ok;
+    __syncthreads();
+    unsigned char* Ks = sm + stage * Cfg::STAGE_BYTES;
+    unsigned char* Vs = Ks + Cfg::MAT_BYTES;
+    const int j0 = j_lo + sub * SC;
+    // rows from lim on (past p, or past the CTA's range) become zeros and the
+    // new slot's row becomes k_t, v_t
+    const bool fix_tail = lim < j0 + SC;
+    const bool fix_new = jnew >= j0 && jnew < j0 + SC && jnew < j_hi;
+    if (fix_tail || fix_new) {  // uniform over the CTA
+      for (int i = tid; i < SC * RCH; i += 128) {
+        const int r = i / RCH, c = i % RCH, j = j0 + r;
+        uint4* kd = reinterpret_cast<uint4*>(Ks + step_tile_off<HD>(r, c));
+        uint4* vd = reinterpret_cast<uint4*>(Vs + step_tile_off<HD>(r, c));
+        if (j == jnew) {
+          *kd = reinterpret_cast<const uint4*>(k_t + noff)[c];
+          *vd = reinterpret_cast<const uint4*>(v_t + noff)[c];
+        } else if (j >= lim) {
+          *kd = make_uint4(0u, 0u, 0u, 0u);
+          *vd = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_shared();  // these writes come before the next tensor copy into the buffer
+      __syncthreads();
+    }
+    if (sub == 0) {
+#pragma unroll
+      for (int ks = 0; ks < HD / 16; ++ks)
+        ldsm_x4(qa[ks], smem_u32(Qs + ((mi & 1) * 8 + l7) * KP + 16 * ks + (mi >> 1) * 8));
+    }
+    const int r0 = 16 * warp;
+    const uint32_t kb_base = sm_base + stage * Cfg::STAGE_BYTES, vb_base = kb_base + Cfg::MAT_BYTES;
+    // scores S[head, slot] for this warp's 16 slots (two n8 tiles), raw
+    float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int ks = 0; ks < HD / 16; ++ks) {
+      uint32_t kb[4];
+      ldsm_x4(kb, kb_base + step_tile_off<HD>(r0 + (mi >> 1) * 8 + l7, 2 * ks + (mi & 1)));
+      mma_bf16_16816(sc[0], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], kb[0], kb[1]);
+      mma_bf16_16816(sc[1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], kb[2], kb[3]);
+    }
+    const int nval = lim - (j0 + r0);  // this warp's slots [0, nval) are in the window
+    float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int row = 32 * warp + 16 * mt + gq + (e >= 2 ? 8 : 0);  // position
-        const int col = 8 * nt + 2 * tq + (e & 1);                      // head
-        Sc[col * CH + row] = row < n_here ? sacc[mt][nt][e] * scale_log2 : -INFINITY;
+        const int col = 8 * nt + 2 * tq + (e & 1);
+        sc[nt][e] = col < nval ? sc[nt][e] : -INFINITY;
+        if (e < 2) mx0 = fmaxf(mx0, sc[nt][e]);
+        else mx1 = fmaxf(mx1, sc[nt][e]);
       }
-  __syncthreads();
-  // per head max and exp-sum (one warp per head, heads strided over the
-  // warps); P in bf16, rows past the group zero
-  for (int hh = warp; hh < 16; hh += NWARP) {
-    if (hh >= group) {
-      for (int i = lane; i < CH; i += 32) Ps[hh * PP + i] = __float2bfloat16_rn(0.f);
-      continue;
-    }
-    float m = -INFINITY;
-    for (int i = lane; i < CH; i += 32) m = fmaxf(m, Sc[hh * CH + i]);
 #pragma unroll
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const float mu = (m == -INFINITY) ? 0.f : m;
-    float l = 0.f;
-    for (int i = lane; i < CH; i += 32) {
-      const __nv_bfloat16 e = __float2bfloat16_rn(ex2_approx(Sc[hh * CH + i] - mu));
-      Ps[hh * PP + i] = e;
-      l += __bfloat162float(e);  // the sum of the probabilities P·V uses
+    for (int off = 1; off <= 2; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
     }
+    // the scale is positive, so the max of the raw scores gives the max of
+    // the scaled ones
+    const float mn0 = fmaxf(m0, mx0 * scale_log2), mn1 = fmaxf(m1, mx1 * scale_log2);
+    const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
+    const float c0 = ex2_approx(m0 - mu0), c1 = ex2_approx(m1 - mu1);  // 0 while nothing was seen
+    m0 = mn0;
+    m1 = mn1;
+    uint32_t pa[4];
 #pragma unroll
-    for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (lane == 0) {
-      red_m[hh] = m;
-      red_l[hh] = l;
+    for (int nt = 0; nt < 2; ++nt) {
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(ex2_approx(fmaf(sc[nt][0], scale_log2, -mu0)),
+                                                       ex2_approx(fmaf(sc[nt][1], scale_log2, -mu0)));
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(ex2_approx(fmaf(sc[nt][2], scale_log2, -mu1)),
+                                                       ex2_approx(fmaf(sc[nt][3], scale_log2, -mu1)));
+      pa[2 * nt] = *reinterpret_cast<const uint32_t*>(&lo);
+      pa[2 * nt + 1] = *reinterpret_cast<const uint32_t*>(&hi);
     }
+    if (!__all_sync(0xffffffffu, c0 == 1.f && c1 == 1.f)) {  // a max moved: rescale
+#pragma unroll
+      for (int nt = 0; nt < HD / 8; ++nt) {
+        o[nt][0] *= c0;
+        o[nt][1] *= c0;
+        o[nt][2] *= c1;
+        o[nt][3] *= c1;
+      }
+      ol[0] *= c0;
+      ol[1] *= c0;
+      ol[2] *= c1;
+      ol[3] *= c1;
+    }
+    // O[head, d] += P[head, slot] · V[slot, d]; A = P (k = slots 0-7 | 8-15)
+#pragma unroll
+    for (int jj = 0; jj < HD / 16; ++jj) {
+      uint32_t vb[4];
+      ldsm_x4_t(vb, vb_base + step_tile_off<HD>(r0 + (mi & 1) * 8 + l7, 2 * jj + (mi >> 1)));
+      mma_bf16_16816(o[2 * jj], pa[0], pa[1], pa[2], pa[3], vb[0], vb[1]);
+      mma_bf16_16816(o[2 * jj + 1], pa[0], pa[1], pa[2], pa[3], vb[2], vb[3]);
+    }
+    mma_bf16_16816(ol, pa[0], pa[1], pa[2], pa[3], kOnes, kOnes);
+    // every warp has passed this iteration's barrier, so the buffer of the
+    // previous sub-chunk is free for the one STG - 1 ahead
+    if (tid == 0 && sub + STG - 1 < nsub) issue((sub + STG - 1) % STG, sub + STG - 1);
+  }
+  __syncthreads();  // the stage buffers now hold the merge (every copy has landed: each was waited for)
+
+  // merge the four warps: per head M = max over warps, each warp's share
+  // scaled by exp2(m_w - M) into its own slice (plain stores; shared-memory
+  // atomics from three CTAs per SM would serialise), the slices summed as the
+  // partial is written
+  float* Ow = reinterpret_cast<float*>(sm);                    // [4][16][HD]
+  float* wm = reinterpret_cast<float*>(sm + Cfg::WM_OFF);      // [4][16]
+  float* wl = wm + 64;                                         // [4][16]
+  if (tq == 0) {
+    wm[warp * 16 + gq] = m0;
+    wm[warp * 16 + gq + 8] = m1;
+    wl[warp * 16 + gq] = ol[0];
+    wl[warp * 16 + gq + 8] = ol[2];
   }
   __syncthreads();
-  // outputs: heads (m16) x head dim (n8 tiles over the warps), k over positions
-  for (int nt = warp; nt < HD / 8; nt += NWARP) {
-    float oacc[4] = {0.f, 0.f, 0.f, 0.f};
-    const int n = 8 * nt + gq;  // head-dim column of the B fragment
+  float M0 = -INFINITY, M1 = -INFINITY;
 #pragma unroll
-    for (int ks = 0; ks < CH / 16; ++ks) {
-      const int kc = 16 * ks + 2 * tq;
-      const uint32_t a0r = *reinterpret_cast<const uint32_t*>(Ps + gq * PP + kc);
-      const uint32_t a1r = *reinterpret_cast<const uint32_t*>(Ps + (gq + 8) * PP + kc);
-      const uint32_t a2r = *reinterpret_cast<const uint32_t*>(Ps + gq * PP + kc + 8);
-      const uint32_t a3r = *reinterpret_cast<const uint32_t*>(Ps + (gq + 8) * PP + kc + 8);
-      const unsigned short* vb = reinterpret_cast<const unsigned short*>(Vs);
-      const uint32_t b0r = (uint32_t)vb[kc * KP + n] | ((uint32_t)vb[(kc + 1) * KP + n] << 16);
-      const uint32_t b1r = (uint32_t)vb[(kc + 8) * KP + n] | ((uint32_t)vb[(kc + 9) * KP + n] << 16);
-      mma_bf16_16816(oacc, a0r, a1r, a2r, a3r, b0r, b1r);
-    }
+  for (int w = 0; w < 4; ++w) {
+    M0 = fmaxf(M0, wm[w * 16 + gq]);
+    M1 = fmaxf(M1, wm[w * 16 + gq + 8]);
+  }
+  const float f0 = M0 == -INFINITY ? 0.f : ex2_approx(m0 - M0);
+  const float f1 = M1 == -INFINITY ? 0.f : ex2_approx(m1 - M1);
+  float* mine = Ow + warp * 16 * HD;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int hh = gq + (e >= 2 ? 8 : 0);
-      const int dd = 8 * nt + 2 * tq + (e & 1);
-      if (hh < group) {
-        float* dst = ws + ((((int64_t)b * Hq + g * group + hh) * nsplit + split) * (HD + 2));
-        dst[2 + dd] = oacc[e];
-        if (dd == 0) {
-          dst[0] = red_m[hh];
-          dst[1] = red_l[hh];
-        }
-      }
+  for (int nt = 0; nt < HD / 8; ++nt) {
+    const int col = 8 * nt + 2 * tq;
+    *reinterpret_cast<float2*>(mine + gq * HD + col) = make_float2(o[nt][0] * f0, o[nt][1] * f0);
+    *reinterpret_cast<float2*>(mine + (gq + 8) * HD + col) = make_float2(o[nt][2] * f1, o[nt][3] * f1);
+  }
+  if (!__syncthreads_and(ok)) return;  // a copy never landed: the status word says so
+  for (int i = tid; i < group * HD; i += 128) {
+    const int hh = i / HD, dd = i % HD;
+    float* dst = ws + ((((int64_t)b * Hq + g * group + hh) * nsplit + split) * (HD + 2));
+    dst[2 + dd] = Ow[hh * HD + dd] + Ow[(16 + hh) * HD + dd] + Ow[(32 + hh) * HD + dd] + Ow[(48 + hh) * HD + dd];
+    if (dd == 0) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w * 16 + hh]);
+      float l = 0.f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w)
+        if (M != -INFINITY && wm[w * 16 + hh] != -INFINITY) l = fmaf(wl[w * 16 + hh], ex2_approx(wm[w * 16 + hh] - M), l);
+      dst[0] = M;
+      dst[1] = l;
     }
   }
 }
@@ -514,6 +615,8 @@ __global__ void __launch_bounds__(StepCfg<HD>::CH) swa_step_split_kernel(
 template <int HD>
 __global__ void swa_step_combine_kernel(const float* __restrict__ ws, __nv_bfloat16* __restrict__ o_t,
                                         int64_t* __restrict__ pos, int Hq, int nsplit) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int hq = blockIdx.x, b = blockIdx.y;
   const int dd = threadIdx.x;
   const float* base = ws + ((int64_t)b * Hq + hq) * nsplit * (HD + 2);
@@ -534,8 +637,9 @@ __global__ void swa_step_combine_kernel(const float* __restrict__ ws, __nv_bfloa
 }
 
 // Bytes of split partials: (max, sum, d outputs) per (batch, query head,
-// split).  SIZE_MAX when the product does not fit in size_t, so that no
-// workspace (and no built-in scratch) is ever taken as large enough.
+// split), for at most ceil(W / CH) splits.  SIZE_MAX when the product does
+// not fit in size_t, so that no workspace (and no built-in scratch) is ever
+// taken as large enough.
 size_t swa_step_workspace(int64_t B, int Hq, int d, int64_t W) {
   const int ch = d <= 64 ? StepCfg<64>::CH : StepCfg<128>::CH;
   const uint64_t nsplit = static_cast<uint64_t>((W + ch - 1) / ch);
@@ -547,31 +651,66 @@ size_t swa_step_workspace(int64_t B, int Hq, int d, int64_t W) {
   return static_cast<size_t>(n);
 }
 
+// Slots per CTA: as many splits as three CTAs per SM take over the batch and
+// KV heads (the kernel holds three per SM at d <= 64), at least 128 slots (so the
+// partials fit the workspace size above, which counts splits of 128 slots,
+// or 64 for d = 128) and a multiple of 64.
+static int swa_step_chunk(int64_t B, int Hkv, int64_t W) {
+  const int64_t per_split = static_cast<int64_t>(Hkv) * B;
+  const int64_t target = std::max<int64_t>(1, 3 * sm_count() / per_split);
+  const int64_t c = (W + target - 1) / target;
+  return static_cast<int>(std::max<int64_t>(128, (c + 63) / 64 * 64));
+}
+
 template <int HD>
-static void swa_step_go(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring, int64_t* pos,
-                        void* o_t, int64_t B, int Hq, int Hkv, int64_t W, float scale, void* ws, cudaStream_t s) {
-  constexpr int CH = StepCfg<HD>::CH;
-  const int nsplit = (int)((W + CH - 1) / CH);
-  dim3 g1(nsplit, Hkv, (unsigned)B);
-  swa_step_split_kernel<HD><<<g1, CH, 0, s>>>(
-      reinterpret_cast<const __nv_bfloat16*>(q_t), reinterpret_cast<const __nv_bfloat16*>(k_t),
-      reinterpret_cast<const __nv_bfloat16*>(v_t), reinterpret_cast<__nv_bfloat16*>(k_ring),
-      reinterpret_cast<__nv_bfloat16*>(v_ring), pos, reinterpret_cast<float*>(ws), Hq, Hkv, W,
-      scale * 1.4426950408889634f, nsplit);
-  dim3 g2(Hq, (unsigned)B);
-  swa_step_combine_kernel<HD><<<g2, HD, 0, s>>>(reinterpret_cast<const float*>(ws),
-                                                 reinterpret_cast<__nv_bfloat16*>(o_t), pos, Hq, nsplit);
+static int swa_step_go(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring, int64_t* pos,
+                       void* o_t, int64_t B, int Hq, int Hkv, int64_t W, float scale, void* ws, cudaStream_t s) {
+  using Cfg = StepCfg<HD>;
+  auto split_kern = swa_step_split_kernel<HD>;
+  static PerDeviceOnce attr;
+  const int arc = once_per_device(attr, [&] {
+    return cudaFuncSetAttribute(split_kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) == cudaSuccess
+               ? SAMBA_OK
+               : fail(SAMBA_ERR_CUDA, "samba_swa_step: cannot set shared memory size");
+  });
+  if (arc != SAMBA_OK) return arc;
+  // the rings as [B][W][Hkv][d]; boxes of one panel x one head x 64 slots
+  CUtensorMap mk, mv;
+  const uint64_t dims[4] = {(uint64_t)HD, (uint64_t)Hkv, (uint64_t)W, (uint64_t)B};
+  const uint64_t strides[3] = {(uint64_t)HD * 2, (uint64_t)Hkv * HD * 2, (uint64_t)W * Hkv * HD * 2};
+  const uint32_t box[4] = {(uint32_t)Cfg::PW, 1u, (uint32_t)Cfg::SC, 1u};
+  const CUtensorMapSwizzle sw = Cfg::RB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : (Cfg::RB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+  int rc = encode_tiled(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, k_ring, dims, strides, box, sw, "swa_step K ring");
+  if (rc) return rc;
+  rc = encode_tiled(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, v_ring, dims, strides, box, sw, "swa_step V ring");
+  if (rc) return rc;
+  const int chunk = swa_step_chunk(B, Hkv, W);
+  const int nsplit = (int)((W + chunk - 1) / chunk);
+  cudaError_t e = launch_pdl(split_kern, dim3(nsplit, Hkv, (unsigned)B), dim3(Cfg::THREADS), Cfg::SMEM, s, mk, mv,
+                             reinterpret_cast<const __nv_bfloat16*>(q_t), reinterpret_cast<const __nv_bfloat16*>(k_t),
+                             reinterpret_cast<const __nv_bfloat16*>(v_t), reinterpret_cast<__nv_bfloat16*>(k_ring),
+                             reinterpret_cast<__nv_bfloat16*>(v_ring), (const int64_t*)pos,
+                             reinterpret_cast<float*>(ws), Hq, Hkv, static_cast<int>(W), scale * 1.4426950408889634f,
+                             nsplit, chunk);
+  if (e != cudaSuccess) return fail(SAMBA_ERR_CUDA, "samba_swa_step: launch failed: %s", cudaGetErrorString(e));
+  e = launch_pdl(swa_step_combine_kernel<HD>, dim3(Hq, (unsigned)B), dim3(HD), 0, s, (const float*)ws,
+                 reinterpret_cast<__nv_bfloat16*>(o_t), pos, Hq, nsplit);
+  if (e != cudaSuccess) return fail(SAMBA_ERR_CUDA, "samba_swa_step: launch failed: %s", cudaGetErrorString(e));
+  return SAMBA_OK;
 }
 
 int launch_swa_step(const void* q_t, const void* k_t, const void* v_t, void* k_ring, void* v_ring, int64_t* pos,
                     void* o_t, int64_t B, int Hq, int Hkv, int d, int64_t W, float scale, void* ws, cudaStream_t s) {
   if (B > 65535) return fail(SAMBA_ERR_UNSUPPORTED, "samba_swa_step: batch too large");
+  int rc;
   switch (d) {
-    case 16: swa_step_go<16>(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, B, Hq, Hkv, W, scale, ws, s); break;
-    case 32: swa_step_go<32>(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, B, Hq, Hkv, W, scale, ws, s); break;
-    case 64: swa_step_go<64>(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, B, Hq, Hkv, W, scale, ws, s); break;
-    default: swa_step_go<128>(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, B, Hq, Hkv, W, scale, ws, s); break;
+    case 16: rc = swa_step_go<16>(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, B, Hq, Hkv, W, scale, ws, s); break;
+    case 32: rc = swa_step_go<32>(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, B, Hq, Hkv, W, scale, ws, s); break;
+    case 64: rc = swa_step_go<64>(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, B, Hq, Hkv, W, scale, ws, s); break;
+    default: rc = swa_step_go<128>(q_t, k_t, v_t, k_ring, v_ring, pos, o_t, B, Hq, Hkv, W, scale, ws, s); break;
   }
+  if (rc != SAMBA_OK) return rc;
   return check_launch("samba_swa_step");
 }
 

@@ -155,34 +155,57 @@ def random_swa_weights(d_model, Hq, Hkv, d, window, seed, device="cuda"):
 @dataclass
 class MambaDecodeState:
     """Decode state of a Mamba layer: the SSM state and the conv state (the
-    conv of one position updates its state in place)."""
+    conv of one position updates its state in place), and the zero-filled
+    workspace of the split-K projections (None: tiled projections)."""
     h: torch.Tensor                      # [B, D, N] fp32
     conv: torch.Tensor                   # [B, D, K-1] fp32
+    gemm_ws: torch.Tensor = field(default=None)
 
 
 @dataclass
 class SwaDecodeState:
-    """Decode state of an SWA layer: the K/V ring and the next position."""
+    """Decode state of an SWA layer: the K/V ring and the next position, the
+    SWA step's workspace and the projections' (as for the Mamba layer)."""
     k_ring: torch.Tensor                 # [B, W, Hkv, d] bf16
     v_ring: torch.Tensor
     pos: torch.Tensor                    # [B] int64
     workspace: torch.Tensor = field(default=None)
+    gemm_ws: torch.Tensor = field(default=None)
 
 
-def mamba_decode_state(h_final, conv_state):
+def _gemm_workspace(M, widths, device):
+    """One zero-filled workspace for projections of M rows to each of the
+    given widths, run one after another (None when M is above the split-K
+    limit)."""
+    n = max(ops.gemm_workspace_size(M, w) for w in widths)
+    return torch.zeros((n,), dtype=torch.uint8, device=device) if n > 0 else None
+
+
+def mamba_decode_state(h_final, conv_state, w: MambaLayerWeights = None, split_k=True):
     """The decode state after a prefill (mamba_layer_prefill's h_final and
-    conv state)."""
-    return MambaDecodeState(h=h_final.clone(), conv=conv_state.clone())
+    conv state).  Given the layer's weights (and ``split_k``), it also
+    carries the workspace of the split-K projections."""
+    Bsz = h_final.shape[0]
+    ws = None
+    if w is not None and split_k:
+        D, N, K, R = w.dims
+        ws = _gemm_workspace(Bsz, (2 * D, R + 2 * N, D, w.out_proj.shape[0]), h_final.device)
+    return MambaDecodeState(h=h_final.clone(), conv=conv_state.clone(), gemm_ws=ws)
 
 
-def swa_decode_state(k, v, window, heads_q):
+def swa_decode_state(k, v, w: SwaLayerWeights, split_k=True):
     """The decode state after a prefill (swa_layer_prefill's k, v): the ring
-    of the last W positions."""
-    k_ring, v_ring, pos = ops.swa_ring_fill(k, v, window)
-    Bsz, _, _, d = k.shape
-    ws = torch.empty((max(ops.swa_step_workspace_size(Bsz, heads_q, d, window), 16),), dtype=torch.uint8,
-                     device=k.device)
-    return SwaDecodeState(k_ring, v_ring, pos, ws)
+    of the last W positions, the SWA step's workspace and (with ``split_k``)
+    the split-K projections' workspace."""
+    k_ring, v_ring, pos = ops.swa_ring_fill(k, v, w.window)
+    Bsz = k.shape[0]
+    ws = torch.zeros((max(ops.swa_step_workspace_size(Bsz, w.heads_q, w.head_dim, w.window), 16),),
+                     dtype=torch.uint8, device=k.device)
+    gws = None
+    if split_k:
+        nqkv = (w.heads_q + 2 * w.heads_kv) * w.head_dim
+        gws = _gemm_workspace(Bsz, (nqkv, w.o_proj.shape[0]), k.device)
+    return SwaDecodeState(k_ring, v_ring, pos, ws, gws)
 
 
 def mamba_layer_step(hidden_t, w: MambaLayerWeights, st: MambaDecodeState, stream=None, taps=None):
@@ -198,20 +221,20 @@ def mamba_layer_step(hidden_t, w: MambaLayerWeights, st: MambaDecodeState, strea
     dev = hidden_t.device
     x = torch.empty((Bsz, D), dtype=torch.bfloat16, device=dev)
     z = torch.empty_like(x)
-    ops.gemm(hidden_t, w.in_proj, outs=[(x, 0, D, None), (z, D, 2 * D, None)], stream=stream)
+    ops.gemm(hidden_t, w.in_proj, outs=[(x, 0, D, None), (z, D, 2 * D, None)], workspace=st.gemm_ws, stream=stream)
     u = ops.conv1d_fwd(x.view(Bsz, 1, D), w.conv_w, w.conv_b, conv_state_in=st.conv, silu=True,
                        conv_state_out=st.conv, stream=stream).view(Bsz, D)
     dt_low = torch.empty((Bsz, R), dtype=torch.bfloat16, device=dev)
     Bt = torch.empty((Bsz, N), dtype=torch.float32, device=dev)
     Ct = torch.empty_like(Bt)
     ops.gemm(u, w.x_proj, outs=[(dt_low, 0, R, None), (Bt, R, R + N, None), (Ct, R + N, R + 2 * N, None)],
-             stream=stream)
+             workspace=st.gemm_ws, stream=stream)
     delta = torch.empty((Bsz, D), dtype=torch.float32, device=dev)
-    ops.gemm(dt_low, w.dt_proj, outs=[(delta, 0, D, w.dt_bias)], stream=stream)
+    ops.gemm(dt_low, w.dt_proj, outs=[(delta, 0, D, w.dt_bias)], workspace=st.gemm_ws, stream=stream)
     y = ops.scan_step(st.h, None, u, delta, w.A, Bt, Ct, D=w.D, z_t=z, y_dtype=torch.bfloat16, stream=stream)
     if taps is not None:
         taps.update(x=x, z=z, u=u, delta=delta, B=Bt, C=Ct, y=y)
-    return ops.gemm(y, w.out_proj, stream=stream)
+    return ops.gemm(y, w.out_proj, workspace=st.gemm_ws, stream=stream)
 
 
 def swa_layer_step(hidden_t, w: SwaLayerWeights, st: SwaDecodeState, stream=None):
@@ -225,6 +248,7 @@ def swa_layer_step(hidden_t, w: SwaLayerWeights, st: SwaDecodeState, stream=None
     v = torch.empty_like(k)
     nq, nk = Hq * d, Hkv * d
     ops.gemm(hidden_t, w.qkv_proj, outs=[(q.view(Bsz, nq), 0, nq, None), (k.view(Bsz, nk), nq, nq + nk, None),
-                                        (v.view(Bsz, nk), nq + nk, nq + 2 * nk, None)], stream=stream)
+                                        (v.view(Bsz, nk), nq + nk, nq + 2 * nk, None)],
+             workspace=st.gemm_ws, stream=stream)
     o = ops.swa_step(q, k, v, st.k_ring, st.v_ring, st.pos, w.window, workspace=st.workspace, stream=stream)
-    return ops.gemm(o.view(Bsz, nq), w.o_proj, stream=stream)
+    return ops.gemm(o.view(Bsz, nq), w.o_proj, workspace=st.gemm_ws, stream=stream)

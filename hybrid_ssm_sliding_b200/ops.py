@@ -254,12 +254,20 @@ def scan_step(h, conv_state, x_t, delta_t, A, B_t, C_t, D=None, z_t=None, conv_w
     return y_t
 
 
-def gemm(a, w, outs=None, out_dtype=torch.bfloat16, bias=None, stream=None):
+def gemm_workspace_size(M, N) -> int:
+    """Bytes of workspace the split-K form of samba_gemm uses for M rows and
+    N columns (0 when M > 32)."""
+    return int(L.load().samba_gemm_workspace_size(M, N))
+
+
+def gemm(a, w, outs=None, out_dtype=torch.bfloat16, bias=None, workspace=None, stream=None):
     """C = a @ w.T on the tensor cores (see samba_gemm): a [M, K] bf16 (rows
     may be strided), w [N, K] bf16.  ``outs`` is a list of up to three
     (tensor, col0, col1, bias) entries that receive columns [col0, col1) of C
     (tensors 2-D [M, col1 - col0], row stride any, bf16 or fp32); by default
-    one new [M, N] tensor of out_dtype (with ``bias``) is returned."""
+    one new [M, N] tensor of out_dtype (with ``bias``) is returned.
+    ``workspace`` (uint8, zero-filled before its first use, left zero-filled
+    by every call) selects the split-K form for M <= 32."""
     if a.dim() != 2 or w.dim() != 2:
         raise ValueError("a and w must be 2-D")
     if a.dtype != torch.bfloat16 or w.dtype != torch.bfloat16:
@@ -289,6 +297,9 @@ def gemm(a, w, outs=None, out_dtype=torch.bfloat16, bias=None, stream=None):
         o = args.out[i]
         o.ptr, o.bias, o.ld, o.col0, o.col1, o.dtype = L.ptr(t), L.ptr(b), t.stride(0), c0, c1, L.dtype_code(t)
     args.nout = len(outs)
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8)
+        args.workspace, args.workspace_bytes = L.ptr(workspace), workspace.numel()
     L.check(L.load().samba_gemm(ctypes.byref(args), L.stream_handle(stream)))
     return ret if ret is not None else [o[0] for o in outs]
 

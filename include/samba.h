@@ -357,9 +357,24 @@ int samba_swa_fwd(const samba_swa_args* args, samba_stream_t stream);
  * [M, col1 - col0] matrix with row stride ld (elements), in bf16 or fp32,
  * plus bias[col - col0] when bias is not NULL.  Columns outside every range
  * are dropped.
+ *
+ * Workspace (optional; only for M <= 32, a decode step's rows): with a
+ * workspace of at least samba_gemm_workspace_size(M, N) bytes the call
+ * splits K over all SMs, so that the whole weight is streamed at once even
+ * though C has few tiles; partial sums meet in the workspace in fp32 (their
+ * order of addition, hence the last bits of C, may vary from run to run).
+ * The workspace is caller-owned device memory, 16-byte aligned, and must be
+ * zero-filled before its first use; every call that returns SAMBA_OK and
+ * completes without a device error leaves it zero-filled again, so one
+ * workspace serves any number of calls made one after another (on one
+ * stream, or otherwise ordered).  Calls that may run at the same time need
+ * workspaces of their own.  After a call whose status word reports an error
+ * its content is undefined: fill it with zeros again.  Without a workspace
+ * (NULL, or fewer bytes) the call tiles C as usual.
  * Errors: SAMBA_ERR_INVALID_ARG for a missing operand or output, a
  * non-positive size, a stride below its row length or not a multiple of 8, an
- * empty or out-of-range column range or a misaligned pointer;
+ * empty or out-of-range column range or a misaligned pointer (workspace
+ * included);
  * SAMBA_ERR_UNSUPPORTED for M above 65535 * 128, N or K above 2^31 - 1, an
  * output dtype other than SAMBA_F32 / SAMBA_BF16, or nout outside 1..3.
  */
@@ -378,9 +393,15 @@ typedef struct samba_gemm_args {
   int64_t M, N, K;
   samba_gemm_out out[3];
   int32_t nout;
+  void* workspace;         /* NULL, or samba_gemm_workspace_size() bytes (see above) */
+  size_t workspace_bytes;
 } samba_gemm_args;
 
 int samba_gemm(const samba_gemm_args* args, samba_stream_t stream);
+
+/* Bytes of workspace the split-K form of samba_gemm needs for M rows and N
+ * columns (for M <= 32; 0 otherwise, when no workspace is used). */
+size_t samba_gemm_workspace_size(int64_t M, int64_t N);
 
 /* ------------------------------------------------------------ mixer prefill
  * One Mamba mixer (scan) and one SWA mixer on their own inputs (the two token
@@ -467,7 +488,7 @@ int samba_swa_step(const void* q_t, const void* k_t, const void* v_t, void* k_ri
  * process exits.  Calls whose partials do not fit, that is
  * samba_swa_step_workspace_size(batch, heads_q, head_dim, window) > 4 MiB,
  * are rejected with SAMBA_ERR_WORKSPACE before anything is launched; the
- * 16 x 32-head, d = 64, W = 2048 decode needs 1.08 MB.
+ * 16 x 32-head, d = 64, W = 2048 decode needs 2.16 MB.
  *
  * Every call looks up the array's device address (cudaGetSymbolAddress) on
  * the current device; this is a table lookup once the library's device code

@@ -194,12 +194,13 @@ def test_swa_step_noalloc_checks_on_host(lib):
 def test_gemm_rejects_bad_arguments_on_host(lib):
     f = 0x80000
 
-    def call(M=128, N=256, K=64, lda=64, ldb=64, nout=1, ptr=f, col0=0, col1=256, ld=256, dtype=1, A=f):
+    def call(M=128, N=256, K=64, lda=64, ldb=64, nout=1, ptr=f, col0=0, col1=256, ld=256, dtype=1, A=f, ws=None):
         a = L.GemmArgs()
         a.A, a.B, a.lda, a.ldb, a.M, a.N, a.K = A, f, lda, ldb, M, N, K
         o = a.out[0]
         o.ptr, o.bias, o.ld, o.col0, o.col1, o.dtype = ptr, None, ld, col0, col1, dtype
         a.nout = nout
+        a.workspace, a.workspace_bytes = ws, 1 << 20
         return lib.samba_gemm(ctypes.byref(a), None)
 
     assert call(A=None) == L.SAMBA_ERR_INVALID_ARG
@@ -215,6 +216,21 @@ def test_gemm_rejects_bad_arguments_on_host(lib):
     assert call(ld=100) == L.SAMBA_ERR_INVALID_ARG          # row stride below the range
     assert call(dtype=7) == L.SAMBA_ERR_UNSUPPORTED
     assert call(M=65535 * 128 + 1) == L.SAMBA_ERR_UNSUPPORTED
+    assert call(M=16, ws=f + 4) == L.SAMBA_ERR_INVALID_ARG    # misaligned workspace
+
+
+def test_gemm_workspace_size(lib):
+    """fp32 partial sums for 128-row blocks of the weight x 16 or 32 rows, and
+    four counters per block, rounded up to 256 bytes; none above 32 rows."""
+    def want(M, N):
+        nblk = -(-N // 128)
+        mp = 16 if M <= 16 else 32
+        return -(-(nblk * 128 * mp * 4 + nblk * 16) // 256) * 256
+
+    for M, N in ((1, 1), (16, 8192), (17, 160), (32, 4096), (3, 129)):
+        assert lib.samba_gemm_workspace_size(M, N) == want(M, N)
+    assert lib.samba_gemm_workspace_size(33, 4096) == 0
+    assert lib.samba_gemm_workspace_size(0, 4096) == 0
 
 
 def test_scan_bwd_rejects_bad_arguments_on_host(lib):

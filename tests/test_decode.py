@@ -76,17 +76,31 @@ def test_prefill_then_scan_steps_match_oracle(dt, N):
 
 
 # ------------------------------------------------------------------ SWA step
-@pytest.mark.parametrize("L1,W,Hq,Hkv,d", [(10, 16, 8, 2, 64), (40, 16, 4, 4, 32), (300, 256, 32, 4, 64),
-                                           (1, 700, 8, 1, 64), (600, 300, 16, 1, 16), (200, 150, 8, 2, 128)])
-def test_ring_fill_then_swa_steps_match_oracle(L1, W, Hq, Hkv, d):
-    Bsz, steps = 2, 24
+@pytest.mark.parametrize("L1,W,Hq,Hkv,d,Bsz,poison", [
+    (10, 16, 8, 2, 64, 2, False), (40, 16, 4, 4, 32, 2, False), (300, 256, 32, 4, 64, 2, False),
+    (1, 700, 8, 1, 64, 2, False), (600, 300, 16, 1, 16, 2, False), (200, 150, 8, 2, 128, 2, False),
+    # slots past the newest position start as NaN: they hold no position and
+    # must not reach the output
+    (5, 300, 8, 2, 64, 3, True), (100, 2048, 32, 4, 64, 16, True), (3, 64, 4, 1, 128, 2, True),
+    # a full 2048-slot ring at the decode batch width: several splits of
+    # several sub-chunks per CTA
+    (2100, 2048, 32, 4, 64, 16, False),
+    # one sequence over a long ring: many splits
+    (9000, 8192, 8, 1, 64, 1, False),
+])
+def test_ring_fill_then_swa_steps_match_oracle(L1, W, Hq, Hkv, d, Bsz, poison):
+    steps = 24
     g = torch.Generator(device="cuda")
     g.manual_seed(L1 + W)
     Ln = L1 + steps
     q = torch.randn((Bsz, Ln, Hq, d), generator=g, device="cuda").to(torch.bfloat16)
     k = torch.randn((Bsz, Ln, Hkv, d), generator=g, device="cuda").to(torch.bfloat16)
     v = torch.randn((Bsz, Ln, Hkv, d), generator=g, device="cuda").to(torch.bfloat16)
-    kr, vr, pos = ops.swa_ring_fill(k[:, :L1].contiguous(), v[:, :L1].contiguous(), W)
+    kr = vr = None
+    if poison:
+        kr = torch.full((Bsz, W, Hkv, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+        vr = torch.full((Bsz, W, Hkv, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    kr, vr, pos = ops.swa_ring_fill(k[:, :L1].contiguous(), v[:, :L1].contiguous(), W, k_ring=kr, v_ring=vr)
     rk, rv, rpos = orc.ring_fill(host64(k[:, :L1]), host64(v[:, :L1]), W)
     full, _ = orc.swa(host64(q), host64(k), host64(v), W)
     ws = torch.zeros((ops.swa_step_workspace_size(Bsz, Hq, d, W),), dtype=torch.uint8, device="cuda")
@@ -104,6 +118,29 @@ def test_ring_fill_then_swa_steps_match_oracle(L1, W, Hq, Hkv, d):
     slots = [p % W for p in range(Ln - keep, Ln)]
     np.testing.assert_array_equal(host64(kr)[:, slots], rk[:, slots])
     np.testing.assert_array_equal(host64(vr)[:, slots], rv[:, slots])
+    if poison and Ln < W:    # the slots never written keep their NaN
+        assert torch.isnan(kr[:, Ln:].float()).all() and torch.isnan(vr[:, Ln:].float()).all()
+
+
+def test_swa_step_at_a_large_batch():
+    """16384 sequences of one step (a grid of 65536 split CTAs): sampled
+    sequences against the oracle, every pos advanced."""
+    Bsz, Hq, Hkv, d, W, L1 = 16384, 8, 4, 16, 200, 150
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    k = torch.randn((Bsz, L1 + 1, Hkv, d), generator=g, device="cuda").to(torch.bfloat16)
+    v = torch.randn((Bsz, L1 + 1, Hkv, d), generator=g, device="cuda").to(torch.bfloat16)
+    q = torch.randn((Bsz, Hq, d), generator=g, device="cuda").to(torch.bfloat16)
+    kr, vr, pos = ops.swa_ring_fill(k[:, :L1].contiguous(), v[:, :L1].contiguous(), W)
+    o_t = ops.swa_step(q, k[:, L1].contiguous(), v[:, L1].contiguous(), kr, vr, pos, W)
+    torch.cuda.synchronize()
+    assert ops.get_status() == 0
+    assert torch.equal(pos.cpu(), torch.full((Bsz,), L1 + 1, dtype=torch.int64))
+    for b in (0, 1, 777, 8191, 16383):
+        full, _ = orc.swa(host64(q[b:b + 1, None].expand(1, L1 + 1, Hq, d).contiguous()), host64(k[b:b + 1]),
+                          host64(v[b:b + 1]), W)
+        err = np.abs(host64(o_t[b]) - full[0, L1])
+        assert err.max() <= SWA_MAX_ABS, (b, err.max())
 
 
 def test_decode_checkpoint_restore_is_bit_identical():

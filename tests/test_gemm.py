@@ -97,3 +97,66 @@ def test_in_projection_split_into_x_and_z():
     ref, mag = A64 @ W64.T, np.abs(A64) @ np.abs(W64).T
     _check(x, ref[:, :D], mag[:, :D], torch.bfloat16, "gemm in-proj x")
     _check(z, ref[:, D:], mag[:, D:], torch.bfloat16, "gemm in-proj z")
+
+
+# ----------------------------------------------------------- split-K (M <= 32)
+@pytest.mark.parametrize("M,N,K,dt", [
+    (16, 8192, 2048, torch.bfloat16),   # Mamba input projection, 16 sequences decoding
+    (16, 160, 4096, torch.float32),     # selective-parameter projection: 2 blocks of the weight, 64 k-steps each
+    (16, 4096, 128, torch.float32),     # Δ up-projection: two k-steps per block
+    (16, 2048, 4096, torch.bfloat16),   # Mamba output projection
+    (1, 2560, 2048, torch.bfloat16),    # one sequence
+    (3, 300, 200, torch.float32),       # ragged N and K (K not a multiple of 64)
+    (17, 1000, 64, torch.bfloat16),     # 17 rows: the 32-row form; one k-step per block (direct store)
+    (32, 777, 4104, torch.float32),     # 32 rows, ragged everything
+])
+def test_split_k_gemm_matches_float64_and_leaves_the_workspace_zero(M, N, K, dt):
+    a, w = _operands(M, N, K, 3 * M + N + K, lda=(K + 7) // 8 * 8)
+    nbytes = ops.gemm_workspace_size(M, N)
+    assert nbytes > 0
+    ws = torch.zeros((nbytes,), dtype=torch.uint8, device="cuda")
+    A64, W64 = host64(a), host64(w)
+    ref, mag = A64 @ W64.T, np.abs(A64) @ np.abs(W64).T
+    for rep in range(3):      # the same workspace, call after call
+        c = torch.full((M, N), float("nan"), dtype=dt, device="cuda")
+        ops.gemm(a, w, outs=[(c, 0, N, None)], workspace=ws)
+        torch.cuda.synchronize()
+        assert ops.get_status() == 0
+        _check(c, ref, mag, dt, f"split-K gemm {M}x{N}x{K} call {rep}")
+        assert int(torch.count_nonzero(ws)) == 0, "workspace not returned to zero"
+
+
+def test_split_k_column_split_with_bias():
+    """The decode form of the selective-parameter projection: three column
+    ranges (bf16; fp32 with a bias; fp32 into a wider matrix) from 16 rows."""
+    M, N, K = 16, 160, 4096
+    a, w = _operands(M, N, K, 21, lda=K + 64)
+    ws = torch.zeros((ops.gemm_workspace_size(M, N),), dtype=torch.uint8, device="cuda")
+    dt_low = torch.full((M, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    bias = torch.randn((16,), device="cuda")
+    Bm = torch.full((M, 16), float("nan"), device="cuda")
+    wide = torch.full((M, 40), float("nan"), device="cuda")
+    Cm = wide[:, 8:24]
+    ops.gemm(a, w, outs=[(dt_low, 0, 128, None), (Bm, 128, 144, bias), (Cm, 144, 160, None)], workspace=ws)
+    torch.cuda.synchronize()
+    assert ops.get_status() == 0
+    A64, W64 = host64(a), host64(w)
+    ref, mag = A64 @ W64.T, np.abs(A64) @ np.abs(W64).T
+    _check(dt_low, ref[:, :128], mag[:, :128], torch.bfloat16, "split-K split dt_low")
+    _check(Bm, ref[:, 128:144] + host64(bias), mag[:, 128:144], torch.float32, "split-K split B")
+    _check(Cm, ref[:, 144:], mag[:, 144:], torch.float32, "split-K split C")
+    assert torch.isnan(wide[:, :8]).all() and torch.isnan(wide[:, 24:]).all()
+    assert int(torch.count_nonzero(ws)) == 0
+
+
+def test_split_k_agrees_with_the_tiled_form():
+    """The same 16-row product with and without a workspace: the two forms
+    add the k-steps in different orders, so they agree to fp32 rounding."""
+    M, N, K = 16, 4096, 2048
+    a, w = _operands(M, N, K, 22)
+    ws = torch.zeros((ops.gemm_workspace_size(M, N),), dtype=torch.uint8, device="cuda")
+    c1 = ops.gemm(a, w, out_dtype=torch.float32, workspace=ws)
+    c2 = ops.gemm(a, w, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    mag = host64(a).__abs__() @ host64(w).__abs__().T
+    assert np.max(np.abs(host64(c1) - host64(c2)) / (1e-5 * mag)) <= 1.0

@@ -54,18 +54,20 @@ def _swa_ref(hidden, w):
                          w.window)
 
 
-@pytest.mark.parametrize("Bsz,Ln,s,dm,D,N,R", [
-    (2, 100, 6, 256, 512, 16, 32),     # batch 2, a ragged prompt
-    (16, 33, 4, 128, 256, 8, 16),      # the decode batch width of the serving workload
-    (1, 1, 5, 128, 256, 16, 16),       # a one-token prompt: the conv state is mostly the zero start
-    (3, 64, 130, 64, 128, 16, 8),      # more steps than prompt tokens
+@pytest.mark.parametrize("Bsz,Ln,s,dm,D,N,R,split_k", [
+    (2, 100, 6, 256, 512, 16, 32, True),     # batch 2, a ragged prompt
+    (16, 33, 4, 128, 256, 8, 16, True),      # the decode batch width of the serving workload
+    (16, 33, 4, 128, 256, 8, 16, False),     # the same with tiled projections
+    (1, 1, 5, 128, 256, 16, 16, True),       # a one-token prompt: the conv state is mostly the zero start
+    (3, 64, 130, 64, 128, 16, 8, True),      # more steps than prompt tokens
+    (40, 20, 3, 128, 256, 16, 16, True),     # above 32 sequences: tiled projections
 ])
-def test_mamba_layer_step_continues_the_prefill(Bsz, Ln, s, dm, D, N, R):
+def test_mamba_layer_step_continues_the_prefill(Bsz, Ln, s, dm, D, N, R, split_k):
     w = layers.random_mamba_weights(dm, D, N, 4, R, seed=7 * Ln + s)
     hidden = _hidden(Bsz, Ln + s, dm, Ln + s)
     out_p, h_final, cs = layers.mamba_layer_prefill(hidden[:, :Ln].contiguous(), w)
     h_pre = h_final.clone()
-    st = layers.mamba_decode_state(h_final, cs)
+    st = layers.mamba_decode_state(h_final, cs, w, split_k=split_k)
     outs, taps = [], []
     for j in range(s):
         taps.append({})
@@ -106,7 +108,7 @@ def test_swa_layer_step_continues_the_prefill(Bsz, Ln, s, dm, Hq, Hkv, d, W):
     w = layers.random_swa_weights(dm, Hq, Hkv, d, W, seed=Ln + W + s)
     hidden = _hidden(Bsz, Ln + s, dm, Ln + 3 * s)
     out_p, k, v = layers.swa_layer_prefill(hidden[:, :Ln].contiguous(), w)
-    st = layers.swa_decode_state(k, v, W, Hq)
+    st = layers.swa_decode_state(k, v, w)
     outs = [layers.swa_layer_step(hidden[:, Ln + j].contiguous(), w, st) for j in range(s)]
     torch.cuda.synchronize()
     assert ops.get_status() == 0
@@ -144,10 +146,10 @@ def test_layer_stack_serving_loop():
         seen[i].append(h)
         if kind == "mamba":
             out, hf, cs = layers.mamba_layer_prefill(h, w)
-            states.append(layers.mamba_decode_state(hf, cs))
+            states.append(layers.mamba_decode_state(hf, cs, w))
         else:
             out, k, v = layers.swa_layer_prefill(h, w)
-            states.append(layers.swa_decode_state(k, v, W, Hq))
+            states.append(layers.swa_decode_state(k, v, w))
         got[i].append(out)
         h = out
     for j in range(s):
@@ -169,7 +171,10 @@ def test_layer_stack_serving_loop():
 def test_decode_steps_replay_in_a_cuda_graph():
     """The steps of one Mamba + SWA pair captured in a CUDA graph of four
     steps and replayed twice give the outputs of the same eight steps run
-    eagerly (state buffers stay in place, so the capture is valid)."""
+    eagerly (state buffers stay in place, so the capture is valid).  The
+    split-K projections add their partial sums in an order that varies from
+    run to run, so the two agree to rounding, not bit for bit: within one
+    bf16 unit plus 1e-2 of the output rms, the layer tests' bound."""
     Bsz, Ln, dm, D, N, R = 16, 64, 128, 256, 16, 16
     Hq, Hkv, d, W = 4, 1, 64, 32
     mw = layers.random_mamba_weights(dm, D, N, 4, R, seed=11)
@@ -179,7 +184,7 @@ def test_decode_steps_replay_in_a_cuda_graph():
     def fresh():
         out, hf, cs = layers.mamba_layer_prefill(tokens[:, :Ln].contiguous(), mw)
         _, k, v = layers.swa_layer_prefill(out, sw)
-        return layers.mamba_decode_state(hf, cs), layers.swa_decode_state(k, v, W, Hq)
+        return layers.mamba_decode_state(hf, cs, mw), layers.swa_decode_state(k, v, sw)
 
     ms, ss = fresh()
     eager = []
@@ -208,4 +213,6 @@ def test_decode_steps_replay_in_a_cuda_graph():
     torch.cuda.synchronize()
     assert ops.get_status() == 0
     for a, b in zip(eager, graphed):
-        assert torch.equal(a, b)
+        a, b = host64(a), host64(b)
+        rms = float(np.sqrt(np.mean(b * b)))
+        assert np.max(np.abs(a - b) / (2.0 ** -7 * np.abs(b) + 1e-2 * rms)) <= 1.0
