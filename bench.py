@@ -720,7 +720,8 @@ def run_serve(args, wl, dev, rank, world):
     y_out = torch.empty((Bsz, D), dtype=torch.bfloat16, device=dev)
     o_out = torch.empty((Bsz, wl.heads_q, wl.head_dim), dtype=torch.bfloat16, device=dev)
     delta_in = torch.full((Bsz, D), -3.0, device=dev)
-    bc_in = torch.randn((Bsz, 2 * N), generator=g, device=dev)
+    b_in = torch.randn((Bsz, N), generator=g, device=dev)
+    c_in = torch.randn((Bsz, N), generator=g, device=dev)
     q_in, kv_in = bf(Bsz, wl.heads_q, wl.head_dim), bf(Bsz, wl.heads_kv, wl.head_dim)
     kernels = {
         "in_proj": lambda i: ops.gemm(x_in, mam[i].in_proj, outs=[(xz_out, 0, 2 * D, None)],
@@ -738,8 +739,8 @@ def run_serve(args, wl, dev, rank, world):
         "conv": lambda i: ops.conv1d_fwd(u_in.view(Bsz, 1, D), mam[i].conv_w, mam[i].conv_b,
                                          conv_state_in=mst[i].conv, conv_state_out=mst[i].conv,
                                          u=u_out.view(Bsz, 1, D)),
-        "scan_step": lambda i: ops.scan_step(mst[i].h, None, u_in, delta_in, mam[i].A, bc_in[:, :N].contiguous(),
-                                             bc_in[:, N:].contiguous(), D=mam[i].D, z_t=y_in, y_t=y_out),
+        "scan_step": lambda i: ops.scan_step(mst[i].h, None, u_in, delta_in, mam[i].A, b_in, c_in, D=mam[i].D,
+                                             z_t=y_in, y_t=y_out),
         "swa_step": lambda i: ops.swa_step(q_in, kv_in, kv_in, sst[i].k_ring, sst[i].v_ring, sst[i].pos, W,
                                            o_t=o_out, workspace=sst[i].workspace),
     }

@@ -122,6 +122,52 @@ def test_ring_fill_then_swa_steps_match_oracle(L1, W, Hq, Hkv, d, Bsz, poison):
         assert torch.isnan(kr[:, Ln:].float()).all() and torch.isnan(vr[:, Ln:].float()).all()
 
 
+@pytest.mark.parametrize("Bsz,Hq,Hkv,d,W,L1", [(1, 8, 2, 64, 256, 300), (2, 4, 1, 32, 64, 20), (1, 16, 4, 64, 2048, 2100)])
+@pytest.mark.parametrize("graph", [False, True])
+def test_back_to_back_swa_steps_on_one_ring(Bsz, Hq, Hkv, d, W, L1, graph):
+    """Steps on the same ring launched one right after the other (all inputs
+    prepared beforehand, nothing else on the stream in between), eagerly and
+    captured in a CUDA graph: each step starts reading the ring before the
+    previous one has finished, and must still see the key that step wrote."""
+    steps = 40
+    g = torch.Generator(device="cuda")
+    g.manual_seed(Bsz * 100 + W)
+    Ln = L1 + steps
+    q = torch.randn((Bsz, Ln, Hq, d), generator=g, device="cuda").to(torch.bfloat16)
+    k = torch.randn((Bsz, Ln, Hkv, d), generator=g, device="cuda").to(torch.bfloat16)
+    v = torch.randn((Bsz, Ln, Hkv, d), generator=g, device="cuda").to(torch.bfloat16)
+    kr, vr, pos = ops.swa_ring_fill(k[:, :L1].contiguous(), v[:, :L1].contiguous(), W)
+    ins = [(q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous()) for t in range(L1, Ln)]
+    outs = [torch.empty((Bsz, Hq, d), dtype=torch.bfloat16, device="cuda") for _ in ins]
+    ws = torch.empty((ops.swa_step_workspace_size(Bsz, Hq, d, W),), dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+
+    def run():
+        for (qt, kt, vt), ot in zip(ins, outs):
+            ops.swa_step(qt, kt, vt, kr, vr, pos, W, o_t=ot, workspace=ws)
+
+    if graph:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        gr = torch.cuda.CUDAGraph()
+        kr0, vr0, pos0 = kr.clone(), vr.clone(), pos.clone()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(gr, stream=side):
+                run()
+        torch.cuda.current_stream().wait_stream(side)
+        kr.copy_(kr0), vr.copy_(vr0), pos.copy_(pos0)   # the capture ran nothing; restore to be safe
+        gr.replay()
+    else:
+        run()
+    torch.cuda.synchronize()
+    assert ops.get_status() == 0
+    assert torch.equal(pos.cpu(), torch.full((Bsz,), Ln, dtype=torch.int64))
+    full, _ = orc.swa(host64(q), host64(k), host64(v), W)
+    for i, t in enumerate(range(L1, Ln)):
+        err = np.abs(host64(outs[i]) - full[:, t])
+        assert err.max() <= SWA_MAX_ABS and err.mean() <= SWA_MEAN_ABS, (t, err.max())
+
+
 def test_swa_step_at_a_large_batch():
     """16384 sequences of one step (a grid of 65536 split CTAs): sampled
     sequences against the oracle, every pos advanced."""
