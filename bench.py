@@ -879,15 +879,18 @@ def run_train(args, wl, dev, rank, world):
     ws_scan = torch.empty((ops.scan_bwd_workspace_size(Bsz, Ln, D, N),), dtype=torch.uint8, device=dev)
     ws_swa = torch.empty((ops.swa_bwd_workspace_size(Bsz, Ln, wl.heads_q),), dtype=torch.uint8, device=dev)
     scan_in = dict(D=inp["D"], z=inp["z"], conv_w=inp["conv_w"], conv_b=inp["conv_b"])
+    # the forward stores the state at every 16-token chunk start; the
+    # backward starts its chunks from them instead of recomputing them
+    ckpt = torch.empty(ops.scan_ckpt_shape(Bsz, Ln, D, N), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
     def fwd():
-        ops.selective_scan_fwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], y=y, **scan_in)
+        ops.selective_scan_fwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], y=y, h_ckpt=ckpt, **scan_in)
         ops.swa_fwd(inp["q"], inp["k"], inp["v"], wl.window, o=o, lse=lse)
 
     def bwd_scan():
         return ops.selective_scan_bwd(grads["dy"], inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"],
-                                      workspace=ws_scan, **scan_in)
+                                      workspace=ws_scan, ckpt=ckpt, **scan_in)
 
     def bwd_swa():
         ops.swa_bwd(grads["do"], inp["q"], inp["k"], inp["v"], o, lse, wl.window, dq=dq, dk=dk, dv=dv,
@@ -950,7 +953,8 @@ def run_train(args, wl, dev, rank, world):
     roof = {k: kernels[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
     roof["kernel"] = "scan_bwd_kernel" if dom == "scan_bwd" else "swa_bwd_kv_kernel + swa_bwd_q_kernel"
     cfg = workload_config(wl)
-    cfg["step"] = "scan and SWA forward (with log-sum-exp), then scan and SWA backward from seeded dy, dO"
+    cfg["step"] = ("scan and SWA forward (with log-sum-exp and the scan's 16-token state checkpoints), then scan "
+                   "and SWA backward from seeded dy, dO")
     return {
         "metric": TRAIN_METRIC, "value": whole_job_rate(wl.batch * wl.seqlen, world, ms_step), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,

@@ -33,7 +33,7 @@ class ScanArgs(ctypes.Structure):
         ("conv_state_out", _vp), ("h0", _vp), ("h_final", _vp), ("y", _vp),
         ("batch", _i64), ("seqlen", _i64), ("dim", _i64),
         ("dstate", _i32), ("dconv", _i32), ("x_dtype", _i32), ("z_dtype", _i32), ("y_dtype", _i32),
-        ("flags", ctypes.c_uint32), ("delta_sum", _vp),
+        ("flags", ctypes.c_uint32), ("delta_sum", _vp), ("h_ckpt", _vp),
     ]
 
 
@@ -46,7 +46,7 @@ class ScanBwdArgs(ctypes.Structure):
         ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
         ("batch", _i64), ("seqlen", _i64), ("dim", _i64),
         ("dstate", _i32), ("dconv", _i32), ("x_dtype", _i32), ("z_dtype", _i32), ("y_dtype", _i32),
-        ("flags", ctypes.c_uint32),
+        ("flags", ctypes.c_uint32), ("ckpt", _vp),
     ]
 
 

@@ -17,7 +17,8 @@
 // scan warps do.  The walk needs h_{t-1} in reverse order, so it is
 // recomputed: a first pass runs the recurrence forward over the whole
 // sequence and stores the state at the start of every 16-token chunk in the
-// workspace; the reverse pass then takes the chunks last to first, recomputes
+// workspace (or the forward kernel has stored them, and the pass is
+// skipped); the reverse pass then takes the chunks last to first, recomputes
 // the chunk's 16 states into shared memory from its checkpoint, and walks it
 // backwards.  Per chunk, all 128 threads share the per-(token, channel) work
 // (conv, softplus, gate, and their gradients) with thread = (channel, token
@@ -136,7 +137,8 @@ struct ScanBwdParams {
   float* dconv_b;
   float* dh0;
   float* dconv_state;
-  float* ckpt;  // [B, nchunks, N, D]
+  float* ckpt;  // [B, nchunks, N, D]: the workspace's, or the forward's
+  bool ckpt_given;  // the forward wrote ckpt: no first pass
   float* part;  // [D/32 blocks][2 (dB, dC)][B, L, N]
   int64_t L, D;
   int K;
@@ -326,8 +328,8 @@ __global__ void __launch_bounds__(32 * nwarps(N), 3) scan_bwd_kernel(const ScanB
   float h[SPL];
 #pragma unroll
   for (int j = 0; j < SPL; ++j) h[j] = (p.h0 && lane_ok) ? p.h0[(b * D + ch_l) * N + warp * SPL + j] : 0.f;
-  fetch(0, false, R);
-  for (int c = 0; c < p.nchunks; ++c) {
+  if (!p.ckpt_given) fetch(0, false, R);
+  for (int c = 0; c < (p.ckpt_given ? 0 : p.nchunks); ++c) {
     const int nv = chunk_len(c);
     stage(c, false, R);
     if (c + 1 < p.nchunks) fetch(c + 1, false, R);
@@ -637,7 +639,8 @@ int launch_scan_bwd(const samba_scan_bwd_args& a, cudaStream_t s) {
   p.dconv_b = a.dconv_b;
   p.dh0 = a.dh0;
   p.dconv_state = a.dconv_state;
-  p.ckpt = reinterpret_cast<float*>(a.workspace);
+  p.ckpt = a.ckpt ? const_cast<float*>(a.ckpt) : reinterpret_cast<float*>(a.workspace);
+  p.ckpt_given = a.ckpt != nullptr;
   p.part = reinterpret_cast<float*>(static_cast<unsigned char*>(a.workspace) +
                                     ckpt_bytes(a.batch, a.seqlen, a.dim, a.dstate));
   p.L = a.seqlen;

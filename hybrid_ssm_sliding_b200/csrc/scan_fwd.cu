@@ -61,6 +61,8 @@ struct ScanParams {
   const float* h0;
   float* h_final;
   float* delta_sum;  // [B, D] sum over t of Δ, or null
+  float* h_ckpt;     // [B, nck, N, D] state at the start of every 16-token chunk, or null
+  int nck;           // ceil(L / 16)
   const void* x;  // for the conv state at the end
   void* y;
   int64_t L, D;
@@ -217,7 +219,7 @@ __device__ __forceinline__ float softplus_fast(float w) {
 //   epilogue : y <- (Σ PART[k] + D·u)·silu(z); arrives epi_done[k]
 //              (waits scan_done[k])
 // empty[s] collects the prologue and scan warps (the readers of stage s).
-template <int N, typename XT, typename YT, int POLY>
+template <int N, typename XT, typename YT, int POLY, bool CKPT>
 __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
     scan_fwd_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_z,
                     const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_b,
@@ -491,6 +493,19 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
     a2p[q] = pk2(a[0], a[1]);
     hp[q] = pk2(hh[0], hh[1]);
   }
+  // checkpoint cidx: the state before token 16 * cidx ([b][cidx][n][D])
+  auto store_ckpt = [&](int64_t cidx) {
+    if (!cval || cidx >= p.nck) return;
+    float* dst = p.h_ckpt + ((int64_t)b * p.nck + cidx) * N * p.D + c;
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+      const float2 hv = up2(hp[q]);
+      dst[(int64_t)(n0 + 2 * q) * p.D] = hv.x;
+      if (2 * q + 1 < NS) dst[(int64_t)(n0 + 2 * q + 1) * p.D] = hv.y;
+    }
+  };
+  static_assert(T % 16 == 0, "tiles hold whole 16-token chunks");
+  if constexpr (CKPT) store_ckpt(0);
 
   for (int i = 0; i < ntiles; ++i) {
     const int s = i % STAGES, k = i % SLOTS, r = i / SLOTS;
@@ -590,6 +605,9 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
 #pragma unroll
         for (int q = 0; q < G; ++q)
           if (cown) part[(tg0 + q) * CB * GL] = pv[q];  // idle lanes would alias other channels
+        if constexpr (CKPT) {
+          if ((tg0 + G) % 16 == 0) store_ckpt(((int64_t)i * T + tg0 + G) / 16);
+        }
       }
     }
     __syncwarp();
@@ -638,11 +656,13 @@ static int choose_cu(int64_t B, int64_t D) {
   return best;
 }
 
-template <int N, typename XT, typename YT>
+// CKPT: the variant that also stores the chunk checkpoints (a separate
+// instantiation, so that the kernel without them is unchanged).
+template <int N, typename XT, typename YT, bool CKPT>
 static int launch_scan_t(const samba_scan_args& a, cudaStream_t stream) {
   using Ly = ScanLayout<N, XT>;
   constexpr int POLY = SAMBA_SCAN_POLY;
-  auto kern = scan_fwd_kernel<N, XT, YT, POLY>;
+  auto kern = scan_fwd_kernel<N, XT, YT, POLY, CKPT>;
   static PerDeviceOnce attr;
   const int arc = once_per_device(attr, [&] {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::SMEM) == cudaSuccess
@@ -686,6 +706,8 @@ static int launch_scan_t(const samba_scan_args& a, cudaStream_t stream) {
   p.h0 = a.h0;
   p.h_final = a.h_final;
   p.delta_sum = a.delta_sum;
+  p.h_ckpt = a.h_ckpt;
+  p.nck = static_cast<int>((a.seqlen + 15) / 16);
   p.x = a.x;
   p.y = a.y;
   p.L = a.seqlen;
@@ -705,13 +727,18 @@ static int launch_scan_t(const samba_scan_args& a, cudaStream_t stream) {
   return check_launch("samba_selective_scan_fwd");
 }
 
+template <int N, bool CKPT>
+static int launch_scan_c(const samba_scan_args& a, cudaStream_t s) {
+  const bool xb = a.x_dtype == SAMBA_BF16, yb = a.y_dtype == SAMBA_BF16;
+  if (xb && yb) return launch_scan_t<N, __nv_bfloat16, __nv_bfloat16, CKPT>(a, s);
+  if (xb && !yb) return launch_scan_t<N, __nv_bfloat16, float, CKPT>(a, s);
+  if (!xb && yb) return launch_scan_t<N, float, __nv_bfloat16, CKPT>(a, s);
+  return launch_scan_t<N, float, float, CKPT>(a, s);
+}
+
 template <int N>
 static int launch_scan_n(const samba_scan_args& a, cudaStream_t s) {
-  const bool xb = a.x_dtype == SAMBA_BF16, yb = a.y_dtype == SAMBA_BF16;
-  if (xb && yb) return launch_scan_t<N, __nv_bfloat16, __nv_bfloat16>(a, s);
-  if (xb && !yb) return launch_scan_t<N, __nv_bfloat16, float>(a, s);
-  if (!xb && yb) return launch_scan_t<N, float, __nv_bfloat16>(a, s);
-  return launch_scan_t<N, float, float>(a, s);
+  return a.h_ckpt ? launch_scan_c<N, true>(a, s) : launch_scan_c<N, false>(a, s);
 }
 
 int launch_scan(const samba_scan_args& a, cudaStream_t s) {

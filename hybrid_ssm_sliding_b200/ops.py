@@ -63,9 +63,14 @@ def conv1d_fwd(x, w, bias=None, conv_state_in=None, silu=True, u=None, u_dtype=N
     return u
 
 
+def scan_ckpt_shape(batch, seqlen, dim, dstate):
+    """Shape of the forward's chunk checkpoints (samba_scan_args.h_ckpt)."""
+    return (batch, (seqlen + 15) // 16, dstate, dim)
+
+
 def _scan_struct(x, delta, A, B, C, D=None, z=None, conv_w=None, conv_b=None, conv_state_in=None,
                  h0=None, y=None, y_dtype=None, h_final=None, conv_state_out=None,
-                 delta_softplus=True, conv_silu=True, fuse_conv=None, delta_sum=None):
+                 delta_softplus=True, conv_silu=True, fuse_conv=None, delta_sum=None, h_ckpt=None):
     _need(x, "x")
     Bsz, Ln, Dm = x.shape
     N = A.shape[1]
@@ -85,6 +90,7 @@ def _scan_struct(x, delta, A, B, C, D=None, z=None, conv_w=None, conv_b=None, co
     _opt(h0, "h0", torch.float32, (Bsz, Dm, N))
     _opt(h_final, "h_final", torch.float32, (Bsz, Dm, N))
     _opt(delta_sum, "delta_sum", torch.float32, (Bsz, Dm))
+    _opt(h_ckpt, "h_ckpt", torch.float32, scan_ckpt_shape(Bsz, Ln, Dm, N))
     if y is None:
         y = torch.empty_like(x, dtype=y_dtype or x.dtype)
     _need(y, "y", None, x.shape)
@@ -93,16 +99,19 @@ def _scan_struct(x, delta, A, B, C, D=None, z=None, conv_w=None, conv_b=None, co
     a = L.ScanArgs(L.ptr(x), L.ptr(z), L.ptr(delta), L.ptr(A), L.ptr(B), L.ptr(C), L.ptr(D), L.ptr(conv_w),
                    L.ptr(conv_b), L.ptr(conv_state_in), L.ptr(conv_state_out), L.ptr(h0), L.ptr(h_final),
                    L.ptr(y), Bsz, Ln, Dm, N, K, L.dtype_code(x), L.dtype_code(z) if z is not None else 0,
-                   L.dtype_code(y), flags, L.ptr(delta_sum))
+                   L.dtype_code(y), flags, L.ptr(delta_sum), L.ptr(h_ckpt))
     return a, y
 
 
 def selective_scan_fwd(x, delta, A, B, C, D=None, z=None, conv_w=None, conv_b=None, conv_state_in=None,
                        h0=None, y=None, y_dtype=None, h_final=None, conv_state_out=None,
-                       delta_softplus=True, conv_silu=True, fuse_conv=None, delta_sum=None, stream=None):
-    """Fused selective-scan prefill (see samba_selective_scan_fwd).  Returns y."""
+                       delta_softplus=True, conv_silu=True, fuse_conv=None, delta_sum=None, h_ckpt=None,
+                       stream=None):
+    """Fused selective-scan prefill (see samba_selective_scan_fwd).  Returns y.
+    ``h_ckpt`` ([B, ceil(L/16), N, D] fp32) receives the state at every
+    16-token chunk start, for selective_scan_bwd(ckpt=...)."""
     a, y = _scan_struct(x, delta, A, B, C, D, z, conv_w, conv_b, conv_state_in, h0, y, y_dtype, h_final,
-                        conv_state_out, delta_softplus, conv_silu, fuse_conv, delta_sum)
+                        conv_state_out, delta_softplus, conv_silu, fuse_conv, delta_sum, h_ckpt)
     L.check(L.load().samba_selective_scan_fwd(ctypes.byref(a), L.stream_handle(stream)))
     return y
 
@@ -113,11 +122,12 @@ def scan_bwd_workspace_size(batch, seqlen, dim, dstate):
 
 def selective_scan_bwd(dy, x, delta, A, B, C, D=None, z=None, conv_w=None, conv_b=None, conv_state_in=None,
                        h0=None, delta_softplus=True, conv_silu=True, fuse_conv=None, want_dh0=False,
-                       want_dconv_state=False, workspace=None, stream=None):
+                       want_dconv_state=False, workspace=None, ckpt=None, stream=None):
     """Gradients of selective_scan_fwd's y given dy (see
     samba_selective_scan_bwd).  Returns a dict with dx, ddelta, dA, dB, dC
     and, where the forward input exists, dz, dD, dconv_w, dconv_b, plus dh0 /
-    dconv_state when asked for."""
+    dconv_state when asked for.  ``ckpt``: the forward's h_ckpt for these
+    inputs (the backward then skips its own checkpoint pass)."""
     _need(x, "x")
     Bsz, Ln, Dm = x.shape
     N = A.shape[1]
@@ -135,6 +145,7 @@ def selective_scan_bwd(dy, x, delta, A, B, C, D=None, z=None, conv_w=None, conv_
     _opt(conv_b, "conv_b", torch.float32, (Dm,))
     _opt(conv_state_in, "conv_state_in", torch.float32, (Bsz, Dm, K - 1))
     _opt(h0, "h0", torch.float32, (Bsz, Dm, N))
+    _opt(ckpt, "ckpt", torch.float32, scan_ckpt_shape(Bsz, Ln, Dm, N))
     dev = x.device
     f32 = dict(dtype=torch.float32, device=dev)
     out = {"dx": torch.empty_like(x), "ddelta": torch.empty((Bsz, Ln, Dm), **f32), "dA": torch.empty((Dm, N), **f32),
@@ -156,7 +167,7 @@ def selective_scan_bwd(dy, x, delta, A, B, C, D=None, z=None, conv_w=None, conv_
                       L.ptr(out["dC"]), L.ptr(out["dD"]), L.ptr(out["dconv_w"]), L.ptr(out["dconv_b"]),
                       L.ptr(out["dh0"]), L.ptr(out["dconv_state"]), L.ptr(workspace),
                       workspace.numel() * workspace.element_size(), Bsz, Ln, Dm, N, K, L.dtype_code(x),
-                      L.dtype_code(z) if z is not None else 0, L.dtype_code(dy), flags)
+                      L.dtype_code(z) if z is not None else 0, L.dtype_code(dy), flags, L.ptr(ckpt))
     L.check(L.load().samba_selective_scan_bwd(ctypes.byref(a), L.stream_handle(stream)))
     return out
 

@@ -163,6 +163,10 @@ typedef struct samba_scan_args {
   int32_t x_dtype, z_dtype, y_dtype;
   uint32_t flags;
   float* delta_sum;            /* [B, D] fp32, or NULL: sum over t of Δ_t     */
+  float* h_ckpt;               /* [B, ceil(L/16), N, D] fp32, or NULL: the
+                                  state at the start of every 16-token chunk
+                                  (h0 for the first), the checkpoints
+                                  samba_selective_scan_bwd can start from     */
 } samba_scan_args;
 
 int samba_selective_scan_fwd(const samba_scan_args* args, samba_stream_t stream);
@@ -181,6 +185,8 @@ int samba_selective_scan_fwd(const samba_scan_args* args, samba_stream_t stream)
  * dconv_b, dconv_state).  The forward states are recomputed: a first pass
  * stores the state at the start of every 16-token chunk in the workspace,
  * then every chunk is recomputed and walked from its last token to its first.
+ * When `ckpt` holds the checkpoints the forward wrote (samba_scan_args.h_ckpt,
+ * same inputs), the first pass is skipped and the chunks start from them.
  *
  * Inputs are those of the forward (same shapes, dtypes and flags; y_dtype is
  * the dtype of dy).  Outputs:
@@ -232,6 +238,8 @@ typedef struct samba_scan_bwd_args {
   int32_t dstate, dconv;
   int32_t x_dtype, z_dtype, y_dtype;
   uint32_t flags;
+  const float* ckpt;           /* NULL, or the forward's h_ckpt for these inputs:
+                                  the first pass is then skipped              */
 } samba_scan_bwd_args;
 
 /* Bytes of workspace samba_selective_scan_bwd needs (the chunk checkpoints,

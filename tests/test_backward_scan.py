@@ -50,12 +50,22 @@ def _check(name, got, ref, bf16_keys=()):
     return worst
 
 
-def _run(inp, dy, with_conv=True, with_z=True, with_D=True, softplus=True, h0=None, cs=None, conv_silu=True):
+def _fwd_ckpt(inp, **kw):
+    """The forward on the same inputs, writing its 16-token chunk checkpoints."""
+    Bsz, Ln, D = inp["x"].shape
+    ck = torch.full(ops.scan_ckpt_shape(Bsz, Ln, D, inp["A"].shape[1]), float("nan"), device="cuda")
+    ops.selective_scan_fwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], h_ckpt=ck, **kw)
+    return ck
+
+
+def _run(inp, dy, with_conv=True, with_z=True, with_D=True, softplus=True, h0=None, cs=None, conv_silu=True,
+         fwd_ckpt=False):
     kw = dict(D=inp["D"] if with_D else None, z=inp["z"] if with_z else None,
               conv_w=inp["conv_w"] if with_conv else None, conv_b=inp["conv_b"] if with_conv else None,
               conv_state_in=cs, h0=h0, delta_softplus=softplus, conv_silu=conv_silu)
+    ck = _fwd_ckpt(inp, **kw) if fwd_ckpt else None
     got = ops.selective_scan_bwd(dy, inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], want_dh0=True,
-                                 want_dconv_state=with_conv, **kw)
+                                 want_dconv_state=with_conv, ckpt=ck, **kw)
     torch.cuda.synchronize()
     assert ops.get_status() == 0
     ref = orc.selective_scan_bwd(host64(dy), host64(inp["x"]), host64(inp["delta"]), host64(inp["A"]),
@@ -75,7 +85,8 @@ def _run(inp, dy, with_conv=True, with_z=True, with_D=True, softplus=True, h0=No
     (1, 300, 64, 16, 4, torch.bfloat16),
     (2, 129, 96, 8, 4, torch.bfloat16),
 ])
-def test_scan_bwd_matches_oracle(Bsz, Ln, D, N, K, dt):
+@pytest.mark.parametrize("fwd_ckpt", [False, True])
+def test_scan_bwd_matches_oracle(Bsz, Ln, D, N, K, dt, fwd_ckpt):
     wl = Workload("sb", Bsz, Ln, D, N, K, 1, 1, 16, 16, 200 + Ln, act_dtype=dt)
     inp = make_prefill_inputs(wl, device="cuda", with_attention=False)
     dy = make_output_grads(wl, device="cuda", with_attention=False)["dy"]
@@ -83,9 +94,9 @@ def test_scan_bwd_matches_oracle(Bsz, Ln, D, N, K, dt):
     g.manual_seed(7)
     h0 = torch.randn((Bsz, D, N), generator=g, device="cuda")
     cs = torch.randn((Bsz, D, K - 1), generator=g, device="cuda")
-    got, ref = _run(inp, dy, h0=h0, cs=cs)
+    got, ref = _run(inp, dy, h0=h0, cs=cs, fwd_ckpt=fwd_ckpt)
     bf = ("dx", "dz") if dt == torch.bfloat16 else ()
-    _check(f"scan bwd B{Bsz} L{Ln} D{D} N{N} K{K} {str(dt)[6:]}", got, ref, bf)
+    _check(f"scan bwd B{Bsz} L{Ln} D{D} N{N} K{K} {str(dt)[6:]}{' fwd ckpt' if fwd_ckpt else ''}", got, ref, bf)
 
 
 @pytest.mark.parametrize("conv,z,Dk,sp,silu", [
@@ -101,7 +112,7 @@ def test_scan_bwd_optional_parts(conv, z, Dk, sp, silu):
         # without softplus the step sizes are taken as given: pass positive ones
         inp["delta"] = torch.nn.functional.softplus(inp["delta"]).contiguous()
     dy = make_output_grads(wl, device="cuda", with_attention=False)["dy"]
-    got, ref = _run(inp, dy, with_conv=conv, with_z=z, with_D=Dk, softplus=sp, conv_silu=silu)
+    got, ref = _run(inp, dy, with_conv=conv, with_z=z, with_D=Dk, softplus=sp, conv_silu=silu, fwd_ckpt=conv)
     _check(f"scan bwd options conv={conv} z={z} D={Dk} softplus={sp} silu={silu}", got, ref)
 
 
@@ -119,8 +130,8 @@ def test_scan_bwd_long_sequence():
     wl = Workload("sbl", 2, 4096, 256, 16, 4, 1, 1, 16, 16, 302)
     inp = make_prefill_inputs(wl, device="cuda", with_attention=False)
     dy = make_output_grads(wl, device="cuda", with_attention=False)["dy"]
-    got, ref = _run(inp, dy)
-    _check("scan bwd B2 L4096 D256 bf16", got, ref, ("dx", "dz"))
+    got, ref = _run(inp, dy, fwd_ckpt=True)
+    _check("scan bwd B2 L4096 D256 bf16 fwd ckpt", got, ref, ("dx", "dz"))
 
 
 def test_scan_bwd_training_workload_sampled_channels():
@@ -132,8 +143,10 @@ def test_scan_bwd_training_workload_sampled_channels():
     wl = WORKLOADS["train_4k"]
     inp = make_prefill_inputs(wl, device="cuda", with_attention=False)
     dy = make_output_grads(wl, device="cuda", with_attention=False)["dy"]
-    got = ops.selective_scan_bwd(dy, inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"], z=inp["z"],
-                                 conv_w=inp["conv_w"], conv_b=inp["conv_b"], want_dh0=True)
+    kw = dict(D=inp["D"], z=inp["z"], conv_w=inp["conv_w"], conv_b=inp["conv_b"])
+    ck = _fwd_ckpt(inp, y_dtype=torch.bfloat16, **kw)   # as the training step runs it
+    got = ops.selective_scan_bwd(dy, inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], want_dh0=True, ckpt=ck,
+                                 **kw)
     torch.cuda.synchronize()
     assert ops.get_status() == 0
     rng = np.random.default_rng(5)

@@ -185,3 +185,32 @@ def test_full_size_sampled_channels(name):
     yb, hb, _ = _run_gpu(inp, y_dtype=torch.bfloat16)
     assert torch.equal(hb, hf)
     assert torch.equal(yb, y.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("Bsz,Ln,D,N,dt", [(2, 75, 40, 16, torch.float32), (1, 64, 32, 8, torch.bfloat16),
+                                           (1, 5, 16, 4, torch.float32)])
+def test_forward_checkpoints_are_the_chunk_start_states(Bsz, Ln, D, N, dt):
+    """h_ckpt[:, c] is the state before token 16 c: h0 for c = 0, else the
+    oracle's final state after the first 16 c tokens (same inputs, conv state
+    and h0)."""
+    wl = Workload("ck", Bsz, Ln, D, N, 4, 1, 1, 16, 16, 400 + Ln, act_dtype=dt)
+    inp = make_prefill_inputs(wl, device="cuda", with_attention=False)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(9)
+    h0 = torch.randn((Bsz, D, N), generator=g, device="cuda")
+    cs = torch.randn((Bsz, D, 3), generator=g, device="cuda")
+    ck = torch.full(ops.scan_ckpt_shape(Bsz, Ln, D, N), float("nan"), device="cuda")
+    kw = dict(D=inp["D"], z=inp["z"], conv_w=inp["conv_w"], conv_b=inp["conv_b"], conv_state_in=cs, h0=h0)
+    ops.selective_scan_fwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], h_ckpt=ck, **kw)
+    torch.cuda.synchronize()
+    assert ops.get_status() == 0
+    got = host64(ck)                                     # [B, nck, N, D]
+    np.testing.assert_array_equal(got[:, 0], host64(h0).transpose(0, 2, 1))
+    for c in range(1, got.shape[1]):
+        t = 16 * c
+        ref = orc.selective_scan(host64(inp["x"][:, :t]), host64(inp["delta"][:, :t]), host64(inp["A"]),
+                                 host64(inp["B"][:, :t]), host64(inp["C"][:, :t]), host64(inp["D"]),
+                                 host64(inp["z"][:, :t]), h0=host64(h0), conv_w=host64(inp["conv_w"]),
+                                 conv_b=host64(inp["conv_b"]), conv_state=host64(cs), magnitudes=True)
+        e = scan_errors(got[:, c].transpose(0, 2, 1), ref["h"], ref["h_mag"])
+        assert e["rel_to_mag"] <= SCAN_TOL, (c, e["rel_to_mag"])
