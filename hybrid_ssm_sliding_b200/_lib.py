@@ -13,12 +13,14 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsamba.so")
+# SAMBA_LIBRARY=debug loads the debug build (libsamba_debug.so: the same
+# kernels with device-side index checks); it is never a fallback
+LIB_PATH = os.path.join(_HERE, "libsamba_debug.so" if os.environ.get("SAMBA_LIBRARY") == "debug" else "libsamba.so")
 
 SAMBA_F32, SAMBA_BF16 = 0, 1
 SAMBA_OK = 0
 SAMBA_ERR_INVALID_ARG, SAMBA_ERR_UNSUPPORTED, SAMBA_ERR_WORKSPACE = -1, -2, -3
-SAMBA_ERR_CUDA, SAMBA_ERR_TIMEOUT = -4, -5
+SAMBA_ERR_CUDA, SAMBA_ERR_TIMEOUT, SAMBA_ERR_CHECK = -4, -5, -6
 SCAN_FUSE_CONV, SCAN_DELTA_SOFTPLUS, SCAN_CONV_SILU = 1, 2, 4
 
 _vp = ctypes.c_void_p
@@ -97,6 +99,7 @@ def load() -> ctypes.CDLL:
     lib.samba_last_error.restype = ctypes.c_char_p
     lib.samba_get_status.argtypes = [_vp]
     lib.samba_selftest_wait_timeout.argtypes = [_vp]
+    lib.samba_selftest_check.argtypes = [_vp]
     lib.samba_conv1d_fwd.argtypes = [_vp, ctypes.c_int, _vp, _vp, _vp, _vp, ctypes.c_int, _vp,
                                      _i64, _i64, _i64, ctypes.c_int, ctypes.c_int, _vp]
     lib.samba_selective_scan_fwd.argtypes = [ctypes.POINTER(ScanArgs), _vp]
@@ -127,7 +130,7 @@ def load() -> ctypes.CDLL:
     for name in ("samba_conv1d_fwd", "samba_selective_scan_fwd", "samba_swa_fwd", "samba_mixer_prefill",
                  "samba_scan_step", "samba_swa_ring_fill", "samba_swa_step", "samba_get_status",
                  "samba_scan_carry", "samba_conv_state", "samba_gemm", "samba_selective_scan_bwd", "samba_swa_bwd",
-                 "samba_selftest_wait_timeout", "samba_swa_step_noalloc"):
+                 "samba_selftest_wait_timeout", "samba_swa_step_noalloc", "samba_selftest_check"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib

@@ -104,6 +104,10 @@ int samba_selftest_wait_timeout(samba_stream_t stream) {
   return launch_selftest_wait(reinterpret_cast<cudaStream_t>(stream));
 }
 
+int samba_selftest_check(samba_stream_t stream) {
+  return launch_selftest_check(reinterpret_cast<cudaStream_t>(stream));
+}
+
 int samba_conv1d_fwd(const void* x, int x_dtype, const float* w, const float* bias, const float* conv_state_in,
                      void* u, int u_dtype, float* conv_state_out, int64_t batch, int64_t seqlen, int64_t dim,
                      int dconv, int silu, samba_stream_t stream) {

@@ -43,6 +43,19 @@ __device__ __forceinline__ void report_timeout(int where) {
   (void)where;
 }
 
+// Index checks of the debug build (-DSAMBA_DEBUG): `if (SAMBA_CHECK(i < n))
+// store;` skips the store and records SAMBA_ERR_CHECK when the index is out
+// of range.  In the release build the condition is the constant true.
+#ifdef SAMBA_DEBUG
+__device__ __forceinline__ bool check_index(bool ok) {
+  if (!ok) atomicCAS(&g_status, 0, SAMBA_ERR_CHECK);
+  return ok;
+}
+#define SAMBA_CHECK(cond) ::samba::check_index(static_cast<bool>(cond))
+#else
+#define SAMBA_CHECK(cond) true
+#endif
+
 // ------------------------------------------------------------------ bf16 / f32
 template <typename T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }

@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t r[32];
         tmem_ld32(t_row + c0, r);  // warp-collective: every lane, whatever its row
         tc_wait_ld();
-        if (row >= p.M) continue;
+        if (row >= p.M || !SAMBA_CHECK(row >= 0 && n0 + c0 < p.N)) continue;
 #pragma unroll
         for (int j = 0; j < 32; j += 8) {
           const int64_t col = n0 + c0 + j;  // 8 consecutive columns
@@ -280,7 +280,7 @@ struct SkinnyCfg {
 
 template <int MP>
 __device__ __forceinline__ void skinny_store(const SkinnyParams& p, int64_t n, const float (&v)[MP]) {
-  if (n >= p.N) return;
+  if (n >= p.N || !SAMBA_CHECK(n >= 0 && p.M <= MP)) return;
 #pragma unroll
   for (int o = 0; o < 3; ++o) {
     if (o >= p.nout) break;
@@ -454,6 +454,7 @@ __global__ void __launch_bounds__(192, 1)
         skinny_store<MP>(p, n, v);
         continue;
       }
+      if (!SAMBA_CHECK(nb * 4 + warp < p.T / kb * 4)) continue;  // the workspace holds nblk blocks
       float4* row = reinterpret_cast<float4*>(p.acc + n * MP);
 #pragma unroll
       for (int q = 0; q < MP / 4; ++q) atomicAdd(row + q, make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));

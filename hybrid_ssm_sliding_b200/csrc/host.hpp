@@ -58,6 +58,7 @@ int take_status_swa(cudaStream_t s);
 int take_status_misc(cudaStream_t s);
 int take_status_gemm(cudaStream_t s);
 int launch_gemm(const samba_gemm_args& a, cudaStream_t stream);
+int launch_selftest_check(cudaStream_t s);
 size_t gemm_workspace_size(int64_t M, int64_t N);
 size_t scan_bwd_workspace(int64_t B, int64_t L, int64_t D, int N);
 int launch_scan_bwd(const samba_scan_bwd_args& a, cudaStream_t stream);

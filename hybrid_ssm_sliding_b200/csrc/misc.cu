@@ -87,6 +87,7 @@ __global__ void conv1d_step_kernel(const XT* __restrict__ x, const float* __rest
     float acc = bias ? bias[c] : 0.f;
     for (int k = 0; k < K; ++k) acc = fmaf(w[c * K + k], xp[k], acc);
     if (silu) acc = silu_dev(acc);
+    if (!SAMBA_CHECK(e >= 0 && e < n && K <= 4)) continue;
     u[e] = from_f32<UT>(acc);
     for (int k = 0; k < K - 1; ++k) cs_out[e * (K - 1) + k] = xp[k + 1];
   }
@@ -221,10 +222,10 @@ __global__ void __launch_bounds__(256) scan_step_kernel(
     hv[n] = fmaf(ex2_approx(dlt * (av[n] * kLog2e)), hv[n], du * bv[n]);
     acc = fmaf(cv[n], hv[n], acc);
   }
-  st_states<NS>(hp, hv);
+  if (SAMBA_CHECK(b < (int64_t)gridDim.y && c < D)) st_states<NS>(hp, hv);
   acc += __shfl_xor_sync(gmask, acc, 1);
   acc += __shfl_xor_sync(gmask, acc, 2);
-  if (j == 0) {
+  if (j == 0 && SAMBA_CHECK(e < (int64_t)gridDim.y * D)) {
     float yv = acc + (Dskip ? dsk * u : 0.f);
     if (z_t) yv *= silu_dev(zv);
     y_t[e] = from_f32<YT>(yv);
@@ -445,7 +446,7 @@ __global__ void __launch_bounds__(128) swa_step_split_kernel(
                                : make_uint4(0u, 0u, 0u, 0u);
     reinterpret_cast<uint4*>(Qs + hh * KP)[c] = v;
   }
-  if (jnew >= j_lo && jnew < j_hi && tid < RCH) {  // the new key and value into their slot
+  if (jnew >= j_lo && jnew < j_hi && tid < RCH && SAMBA_CHECK(jnew >= 0 && jnew < W)) {  // the new key and value into their slot
     const int64_t roff = ((int64_t)b * W + jnew) * row_stride + (int64_t)g * HD;
     reinterpret_cast<uint4*>(k_ring + roff)[tid] = reinterpret_cast<const uint4*>(k_t + noff)[tid];
     reinterpret_cast<uint4*>(v_ring + roff)[tid] = reinterpret_cast<const uint4*>(v_t + noff)[tid];
@@ -596,6 +597,7 @@ __global__ void __launch_bounds__(128) swa_step_split_kernel(
   if (!__syncthreads_and(ok)) return;  // a copy never landed: the status word says so
   for (int i = tid; i < group * HD; i += 128) {
     const int hh = i / HD, dd = i % HD;
+    if (!SAMBA_CHECK(g * group + hh < Hq && split < nsplit && b < (int)gridDim.z)) continue;
     float* dst = ws + ((((int64_t)b * Hq + g * group + hh) * nsplit + split) * (HD + 2));
     dst[2 + dd] = Ow[hh * HD + dd] + Ow[(16 + hh) * HD + dd] + Ow[(32 + hh) * HD + dd] + Ow[(48 + hh) * HD + dd];
     if (dd == 0) {
@@ -632,6 +634,7 @@ __global__ void swa_step_combine_kernel(const float* __restrict__ ws, __nv_bfloa
     l = fmaf(base[s * (HD + 2) + 1], f, l);
     acc = fmaf(base[s * (HD + 2) + 2 + dd], f, acc);
   }
+  if (!SAMBA_CHECK(hq < Hq && dd < HD && b < (int)gridDim.y)) return;
   o_t[((int64_t)b * Hq + hq) * HD + dd] = __float2bfloat16_rn(acc / l);
   if (hq == 0 && dd == 0) pos[b] += 1;
 }
@@ -734,6 +737,24 @@ __global__ void selftest_wait_kernel() {
 int launch_selftest_wait(cudaStream_t s) {
   selftest_wait_kernel<<<1, 32, 0, s>>>();
   return check_launch("samba_selftest_wait_timeout");
+}
+
+#ifdef SAMBA_DEBUG
+// A store whose index is one past its 16-element buffer: the check skips it.
+__device__ float g_check_buf[16];
+__global__ void selftest_check_kernel(int i) {
+  if (threadIdx.x == 0 && SAMBA_CHECK(i >= 0 && i < 16)) g_check_buf[i] = 1.f;
+}
+#endif
+
+int launch_selftest_check(cudaStream_t s) {
+#ifdef SAMBA_DEBUG
+  selftest_check_kernel<<<1, 32, 0, s>>>(16);
+  return check_launch("samba_selftest_check");
+#else
+  (void)s;
+  return fail(SAMBA_ERR_UNSUPPORTED, "samba_selftest_check: the release build has no device-side checks");
+#endif
 }
 
 }  // namespace samba

@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(32 * nwarps(N), 3) scan_bwd_kernel(const ScanB
     // (b) the gate's gradient dz = dy · (C·h + D u) · silu'(z); the sums are
     // then cleared for the reverse walk's dΔ
     for (int t = pt; t < kTc; t += NW) {
-      if (z && t < nv && ch_ok) {
+      if (z && t < nv && ch_ok && SAMBA_CHECK(t0 + t < L && b < (int64_t)gridDim.y)) {
         const float ypre = S.part[0][t][pc] + dsk * S.u[t][pc];
         stv<XT>(p.dz, (b * L + t0 + t) * D + ch_p, ypre * S.dydsz[t][pc]);
       }
@@ -450,7 +450,7 @@ __global__ void __launch_bounds__(32 * nwarps(N), 3) scan_bwd_kernel(const ScanB
       float* dst = p.part + static_cast<int64_t>(blockIdx.x) * 2 * BLN + (b * L + t0) * N;
       for (int i = tid; i < 2 * nv * N; i += kThreads) {
         const int w = i / (nv * N), r = i - w * (nv * N);
-        dst[w * BLN + r] = S.dbc[w][r / N][r % N];
+        if (SAMBA_CHECK((b * L + t0) * N + r < BLN)) dst[w * BLN + r] = S.dbc[w][r / N][r % N];
       }
     }
     // (d) du, dΔ, the conv's SiLU; accumulate dD and the conv parameter sums
@@ -460,7 +460,7 @@ __global__ void __launch_bounds__(32 * nwarps(N), 3) scan_bwd_kernel(const ScanB
         const float du = dsk * S.gy[t][pc] + S.part[1][t][pc];
         const float ddt = S.part[0][t][pc];
         const int64_t e = (b * L + t0 + t) * D + ch_p;
-        if (ch_ok) p.ddelta[e] = ddt * S.sg[t][pc];
+        if (ch_ok && SAMBA_CHECK(e < (int64_t)gridDim.y * L * D)) p.ddelta[e] = ddt * S.sg[t][pc];
         accD = fmaf(S.gy[t][pc], S.u[t][pc], accD);
         if (fuse) {
           const float pre = S.cpre[t][pc];
@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(32 * nwarps(N), 3) scan_bwd_kernel(const ScanB
         #pragma unroll
         for (int k = 0; k < 4; ++k)
           if (k < K) v = fmaf(cw[k], S.dc[t + (K - 1) - k][pc], v);
-        if (ch_ok) stv<XT>(p.dx, (b * L + t0 + t) * D + ch_p, v);
+        if (ch_ok && SAMBA_CHECK(t0 + t < L && b < (int64_t)gridDim.y)) stv<XT>(p.dx, (b * L + t0 + t) * D + ch_p, v);
       }
     }
     __syncthreads();

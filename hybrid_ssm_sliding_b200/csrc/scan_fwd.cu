@@ -332,8 +332,9 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
         const int64_t tok = t0 + eg * TPE + q;
         const float acc = (pv[q].x + pv[q].y) + (pv[q].z + pv[q].w);
         const float g = p.has_z ? silu_fast(ev[q].y) : 1.f;
-        if (cval && tok < L)
-          reinterpret_cast<YT*>(p.y)[((int64_t)b * L + tok) * p.D + c] = from_f32<YT>((acc + ev[q].x) * g);
+        const int64_t yi = ((int64_t)b * L + tok) * p.D + c;
+        if (cval && tok < L && SAMBA_CHECK(yi >= 0 && yi < (int64_t)gridDim.y * L * p.D))
+          reinterpret_cast<YT*>(p.y)[yi] = from_f32<YT>((acc + ev[q].x) * g);
       }
     }
     return;
@@ -496,6 +497,7 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
   // checkpoint cidx: the state before token 16 * cidx ([b][cidx][n][D])
   auto store_ckpt = [&](int64_t cidx) {
     if (!cval || cidx >= p.nck) return;
+    if (!SAMBA_CHECK(b < (int64_t)gridDim.y && c < p.D && n0 + NS <= N)) return;
     float* dst = p.h_ckpt + ((int64_t)b * p.nck + cidx) * N * p.D + c;
 #pragma unroll
     for (int q = 0; q < NP; ++q) {
@@ -617,7 +619,7 @@ __global__ void __launch_bounds__(SAMBA_SCAN_MAXTHREADS, 1)
     }
   }
   if (*abort_flag) return;
-  if (cval && p.h_final) {
+  if (cval && p.h_final && SAMBA_CHECK(b < (int64_t)gridDim.y && c < p.D && n0 + NS <= N)) {
 #pragma unroll
     for (int q = 0; q < NP; ++q) {
       const float2 hv = up2(hp[q]);

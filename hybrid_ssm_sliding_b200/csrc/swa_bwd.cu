@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
 #pragma unroll
             for (int c = 0; c < 16; ++c) t16[c] = 0u;
           }
-          if (j < p.L) {
+          if (j < p.L && SAMBA_CHECK(j >= 0 && b < p.B && g < p.Hkv)) {
             uint4 v0, v1;
             v0.x = pack_bf16x2(__uint_as_float(t16[0]) * mul, __uint_as_float(t16[1]) * mul);
             v0.y = pack_bf16x2(__uint_as_float(t16[2]) * mul, __uint_as_float(t16[3]) * mul);
@@ -643,7 +643,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, GROUP>::THREADS, 1)
         uint32_t t16[16];
         tmem_ld16(tmem + lane_off + Cfg::COL_DQ + 16 * q, t16);
         tc_wait_ld();
-        if (irow >= p.L) continue;
+        if (irow >= p.L || !SAMBA_CHECK(irow >= 0 && b < p.B && g * GROUP + hh < p.Hq)) continue;
         uint4 v0, v1;
         const float mul = p.scale;
         v0.x = pack_bf16x2(__uint_as_float(t16[0]) * mul, __uint_as_float(t16[1]) * mul);

@@ -524,7 +524,7 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
         for (int c = 0; c < 16; ++c) o[16 * q + c] = t16[c];
       }
-      if (irow < p.L) {
+      if (irow < p.L && SAMBA_CHECK(b < p.B && irow >= 0 && g * GROUP + hh < p.Hq)) {
         const float inv = 1.f / l_run;
         const int h = g * GROUP + hh;
         __nv_bfloat16* dst = p.o + ((static_cast<int64_t>(b) * p.L + irow) * p.Hq + h) * HD;

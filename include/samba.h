@@ -66,7 +66,8 @@ enum {
   SAMBA_ERR_UNSUPPORTED = -2,
   SAMBA_ERR_WORKSPACE = -3,
   SAMBA_ERR_CUDA = -4,
-  SAMBA_ERR_TIMEOUT = -5
+  SAMBA_ERR_TIMEOUT = -5,
+  SAMBA_ERR_CHECK = -6          /* debug build only: a device-side index check failed */
 };
 
 /* flags of samba_scan_args.flags */
@@ -84,7 +85,15 @@ const char* samba_last_error(void);
 
 /* Synchronises `stream`, then returns and clears this device's status word:
  * SAMBA_OK, or SAMBA_ERR_TIMEOUT if a kernel gave up a device-side wait since
- * the last call.  Returns SAMBA_ERR_CUDA if the synchronisation itself fails. */
+ * the last call, or (debug build) SAMBA_ERR_CHECK if a device-side index
+ * check failed.  Returns SAMBA_ERR_CUDA if the synchronisation itself fails.
+ *
+ * Debug build: libsamba_debug.so (hybrid_ssm_sliding_b200/build.py --debug)
+ * is the same library compiled with SAMBA_DEBUG.  Its kernels check the
+ * index of every global output store against the extent of the tensor it
+ * writes (computed from the call's sizes); a failed check skips the store and
+ * records SAMBA_ERR_CHECK instead of trapping, so the context stays usable.
+ * The release build compiles the checks away. */
 int samba_get_status(samba_stream_t stream);
 
 /* Self-test of the failure path: launches one small kernel that waits on an
@@ -95,6 +104,13 @@ int samba_get_status(samba_stream_t stream);
  * was issued.  Not part of the mixers; it exists so the timeout handling can
  * be tested on a GPU without faulting or hanging it. */
 int samba_selftest_wait_timeout(samba_stream_t stream);
+
+/* Self-test of the debug build's checks: launches one small kernel whose
+ * guarded store has an index past its (16-element, library-owned) buffer;
+ * the check skips the store and records SAMBA_ERR_CHECK, which
+ * samba_get_status(stream) then returns.  Returns SAMBA_OK if the launch was
+ * issued, SAMBA_ERR_UNSUPPORTED in the release build (no checks there). */
+int samba_selftest_check(samba_stream_t stream);
 
 /* ------------------------------------------------------------------ conv1d
  * Causal depthwise conv1d over time, the conv that a Mamba layer puts in front

@@ -38,6 +38,21 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, name), name
 
 
+def test_debug_build_exports_every_declared_symbol():
+    """libsamba_debug.so: the same sources with the device-side checks; it
+    must export the same entry points (loaded here by path, beside the
+    release library the other tests use)."""
+    dbg = ctypes.CDLL(B.build(debug=True))
+    for name in declared_functions():
+        assert hasattr(dbg, name), name
+
+
+def test_release_build_has_no_check_selftest(lib):
+    """Without SAMBA_DEBUG the check self-test refuses on the host (it
+    launches nothing, so no GPU is needed)."""
+    assert lib.samba_selftest_check(None) == L.SAMBA_ERR_UNSUPPORTED
+
+
 def test_version(lib):
     assert lib.samba_version() >= 100
 
