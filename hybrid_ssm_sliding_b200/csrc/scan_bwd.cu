@@ -414,18 +414,22 @@ __global__ void __launch_bounds__(32 * nwarps(N), 3) scan_bwd_kernel(const ScanB
         const float gyv = valid ? S.gy[t][lane] : 0.f;
         const float dt = valid ? S.dt[t][lane] : 0.f;
         const float uv = valid ? S.u[t][lane] : 0.f;
+        const float du = dt * uv;  // rounded as in (a)
         float gB = 0.f, ddt = 0.f;
 #pragma unroll
         for (int j = 0; j < SPL; ++j) {
           const int n = warp * SPL + j;
           const float ht = valid ? S.H[t][n][lane] : 0.f;
-          const float hprev = !valid ? 0.f : (t > 0 ? S.H[t - 1][n][lane] : hs[j]);
+          const float bv = S.Bv[t][n];
+          // exp(Δ A) h_{t-1} = h_t - Δ u B: (a) formed h_t as that sum, so
+          // the decayed previous state needs neither h_{t-1} nor the product
+          const float dh = ht - du * bv;
           g[j] = fmaf(S.Cv[t][n], gyv, g[j]);
           const float decay = ex2_fast(dt * Al[j]);
-          const float gdh = g[j] * decay * hprev;
-          q[i * 2 * SPL + j] = gyv * ht;            // dC contribution
-          q[i * 2 * SPL + SPL + j] = g[j] * dt * uv;  // dB contribution
-          gB = fmaf(g[j], S.Bv[t][n], gB);
+          const float gdh = g[j] * dh;
+          q[i * 2 * SPL + j] = gyv * ht;       // dC contribution
+          q[i * 2 * SPL + SPL + j] = g[j] * du;  // dB contribution
+          gB = fmaf(g[j], bv, gB);
           ddt = fmaf(gdh, Al[j] * (1.0f / kLog2e), ddt);
           dAacc[j] = fmaf(gdh, dt, dAacc[j]);
           g[j] *= decay;
