@@ -257,6 +257,10 @@ __global__ void __launch_bounds__(192, 1)
 // is launched as a programmatic dependent of the kernel before it (pdl.cuh):
 // the first stages' weight tiles are requested before the wait for that
 // kernel, A's tiles and every global write after it.
+#ifndef SAMBA_SKINNY_MIN_KSTEPS
+#define SAMBA_SKINNY_MIN_KSTEPS 4  // fixed by measurement (serving loop: 1, 2, 4, 8 -> 266, 258, 254, 254 us per step)
+#endif
+
 struct SkinnyParams {
   int64_t M, N, K;
   GemmOut out[3];
@@ -538,7 +542,10 @@ static int launch_skinny_t(const samba_gemm_args& a, cudaStream_t stream) {
   p.acc = reinterpret_cast<float*>(a.workspace);
   p.cnt = reinterpret_cast<uint32_t*>(reinterpret_cast<unsigned char*>(a.workspace) +
                                       static_cast<size_t>(nblk) * Cfg::BN * MP * 4);
-  const unsigned grid = (unsigned)std::min<int64_t>(p.T, sm_count());
+  // At least SAMBA_SKINNY_MIN_KSTEPS k-steps per CTA (a block's whole K when
+  // it has fewer): fewer partial sums meet in the workspace for small weights.
+  const int64_t min_ks = std::min<int64_t>(p.kb, SAMBA_SKINNY_MIN_KSTEPS);
+  const unsigned grid = (unsigned)std::min<int64_t>((p.T + min_ks - 1) / min_ks, sm_count());
   const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM, stream, ma, mb, p);
   if (e != cudaSuccess) return fail(SAMBA_ERR_CUDA, "samba_gemm: launch failed: %s", cudaGetErrorString(e));
   return check_launch("samba_gemm");
