@@ -896,10 +896,17 @@ def run_train(args, wl, dev, rank, world):
         ops.swa_bwd(grads["do"], inp["q"], inp["k"], inp["v"], o, lse, wl.window, dq=dq, dk=dk, dv=dv,
                     workspace=ws_swa)
 
+    aux = torch.cuda.Stream()
+
     def step():
+        # the two backward passes are independent: the attention's runs on a
+        # second stream and takes the SMs the scan's last wave leaves free
         fwd()
-        bwd_scan()
-        bwd_swa()
+        ops.mixer_bwd(dict(dy=grads["dy"], x=inp["x"], delta=inp["delta"], A=inp["A"], B=inp["B"], C=inp["C"],
+                           workspace=ws_scan, ckpt=ckpt, **scan_in),
+                      dict(do=grads["do"], q=inp["q"], k=inp["k"], v=inp["v"], o=o, lse=lse, window=wl.window,
+                           dq=dq, dk=dk, dv=dv, workspace=ws_swa),
+                      aux_stream=aux)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -954,7 +961,7 @@ def run_train(args, wl, dev, rank, world):
     roof["kernel"] = "scan_bwd_kernel" if dom == "scan_bwd" else "swa_bwd_kv_kernel + swa_bwd_q_kernel"
     cfg = workload_config(wl)
     cfg["step"] = ("scan and SWA forward (with log-sum-exp and the scan's 16-token state checkpoints), then scan "
-                   "and SWA backward from seeded dy, dO")
+                   "and SWA backward from seeded dy, dO (samba_mixer_bwd, the SWA backward on a second stream)")
     return {
         "metric": TRAIN_METRIC, "value": whole_job_rate(wl.batch * wl.seqlen, world, ms_step), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,

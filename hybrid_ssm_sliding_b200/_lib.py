@@ -126,11 +126,12 @@ def load() -> ctypes.CDLL:
     lib.samba_swa_bwd_workspace_size.argtypes = [_i64, _i64, _i32]
     lib.samba_swa_bwd_workspace_size.restype = ctypes.c_size_t
     lib.samba_swa_bwd.argtypes = [ctypes.POINTER(SwaBwdArgs), _vp]
+    lib.samba_mixer_bwd.argtypes = [ctypes.POINTER(ScanBwdArgs), ctypes.POINTER(SwaBwdArgs), _vp, _vp]
     lib.samba_conv_state.argtypes = [_vp, ctypes.c_int, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp]
     for name in ("samba_conv1d_fwd", "samba_selective_scan_fwd", "samba_swa_fwd", "samba_mixer_prefill",
                  "samba_scan_step", "samba_swa_ring_fill", "samba_swa_step", "samba_get_status",
                  "samba_scan_carry", "samba_conv_state", "samba_gemm", "samba_selective_scan_bwd", "samba_swa_bwd",
-                 "samba_selftest_wait_timeout", "samba_swa_step_noalloc", "samba_selftest_check"):
+                 "samba_selftest_wait_timeout", "samba_swa_step_noalloc", "samba_selftest_check", "samba_mixer_bwd"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib

@@ -168,8 +168,7 @@ size_t samba_scan_bwd_workspace_size(int64_t batch, int64_t seqlen, int64_t dim,
   return scan_bwd_workspace(batch, seqlen, dim, dstate);
 }
 
-int samba_selective_scan_bwd(const samba_scan_bwd_args* a, samba_stream_t stream) {
-  const char* who = "samba_selective_scan_bwd";
+static int check_scan_bwd(const samba_scan_bwd_args* a, const char* who) {
   if (!a) return fail(SAMBA_ERR_INVALID_ARG, "%s: null args", who);
   // the forward's checks on the shared fields
   samba_scan_args f = {};
@@ -208,6 +207,12 @@ int samba_selective_scan_bwd(const samba_scan_bwd_args* a, samba_stream_t stream
   const size_t need = scan_bwd_workspace(a->batch, a->seqlen, a->dim, a->dstate);
   if (!a->workspace || need == SIZE_MAX || a->workspace_bytes < need)
     return fail(SAMBA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed", who, need);
+  return SAMBA_OK;
+}
+
+int samba_selective_scan_bwd(const samba_scan_bwd_args* a, samba_stream_t stream) {
+  const int rc = check_scan_bwd(a, "samba_selective_scan_bwd");
+  if (rc != SAMBA_OK) return rc;
   return launch_scan_bwd(*a, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -216,8 +221,7 @@ size_t samba_swa_bwd_workspace_size(int64_t batch, int64_t seqlen, int32_t heads
   return swa_bwd_workspace(batch, seqlen, heads_q);
 }
 
-int samba_swa_bwd(const samba_swa_bwd_args* a, samba_stream_t stream) {
-  const char* who = "samba_swa_bwd";
+static int check_swa_bwd(const samba_swa_bwd_args* a, const char* who) {
   if (!a) return fail(SAMBA_ERR_INVALID_ARG, "%s: null args", who);
   samba_swa_args f = {};
   f.q = a->q;
@@ -241,7 +245,53 @@ int samba_swa_bwd(const samba_swa_bwd_args* a, samba_stream_t stream) {
   const size_t need = swa_bwd_workspace(a->batch, a->seqlen, a->heads_q);
   if (!a->workspace || need == SIZE_MAX || a->workspace_bytes < need)
     return fail(SAMBA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed", who, need);
+  return SAMBA_OK;
+}
+
+int samba_swa_bwd(const samba_swa_bwd_args* a, samba_stream_t stream) {
+  const int rc = check_swa_bwd(a, "samba_swa_bwd");
+  if (rc != SAMBA_OK) return rc;
   return launch_swa_bwd(*a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int samba_mixer_bwd(const samba_scan_bwd_args* scan, const samba_swa_bwd_args* swa, samba_stream_t stream,
+                    samba_stream_t aux) {
+  const char* who = "samba_mixer_bwd";
+  int rc = check_scan_bwd(scan, who);
+  if (rc != SAMBA_OK) return rc;
+  rc = check_swa_bwd(swa, who);
+  if (rc != SAMBA_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaStream_t a = reinterpret_cast<cudaStream_t>(aux);
+  if (!a) {
+    rc = launch_scan_bwd(*scan, s);
+    if (rc != SAMBA_OK) return rc;
+    return launch_swa_bwd(*swa, s);
+  }
+  // The scan's backward goes first on `stream`; the attention's, forked onto
+  // `aux`, takes the SMs the scan leaves free and is joined back, so that the
+  // call as a whole stays ordered on `stream`.
+  cudaEvent_t fork = nullptr, join = nullptr;
+  if (cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess)
+    return fail(SAMBA_ERR_CUDA, "%s: event creation failed", who);
+  if (cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {
+    cudaEventDestroy(fork);
+    return fail(SAMBA_ERR_CUDA, "%s: event creation failed", who);
+  }
+  if (cudaEventRecord(fork, s) != cudaSuccess || cudaStreamWaitEvent(a, fork, 0) != cudaSuccess) {
+    rc = fail(SAMBA_ERR_CUDA, "%s: cannot fork the aux stream", who);
+  } else {
+    rc = launch_scan_bwd(*scan, s);
+    // After a failed scan launch the attention is not started; the join below
+    // still orders `stream` after whatever reached `aux`.
+    if (rc == SAMBA_OK) rc = launch_swa_bwd(*swa, a);
+    if ((cudaEventRecord(join, a) != cudaSuccess || cudaStreamWaitEvent(s, join, 0) != cudaSuccess) &&
+        rc == SAMBA_OK)
+      rc = fail(SAMBA_ERR_CUDA, "%s: cannot join the aux stream", who);
+  }
+  cudaEventDestroy(fork);
+  cudaEventDestroy(join);
+  return rc;
 }
 
 int samba_gemm(const samba_gemm_args* a, samba_stream_t stream) {

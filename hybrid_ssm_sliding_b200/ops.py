@@ -128,6 +128,17 @@ def selective_scan_bwd(dy, x, delta, A, B, C, D=None, z=None, conv_w=None, conv_
     and, where the forward input exists, dz, dD, dconv_w, dconv_b, plus dh0 /
     dconv_state when asked for.  ``ckpt``: the forward's h_ckpt for these
     inputs (the backward then skips its own checkpoint pass)."""
+    a, out, _ws = _scan_bwd_struct(dy, x, delta, A, B, C, D, z, conv_w, conv_b, conv_state_in, h0, delta_softplus,
+                                   conv_silu, fuse_conv, want_dh0, want_dconv_state, workspace, ckpt)
+    L.check(L.load().samba_selective_scan_bwd(ctypes.byref(a), L.stream_handle(stream)))
+    return out
+
+
+def _scan_bwd_struct(dy, x, delta, A, B, C, D=None, z=None, conv_w=None, conv_b=None, conv_state_in=None,
+                     h0=None, delta_softplus=True, conv_silu=True, fuse_conv=None, want_dh0=False,
+                     want_dconv_state=False, workspace=None, ckpt=None):
+    """The samba_scan_bwd_args of selective_scan_bwd, its output dict and the
+    workspace (kept alive by the caller until the call is enqueued)."""
     _need(x, "x")
     Bsz, Ln, Dm = x.shape
     N = A.shape[1]
@@ -168,8 +179,7 @@ def selective_scan_bwd(dy, x, delta, A, B, C, D=None, z=None, conv_w=None, conv_
                       L.ptr(out["dh0"]), L.ptr(out["dconv_state"]), L.ptr(workspace),
                       workspace.numel() * workspace.element_size(), Bsz, Ln, Dm, N, K, L.dtype_code(x),
                       L.dtype_code(z) if z is not None else 0, L.dtype_code(dy), flags, L.ptr(ckpt))
-    L.check(L.load().samba_selective_scan_bwd(ctypes.byref(a), L.stream_handle(stream)))
-    return out
+    return a, out, workspace
 
 
 def _swa_struct(q, k, v, window, scale=None, o=None, lse=None):
@@ -201,6 +211,13 @@ def swa_bwd_workspace_size(batch, seqlen, heads_q):
 def swa_bwd(do, q, k, v, o, lse, window, scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
     """Gradients of swa_fwd given dO (see samba_swa_bwd): o and lse are the
     forward's outputs for the same q, k, v.  Returns (dq, dk, dv)."""
+    a, grads, _ws = _swa_bwd_struct(do, q, k, v, o, lse, window, scale, dq, dk, dv, workspace)
+    L.check(L.load().samba_swa_bwd(ctypes.byref(a), L.stream_handle(stream)))
+    return grads
+
+
+def _swa_bwd_struct(do, q, k, v, o, lse, window, scale=None, dq=None, dk=None, dv=None, workspace=None):
+    """The samba_swa_bwd_args of swa_bwd, (dq, dk, dv) and the workspace."""
     _need(q, "q", torch.bfloat16)
     Bsz, Ln, Hq, d = q.shape
     Hkv = k.shape[2]
@@ -221,8 +238,20 @@ def swa_bwd(do, q, k, v, o, lse, window, scale=None, dq=None, dk=None, dv=None, 
     a = L.SwaBwdArgs(L.ptr(q), L.ptr(k), L.ptr(v), L.ptr(o), L.ptr(lse), L.ptr(do), L.ptr(dq), L.ptr(dk), L.ptr(dv),
                      L.ptr(workspace), workspace.numel() * workspace.element_size(), Bsz, Ln, int(window), Hq, Hkv, d,
                      float(scale) if scale else 0.0)
-    L.check(L.load().samba_swa_bwd(ctypes.byref(a), L.stream_handle(stream)))
-    return dq, dk, dv
+    return a, (dq, dk, dv), workspace
+
+
+def mixer_bwd(scan: dict, swa: dict, stream=None, aux_stream=None):
+    """The backward of both mixers (see samba_mixer_bwd): ``scan`` and
+    ``swa`` hold the keyword arguments of selective_scan_bwd and swa_bwd
+    (without stream).  With ``aux_stream`` the attention's backward runs
+    there, beside the scan's.  Returns (scan gradients dict, (dq, dk, dv))."""
+    sa, sgrads, ws1 = _scan_bwd_struct(**scan)
+    wa, wgrads, ws2 = _swa_bwd_struct(**swa)
+    L.check(L.load().samba_mixer_bwd(ctypes.byref(sa), ctypes.byref(wa), L.stream_handle(stream),
+                                     L.stream_handle(aux_stream) if aux_stream is not None else None))
+    del ws1, ws2
+    return sgrads, wgrads
 
 
 def mixer_prefill(scan: dict, swa: dict, stream=None, aux_stream=None):

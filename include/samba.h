@@ -307,6 +307,17 @@ size_t samba_swa_bwd_workspace_size(int64_t batch, int64_t seqlen, int32_t heads
 
 int samba_swa_bwd(const samba_swa_bwd_args* args, samba_stream_t stream);
 
+/* The backward of both mixers (a training step's gradients of the two token
+ * mixers; their backward passes are independent): samba_selective_scan_bwd
+ * and samba_swa_bwd on their own arguments, with the same checks and errors.
+ * With aux == NULL both run in order on `stream`; otherwise the scan's
+ * backward runs on `stream` and the attention's on `aux`, forked from and
+ * joined back into `stream` with events, so that the attention's kernels can
+ * take the SMs the scan's last wave leaves free and the call as a whole stays
+ * ordered on `stream`. */
+int samba_mixer_bwd(const samba_scan_bwd_args* scan, const samba_swa_bwd_args* swa, samba_stream_t stream,
+                    samba_stream_t aux);
+
 /* ------------------------------------------------------ sequence segments
  * A sequence split into consecutive segments (for example one per GPU) can be
  * scanned segment by segment with exactly the result of one pass, because the

@@ -18,7 +18,7 @@ import torch
 import oracle.samba_oracle as orc
 from hybrid_ssm_sliding_b200 import build as B
 from hybrid_ssm_sliding_b200 import ops
-from hybrid_ssm_sliding_b200.workloads import WORKLOADS, make_output_grads, make_prefill_inputs
+from hybrid_ssm_sliding_b200.workloads import WORKLOADS, Workload, make_output_grads, make_prefill_inputs
 from tests._helpers import host64, record_margin
 
 pytestmark = pytest.mark.gpu
@@ -137,3 +137,40 @@ def test_swa_bwd_training_workload_sampled_blocks():
             ratio = _ratio(host64(gt[b:b + 1, j0:j0 + 64]), rr[:, a:a + 64], mags[key][:, a:a + 64])
             record_margin(f"swa bwd train_4k {key} keys {j0}..{j0 + 63} of b{b}", key, worst_over_bound=ratio)
             assert ratio <= 1.0, (key, b, j0, ratio)
+
+
+@pytest.mark.parametrize("use_aux", [False, True])
+def test_mixer_bwd_equals_separate_calls(use_aux):
+    """samba_mixer_bwd (both backward passes, the attention's on a second
+    stream when given one) against samba_selective_scan_bwd and samba_swa_bwd
+    called one after the other: the attention's gradients bit for bit, the
+    scan's up to the order of its atomic sums (the per-token sums over the
+    state groups too, so a bf16 gradient may round one unit apart)."""
+    wl = Workload("mb", 2, 300, 64, 16, 4, 8, 2, 64, 128, 61)
+    inp = make_prefill_inputs(wl, device="cuda")
+    gr = make_output_grads(wl, device="cuda")
+    kw = dict(D=inp["D"], z=inp["z"], conv_w=inp["conv_w"], conv_b=inp["conv_b"])
+    lse = torch.empty((2, 8, 300), device="cuda")
+    o = ops.swa_fwd(inp["q"], inp["k"], inp["v"], 128, lse=lse)
+    scan = dict(dy=gr["dy"], x=inp["x"], delta=inp["delta"], A=inp["A"], B=inp["B"], C=inp["C"], **kw)
+    swa = dict(do=gr["do"], q=inp["q"], k=inp["k"], v=inp["v"], o=o, lse=lse, window=128)
+    ref_scan = ops.selective_scan_bwd(**scan)
+    ref_swa = ops.swa_bwd(**swa)
+    aux = torch.cuda.Stream() if use_aux else None
+    got_scan, got_swa = ops.mixer_bwd(scan, swa, aux_stream=aux)
+    torch.cuda.synchronize()
+    assert ops.get_status() == 0
+    bad = []
+    for name, a, b in zip(("dq", "dk", "dv"), got_swa, ref_swa):
+        if not torch.equal(a, b):
+            bad.append(f"{name}: max diff {float((a.float() - b.float()).abs().max()):.3e}")
+    for key, ref in ref_scan.items():
+        if ref is None:
+            assert got_scan[key] is None
+            continue
+        g, r = host64(got_scan[key]), host64(ref)
+        bf = 2.0 ** -7 * np.abs(r) if ref.dtype == torch.bfloat16 else 0.0  # one bf16 unit
+        bound = bf + 1e-5 * (np.max(np.abs(r)) or 1.0)
+        if not np.all(np.abs(g - r) <= bound):
+            bad.append(f"{key}: worst {float(np.max(np.abs(g - r) / bound)):.2f} x the bound")
+    assert not bad, "; ".join(bad)
