@@ -36,6 +36,10 @@
 
 namespace samba {
 
+#ifndef SAMBA_SCAN_BWD_CTAS
+#define SAMBA_SCAN_BWD_CTAS 4  // CTAs per SM the launch bounds aim at
+#endif
+
 namespace {
 
 constexpr int kCh = 32;      // channels per CTA (one per lane)
@@ -149,7 +153,6 @@ struct ScanBwdParams {
 template <int N>
 struct ScanBwdSmem {
   float x[kTc + kHalo][kCh];   // inputs of the chunk and the 3 before it
-  float cpre[kTc][kCh];        // conv output before its SiLU
   float u[kTc][kCh];
   float dt[kTc][kCh];
   float sg[kTc][kCh];          // σ(delta): d softplus / d delta
@@ -157,10 +160,12 @@ struct ScanBwdSmem {
   float dydsz[kTc][kCh];       // dy · silu'(z)
   float Bv[kTc][N];
   float Cv[kTc][N];
-  float H[kTc][N][kCh];        // h_t of the chunk
+  union {
+    float H[kTc][N][kCh];      // h_t of the chunk (during the chunks)
+    float red[3 + 4][nwarps(N)][kCh];  // per-channel sums of the token lanes (dD, dconv_b, dconv_w[K]; at the end)
+  };
   float part[2][kTc][kCh];     // sums over the warps' states: [0] C·h (forward) / dΔ (reverse), [1] du
   float dc[kTc + kHalo][kCh];  // conv-output gradient, rows kTc.. = first rows of the later chunk
-  float red[3 + 4][nwarps(N)][kCh];  // per-channel sums of the token lanes (dD, dconv_b, dconv_w[K])
   float dbc[2][kTc][N];        // this block's dB, dC of the chunk (summed over its channels)
 };
 
@@ -177,7 +182,7 @@ struct ChunkRegs {
 };
 
 template <int N, typename XT, typename YT>
-__global__ void __launch_bounds__(32 * nwarps(N), 3) scan_bwd_kernel(const ScanBwdParams p) {
+__global__ void __launch_bounds__(32 * nwarps(N), SAMBA_SCAN_BWD_CTAS) scan_bwd_kernel(const ScanBwdParams p) {
   constexpr int NW = nwarps(N);
   constexpr int kThreads = 32 * NW;
   constexpr int SPL = N / NW;  // states per lane
@@ -300,7 +305,6 @@ __global__ void __launch_bounds__(32 * nwarps(N), 3) scan_bwd_kernel(const ScanB
         dt = splus ? softplus_b(w) : w;
         if (full) sg = splus ? sigmoid_dev(w) : 1.f;
       }
-      S.cpre[t][pc] = pre;
       S.u[t][pc] = u;
       S.dt[t][pc] = dt;
       if (full) {
@@ -467,7 +471,11 @@ __global__ void __launch_bounds__(32 * nwarps(N), 3) scan_bwd_kernel(const ScanB
         if (ch_ok && SAMBA_CHECK(e < (int64_t)gridDim.y * L * D)) p.ddelta[e] = ddt * S.sg[t][pc];
         accD = fmaf(S.gy[t][pc], S.u[t][pc], accD);
         if (fuse) {
-          const float pre = S.cpre[t][pc];
+          // the conv output before its SiLU, again from the staged inputs
+          float pre = cb;
+          #pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (k < K) pre = fmaf(cw[k], S.x[t + kHalo - (K - 1) + k][pc], pre);
           if (csilu) {
             const float sgp = sigmoid_dev(pre);
             dcv = du * sgp * (1.f + pre * (1.f - sgp));
