@@ -106,6 +106,22 @@ def load_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def recorded_traffic(kind, workload, src):
+    """DRAM bytes per launch of one kernel on one workload, as an ncu capture
+    recorded them (read + write), or None when there is no capture or the
+    kernel's sources have changed since it was taken."""
+    from hybrid_ssm_sliding_b200 import build as B
+
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            ent = json.load(f).get(kind, {}).get(workload)
+        if ent and ent.get("kernel_hash") == B.kernel_hash(src):
+            return ent["bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
 def workload_config(wl):
     return {"workload": wl.name, "batch": wl.batch, "seq_len": wl.seqlen, "d_inner": wl.dim, "d_state": wl.dstate,
             "d_conv": wl.dconv, "heads_q": wl.heads_q, "heads_kv": wl.heads_kv, "head_dim": wl.head_dim,
@@ -953,8 +969,9 @@ def run_train(args, wl, dev, rank, world):
                     "frac": swa_tfs / peaks["bf16_tflops"], "traffic": None, "ms": ms_bswa, "band_flops": fl,
                     "peak_source": peaks["source"] + " burst"},
         "scan_bwd": {"bound": "hbm", "achieved": scan_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": scan_gbs / peaks["hbm_gbs"], "traffic": None, "ms": ms_bscan, "algorithmic_bytes": sb,
-                     "peak_source": peaks["source"]},
+                     "frac": scan_gbs / peaks["hbm_gbs"],
+                     "traffic": recorded_traffic("scan_bwd", wl.name, "scan_bwd"), "ms": ms_bscan,
+                     "algorithmic_bytes": sb, "peak_source": peaks["source"]},
     }
     dom = "scan_bwd" if ms_bscan >= ms_bswa else "swa_bwd"
     roof = {k: kernels[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
@@ -1293,16 +1310,8 @@ def main():
     mhz = (clk or {}).get("sm_mhz") or (clk or {}).get("sm_max_mhz") or 1965.0
     scan_roof["mufu"] = mufu_roof(scan_mufu_ops(wl), ms_scan, sms, mhz)
     swa_roof["mufu"] = mufu_roof(swa_exps(wl), ms_swa, sms, mhz)
-    traffic_file = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(traffic_file):
-        try:
-            tr = json.load(open(traffic_file))
-            for name, src, roof in (("scan", "scan_fwd", scan_roof), ("swa", "swa_fwd", swa_roof)):
-                ent = tr.get(name, {}).get(wl.name)
-                if ent and ent.get("kernel_hash") == B.kernel_hash(src):
-                    roof["traffic"] = ent["bytes_per_launch"]
-        except Exception:
-            pass
+    scan_roof["traffic"] = recorded_traffic("scan", wl.name, "scan_fwd")
+    swa_roof["traffic"] = recorded_traffic("swa", wl.name, "swa_fwd")
     dominant = swa_roof if ms_swa >= ms_scan else scan_roof
     roofline = {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
     roofline["kernel"] = "swa_fwd_kernel" if dominant is swa_roof else "scan_fwd_kernel"
