@@ -1092,15 +1092,19 @@ def run_decode(args, wl, lib, dev, rank, world):
     for name, ms, nb in (("scan_step", ms_scan, sb), ("swa_step", ms_swa, wb)):
         gbs = nb / (ms / 1e3) / 1e9
         kern[name] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                      "frac": gbs / peaks["hbm_gbs"], "traffic": None, "ms": ms, "algorithmic_bytes": nb,
-                      "peak_source": peaks["source"]}
+                      "frac": gbs / peaks["hbm_gbs"], "traffic": recorded_traffic(name, wl.name, "misc"),
+                      "ms": ms, "algorithmic_bytes": nb, "peak_source": peaks["source"]}
     dom = "swa_step" if ms_swa >= ms_scan else "scan_step"
     roofline = {k: kern[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
     roofline["kernel"] = dom
 
     # end to end: every step copies its inputs from pinned host memory (all of
     # a step's inputs packed in one buffer, one copy) and reads y_t and o_t
-    # back (one copy), around the library calls; 32 steps in a CUDA graph
+    # back (one copy), around the library calls; 32 steps in a CUDA graph.
+    # The steps are pipelined over two device buffer sets and three streams
+    # (copy in, compute, copy out), as a serving loop would run them: the
+    # inputs of step s+1 arrive and the outputs of step s-1 leave while step
+    # s computes.
     e2e = None
     if not args.no_e2e:
         keys = list(steps_in[0].keys())
@@ -1119,29 +1123,53 @@ def run_decode(args, wl, lib, dev, rank, world):
             for k in keys:
                 hp[offs[k]:offs[k] + nbytes(si[k])].copy_(si[k].cpu().reshape(-1).view(torch.uint8))
             host_packs.append(hp)
-        dev_pack = torch.empty(pack_bytes, dtype=torch.uint8, device=dev)
-        dev_in = {k: dev_pack[offs[k]:offs[k] + nbytes(steps_in[0][k])].view(steps_in[0][k].dtype)
-                  .view(steps_in[0][k].shape) for k in keys}
         y_bytes = (nbytes(y_t) + 255) // 256 * 256
-        out_pack = torch.empty(y_bytes + nbytes(o_t), dtype=torch.uint8, device=dev)
-        y_view = out_pack[:nbytes(y_t)].view(y_t.dtype).view(y_t.shape)
-        o_view = out_pack[y_bytes:].view(o_t.dtype).view(o_t.shape)
-        host_out = torch.empty(out_pack.numel(), dtype=torch.uint8).pin_memory()
-        h2d, d2h = pack_bytes, out_pack.numel()
+        sets = []
+        for j in range(2):
+            dev_pack = torch.empty(pack_bytes, dtype=torch.uint8, device=dev)
+            out_pack = torch.empty(y_bytes + nbytes(o_t), dtype=torch.uint8, device=dev)
+            sets.append({
+                "pack": dev_pack,
+                "in": {k: dev_pack[offs[k]:offs[k] + nbytes(steps_in[0][k])].view(steps_in[0][k].dtype)
+                       .view(steps_in[0][k].shape) for k in keys},
+                "out": out_pack,
+                "y": out_pack[:nbytes(y_t)].view(y_t.dtype).view(y_t.shape),
+                "o": out_pack[y_bytes:].view(o_t.dtype).view(o_t.shape),
+                "in_done": torch.cuda.Event(), "comp_done": torch.cuda.Event(), "out_done": torch.cuda.Event()})
+        host_out = torch.empty(sets[0]["out"].numel(), dtype=torch.uint8).pin_memory()
+        h2d, d2h = pack_bytes, sets[0]["out"].numel()
+        s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
-        def e2e_one(s_, ly):
-            dev_pack.copy_(host_packs[s_], non_blocking=True)
-            scan_one(dev_in, ly, y_view)
-            swa_one(dev_in, ly, o_view)
-            host_out.copy_(out_pack, non_blocking=True)
+        def e2e_steps():
+            cur = torch.cuda.current_stream()
+            for st in (s_in, s_comp, s_out):
+                st.wait_stream(cur)
+            for s_ in range(G):
+                st, ly = sets[s_ % 2], layers[s_ % NLY]
+                if s_ >= 2:
+                    s_in.wait_event(st["comp_done"])     # step s-2 has read this input pack
+                with torch.cuda.stream(s_in):
+                    st["pack"].copy_(host_packs[s_], non_blocking=True)
+                    st["in_done"].record(s_in)
+                s_comp.wait_event(st["in_done"])
+                if s_ >= 2:
+                    s_comp.wait_event(st["out_done"])    # the outputs of step s-2 have been read back
+                with torch.cuda.stream(s_comp):
+                    scan_one(st["in"], ly, st["y"])
+                    swa_one(st["in"], ly, st["o"])
+                    st["comp_done"].record(s_comp)
+                s_out.wait_event(st["comp_done"])
+                with torch.cuda.stream(s_out):
+                    host_out.copy_(st["out"], non_blocking=True)
+                    st["out_done"].record(s_out)
+            for st in (s_in, s_comp, s_out):
+                cur.wait_stream(st)
 
-        for s_ in range(2):
-            e2e_one(s_, layers[s_ % NLY])
+        e2e_steps()
         torch.cuda.synchronize()
         g_e2e = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_e2e):
-            for s_ in range(G):
-                e2e_one(s_, layers[s_ % NLY])
+            e2e_steps()
         g_e2e.replay()
         torch.cuda.synchronize()
         if world > 1:
