@@ -436,6 +436,119 @@ def _oracle_serve_unit(args):
         return reps, time.perf_counter() - t0
 
 
+def _oracle_layers_unit(args):
+    """The oracle's Mamba layer (kind "mamba") or the projections of its SWA
+    layer (kind "swa_proj": swa_layer with a one-key window, so that its
+    attention costs next to nothing) on n_tok tokens of one sequence at the
+    workload's widths, random float64 weights of the layer shapes.  Returns
+    the tokens done."""
+    kind, n_tok, dm, D, N, K, R, Hq, Hkv, d, seed = args
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    import oracle.samba_oracle as orc
+
+    rng = np.random.default_rng(seed)
+    hidden = rng.standard_normal((1, n_tok, dm))
+    with threadpool_limits(1):
+        if kind == "mamba":
+            orc.mamba_layer(hidden, rng.standard_normal((2 * D, dm)) / dm ** 0.5, rng.uniform(-0.5, 0.5, (D, K)),
+                            rng.uniform(-0.5, 0.5, D), rng.standard_normal((R + 2 * N, D)) / D ** 0.5,
+                            rng.standard_normal((D, R)) / R ** 0.5, rng.uniform(-6.9, -2.3, D),
+                            -np.tile(np.arange(1, N + 1, dtype=np.float64), (D, 1)), rng.standard_normal(D),
+                            rng.standard_normal((dm, D)) / D ** 0.5)
+        else:
+            orc.swa_layer(hidden, rng.standard_normal(((Hq + 2 * Hkv) * d, dm)) / dm ** 0.5,
+                          rng.standard_normal((dm, Hq * d)) / (Hq * d) ** 0.5, Hq, Hkv, d, 1)
+    return n_tok
+
+
+def oracle_layers_throughput(wl, pool, scale=1.0, seed=0):
+    """Tokens/s of the oracle's Mamba layer plus SWA layer on the host cores,
+    from three timed samples: the Mamba layer on one unit of n tokens per
+    core; the SWA layer's projections (the layer with a one-key window) on
+    one unit per core; its attention at the full window as in the prefill
+    baseline (blocks of 64 rows of one KV head's query heads)."""
+    P = host_cores()
+    n_tok = max(32, int(1024 * scale))
+    dims = (wl.d_model, wl.dim, wl.dstate, wl.dconv, wl.dt_rank, wl.heads_q, wl.heads_kv, wl.head_dim)
+    _timed_map(pool, _oracle_layers_unit, [("swa_proj", 8, 64, 64, 4, 4, 8, 2, 1, 16, 0)] * P)   # workers import
+    m_done, t_m = _timed_map(pool, _oracle_layers_unit, [("mamba", n_tok) + dims + (seed * 1000 + i,)
+                                                         for i in range(P)])
+    p_done, t_p = _timed_map(pool, _oracle_layers_unit, [("swa_proj", n_tok) + dims + (seed * 1000 + i,)
+                                                         for i in range(P)])
+    group = wl.heads_q // wl.heads_kv
+    sw_units = [(group, wl.head_dim, wl.window, 2, seed * 1000 + i) for i in range(2 * P)]
+    a_done, t_a = _timed_map(pool, _oracle_swa_unit, sw_units)
+    per_token = t_m / m_done + t_p / p_done + t_a / a_done * wl.heads_kv
+    sample = (f"{P} processes on {cpu_model()}: the Mamba layer on {P} units of {n_tok} tokens ({t_m:.1f} s), the "
+              f"SWA layer's projections on {P} units of {n_tok} tokens ({t_p:.1f} s), its attention on "
+              f"{len(sw_units)} units of 2 x 64 query rows x {group} heads at W = {wl.window} ({t_a:.1f} s); "
+              f"d_model {wl.d_model}, d_inner {wl.dim}; float64 NumPy; extrapolated to tokens/s (attention x "
+              f"{wl.heads_kv} KV heads per token)")
+    return 1.0 / per_token, P, sample
+
+
+def _oracle_train_unit(args):
+    """One training step's worth of the oracle on a sample: kind "scan" runs
+    selective_scan and selective_scan_bwd on n_chan channels x n_tok tokens
+    and returns channel-tokens done; kind "swa" runs swa and swa_bwd on one
+    KV head and its `group` query heads over n_tok tokens and returns
+    full-window row equivalents done (the band's (query, key) pairs over W)."""
+    kind, n_chan, n_tok, N, K, group, d, W, seed = args
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    import oracle.samba_oracle as orc
+
+    rng = np.random.default_rng(seed)
+    with threadpool_limits(1):
+        if kind == "scan":
+            x = rng.standard_normal((1, n_tok, n_chan))
+            z = rng.standard_normal((1, n_tok, n_chan))
+            delta = rng.uniform(-6.9, -2.3, (1, n_tok, n_chan))
+            A = -np.tile(np.arange(1, N + 1, dtype=np.float64), (n_chan, 1))
+            Bm, Cm = rng.standard_normal((1, n_tok, N)), rng.standard_normal((1, n_tok, N))
+            Dsk = rng.standard_normal(n_chan)
+            cw, cb = rng.uniform(-0.5, 0.5, (n_chan, K)), rng.uniform(-0.5, 0.5, n_chan)
+            orc.selective_scan(x, delta, A, Bm, Cm, Dsk, z, conv_w=cw, conv_b=cb)
+            orc.selective_scan_bwd(rng.standard_normal((1, n_tok, n_chan)), x, delta, A, Bm, Cm, Dsk, z,
+                                   conv_w=cw, conv_b=cb)
+            return float(n_chan * n_tok)
+        q = rng.standard_normal((1, n_tok, group, d))
+        k = rng.standard_normal((1, n_tok, 1, d))
+        v = rng.standard_normal((1, n_tok, 1, d))
+        orc.swa(q, k, v, W)
+        orc.swa_bwd(rng.standard_normal((1, n_tok, group, d)), q, k, v, W)
+        pairs = sum(min(i + 1, W) for i in range(n_tok))
+        return pairs / W
+
+
+def oracle_train_throughput(wl, pool, scale=1.0, seed=0):
+    """Training-step tokens/s of the oracle on the host cores: the scan's
+    forward and backward on one unit of 32 channels x n tokens per core, the
+    attention's forward and backward on one unit per core of one KV head over
+    W + 256 tokens, extrapolated by channels and by the band's pairs."""
+    P = host_cores()
+    n_tok = max(256, int(16384 * scale))
+    group = wl.heads_q // wl.heads_kv
+    _timed_map(pool, _oracle_train_unit, [("scan", 8, 64, wl.dstate, wl.dconv, 1, 16, 16, 0)] * P)   # workers import
+    sc_units = [("scan", 32, n_tok, wl.dstate, wl.dconv, group, wl.head_dim, wl.window, seed * 1000 + i)
+                for i in range(P)]
+    sw_tok = wl.window + max(64, int(256 * scale))
+    sw_units = [("swa", 0, sw_tok, wl.dstate, wl.dconv, group, wl.head_dim, wl.window, seed * 1000 + i)
+                for i in range(P)]
+    sc_done, t_sc = _timed_map(pool, _oracle_train_unit, sc_units)
+    sw_done, t_sw = _timed_map(pool, _oracle_train_unit, sw_units)
+    per_token = t_sc / sc_done * wl.dim + t_sw / sw_done * wl.heads_kv
+    sample = (f"{P} processes on {cpu_model()}: the scan's forward and backward on {P} units of 32 channels x "
+              f"{n_tok} tokens ({t_sc:.1f} s), the attention's forward and backward on {P} units of one KV head "
+              f"with {group} query heads over {sw_tok} tokens at W = {wl.window} ({t_sw:.1f} s); float64 NumPy; "
+              f"extrapolated to tokens/s (scan x {wl.dim} channels, attention by the band's pairs x "
+              f"{wl.heads_kv} KV heads per token)")
+    return 1.0 / per_token, P, sample
+
+
 def oracle_serve_throughput(wl, pool, scale=1.0, seed=0, pairs=None):
     """Decode tokens/s of the oracle's layer steps on the host cores: one unit
     per core of `reps` steps of one sequence through one layer pair (the steps
@@ -575,6 +688,58 @@ def run_layers(args, wl, dev, rank, world):
     roof = {"bound": "tensor", "achieved": tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
             "frac": tfs / peaks["bf16_tflops"], "traffic": None, "kernel": "gemm_kernel (input projection)",
             "ms": ms_in, "flops": fl_in, "peak_source": peaks["source"] + " burst"}
+    # ---- end to end: every step copies the hidden state in from pinned host
+    # memory and reads both layers' outputs back, pipelined over two device
+    # buffers and three streams (copy in, compute, copy out) as in the mixer
+    # prefill line
+    e2e = None
+    if not args.no_e2e:
+        host_h = hidden.cpu().pin_memory()
+        host_out = [torch.empty(host_h.shape, dtype=host_h.dtype).pin_memory() for _ in range(2)]
+        sets = [{"h": hidden if j == 0 else torch.empty_like(hidden), "in_done": torch.cuda.Event(),
+                 "comp_done": torch.cuda.Event()} for j in range(2)]
+        s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+
+        def e2e_step(i):
+            st = sets[i % 2]
+            if i >= 2:
+                s_in.wait_event(st["comp_done"])     # step i-2 has read this buffer
+            with torch.cuda.stream(s_in):
+                st["h"].copy_(host_h, non_blocking=True)
+                st["in_done"].record(s_in)
+            s_comp.wait_event(st["in_done"])
+            with torch.cuda.stream(s_comp):
+                m_out = layers.mamba_layer_prefill(st["h"], mw)[0]
+                w_out = layers.swa_layer_prefill(st["h"], sw)[0]
+                st["comp_done"].record(s_comp)
+            s_out.wait_event(st["comp_done"])
+            with torch.cuda.stream(s_out):
+                for t_, h_ in ((m_out, host_out[0]), (w_out, host_out[1])):
+                    t_.record_stream(s_out)           # not reused before this copy has run
+                    h_.copy_(t_, non_blocking=True)
+
+        e2e_step(0)
+        e2e_step(1)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(4, args.e2e_steps)
+        a.record(s_in)
+        for i in range(n_e2e):
+            e2e_step(i)
+        b.record(s_out)
+        torch.cuda.synchronize()
+        ms_e2e = max_over_ranks(a.elapsed_time(b) / n_e2e, dev)
+        nb = host_h.numel() * host_h.element_size()
+        e2e = {"value": whole_job_rate(wl.batch * wl.seqlen, world, ms_e2e), "unit": UNIT,
+               "h2d_bytes_per_step": nb, "d2h_bytes_per_step": 2 * nb, "ms_per_step": ms_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        with oracle_pool() as pool:
+            v, cores, sample = oracle_layers_throughput(wl, pool)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
     cfg = workload_config(wl)
     cfg.update({"d_model": wl.d_model, "dt_rank": wl.dt_rank,
                 "layer_gemm_flops_per_step": layer_gemm_flops(wl)})
@@ -583,7 +748,7 @@ def run_layers(args, wl, dev, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (random weights of the layer shapes)", "config": cfg, "roofline": roof,
-        "cpu_baseline": None, "e2e": None, "clocks": clk, "gpu_launches": 11 * args.steps,
+        "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "gpu_launches": 11 * args.steps,
         "status": ops.get_status(),
     }
 
@@ -940,15 +1105,23 @@ def run_train(args, wl, dev, rank, world):
 
     aux = torch.cuda.Stream()
 
-    def step():
+    def train_step(ins, gr):
+        """Forward and backward of both mixers on the activations `ins` and
+        output gradients `gr` (the parameters A, D and the conv stay put);
+        returns the scan's and the attention's gradients."""
+        sin = dict(scan_in, z=ins["z"])
+        ops.selective_scan_fwd(ins["x"], ins["delta"], inp["A"], ins["B"], ins["C"], y=y, h_ckpt=ckpt, **sin)
+        ops.swa_fwd(ins["q"], ins["k"], ins["v"], wl.window, o=o, lse=lse)
         # the two backward passes are independent: the attention's runs on a
         # second stream and takes the SMs the scan's last wave leaves free
-        fwd()
-        ops.mixer_bwd(dict(dy=grads["dy"], x=inp["x"], delta=inp["delta"], A=inp["A"], B=inp["B"], C=inp["C"],
-                           workspace=ws_scan, ckpt=ckpt, **scan_in),
-                      dict(do=grads["do"], q=inp["q"], k=inp["k"], v=inp["v"], o=o, lse=lse, window=wl.window,
-                           dq=dq, dk=dk, dv=dv, workspace=ws_swa),
-                      aux_stream=aux)
+        return ops.mixer_bwd(dict(dy=gr["dy"], x=ins["x"], delta=ins["delta"], A=inp["A"], B=ins["B"], C=ins["C"],
+                                  workspace=ws_scan, ckpt=ckpt, **sin),
+                             dict(do=gr["do"], q=ins["q"], k=ins["k"], v=ins["v"], o=o, lse=lse, window=wl.window,
+                                  dq=dq, dk=dk, dv=dv, workspace=ws_swa),
+                             aux_stream=aux)
+
+    def step():
+        train_step(inp, grads)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -1002,6 +1175,70 @@ def run_train(args, wl, dev, rank, world):
     dom = "scan_bwd" if ms_bscan >= ms_bswa else "swa_bwd"
     roof = {k: kernels[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
     roof["kernel"] = "scan_bwd_kernel" if dom == "scan_bwd" else "swa_bwd_kv_kernel + swa_bwd_q_kernel"
+    # ---- end to end: every step copies its activations (x, z, delta, B, C,
+    # q, k, v) and output gradients (dy, dO) in from pinned host memory and
+    # reads the parameters' gradients (dA, dD, dconv_w, dconv_b) back; the
+    # activations' gradients stay on the device for the layer below.
+    # Pipelined over two device buffer sets and three streams (copy in,
+    # compute, copy out) as in the mixer prefill line.
+    e2e = None
+    if not args.no_e2e:
+        act_keys, grad_keys = ("x", "z", "delta", "B", "C", "q", "k", "v"), ("dy", "do")
+        param_grads = ("dA", "dD", "dconv_w", "dconv_b")
+        host_act = {k: inp[k].cpu().pin_memory() for k in act_keys}
+        host_gr = {k: grads[k].cpu().pin_memory() for k in grad_keys}
+        sets = []
+        for j in range(2):
+            sets.append({"ins": {k: inp[k] if j == 0 else torch.empty_like(inp[k]) for k in act_keys},
+                         "gr": {k: grads[k] if j == 0 else torch.empty_like(grads[k]) for k in grad_keys},
+                         "in_done": torch.cuda.Event(), "comp_done": torch.cuda.Event()})
+        e2e_sg = train_step(inp, grads)[0]
+        host_pg = {k: torch.empty(e2e_sg[k].shape, dtype=e2e_sg[k].dtype).pin_memory() for k in param_grads}
+        s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+
+        def e2e_step(i):
+            st = sets[i % 2]
+            if i >= 2:
+                s_in.wait_event(st["comp_done"])     # step i-2 has read these buffers
+            with torch.cuda.stream(s_in):
+                for k in act_keys:
+                    st["ins"][k].copy_(host_act[k], non_blocking=True)
+                for k in grad_keys:
+                    st["gr"][k].copy_(host_gr[k], non_blocking=True)
+                st["in_done"].record(s_in)
+            s_comp.wait_event(st["in_done"])
+            with torch.cuda.stream(s_comp):
+                sg = train_step(st["ins"], st["gr"])[0]
+                st["comp_done"].record(s_comp)
+            s_out.wait_event(st["comp_done"])
+            with torch.cuda.stream(s_out):
+                for k in param_grads:
+                    sg[k].record_stream(s_out)         # not reused before this copy has run
+                    host_pg[k].copy_(sg[k], non_blocking=True)
+
+        e2e_step(0)
+        e2e_step(1)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(4, args.e2e_steps)
+        a.record(s_in)
+        for i in range(n_e2e):
+            e2e_step(i)
+        b.record(s_out)
+        torch.cuda.synchronize()
+        ms_e2e = max_over_ranks(a.elapsed_time(b) / n_e2e, dev)
+        h2d = sum(t.numel() * t.element_size() for t in list(host_act.values()) + list(host_gr.values()))
+        d2h = sum(t.numel() * t.element_size() for t in host_pg.values())
+        e2e = {"value": whole_job_rate(wl.batch * wl.seqlen, world, ms_e2e), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        with oracle_pool() as pool:
+            v, cores, sample = oracle_train_throughput(wl, pool)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
     cfg = workload_config(wl)
     cfg["step"] = ("scan and SWA forward (with log-sum-exp and the scan's 16-token state checkpoints), then scan "
                    "and SWA backward from seeded dy, dO (samba_mixer_bwd, the SWA backward on a second stream)")
@@ -1011,7 +1248,7 @@ def run_train(args, wl, dev, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": cfg, "roofline": roof, "kernels": kernels,
         "phases_ms": {"forward": ms_fwd, "scan_backward": ms_bscan, "swa_backward": ms_bswa},
-        "cpu_baseline": None, "e2e": None, "clocks": clk, "gpu_launches": 7 * args.steps,
+        "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "gpu_launches": 7 * args.steps,
         "status": ops.get_status(),
     }
 
