@@ -79,17 +79,26 @@ __global__ void conv1d_step_kernel(const XT* __restrict__ x, const float* __rest
   pdl_launch_dependents();
   pdl_wait();
   const int64_t n = B * D;
+  // The window [state (K - 1 values), x] sits at the end of four registers:
+  // v[j] holds tap k = j - (4 - K), so every index is fixed once the loops
+  // are unrolled (K is 2..4) and the taps never go to local memory.
+  const int off = 4 - K;
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
     const int64_t c = e % D;
-    float xp[4];
-    for (int k = 0; k < K - 1; ++k) xp[k] = cs_in ? cs_in[e * (K - 1) + k] : 0.f;
-    xp[K - 1] = to_f32<XT>(x[e]);
+    float v[4];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) v[j] = (j >= off && cs_in) ? cs_in[e * (K - 1) + (j - off)] : 0.f;
+    v[3] = to_f32<XT>(x[e]);
     float acc = bias ? bias[c] : 0.f;
-    for (int k = 0; k < K; ++k) acc = fmaf(w[c * K + k], xp[k], acc);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (j >= off) acc = fmaf(w[c * K + (j - off)], v[j], acc);
     if (silu) acc = silu_dev(acc);
     if (!SAMBA_CHECK(e >= 0 && e < n && K <= 4)) continue;
     u[e] = from_f32<UT>(acc);
-    for (int k = 0; k < K - 1; ++k) cs_out[e * (K - 1) + k] = xp[k + 1];
+#pragma unroll
+    for (int j = 1; j < 4; ++j)
+      if (j > off) cs_out[e * (K - 1) + (j - off - 1)] = v[j];
   }
 }
 
