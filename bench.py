@@ -1309,16 +1309,19 @@ def run_decode(args, wl, lib, dev, rank, world):
     # One decode step of the mixer pair: the two mixers' steps are independent
     # (each reads its own inputs and state), so the SWA step is forked onto a
     # second stream and both are joined before the next step starts, as the
-    # mixer prefill's two-stream form does; the scan step's CTAs run on the
-    # SMs beside the SWA step's.  The same steps on one stream are timed too.
+    # mixer prefill's two-stream form does.  The SWA step is issued first: its
+    # CTAs take their four slots per SM, and the scan step's CTAs run in the
+    # threads and registers left beside them (issued the other way round, the
+    # scan step's CTAs fill the SMs and the SWA step waits for them).  The same
+    # steps on one stream are timed too.
     aux = torch.cuda.Stream()
 
     def step_pair(si, ly, y_out=None, o_out=None):
         cur = torch.cuda.current_stream()
         aux.wait_stream(cur)
-        scan_one(si, ly, y_out)
         with torch.cuda.stream(aux):
             swa_one(si, ly, o_out)
+        scan_one(si, ly, y_out)
         cur.wait_stream(aux)
 
     g_step = capture(step_pair)
