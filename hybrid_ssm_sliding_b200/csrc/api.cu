@@ -138,7 +138,7 @@ static int check_scan(const samba_scan_args* a, const char* who) {
   if ((a->flags & SAMBA_SCAN_FUSE_CONV) && !a->conv_w)
     return fail(SAMBA_ERR_INVALID_ARG, "%s: FUSE_CONV needs conv_w", who);
   if (a->flags & ~7u) return fail(SAMBA_ERR_INVALID_ARG, "%s: unknown flag bits", who);
-  const void* ptrs[] = {a->x, a->z, a->delta, a->Bm, a->Cm, a->y};
+  const void* ptrs[] = {a->x, a->z, a->delta, a->Bm, a->Cm, a->y, a->h_ckpt};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SAMBA_ERR_INVALID_ARG, "%s: misaligned pointer", who);
   return SAMBA_OK;
@@ -201,7 +201,7 @@ static int check_scan_bwd(const samba_scan_bwd_args* a, const char* who) {
   const bool fuse = (a->flags & SAMBA_SCAN_FUSE_CONV) != 0;
   if (fuse && (!a->dconv_w || (a->conv_b && !a->dconv_b)))
     return fail(SAMBA_ERR_INVALID_ARG, "%s: dconv_w (and dconv_b with conv_b) are required with FUSE_CONV", who);
-  const void* ptrs[] = {a->dx, a->dz, a->ddelta, a->dB, a->dC, a->workspace};
+  const void* ptrs[] = {a->dx, a->dz, a->ddelta, a->dB, a->dC, a->workspace, a->ckpt};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SAMBA_ERR_INVALID_ARG, "%s: misaligned pointer", who);
   const size_t need = scan_bwd_workspace(a->batch, a->seqlen, a->dim, a->dstate);

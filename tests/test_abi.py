@@ -82,6 +82,7 @@ def _scan_args(**over):
     (dict(conv_w=None), L.SAMBA_ERR_INVALID_ARG),
     (dict(flags=64), L.SAMBA_ERR_INVALID_ARG),
     (dict(x=0x10008), L.SAMBA_ERR_INVALID_ARG),
+    (dict(h_ckpt=0x10004), L.SAMBA_ERR_INVALID_ARG),   # checkpoints are a base pointer too
 ])
 def test_scan_rejects_bad_arguments_on_host(lib, over, code):
     a = _scan_args(**over)
@@ -277,6 +278,37 @@ def test_scan_bwd_rejects_bad_arguments_on_host(lib):
     assert call(dstate=12) == L.SAMBA_ERR_UNSUPPORTED
     assert call(workspace=None) == L.SAMBA_ERR_WORKSPACE
     assert call(workspace_bytes=need - 1) == L.SAMBA_ERR_WORKSPACE
+    assert call(ckpt=f + 4) == L.SAMBA_ERR_INVALID_ARG                   # the forward's checkpoints, misaligned
+
+
+def test_mixer_bwd_checks_both_arguments_before_any_launch(lib):
+    """samba_mixer_bwd validates the scan's and the attention's arguments
+    before it creates its events or launches anything (with or without an
+    aux stream), and returns the first failing check's code."""
+    f = 0x80000
+    s = L.ScanBwdArgs()
+    for k in ("x", "delta", "A", "Bm", "Cm", "dy", "dx", "ddelta", "dA", "dB", "dC", "workspace"):
+        setattr(s, k, f)
+    s.batch, s.seqlen, s.dim, s.dstate, s.dconv = 2, 100, 64, 16, 4
+    s.workspace_bytes = lib.samba_scan_bwd_workspace_size(2, 100, 64, 16)
+    s.x_dtype = s.y_dtype = 1
+    w = L.SwaBwdArgs()
+    for key in ("q", "k", "v", "o", "lse", "dO", "dq", "dk", "dv", "workspace"):
+        setattr(w, key, f)
+    w.workspace_bytes = lib.samba_swa_bwd_workspace_size(2, 100, 8)
+    w.batch, w.seqlen, w.window, w.heads_q, w.heads_kv, w.head_dim = 2, 100, 16, 8, 2, 64
+    for aux in (None, 0x1234):  # the aux handle is never used when a check fails
+        assert lib.samba_mixer_bwd(None, ctypes.byref(w), None, aux) == L.SAMBA_ERR_INVALID_ARG
+        assert lib.samba_mixer_bwd(ctypes.byref(s), None, None, aux) == L.SAMBA_ERR_INVALID_ARG
+        s.dstate = 12
+        assert lib.samba_mixer_bwd(ctypes.byref(s), ctypes.byref(w), None, aux) == L.SAMBA_ERR_UNSUPPORTED
+        s.dstate = 16
+        w.head_dim = 48
+        assert lib.samba_mixer_bwd(ctypes.byref(s), ctypes.byref(w), None, aux) == L.SAMBA_ERR_UNSUPPORTED
+        w.head_dim = 64
+        w.workspace_bytes -= 4
+        assert lib.samba_mixer_bwd(ctypes.byref(s), ctypes.byref(w), None, aux) == L.SAMBA_ERR_WORKSPACE
+        w.workspace_bytes += 4
 
 
 def test_swa_bwd_rejects_bad_arguments_on_host(lib):
