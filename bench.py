@@ -948,8 +948,12 @@ def run_serve(args, wl, dev, rank, world):
         torch.cuda.synchronize()
         ms = a.elapsed_time(b) / (n * G)            # per decode step, all pairs
         gbs = nbytes[name] / (ms / 1e3) / 1e9
+        # DRAM bytes per step where a capture of this class's kernel in this
+        # workload is recorded: per launch, times the launches of a step
+        per_launch = recorded_traffic(name, wl.name, "misc") if name in ("swa_step", "scan_step") else None
         kern[name] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                      "frac": gbs / peaks["hbm_gbs"], "traffic": None, "ms_per_step": ms,
+                      "frac": gbs / peaks["hbm_gbs"],
+                      "traffic": per_launch * SERVE_PAIRS if per_launch is not None else None, "ms_per_step": ms,
                       "algorithmic_bytes_per_step": nbytes[name], "peak_source": peaks["source"]}
         del kg
     dom = max(kern, key=lambda k: kern[k]["ms_per_step"])
