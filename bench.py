@@ -686,7 +686,8 @@ def run_layers(args, wl, dev, rank, world):
     fl_in = 2.0 * M * 2 * wl.dim * wl.d_model
     tfs = fl_in / (ms_in / 1e3) / 1e12
     roof = {"bound": "tensor", "achieved": tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": tfs / peaks["bf16_tflops"], "traffic": None, "kernel": "gemm_kernel (input projection)",
+            "frac": tfs / peaks["bf16_tflops"], "traffic": recorded_traffic("in_proj", wl.name, "gemm"),
+            "kernel": "gemm_kernel (input projection)",
             "ms": ms_in, "flops": fl_in, "peak_source": peaks["source"] + " burst"}
     # ---- end to end: every step copies the hidden state in from pinned host
     # memory and reads both layers' outputs back, pipelined over two device
