@@ -92,3 +92,24 @@ def test_serve_step_bytes_term_by_term():
     assert set(got) == set(want)
     for k in want:
         assert got[k] == bench.SERVE_PAIRS * want[k], k
+
+
+def test_recorded_traffic_only_for_the_captured_source(monkeypatch):
+    """bench.py reports a kernel's DRAM bytes only while its source still
+    hashes to the one the capture was taken from, and only for a recorded
+    (kernel, workload) pair."""
+    import json
+    import os
+
+    from hybrid_ssm_sliding_b200 import build as B
+
+    with open(os.path.join(os.path.dirname(bench.__file__), "profiles", "traffic.json")) as f:
+        rec = json.load(f)
+    ent = rec["scan"]["prefill_128k"]
+    assert ent["bytes_per_launch"] == ent["read"] + ent["write"]
+    monkeypatch.setattr(B, "kernel_hash", lambda src: ent["kernel_hash"])
+    assert bench.recorded_traffic("scan", "prefill_128k", "scan_fwd") == ent["bytes_per_launch"]
+    assert bench.recorded_traffic("scan", "no_such_workload", "scan_fwd") is None
+    assert bench.recorded_traffic("no_such_kernel", "prefill_128k", "scan_fwd") is None
+    monkeypatch.setattr(B, "kernel_hash", lambda src: "0" * 12)    # the source changed since
+    assert bench.recorded_traffic("scan", "prefill_128k", "scan_fwd") is None
